@@ -1,0 +1,183 @@
+"""CPU oracle for the expert-routed quantized matmul (ctypes wrapper of oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline / reference legs of ``bench.py``. The product package never
+imports it.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c with gcc into liboracle.so (plain -O2, IEEE double)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(
+            ["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math", "-ffp-contract=off",
+             "-o", _LIB, _SRC, "-lm", "-lpthread"]
+        )
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        u8p, u16p, u32p, dp, vp = (ctypes.POINTER(t) for t in
+                                   (ctypes.c_uint8, ctypes.c_uint16, ctypes.c_uint32,
+                                    ctypes.c_double, ctypes.c_void_p))
+        u32, u64, i32 = ctypes.c_uint32, ctypes.c_uint64, ctypes.c_int
+        L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_double.restype = ctypes.c_double
+        L.oracle_f16_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_f16_to_double.restype = ctypes.c_double
+        L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_to_double.restype = ctypes.c_double
+        L.oracle_e2m1_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_to_double.restype = ctypes.c_double
+        L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_double_to_f16.argtypes = [ctypes.c_double]
+        L.oracle_double_to_f16.restype = ctypes.c_uint16
+        L.oracle_round_out.argtypes = [ctypes.c_void_p, ctypes.c_void_p, u64, i32]
+        L.oracle_round_out.restype = None
+        L.oracle_row_bytes.argtypes = [i32, i32, u32]
+        L.oracle_row_bytes.restype = u64
+        L.oracle_code.argtypes = [ctypes.c_void_p, i32, i32, u32]
+        L.oracle_code.restype = u32
+        common = [u32, u32, u32, u32, u32, i32, u32, u32, i32, i32]
+        L.oracle_qmm_id.argtypes = [ctypes.c_void_p] * 6 + common
+        L.oracle_qmm_id.restype = ctypes.c_int64
+        L.oracle_qmm_id_sample.argtypes = [ctypes.c_void_p] * 7 + [u64, ctypes.c_void_p] + common
+        L.oracle_qmm_id_sample.restype = i32
+        L.oracle_expert_max_abs_weight.argtypes = [ctypes.c_void_p] * 3 + [u32, u32, u32, u32,
+                                                                            u32, i32, u32]
+        L.oracle_expert_max_abs_weight.restype = ctypes.c_double
+        L.oracle_route.argtypes = [ctypes.c_void_p, u64, u32, u32, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, u64]
+        L.oracle_route.restype = ctypes.c_int64
+        del u8p, u16p, u32p, dp, vp
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ decoders
+
+def bf16_to_double(bits: int) -> float:
+    return lib().oracle_bf16_to_double(int(bits))
+
+
+def f16_to_double(bits: int) -> float:
+    return lib().oracle_f16_to_double(int(bits))
+
+
+def e4m3_to_double(b: int) -> float:
+    return lib().oracle_e4m3_to_double(int(b))
+
+
+def e2m1_to_double(c: int) -> float:
+    return lib().oracle_e2m1_to_double(int(c))
+
+
+def double_to_bf16(v: float) -> int:
+    return lib().oracle_double_to_bf16(float(v))
+
+
+def double_to_f16(v: float) -> int:
+    return lib().oracle_double_to_f16(float(v))
+
+
+def round_out(vals: np.ndarray, out_dtype: int) -> np.ndarray:
+    """Round doubles to the output dtype's storage: float32 array, or uint16 bits."""
+    vals = np.ascontiguousarray(vals, dtype=np.float64)
+    out = np.empty(vals.shape, dtype=np.float32 if out_dtype == 0 else np.uint16)
+    lib().oracle_round_out(_ptr(vals), _ptr(out), vals.size, out_dtype)
+    return out
+
+
+def row_bytes(fmt: int, bits: int, k: int) -> int:
+    return lib().oracle_row_bytes(fmt, bits, k)
+
+
+def code(row: np.ndarray, fmt: int, bits: int, j: int) -> int:
+    row = np.ascontiguousarray(row, dtype=np.uint8)
+    return lib().oracle_code(_ptr(row), fmt, bits, j)
+
+
+# ------------------------------------------------------------------ operation
+
+def _common(P):
+    return [P.m, P.k, P.n, P.group_size, P.bits, P.fmt, P.n_expert_used, P.num_experts,
+            P.x_dtype]
+
+
+def _arrays(P):
+    return [np.ascontiguousarray(a) for a in (P.x, P.ids, P.packed, P.scales, P.aux)]
+
+
+def qmm_id(P, nthreads: int | None = None):
+    """Full output, double [m*n_expert_used, n]; returns (out, number of bad ids)."""
+    arrs = _arrays(P)
+    out = np.empty((P.R, P.n), dtype=np.float64)
+    rc = lib().oracle_qmm_id(*[_ptr(a) for a in arrs], _ptr(out), *_common(P),
+                             nthreads or default_threads())
+    if rc < 0:
+        raise ValueError("oracle rejected the problem")
+    return out, int(rc)
+
+
+def qmm_id_sample(P, pairs: np.ndarray, cols: np.ndarray, nthreads: int | None = None):
+    """out[pairs[i], cols[i]] in double."""
+    arrs = _arrays(P)
+    pairs = np.ascontiguousarray(pairs, dtype=np.uint32)
+    cols = np.ascontiguousarray(cols, dtype=np.uint32)
+    vals = np.empty(pairs.shape, dtype=np.float64)
+    rc = lib().oracle_qmm_id_sample(*[_ptr(a) for a in arrs], _ptr(pairs), _ptr(cols),
+                                    pairs.size, _ptr(vals), *_common(P),
+                                    nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle rejected the sample")
+    return vals
+
+
+def expert_max_abs_weight(P, e: int) -> float:
+    arrs = _arrays(P)
+    return lib().oracle_expert_max_abs_weight(_ptr(arrs[2]), _ptr(arrs[3]), _ptr(arrs[4]), e,
+                                              P.k, P.n, P.group_size, P.bits, P.fmt,
+                                              P.num_experts)
+
+
+def route(ids: np.ndarray, num_experts: int, tile_rows: int):
+    """Reference routing: counts[E+1], offsets[E+2], sorted_pairs[R], tiles[ntiles, 2]."""
+    ids = np.ascontiguousarray(ids, dtype=np.uint32).reshape(-1)
+    R = ids.size
+    counts = np.zeros(num_experts + 1, np.uint32)
+    offsets = np.zeros(num_experts + 2, np.uint32)
+    sp = np.zeros(max(R, 1), np.uint32)
+    max_tiles = R // tile_rows + num_experts + 1
+    tiles = np.zeros((max_tiles, 2), np.uint32)
+    nt = lib().oracle_route(_ptr(ids), R, num_experts, tile_rows, _ptr(counts), _ptr(offsets),
+                            _ptr(sp), _ptr(tiles), max_tiles)
+    if nt < 0:
+        raise ValueError("tile list overflow")
+    return counts, offsets, sp[:R], tiles[:nt]
