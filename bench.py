@@ -1,0 +1,448 @@
+"""Benchmark of the expert-routed quantized matmul on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config decode|canvas|prefill|skewed]
+
+Default workload ("decode"): one MoE decode step for one token: the gate/up
+projection (128 experts, top-8, k=2816, n=1408) followed by the down projection
+(k=704, n=2816), both 4-bit affine with group 64, bf16 x, f32 out. Every step
+uses fresh ids (8 distinct uniform experts), fresh x, and the next of 16 copies
+of the expert weights (6.9 GB rotated, far above the 126 MB L2), so no step
+finds its weights in L2. The K timed steps are replayed from CUDA graphs of up
+to 1000 steps (launch overhead of the graph only, no host work).
+
+Metric: effective HBM GB/s = algorithmic bytes / time, algorithmic bytes = the
+touched experts' packed codes + scales + biases read once, plus x and out.
+Also reported: us per call of each projection, the roofline fraction against
+MEASURED_PEAKS.json's copy bandwidth, the end-to-end number through the Python
+API with host buffers, and the CPU oracle on a bounded sample.
+
+--impl reference times the CPU oracle (the only reference there is) on a
+bounded sample of the same workload. N > 1: independent replicas, one per GPU
+(the operation has no exchange step), value = total bytes / max time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
+N_LAYERS = 16
+GRAPH_STEPS = 1000
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------- setup
+
+class Dist:
+    def __init__(self, gpus):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if torch.cuda.is_available():
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            if torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, v: float) -> float:
+        if not self.pg:
+            return v
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def alg_bytes(P, ids_row_sets) -> float:
+    """Algorithmic bytes of one call: touched experts' codes + scales (+ biases or
+    scale2) read once, x read once, out written once."""
+    from workloads.gen import FMT_AFFINE, FMT_CODEBOOK
+
+    per_row = P.row_bytes + P.groups * (2 if P.fmt in (FMT_AFFINE, FMT_CODEBOOK) else 1)
+    if P.fmt == FMT_AFFINE:
+        per_row += P.groups * 2
+    per_expert = P.n * per_row + (4 if P.fmt == 2 else 0)
+    distinct = np.unique(ids_row_sets[ids_row_sets < P.num_experts]).size
+    xb = P.m * P.k * (4 if P.x_dtype == 0 else 2)
+    ob = P.R * P.n * (4 if P.out_dtype == 0 else 2)
+    cb = (1 << P.bits) * 2 if P.fmt == FMT_CODEBOOK else 0
+    return float(distinct * per_expert + xb + ob + cb)
+
+
+def clocks_sampler(device_index: int):
+    """Start nvidia-smi sampling SM clocks and throttle reasons every 200 ms."""
+    try:
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        sel = ["--id=GPU-" + uuid] if uuid and not uuid.startswith("GPU-") else ["--id=" + uuid]
+    except Exception:
+        sel = []
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    try:
+        return subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                text=True)
+    except Exception:
+        return None
+
+
+def clocks_summary(proc):
+    if proc is None:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    proc.terminate()
+    try:
+        out, _ = proc.communicate(timeout=5)
+    except Exception:
+        proc.kill()
+        out = ""
+    sm, smax, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in out.strip().splitlines():
+        f = [x.strip() for x in line.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            sm.append(float(f[1]))
+            smax.append(float(f[2]))
+        except ValueError:
+            continue
+        for name, val in zip(names, f[5:9]):
+            if val.lower().startswith("active"):
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our workload
+
+class DecodeWorkload:
+    """gate/up + down projections of one decode token, rotating weight copies."""
+
+    def __init__(self, steps_per_graph: int, seed: int = 2):
+        import moe_expert_routed_b200 as M
+        from workloads.torch_io import to_device
+        from workloads import config_problem
+        from workloads.gen import bf16_bits, distinct_uniform_ids
+
+        self.M = M
+        self.projs = [config_problem("decode_gate_up"), config_problem("decode_down")]
+        self.G = steps_per_graph
+        rng = np.random.Generator(np.random.PCG64(seed + 100))
+        self.layers = []
+        for P in self.projs:
+            base = to_device(P)
+            copies = []
+            for _ in range(N_LAYERS):
+                copies.append({k: (v.clone() if k in ("packed", "scales", "aux") else v)
+                               for k, v in base.items()})
+            self.layers.append(copies)
+        # fresh ids and x for every step of the graph
+        self.ids = [torch.from_numpy(distinct_uniform_ids(rng, self.G, 8, P.num_experts)
+                                     .view(np.int32)).cuda() for P in self.projs]
+        self.x = [torch.from_numpy(bf16_bits(rng.standard_normal((self.G, P.k), dtype=np.float32))
+                                   .view(np.int16)).view(torch.bfloat16).cuda() for P in self.projs]
+        self.out = [torch.empty((self.G, 8, P.n), dtype=torch.float32, device="cuda")
+                    for P in self.projs]
+        self.ws = [M.new_workspace(1, 8, P.num_experts) for P in self.projs]
+        self.step_bytes = [
+            [alg_bytes(P, self.ids[i][s].cpu().numpy().view(np.uint32)) for s in range(self.G)]
+            for i, P in enumerate(self.projs)]
+
+    def call(self, proj: int, s: int):
+        P = self.projs[proj]
+        L = self.layers[proj][s % N_LAYERS]
+        self.M.qmm_id(self.x[proj][s:s + 1], self.ids[proj][s:s + 1], L["packed"], L["scales"],
+                      L["aux"], n=P.n, group_size=P.group_size, bits=P.bits, fmt=P.fmt,
+                      num_experts=P.num_experts, out=self.out[proj][s], workspace=self.ws[proj])
+
+    def step(self, s: int, projs=(0, 1)):
+        for p in projs:
+            self.call(p, s)
+
+    def bytes(self, projs=(0, 1)) -> float:
+        return sum(sum(self.step_bytes[p]) for p in projs)
+
+    def capture(self, projs=(0, 1)):
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            for s in range(min(self.G, 4)):
+                self.step(s, projs)  # warm the launch path outside capture
+        torch.cuda.current_stream().wait_stream(st)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for s in range(self.G):
+                self.step(s, projs)
+        torch.cuda.synchronize()
+        return g
+
+
+def time_graph(g, replays: int) -> float:
+    """Seconds for `replays` replays of g, CUDA events on the current stream."""
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / 1e3
+
+
+def e2e_decode(W: DecodeWorkload, steps: int):
+    """Through the public API with host buffers: per step, pinned host x and ids are
+    copied in, both projections run, both outputs are copied back."""
+    M = W.M
+    hx = [W.x[i][: min(steps, W.G)].cpu().pin_memory() for i in range(2)]
+    hid = [W.ids[i][: min(steps, W.G)].cpu().pin_memory() for i in range(2)]
+    hout = [torch.empty((8, P.n), dtype=torch.float32).pin_memory() for P in W.projs]
+    dx = [torch.empty((1, P.k), dtype=torch.bfloat16, device="cuda") for P in W.projs]
+    did = [torch.empty((1, 8), dtype=torch.int32, device="cuda") for _ in W.projs]
+    dout = [torch.empty((1, 8, P.n), dtype=torch.float32, device="cuda") for P in W.projs]
+    n = hx[0].shape[0]
+    h2d = sum(hx[i][0].numel() * 2 + hid[i][0].numel() * 4 for i in range(2))
+    d2h = sum(o.numel() * 4 for o in hout)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(steps):
+        i = s % n
+        for p, P in enumerate(W.projs):
+            dx[p].copy_(hx[p][i:i + 1], non_blocking=True)
+            did[p].copy_(hid[p][i:i + 1], non_blocking=True)
+            L = W.layers[p][s % N_LAYERS]
+            M.qmm_id(dx[p], did[p], L["packed"], L["scales"], L["aux"], n=P.n,
+                     group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
+                     out=dout[p], workspace=W.ws[p])
+            hout[p].copy_(dout[p][0], non_blocking=True)
+    b.record()
+    b.synchronize()
+    secs = a.elapsed_time(b) / 1e3
+    per_step_bytes = W.bytes() / W.G
+    return secs, per_step_bytes, h2d, d2h
+
+
+# ------------------------------------------------------------------- oracle
+
+def oracle_decode_sample(budget_s: float = 12.0):
+    """CPU oracle on a bounded sample of the decode step: every output of the
+    gate/up and down projections of one token (both full calls), repeated until
+    the time budget is used. Returns (GB/s in the metric's unit, seconds, threads,
+    sample description)."""
+    import oracle
+    from workloads import config_problem
+
+    projs = [config_problem("decode_gate_up"), config_problem("decode_down")]
+    threads = oracle.default_threads()
+    nbytes, secs, calls = 0.0, 0.0, 0
+    while secs < budget_s or calls < 2:
+        for P in projs:
+            pairs = np.repeat(np.arange(P.R), P.n)
+            cols = np.tile(np.arange(P.n), P.R)
+            t0 = time.perf_counter()
+            oracle.qmm_id_sample(P, pairs, cols, nthreads=threads)
+            secs += time.perf_counter() - t0
+            nbytes += alg_bytes(P, P.ids.reshape(-1))
+            calls += 1
+        if secs > 4 * budget_s:
+            break
+    return nbytes / secs / 1e9, secs, threads, (
+        f"{calls // 2} full decode steps (gate/up + down, m=1, 8 pairs, all outputs), "
+        f"{secs:.1f} s on {threads} threads")
+
+
+# --------------------------------------------------------------------- main
+
+def run_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return
+    import oracle
+    from workloads import config_problem
+
+    projs = [config_problem("decode_gate_up"), config_problem("decode_down")]
+    threads = oracle.default_threads()
+    # one step = a bounded sample: all 8 pairs x every 8th output column of both projections
+    samples = []
+    for P in projs:
+        cols = np.arange(0, P.n, 8)
+        samples.append((P, np.repeat(np.arange(P.R), cols.size), np.tile(cols, P.R),
+                        alg_bytes(P, P.ids.reshape(-1)) * cols.size / P.n))
+    for _ in range(args.warmup):
+        for P, pr, cl, _b in samples:
+            oracle.qmm_id_sample(P, pr, cl, nthreads=threads)
+    t0 = time.perf_counter()
+    nbytes = 0.0
+    for _ in range(args.steps):
+        for P, pr, cl, b in samples:
+            oracle.qmm_id_sample(P, pr, cl, nthreads=threads)
+            nbytes += b
+    secs = time.perf_counter() - t0
+    value = nbytes / secs / 1e9
+    sample = "every 8th output column of the gate/up and down calls of one decode token (8 pairs)"
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "decode step m=1: gate/up (E128 top8 k2816 n1408) + down (k704 n2816), "
+                               "affine 4-bit g64, bf16 x, f32 out", "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, dist: Dist):
+    import moe_expert_routed_b200 as M
+
+    M.lib()  # fails loudly if the CUDA library is missing
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    dev = dist.local if dist.world > 1 else 0
+    torch.cuda.set_device(dev)
+    K, Wm = args.steps, args.warmup
+    G = min(GRAPH_STEPS, K)
+    W = DecodeWorkload(G)
+    g = W.capture()
+    replays = max(1, K // G)
+    steps_timed = replays * G
+    warm_replays = max(1, -(-Wm // G))
+    for _ in range(warm_replays):
+        g.replay()
+    torch.cuda.synchronize()
+    sampler = clocks_sampler(dev) if dist.rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    dist.barrier()
+    torch.cuda.synchronize()
+    secs = time_graph(g, replays)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = clocks_summary(sampler) if dist.rank == 0 else None
+    secs_max = dist.max(secs)
+    bytes_total = dist.sum(W.bytes() * replays)
+    value = bytes_total / secs_max / 1e9
+    ms_per_step = secs_max / steps_timed * 1e3
+
+    # per-projection calls (separate graphs, outside the timed region)
+    per_call = {}
+    for p, name in ((0, "gate_up"), (1, "down")):
+        gp = W.capture(projs=(p,))
+        gp.replay()
+        t = time_graph(gp, max(1, replays // 2))
+        per_call[name] = {"us_per_call": t / (max(1, replays // 2) * G) * 1e6,
+                          "GB_per_s": W.bytes((p,)) * max(1, replays // 2) / t / 1e9}
+        del gp
+
+    pk = peaks()
+    achieved = W.bytes() * replays / secs / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
+                "kernel": "gemv_kernel<AFF4, NPB=1, fused> (gate/up and down launches)"}
+    e2e_steps = min(max(K // 10, 50), 2000)
+    e_secs, per_step_bytes, h2d, d2h = e2e_decode(W, e2e_steps)
+    e_secs = dist.max(e_secs)
+    e2e = {"value": dist.sum(per_step_bytes * e2e_steps) / e_secs / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "us_per_step": e_secs / e2e_steps * 1e6, "steps": e2e_steps,
+           "path": "moe_expert_routed_b200.qmm_id (Python binding -> C ABI), pinned host buffers"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world, "steps": steps_timed,
+        "warmup": warm_replays * G, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "decode step m=1: gate/up (E128 top8 k2816 n1408) + down (k704 n2816), "
+                               "affine 4-bit g64, bf16 x, f32 out",
+                   "l2": f"inputs larger than L2: {N_LAYERS} rotated weight copies "
+                         f"({N_LAYERS * 0.428:.1f} GB), fresh ids and x every step",
+                   "timing": f"CUDA graph of {G} steps replayed {replays}x, CUDA events",
+                   "parallelism": f"replicas x{dist.world}"},
+        "per_call": per_call,
+        "roofline": roofline,
+        "gpu_launches": 2 * steps_timed,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        v, s, threads, sample = oracle_decode_sample(args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    dist = Dist(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist)
+        else:
+            run_ours(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

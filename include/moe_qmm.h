@@ -1,0 +1,167 @@
+/*
+ * moe_qmm.h -- C ABI of the expert-routed (MoE) quantized matmul for NVIDIA B200 (sm_100a).
+ *
+ * The operation (mlx-native 0.1.0, src/ops/quantized_matmul_id.rs, module
+ * documentation): for every (token, slot) pair p = token * n_expert_used + slot,
+ *
+ *     e = ids[p]
+ *     out[token][slot][col] = sum_{j<k} dequant(W[e][col][j]) * x[token][j]
+ *
+ * Parameters follow that page's QuantizedMatmulIdParams {m, k, n, group_size,
+ * bits, n_expert_used, num_experts}; storage formats, types and the extra
+ * arguments (x / out types, workspace, stream) are appended after them.
+ *
+ * Conventions shared by every entry point:
+ *   * All array arguments are DEVICE pointers owned by the caller. The library
+ *     allocates and frees nothing.
+ *   * Work is enqueued on `stream` and nothing synchronises (the page's encoder
+ *     "does not commit the command buffer"; the caller orders and waits).
+ *   * Scalar validation happens before any CUDA call; a rejected call returns
+ *     MOE_ERR_INVALID_ARGUMENT (invalid per the page's rules: bits outside the
+ *     format's set, any zero m/k/n/group_size/n_expert_used/num_experts, a NULL
+ *     pointer, NVFP4 with group_size != 16 or odd k) or MOE_ERR_UNSUPPORTED
+ *     (valid but not implemented: k % group_size != 0, or sizes beyond the
+ *     documented limits) and enqueues nothing.
+ *   * Expert ids >= num_experts are not an argument error: the output row of
+ *     such a pair is written as zeros and a bit is set in the device error word
+ *     held in the workspace, which moe_qmm_id_poll_error() reads and clears.
+ *   * A launch failure returns MOE_ERR_CUDA.
+ *
+ * Storage (all rows of expert e are contiguous; row (e, col) starts at byte
+ * (e * n + col) * moe_packed_row_bytes(fmt, bits, k)):
+ *   MOE_FMT_AFFINE   bits 4 / 8: 32/bits codes per little-endian u32 word,
+ *                    least significant first; bits 6: 4 codes per 3-byte
+ *                    triplet read as a little-endian 24-bit integer, code j at
+ *                    bit 6*(j mod 4). w = code * scale + bias, scale and bias
+ *                    bf16 [E, n, k/group_size].
+ *   MOE_FMT_CODEBOOK bits 2 / 3 / 4: 32/bits codes per u32 word, least
+ *                    significant first (3-bit words leave bits 30-31 unused).
+ *                    w = codebook[code] * scale, scale f16 [E, n, k/group_size],
+ *                    codebook f16 [2^bits] shared by all experts
+ *                    (turboquant fast_switch_patch.py, _get_dequant_kernel).
+ *   MOE_FMT_NVFP4    bits 4, group_size 16: two E2M1 codes per byte, element 2i
+ *                    in the low nibble. w = e2m1(code) * e4m3(scale) * scale2[e],
+ *                    scale E4M3 bytes [E, n, k/16], scale2 f32 [E]
+ *                    (spark_model quant_dispatch.rs, w4a16_gemv: B packed,
+ *                    B_scale, scale2).
+ */
+#ifndef MOE_QMM_H
+#define MOE_QMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum { MOE_FMT_AFFINE = 0, MOE_FMT_CODEBOOK = 1, MOE_FMT_NVFP4 = 2 } moe_fmt;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_F16 = 2 } moe_dtype;
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARGUMENT = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_BAD_EXPERT_ID = 5,
+    MOE_ERR_TIMEOUT = 6
+} moe_status;
+
+/* Which kernel path computes the call. AUTO picks DECODE when
+ * m * n_expert_used <= MOE_DECODE_MAX_ROUTINGS and GROUPED otherwise. DECODE is
+ * the CUDA-core GEMV (routing fused in when m*n_expert_used <= 64, otherwise read
+ * from the routing prologue); GROUPED is the routing prologue followed by the
+ * tcgen05 expert-grouped GEMM. GROUPED returns MOE_ERR_UNSUPPORTED for shapes it
+ * does not implement (k not a multiple of 8, group_size not a power of two >= 16,
+ * packed rows not a multiple of 8 bytes, num_experts > 1024); AUTO then uses the
+ * routed GEMV instead. */
+typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_GROUPED = 2 } moe_path;
+
+#define MOE_DECODE_MAX_ROUTINGS 64u
+/* Largest num_experts the routing prologue (and so the grouped path) accepts. */
+#define MOE_ROUTE_MAX_EXPERTS 1024u
+
+/*
+ * moe_qmm_id -- the expert-routed quantized matmul.
+ *   x        [m, k] of x_dtype (f32, bf16 or f16), row-major.
+ *   ids      [m, n_expert_used] u32 expert indices.
+ *   packed   [num_experts, n, moe_packed_row_bytes(fmt, bits, k)] bytes.
+ *   scales   [num_experts, n, ceil(k / group_size)]: bf16 (AFFINE), f16 (CODEBOOK),
+ *            E4M3 bytes (NVFP4).
+ *   aux      AFFINE: biases bf16 [num_experts, n, ceil(k/group_size)];
+ *            CODEBOOK: codebook f16 [2^bits]; NVFP4: scale2 f32 [num_experts].
+ *   out      [m, n_expert_used, n] of out_dtype (f32, bf16 or f16); every
+ *            element is written (zeros for out-of-range ids). Results are rounded
+ *            once from the fp32 accumulator, to nearest even.
+ *   workspace, workspace_bytes: device scratch of at least
+ *            moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts) bytes,
+ *            16-byte aligned. Its first 4 bytes are the device error word; they
+ *            must be zero before the first call (cudaMemset once), later calls
+ *            only set bits that moe_qmm_id_poll_error() clears. Calls sharing one
+ *            workspace must be ordered on the GPU (same stream or events).
+ *   Returns MOE_ERR_WORKSPACE_TOO_SMALL if workspace_bytes is short.
+ */
+moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                      const void *aux, void *out, uint32_t m, uint32_t k, uint32_t n,
+                      uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
+                      uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
+                      void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* moe_qmm_id with an explicit kernel path (tests and benchmarks use it to run
+ * both paths on one problem). Same arguments and errors as moe_qmm_id. */
+moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packed,
+                           const void *scales, const void *aux, void *out, uint32_t m, uint32_t k,
+                           uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                           moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                           moe_stream_t stream, moe_path path);
+
+/* Workspace bytes moe_qmm_id needs for these sizes (any path). Returns 0 if the
+ * sizes overflow. */
+size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t num_experts);
+
+/* Bytes of one packed weight row (mlx-native quantized_matmul_id.rs,
+ * expert_weight_bytes per row): AFFINE 4/8 and CODEBOOK ceil(k / (32/bits)) * 4,
+ * AFFINE 6 ceil(k / 4) * 3, NVFP4 k / 2. Returns 0 for an invalid (fmt, bits). */
+size_t moe_packed_row_bytes(moe_fmt fmt, uint32_t bits, uint32_t k);
+
+/*
+ * moe_qmm_id_route -- the routing prologue alone (histogram, exclusive scan,
+ * stable permutation, tile list), as the grouped path runs it. The pages name
+ * its outputs expert_offsets and sorted_token_ids (metrale helpers_b.rs,
+ * launch_grouped_gemm). Bucket b < num_experts holds the pairs routed to expert
+ * b; bucket num_experts holds the pairs whose id is out of range.
+ *   counts        [num_experts + 1] u32: pairs per bucket.
+ *   offsets       [num_experts + 2] u32: exclusive prefix sum of counts.
+ *   sorted_pairs  [m * n_expert_used] u32: pair indices p grouped by bucket in
+ *                 ascending bucket order, ascending p inside a bucket (stable).
+ *   tiles         [max_tiles, 2] u32: (expert, first row) of each run of
+ *                 tile_rows consecutive rows of one expert, experts ascending.
+ *                 max_tiles = (m * n_expert_used) / tile_rows + num_experts + 1.
+ *   tile_count    [1] u32.
+ *   tile_rows     1 .. 65536.
+ * The workspace (moe_qmm_id_workspace_bytes) holds the per-chunk histograms and
+ * the error word. Requires num_experts <= MOE_ROUTE_MAX_EXPERTS.
+ */
+moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_used,
+                            uint32_t num_experts, uint32_t tile_rows, uint32_t *counts,
+                            uint32_t *offsets, uint32_t *sorted_pairs, uint32_t *tiles,
+                            uint32_t *tile_count, void *workspace, size_t workspace_bytes,
+                            moe_stream_t stream);
+
+/* Synchronise `stream`, read and clear the device error word of `workspace`.
+ * Returns MOE_OK, MOE_ERR_BAD_EXPERT_ID (some id was >= num_experts),
+ * MOE_ERR_TIMEOUT (a bounded wait inside a kernel gave up; its outputs are not
+ * valid) or MOE_ERR_CUDA. */
+moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream);
+
+/* Static description of a status code. */
+const char *moe_status_str(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_QMM_H */

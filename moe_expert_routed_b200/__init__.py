@@ -1,0 +1,216 @@
+"""Expert-routed (MoE) quantized matmul for NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/moe_qmm.h`` (``libmoe_qmm.so``,
+built in-tree by ``moe_expert_routed_b200.build``). The binding checks tensor
+shapes, dtypes, devices and buffer lengths, then passes raw device pointers and
+the current CUDA stream to the library; every step of the computation runs in
+the library's kernels. There is no fallback: if the library is missing or a
+tensor is not on a CUDA device, calls raise.
+
+    out = qmm_id(x, ids, packed, scales, aux, n=..., group_size=..., bits=...,
+                 fmt=FMT_AFFINE, num_experts=...)
+    # for every pair p = token*n_expert_used + slot, e = ids[p]:
+    #   out[token, slot, col] = sum_j dequant(W[e, col, j]) * x[token, j]
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4 = 0, 1, 2
+DT_F32, DT_BF16, DT_F16 = 0, 1, 2
+PATH_AUTO, PATH_DECODE, PATH_GROUPED = 0, 1, 2
+_PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "grouped": PATH_GROUPED}
+
+MOE_OK = 0
+STATUS_NAMES = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED",
+    3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_EXPERT_ID",
+    6: "MOE_ERR_TIMEOUT",
+}
+
+_TORCH_DT = {torch.float32: DT_F32, torch.bfloat16: DT_BF16, torch.float16: DT_F16}
+_DT_TORCH = {v: k for k, v in _TORCH_DT.items()}
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_qmm.so")
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_str(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m moe_expert_routed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, u32, sz, i32 = ctypes.c_void_p, ctypes.c_uint32, ctypes.c_size_t, ctypes.c_int
+        L.moe_qmm_id.argtypes = [vp] * 6 + [u32] * 5 + [i32, u32, u32, i32, i32, vp, sz, vp]
+        L.moe_qmm_id.restype = i32
+        L.moe_qmm_id_path.argtypes = L.moe_qmm_id.argtypes + [i32]
+        L.moe_qmm_id_path.restype = i32
+        L.moe_qmm_id_workspace_bytes.argtypes = [u32, u32, u32]
+        L.moe_qmm_id_workspace_bytes.restype = sz
+        L.moe_packed_row_bytes.argtypes = [i32, u32, u32]
+        L.moe_packed_row_bytes.restype = sz
+        L.moe_qmm_id_route.argtypes = [vp, u32, u32, u32, u32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_qmm_id_route.restype = i32
+        L.moe_qmm_id_poll_error.argtypes = [vp, vp]
+        L.moe_qmm_id_poll_error.restype = i32
+        L.moe_status_str.argtypes = [i32]
+        L.moe_status_str.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    try:
+        return lib().moe_status_str(int(status)).decode()
+    except Exception:  # library not loadable
+        return "?"
+
+
+def packed_row_bytes(fmt: int, bits: int, k: int) -> int:
+    return int(lib().moe_packed_row_bytes(fmt, bits, k))
+
+
+def workspace_bytes(m: int, n_expert_used: int, num_experts: int) -> int:
+    return int(lib().moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
+
+
+def new_workspace(m: int, n_expert_used: int, num_experts: int, device="cuda") -> torch.Tensor:
+    """Zero-initialised workspace (the device error word must start at zero)."""
+    nbytes = workspace_bytes(m, n_expert_used, num_experts)
+    if nbytes == 0:
+        raise ValueError("sizes overflow the workspace layout")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_dev(t: torch.Tensor, name: str, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"quantized_matmul_id: {name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"quantized_matmul_id: {name} must be on a CUDA device")
+    if t.device != device:
+        raise ValueError(f"quantized_matmul_id: {name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"quantized_matmul_id: {name} must be contiguous")
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
+def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+           aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
+           out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
+           workspace: torch.Tensor | None = None, path: str = "auto") -> torch.Tensor:
+    """Expert-routed quantized matmul on the current CUDA stream.
+
+    x [m, k] (f32 / bf16 / f16); ids [m, n_expert_used] int32/uint32; packed, scales,
+    aux: raw storage tensors (any dtype, byte lengths checked); returns out
+    [m, n_expert_used, n]. Buffer-size checks and their messages follow
+    mlx-native quantized_matmul_id.rs (quantized_matmul_id).
+    """
+    device = x.device
+    for t, name in ((x, "input"), (ids, "ids"), (packed, "weight"), (scales, "scales"),
+                    (aux, "aux")):
+        _check_dev(t, name, device)
+    if x.dim() != 2:
+        raise ValueError("quantized_matmul_id: input must be [M, K]")
+    if x.dtype not in _TORCH_DT:
+        raise ValueError(f"quantized_matmul_id: unsupported input dtype {x.dtype}")
+    if ids.dim() != 2 or ids.shape[0] != x.shape[0] or ids.element_size() != 4 or \
+            ids.dtype.is_floating_point:
+        raise ValueError("quantized_matmul_id: ids must be a [M, n_expert_used] 32-bit integer tensor")
+    m, k = x.shape
+    n_expert_used = ids.shape[1]
+    if bits not in ({4, 6, 8} if fmt == FMT_AFFINE else {2, 3, 4} if fmt == FMT_CODEBOOK else {4}):
+        raise ValueError(f"quantized_matmul_id: unsupported bits value {bits} for format {fmt}")
+    if m == 0 or k == 0 or n == 0:
+        raise ValueError("quantized_matmul_id: M, K, and N must all be > 0")
+    if group_size <= 0:
+        raise ValueError("quantized_matmul_id: group_size must be > 0")
+    if n_expert_used == 0:
+        raise ValueError("quantized_matmul_id: n_expert_used must be > 0")
+    if num_experts <= 0:
+        raise ValueError("quantized_matmul_id: num_experts must be > 0")
+    rb = packed_row_bytes(fmt, bits, k)
+    if rb == 0:
+        raise ValueError("quantized_matmul_id: invalid format/bits/k combination")
+    total_w = rb * n * num_experts
+    if _nbytes(packed) < total_w:
+        raise ValueError(f"quantized_matmul_id: weight buffer too small: expected at least {total_w} "
+                         f"bytes for {num_experts} experts, got {_nbytes(packed)}")
+    G = (k + group_size - 1) // group_size
+    per_s = {FMT_AFFINE: 2, FMT_CODEBOOK: 2, FMT_NVFP4: 1}[fmt]
+    total_s = num_experts * n * G * per_s
+    if _nbytes(scales) < total_s:
+        raise ValueError(f"quantized_matmul_id: scales buffer too small: expected at least {total_s} "
+                         f"bytes, got {_nbytes(scales)}")
+    aux_need = {FMT_AFFINE: total_s, FMT_CODEBOOK: 2 * (1 << bits), FMT_NVFP4: 4 * num_experts}[fmt]
+    aux_name = {FMT_AFFINE: "biases", FMT_CODEBOOK: "codebook", FMT_NVFP4: "scale2"}[fmt]
+    if _nbytes(aux) < aux_need:
+        raise ValueError(f"quantized_matmul_id: {aux_name} buffer too small: expected at least "
+                         f"{aux_need} bytes, got {_nbytes(aux)}")
+    if out is None:
+        out = torch.empty((m, n_expert_used, n), dtype=out_dtype, device=device)
+    else:
+        _check_dev(out, "out", device)
+        if out.dtype not in _TORCH_DT or out.numel() < m * n_expert_used * n:
+            raise ValueError("quantized_matmul_id: out must hold [M, n_expert_used, N] f32/bf16/f16")
+    if workspace is None:
+        workspace = new_workspace(m, n_expert_used, num_experts, device)
+    else:
+        _check_dev(workspace, "workspace", device)
+    st = lib().moe_qmm_id_path(
+        x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
+        out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used, num_experts,
+        _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], workspace.data_ptr(), _nbytes(workspace),
+        _stream_ptr(device), _PATHS[path])
+    if st != MOE_OK:
+        raise MoeError(st, "moe_qmm_id")
+    return out
+
+
+def route(ids: torch.Tensor, num_experts: int, tile_rows: int,
+          workspace: torch.Tensor | None = None):
+    """Routing prologue alone. Returns (counts[E+1], offsets[E+2], sorted_pairs[R],
+    tiles[tile_count, 2]) as int32 CUDA tensors (values are unsigned)."""
+    if not ids.is_cuda or not ids.is_contiguous() or ids.element_size() != 4:
+        raise ValueError("route: ids must be a contiguous 32-bit CUDA tensor")
+    device = ids.device
+    m, ne = (ids.shape[0], ids.shape[1]) if ids.dim() == 2 else (ids.numel(), 1)
+    R = m * ne
+    counts = torch.empty(num_experts + 1, dtype=torch.int32, device=device)
+    offsets = torch.empty(num_experts + 2, dtype=torch.int32, device=device)
+    sp = torch.empty(max(R, 1), dtype=torch.int32, device=device)
+    max_tiles = R // tile_rows + num_experts + 1
+    tiles = torch.empty((max_tiles, 2), dtype=torch.int32, device=device)
+    tc = torch.empty(1, dtype=torch.int32, device=device)
+    if workspace is None:
+        workspace = new_workspace(m, ne, num_experts, device)
+    st = lib().moe_qmm_id_route(ids.data_ptr(), m, ne, num_experts, tile_rows, counts.data_ptr(),
+                                offsets.data_ptr(), sp.data_ptr(), tiles.data_ptr(), tc.data_ptr(),
+                                workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device))
+    if st != MOE_OK:
+        raise MoeError(st, "moe_qmm_id_route")
+    ntiles = int(tc.item())
+    return counts, offsets, sp[:R], tiles[:ntiles]
+
+
+def poll_error(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream, read and clear the device error word."""
+    return int(lib().moe_qmm_id_poll_error(workspace.data_ptr(), _stream_ptr(workspace.device)))

@@ -1,0 +1,216 @@
+// api.cu -- the C ABI (include/moe_qmm.h): argument validation, workspace
+// layout, path choice and launches. Validation follows the rules of mlx-native
+// quantized_matmul_id.rs (quantized_matmul_id: bits in the allowed set; m, k, n,
+// group_size, n_expert_used, num_experts all > 0; InvalidArgument otherwise) and
+// happens before any CUDA call.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "moe_qmm.h"
+
+namespace moe {
+
+static inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+bool ws_layout(uint64_t R, uint32_t E, WsLayout *L) {
+    if (R > 0xFFFFFFFFull || E >= 0xFFFFFFF0u) return false;
+    size_t off = 0;
+    L->err = 0;
+    L->tile_count = 4;
+    off = 256;
+    L->counts = off; off += al256(4ull * (E + 1ull));
+    L->offsets = off; off += al256(4ull * (E + 2ull));
+    L->sorted_pairs = off; off += al256(4ull * R);
+    const uint64_t max_tiles = R / MIN_TILE_ROWS + E + 1ull;
+    if (max_tiles > 0xFFFFFFFFull) return false;
+    L->max_tiles = (uint32_t)max_tiles;
+    L->tiles = off; off += al256(8ull * max_tiles);
+    const uint64_t chunks = (R + ROUTE_CHUNK - 1) / ROUTE_CHUNK;
+    L->chunks = (uint32_t)chunks;
+    L->chunk_hist = off; off += al256(4ull * chunks * (E + 1ull));
+    L->chunk_base = off; off += al256(4ull * chunks * (E + 1ull));
+    L->total = off;
+    return true;
+}
+
+static uint64_t row_bytes_of(int fmt, uint32_t bits, uint32_t k) {
+    if (fmt == FMT_NVFP4) return k / 2u;
+    if (fmt == FMT_AFFINE && bits == 6) return ((uint64_t)k + 3) / 4 * 3;
+    const uint32_t epw = 32u / bits;
+    return ((uint64_t)k + epw - 1) / epw * 4;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_packed_row_bytes(moe_fmt fmt, uint32_t bits, uint32_t k) {
+    if (kind_of((int)fmt, (int)bits) < 0) return 0;
+    if (fmt == MOE_FMT_NVFP4 && (k & 1u)) return 0;
+    return (size_t)row_bytes_of((int)fmt, bits, k);
+}
+
+size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t num_experts) {
+    WsLayout L;
+    if (!ws_layout((uint64_t)m * n_expert_used, num_experts, &L)) return 0;
+    return L.total;
+}
+
+const char *moe_status_str(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "valid arguments the library does not implement";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_BAD_EXPERT_ID: return "an expert id was >= num_experts (its output rows are zero)";
+        case MOE_ERR_TIMEOUT: return "a bounded device wait gave up; outputs are not valid";
+    }
+    return "unknown status";
+}
+
+static moe_status validate(const void *x, const uint32_t *ids, const void *packed,
+                           const void *scales, const void *aux, const void *out, uint32_t m,
+                           uint32_t k, uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                           moe_dtype out_dtype) {
+    if (kind_of((int)fmt, (int)bits) < 0) return MOE_ERR_INVALID_ARGUMENT;
+    if (!m || !k || !n || !group_size || !n_expert_used || !num_experts) return MOE_ERR_INVALID_ARGUMENT;
+    if ((int)x_dtype < 0 || (int)x_dtype > 2 || (int)out_dtype < 0 || (int)out_dtype > 2)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (!x || !ids || !packed || !scales || !aux || !out) return MOE_ERR_INVALID_ARGUMENT;
+    if (fmt == MOE_FMT_NVFP4 && (group_size != 16 || (k & 1u))) return MOE_ERR_INVALID_ARGUMENT;
+    if (k % group_size != 0) return MOE_ERR_UNSUPPORTED;
+    if ((uint64_t)m * n_expert_used > 0x7FFFFFFFull) return MOE_ERR_UNSUPPORTED;
+    if (row_bytes_of((int)fmt, bits, k) > 0xFFFFFFFFull) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packed,
+                           const void *scales, const void *aux, void *out, uint32_t m, uint32_t k,
+                           uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                           moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                           moe_stream_t stream, moe_path path) {
+    moe_status v = validate(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt,
+                            n_expert_used, num_experts, x_dtype, out_dtype);
+    if (v != MOE_OK) return v;
+    if ((int)path < 0 || (int)path > 2) return MOE_ERR_INVALID_ARGUMENT;
+    if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
+    const uint64_t R = (uint64_t)m * n_expert_used;
+    WsLayout L;
+    if (!ws_layout(R, num_experts, &L)) return MOE_ERR_UNSUPPORTED;
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+
+    QmmArgs a;
+    a.x = x; a.ids = ids; a.packed = (const uint8_t *)packed; a.scales = scales; a.aux = aux;
+    a.out = out; a.m = m; a.k = k; a.n = n; a.group_size = group_size; a.bits = bits;
+    a.n_expert_used = n_expert_used; a.num_experts = num_experts;
+    a.fmt = (int)fmt; a.kind = kind_of((int)fmt, (int)bits);
+    a.x_dtype = (int)x_dtype; a.out_dtype = (int)out_dtype;
+    a.row_bytes = (uint32_t)row_bytes_of((int)fmt, bits, k);
+    a.groups = (k + group_size - 1) / group_size;
+
+    uint8_t *ws = (uint8_t *)workspace;
+    uint32_t *err = (uint32_t *)(ws + L.err);
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool routable = num_experts <= ROUTE_MAX_E;
+    const bool small = R <= MOE_DECODE_MAX_ROUTINGS;
+
+    enum { FUSED, ROUTED_GEMV, GROUPED } choice;
+    if (path == MOE_PATH_GROUPED) {
+        if (!routable || !gemm_supported(a)) return MOE_ERR_UNSUPPORTED;
+        choice = GROUPED;
+    } else if (path == MOE_PATH_DECODE) {
+        if (small) choice = FUSED;
+        else if (routable) choice = ROUTED_GEMV;
+        else return MOE_ERR_UNSUPPORTED;
+    } else {
+        if (small) choice = FUSED;
+        else if (routable && gemm_supported(a)) choice = GROUPED;
+        else if (routable) choice = ROUTED_GEMV;
+        else return MOE_ERR_UNSUPPORTED;
+    }
+
+    cudaError_t ce;
+    if (choice == FUSED) {
+        ce = launch_gemv_fused(a, err, st);
+    } else {
+        uint32_t *counts = (uint32_t *)(ws + L.counts);
+        uint32_t *offsets = (uint32_t *)(ws + L.offsets);
+        uint32_t *sp = (uint32_t *)(ws + L.sorted_pairs);
+        uint32_t *tiles = (uint32_t *)(ws + L.tiles);
+        uint32_t *tc = (uint32_t *)(ws + L.tile_count);
+        const uint32_t tile_rows = choice == GROUPED ? gemm_tile_rows(a) : MIN_TILE_ROWS;
+        const uint32_t max_tiles = (uint32_t)(R / tile_rows + num_experts + 1);
+        ce = launch_route(ids, (uint32_t)R, num_experts, tile_rows, counts, offsets, sp, tiles, tc,
+                          max_tiles, (uint32_t *)(ws + L.chunk_hist),
+                          (uint32_t *)(ws + L.chunk_base), L.chunks, err, out, n, (int)out_dtype,
+                          st);
+        if (ce == cudaSuccess) {
+            if (choice == GROUPED)
+                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, st);
+            else
+                ce = launch_gemv_routed(a, counts, offsets, sp, err, st);
+        }
+    }
+    return ce == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                      const void *aux, void *out, uint32_t m, uint32_t k, uint32_t n,
+                      uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
+                      uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
+                      void *workspace, size_t workspace_bytes, moe_stream_t stream) {
+    return moe_qmm_id_path(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt,
+                           n_expert_used, num_experts, x_dtype, out_dtype, workspace,
+                           workspace_bytes, stream, MOE_PATH_AUTO);
+}
+
+moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_used,
+                            uint32_t num_experts, uint32_t tile_rows, uint32_t *counts,
+                            uint32_t *offsets, uint32_t *sorted_pairs, uint32_t *tiles,
+                            uint32_t *tile_count, void *workspace, size_t workspace_bytes,
+                            moe_stream_t stream) {
+    if (!m || !n_expert_used || !num_experts || !tile_rows || tile_rows > 65536u)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (!ids || !counts || !offsets || !sorted_pairs || !tiles || !tile_count || !workspace)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if ((uintptr_t)workspace & 15u) return MOE_ERR_INVALID_ARGUMENT;
+    if (num_experts > ROUTE_MAX_E) return MOE_ERR_UNSUPPORTED;
+    const uint64_t R = (uint64_t)m * n_expert_used;
+    if (R > 0x7FFFFFFFull) return MOE_ERR_UNSUPPORTED;
+    WsLayout L;
+    if (!ws_layout(R, num_experts, &L)) return MOE_ERR_UNSUPPORTED;
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *ws = (uint8_t *)workspace;
+    const uint32_t max_tiles = (uint32_t)(R / tile_rows + num_experts + 1);
+    cudaError_t ce = launch_route(ids, (uint32_t)R, num_experts, tile_rows, counts, offsets,
+                                  sorted_pairs, tiles, tile_count, max_tiles,
+                                  (uint32_t *)(ws + L.chunk_hist), (uint32_t *)(ws + L.chunk_base),
+                                  L.chunks, (uint32_t *)(ws + L.err), nullptr, 0, 0,
+                                  (cudaStream_t)stream);
+    return ce == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream) {
+    if (!workspace) return MOE_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t w = 0;
+    if (cudaMemcpyAsync(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (w) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(w), st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (w & ERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (w & ERR_BAD_ID) return MOE_ERR_BAD_EXPERT_ID;
+    if (w & ERR_INTERNAL) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// internal.h -- launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Routing prologue sizes.
+constexpr uint32_t ROUTE_CHUNK = 4096;      // ids per histogram / scatter CTA
+constexpr uint32_t ROUTE_THREADS = 256;
+constexpr uint32_t ROUTE_MAX_E = 1024;      // experts (the out-of-range bucket is extra)
+
+// Workspace layout (byte offsets; every section 256-byte aligned).
+struct WsLayout {
+    size_t err;          // u32 error word at offset 0
+    size_t tile_count;   // u32
+    size_t counts;       // (E+1) u32
+    size_t offsets;      // (E+2) u32
+    size_t sorted_pairs; // R u32
+    size_t tiles;        // max_tiles * 2 u32
+    size_t chunk_hist;   // C * (E+1) u32
+    size_t chunk_base;   // C * (E+1) u32
+    size_t total;
+    uint32_t max_tiles;
+    uint32_t chunks;
+};
+
+// Smallest tile height the grouped path uses (sizes the tile list).
+constexpr uint32_t MIN_TILE_ROWS = 64;
+
+bool ws_layout(uint64_t R, uint32_t E, WsLayout *L);
+
+// Routing prologue: histogram -> scan -> stable scatter (+ zero rows of
+// out-of-range pairs when `out` is non-null).
+cudaError_t launch_route(const uint32_t *ids, uint32_t R, uint32_t E, uint32_t tile_rows,
+                         uint32_t *counts, uint32_t *offsets, uint32_t *sorted_pairs,
+                         uint32_t *tiles, uint32_t *tile_count, uint32_t max_tiles,
+                         uint32_t *chunk_hist, uint32_t *chunk_base, uint32_t chunks,
+                         uint32_t *err, void *out, uint32_t n, int out_dtype, cudaStream_t st);
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device:
+// `cache` is a per-kernel array of the largest size already set, per device.
+template <typename K>
+inline cudaError_t ensure_dyn_smem(K kern, size_t bytes, int (&cache)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && cache[dev] >= (int)bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev] = (int)bytes;
+    return e;
+}
+
+struct QmmArgs {
+    const void *x;
+    const uint32_t *ids;
+    const uint8_t *packed;
+    const void *scales;
+    const void *aux;
+    void *out;
+    uint32_t m, k, n, group_size, bits, n_expert_used, num_experts;
+    int fmt, kind, x_dtype, out_dtype;
+    uint32_t row_bytes, groups;
+};
+
+// CUDA-core GEMV with routing fused in (R <= 64).
+cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st);
+// CUDA-core GEMV over the routing prologue's output (any R).
+cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const uint32_t *offsets,
+                               const uint32_t *sorted_pairs, uint32_t *err, cudaStream_t st);
+
+// tcgen05 grouped GEMM over the routing prologue's tiles.
+bool gemm_supported(const QmmArgs &a);
+uint32_t gemm_tile_rows(const QmmArgs &a);
+cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
+                        const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
+                        uint32_t *err, cudaStream_t st);
+
+}  // namespace moe

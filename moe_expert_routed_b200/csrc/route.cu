@@ -1,0 +1,203 @@
+// route.cu -- routing prologue of the grouped path: per-chunk expert histogram,
+// exclusive scan, stable permutation of the (token, slot) pairs and the tile
+// list. It produces the expert_offsets / sorted_token_ids pair that the routed
+// grouped GEMM consumes (metrale helpers_b.rs, launch_grouped_gemm), here with a
+// deterministic order: pairs of one expert stay in ascending pair index.
+//
+// Three launches, no inter-CTA waiting:
+//   route_hist    one CTA per chunk of ROUTE_CHUNK ids: shared-memory histogram
+//   route_scan    one CTA: bucket totals, offsets, per-(chunk, bucket) bases,
+//                 tile list
+//   route_scatter one CTA per chunk: stable ranks inside the chunk from warp
+//                 match masks and per-warp counts, then the scatter
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+__global__ void __launch_bounds__(ROUTE_THREADS)
+route_hist(const uint32_t *__restrict__ ids, uint32_t R, uint32_t E, uint32_t *__restrict__ chunk_hist) {
+    extern __shared__ uint32_t hist[];
+    const uint32_t NB = E + 1;
+    for (uint32_t b = threadIdx.x; b < NB; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    const uint64_t base = (uint64_t)blockIdx.x * ROUTE_CHUNK;
+    const uint64_t end = tmin<uint64_t>(base + ROUTE_CHUNK, R);
+    for (uint64_t i = base + threadIdx.x; i < end; i += blockDim.x) {
+        uint32_t e = __ldg(ids + i);
+        atomicAdd(&hist[e < E ? e : E], 1u);
+    }
+    __syncthreads();
+    for (uint32_t b = threadIdx.x; b < NB; b += blockDim.x)
+        chunk_hist[(size_t)blockIdx.x * NB + b] = hist[b];
+}
+
+// Exclusive scan of one value per thread across the block (blockDim.x <= 1024,
+// multiple of 32). `scratch` holds 33 words. Returns the exclusive prefix and the
+// block total in *total.
+__device__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *scratch, uint32_t *total) {
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        uint32_t t = __shfl_up_sync(0xFFFFFFFFu, inc, d);
+        if (lane >= (uint32_t)d) inc += t;
+    }
+    if (lane == 31) scratch[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = lane < nw ? scratch[lane] : 0u;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            uint32_t t = __shfl_up_sync(0xFFFFFFFFu, s, d);
+            if (lane >= (uint32_t)d) s += t;
+        }
+        if (lane < nw) scratch[lane] = s - (lane < nw ? scratch[lane] : 0u);  // exclusive
+        if (lane == nw - 1) scratch[32] = s;
+    }
+    __syncthreads();
+    uint32_t res = scratch[warp] + inc - v;
+    *total = scratch[32];
+    __syncthreads();
+    return res;
+}
+
+__global__ void __launch_bounds__(1024)
+route_scan(const uint32_t *__restrict__ chunk_hist, uint32_t C, uint32_t E, uint32_t R,
+           uint32_t tile_rows, uint32_t *__restrict__ counts, uint32_t *__restrict__ offsets,
+           uint32_t *__restrict__ chunk_base, uint32_t *__restrict__ tiles,
+           uint32_t *__restrict__ tile_count, uint32_t max_tiles, uint32_t *__restrict__ err) {
+    extern __shared__ uint32_t sm[];
+    const uint32_t NB = E + 1;
+    uint32_t *tot = sm;            // [NB]
+    uint32_t *scratch = sm + NB;   // [33]
+    for (uint32_t b = threadIdx.x; b < NB; b += blockDim.x) {
+        uint32_t s = 0;
+        for (uint32_t c = 0; c < C; c++) s += chunk_hist[(size_t)c * NB + b];
+        tot[b] = s;
+    }
+    __syncthreads();
+    // Each thread owns a contiguous segment of buckets.
+    const uint32_t seg = (NB + blockDim.x - 1) / blockDim.x;
+    const uint32_t b0 = min(threadIdx.x * seg, NB), b1 = min(b0 + seg, NB);
+    uint32_t rows = 0, ntile = 0;
+    for (uint32_t b = b0; b < b1; b++) {
+        rows += tot[b];
+        if (b < E) ntile += (tot[b] + tile_rows - 1) / tile_rows;
+    }
+    uint32_t total_rows, total_tiles;
+    uint32_t row_off = block_exclusive_scan(rows, scratch, &total_rows);
+    uint32_t tile_off = block_exclusive_scan(ntile, scratch, &total_tiles);
+    for (uint32_t b = b0; b < b1; b++) {
+        const uint32_t cnt = tot[b];
+        counts[b] = cnt;
+        offsets[b] = row_off;
+        uint32_t run = row_off;
+        for (uint32_t c = 0; c < C; c++) {
+            chunk_base[(size_t)c * NB + b] = run;
+            run += chunk_hist[(size_t)c * NB + b];
+        }
+        if (b < E) {
+            for (uint32_t r0 = 0; r0 < cnt; r0 += tile_rows, tile_off++) {
+                if (tile_off < max_tiles) {
+                    tiles[2 * (size_t)tile_off] = b;
+                    tiles[2 * (size_t)tile_off + 1] = r0;
+                } else {
+                    atomicOr(err, ERR_INTERNAL);
+                }
+            }
+        }
+        row_off += cnt;
+    }
+    if (threadIdx.x == 0) {
+        offsets[NB] = total_rows;
+        *tile_count = min(total_tiles, max_tiles);
+        if (total_rows != R) atomicOr(err, ERR_INTERNAL);
+    }
+}
+
+__global__ void __launch_bounds__(ROUTE_THREADS)
+route_scatter(const uint32_t *__restrict__ ids, uint32_t R, uint32_t E,
+              const uint32_t *__restrict__ chunk_base, uint32_t *__restrict__ sorted_pairs,
+              uint32_t *__restrict__ err, void *out, uint32_t n, int out_dtype) {
+    extern __shared__ uint32_t sm[];
+    constexpr uint32_t NW = ROUTE_THREADS / 32;
+    const uint32_t NB = E + 1;
+    uint32_t *running = sm;        // [NB]
+    uint32_t *wcnt = sm + NB;      // [NW][NB]
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+    for (uint32_t b = tid; b < NB; b += blockDim.x) {
+        running[b] = chunk_base[(size_t)blockIdx.x * NB + b];
+        for (uint32_t w = 0; w < NW; w++) wcnt[w * NB + b] = 0;
+    }
+    __syncthreads();
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint64_t base = (uint64_t)blockIdx.x * ROUTE_CHUNK;
+    for (uint32_t r = 0; r < ROUTE_CHUNK / ROUTE_THREADS; r++) {
+        const uint64_t first = base + (uint64_t)r * ROUTE_THREADS;
+        if (first >= R) break;  // uniform across the block
+        const uint64_t i = first + tid;
+        const bool valid = i < R;
+        uint32_t b = 0xFFFFFFFFu;
+        if (valid) {
+            uint32_t e = __ldg(ids + i);
+            b = e < E ? e : E;
+        }
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, b);
+        const uint32_t rank = __popc(peers & lt_mask);
+        const bool leader = valid && rank == 0;
+        if (leader) wcnt[warp * NB + b] = __popc(peers);
+        __syncthreads();
+        if (valid) {
+            uint32_t pos = running[b] + rank;
+            for (uint32_t w = 0; w < warp; w++) pos += wcnt[w * NB + b];
+            if (pos < R) sorted_pairs[pos] = (uint32_t)i;
+            else atomicOr(err, ERR_INTERNAL);
+            if (b == E) {
+                atomicOr(err, ERR_BAD_ID);
+                if (out)
+                    for (uint32_t col = 0; col < n; col++) store_out(out, out_dtype, i * n + col, 0.f);
+            }
+        }
+        __syncthreads();
+        if (leader) {
+            bool last = true;
+            uint32_t sum = 0;
+            for (uint32_t w = 0; w < NW; w++) {
+                uint32_t c = wcnt[w * NB + b];
+                sum += c;
+                if (w > warp && c) last = false;
+            }
+            if (last) running[b] += sum;
+        }
+        __syncthreads();
+        if (leader) wcnt[warp * NB + b] = 0;
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const uint32_t *ids, uint32_t R, uint32_t E, uint32_t tile_rows,
+                         uint32_t *counts, uint32_t *offsets, uint32_t *sorted_pairs,
+                         uint32_t *tiles, uint32_t *tile_count, uint32_t max_tiles,
+                         uint32_t *chunk_hist, uint32_t *chunk_base, uint32_t chunks,
+                         uint32_t *err, void *out, uint32_t n, int out_dtype, cudaStream_t st) {
+    const uint32_t NB = E + 1;
+    route_hist<<<chunks, ROUTE_THREADS, NB * sizeof(uint32_t), st>>>(ids, R, E, chunk_hist);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    route_scan<<<1, 1024, (NB + 33) * sizeof(uint32_t), st>>>(
+        chunk_hist, chunks, E, R, tile_rows, counts, offsets, chunk_base, tiles, tile_count,
+        max_tiles, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t sc_smem = (size_t)NB * (1 + ROUTE_THREADS / 32) * sizeof(uint32_t);
+    route_scatter<<<chunks, ROUTE_THREADS, sc_smem, st>>>(ids, R, E, chunk_base, sorted_pairs,
+                                                           err, out, n, out_dtype);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

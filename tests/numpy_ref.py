@@ -126,3 +126,14 @@ def reference(P) -> np.ndarray:
     out = np.zeros((ids.size, P.n))
     out[ok] = np.einsum("pnk,pk->pn", W[ids[ok]], X[tok[ok]])
     return out
+
+
+def dequant_expert(P, e: int) -> np.ndarray:
+    """Weights of one expert [n, k] in float64."""
+    codes = unpack_codes(P.packed[e], P.fmt, P.bits, P.k)
+    g = np.arange(P.k) // P.group_size
+    if P.fmt == FMT_AFFINE:
+        return codes * bf16_to_f64(P.scales[e])[:, g] + bf16_to_f64(P.aux[e])[:, g]
+    if P.fmt == FMT_CODEBOOK:
+        return f16_to_f64(P.aux)[codes] * f16_to_f64(P.scales[e])[:, g]
+    return E2M1_TABLE[codes] * e4m3_to_f64(P.scales[e])[:, g] * float(P.aux[e])

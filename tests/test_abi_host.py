@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and exports
+every entry point the header declares, sizes follow the storage contract, and
+invalid arguments are rejected before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import moe_expert_routed_b200 as M
+import oracle
+from workloads.gen import FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe_qmm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_symbols_exported():
+    names = declared_functions()
+    assert "moe_qmm_id" in names and "moe_qmm_id_route" in names
+    L = M.lib()
+    for name in names:
+        assert hasattr(L, name), name
+
+
+@pytest.mark.parametrize("fmt,bits,k", [(FMT_AFFINE, 4, 2816), (FMT_AFFINE, 4, 704),
+                                        (FMT_AFFINE, 6, 2048), (FMT_AFFINE, 6, 5),
+                                        (FMT_AFFINE, 8, 100), (FMT_CODEBOOK, 3, 2816),
+                                        (FMT_CODEBOOK, 2, 33), (FMT_CODEBOOK, 4, 7),
+                                        (FMT_NVFP4, 4, 4096)])
+def test_row_bytes_match_oracle(fmt, bits, k):
+    assert M.packed_row_bytes(fmt, bits, k) == oracle.row_bytes(fmt, bits, k)
+
+
+def test_row_bytes_invalid():
+    assert M.packed_row_bytes(FMT_AFFINE, 5, 64) == 0
+    assert M.packed_row_bytes(FMT_NVFP4, 4, 63) == 0
+    assert M.packed_row_bytes(FMT_CODEBOOK, 8, 64) == 0
+
+
+def test_workspace_bytes_grows_with_routings():
+    a = M.workspace_bytes(1, 8, 128)
+    b = M.workspace_bytes(4096, 8, 128)
+    assert 0 < a < b and b % 256 == 0
+
+
+def _call(**kw):
+    args = dict(x=16, ids=16, packed=16, scales=16, aux=16, out=16, m=4, k=256, n=128, gs=32,
+                bits=4, fmt=0, topk=2, E=8, xd=0, od=0, ws=4096, wsb=1 << 20, stream=None, path=0)
+    args.update(kw)
+    L = M.lib()
+    return L.moe_qmm_id_path(args["x"], args["ids"], args["packed"], args["scales"], args["aux"],
+                             args["out"], args["m"], args["k"], args["n"], args["gs"], args["bits"],
+                             args["fmt"], args["topk"], args["E"], args["xd"], args["od"],
+                             args["ws"], args["wsb"], args["stream"], args["path"])
+
+
+@pytest.mark.parametrize("kw", [dict(m=0), dict(k=0), dict(n=0), dict(gs=0), dict(topk=0),
+                                dict(E=0), dict(bits=5), dict(bits=3), dict(fmt=3),
+                                dict(fmt=2, bits=4, gs=32), dict(fmt=2, bits=4, gs=16, k=255),
+                                dict(fmt=1, bits=8), dict(x=0), dict(ids=0), dict(packed=0),
+                                dict(scales=0), dict(aux=0), dict(out=0), dict(ws=0),
+                                dict(xd=3), dict(od=-1), dict(path=7), dict(ws=4097)])
+def test_invalid_arguments_rejected_before_cuda(kw):
+    # all pointers are fake host addresses: any CUDA call would fail or fault, so a
+    # clean MOE_ERR_INVALID_ARGUMENT shows validation came first
+    assert _call(**kw) == 1
+
+
+def test_unsupported_and_workspace_errors_before_cuda():
+    assert _call(k=250, gs=32) == 2                  # k % group_size != 0
+    assert _call(wsb=64) == 3                        # workspace too small
+
+
+def test_route_invalid_arguments():
+    L = M.lib()
+    assert L.moe_qmm_id_route(16, 0, 8, 8, 64, 16, 16, 16, 16, 16, 4096, 1 << 20, None) == 1
+    assert L.moe_qmm_id_route(16, 4, 8, 8, 0, 16, 16, 16, 16, 16, 4096, 1 << 20, None) == 1
+    assert L.moe_qmm_id_route(16, 4, 8, 2000, 64, 16, 16, 16, 16, 16, 4096, 1 << 20, None) == 2
+
+
+def test_status_strings():
+    for s in range(7):
+        assert M.status_str(s) and M.status_str(s) != "unknown status"
+
+
+def test_binding_requires_cuda_tensors():
+    x = torch.zeros(4, 256)
+    ids = torch.zeros(4, 2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.qmm_id(x, ids, x, x, x, n=128, group_size=32, bits=4, fmt=0, num_experts=8)
