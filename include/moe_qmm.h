@@ -75,7 +75,7 @@ typedef enum {
  * from the routing prologue); GROUPED is the routing prologue followed by the
  * tcgen05 expert-grouped GEMM. GROUPED returns MOE_ERR_UNSUPPORTED for shapes it
  * does not implement (k not a multiple of 8, group_size not a power of two >= 16,
- * packed rows not a multiple of 8 bytes, num_experts > 1024); AUTO then uses the
+ * packed rows not a multiple of 8 bytes (4 for 3-bit codebook rows), num_experts > 1024); AUTO then uses the
  * routed GEMV instead. */
 typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_GROUPED = 2 } moe_path;
 

@@ -453,7 +453,8 @@ bool gemm_supported(const QmmArgs &a) {
     const uint32_t gs = a.group_size;
     if (gs < 16 || (gs & (gs - 1)) != 0) return false;
     if (a.k % 8 != 0 || a.k % gs != 0) return false;
-    if (a.row_bytes % 8 != 0) return false;
+    // packed codes are read with 8-byte loads (4-byte word loads for 3-bit codebook rows)
+    if (a.row_bytes % (a.kind == K_CB3 ? 4u : 8u) != 0) return false;
     if ((uintptr_t)a.packed % 16 != 0 || (uintptr_t)a.x % 16 != 0) return false;
     if (a.num_experts > ROUTE_MAX_E) return false;
     return true;

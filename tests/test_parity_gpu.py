@@ -132,7 +132,7 @@ def test_fused_decode_out_of_range_ids():
 
 @pytest.mark.parametrize("k,gs,fmt,bits", [(200, 40, FMT_AFFINE, 4), (100, 20, FMT_AFFINE, 6),
                                            (90, 30, FMT_CODEBOOK, 3), (52, 4, FMT_AFFINE, 8),
-                                           (88, 16, FMT_NVFP4, 4)])
+                                           (80, 16, FMT_NVFP4, 4)])
 @pytest.mark.parametrize("m,topk", [(3, 2), (50, 3)])
 def test_unaligned_rows_take_the_gemv(k, gs, fmt, bits, m, topk):
     P = make_problem("unaligned", fmt=fmt, bits=bits, group_size=gs, m=m, k=k, n=45,
@@ -140,6 +140,15 @@ def test_unaligned_rows_take_the_gemv(k, gs, fmt, bits, m, topk):
     out = run(P, "auto")
     torch.cuda.synchronize()
     assert_ok(check_full(P, out), f"unaligned k={k}")
+
+
+def test_ragged_k_is_unsupported_not_wrong():
+    # k % group_size != 0 is valid storage (ceil groups) that this library does not implement
+    P = make_problem("ragged", fmt=FMT_AFFINE, bits=4, group_size=32, m=2, k=100, n=16,
+                     n_expert_used=2, num_experts=4, x_dtype=DT_F32, out_dtype=DT_F32, seed=35)
+    with pytest.raises(M.MoeError) as ei:
+        run(P, "auto")
+    assert ei.value.status == 2
 
 
 @pytest.mark.parametrize("n", [1, 31, 129])
