@@ -19,7 +19,7 @@ LIB = os.path.join(PKG, "libmoe_qmm.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
 SOURCES = ["api.cu", "route.cu", "gemv.cu", "gemm_sm100.cu"]
-HEADERS = ["common.cuh", "ptx.cuh", "internal.h"]
+HEADERS = ["common.cuh", "ptx.cuh", "internal.h", "gemv_common.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

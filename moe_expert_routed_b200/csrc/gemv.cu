@@ -19,18 +19,19 @@
 //   routed (any R): grid.y indexes experts; counts / offsets / sorted_pairs come
 //          from the routing prologue.
 #include "common.cuh"
+#include "gemv_common.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int GEMV_THREADS = 256;
-constexpr int GEMV_LPR = 8;                                      // lanes per row
-constexpr int GEMV_ROWS = GEMV_THREADS / GEMV_LPR;               // 32 rows per CTA
-constexpr uint32_t FUSED_MAX_R = 64;
+__device__ __forceinline__ uint32_t ptx_smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
 constexpr int UNITS_PER_BATCH = 4;
-constexpr size_t GEMV_SMEM_BUDGET = 200 * 1024;
 
 // Words (u32) and codes per unit of each storage kind. A unit is the span a lane
 // handles in one step: 16 bytes, or 48 bytes (64 codes) for 6-bit triplets.
@@ -152,18 +153,7 @@ struct UnitDot {
     }
 };
 
-struct GemvParams {
-    const void *x;
-    const uint32_t *ids;
-    const uint8_t *packed;
-    const void *scales;
-    const void *aux;
-    void *out;
-    uint32_t *err;
-    const uint32_t *counts, *offsets, *sorted_pairs;  // routed mode
-    uint32_t R, k, n, gs, groups, n_expert_used, num_experts, row_bytes, n_units, xstride;
-    int x_dtype, out_dtype, load_mode;
-};
+
 
 template <int KIND, int NPB, bool FUSED>
 __global__ void __launch_bounds__(GEMV_THREADS)
@@ -173,7 +163,7 @@ gemv_kernel(const GemvParams P) {
     __shared__ uint32_t ids_s[FUSED_MAX_R];
     __shared__ uint32_t first_s[FUSED_MAX_R];
     __shared__ uint32_t pairs_s[NPB];
-    __shared__ uint32_t expert_s, npairs_s, pair_base_s;
+    __shared__ uint32_t expert_s, npairs_s;
     __shared__ float cb_s[16];
 
     const uint32_t tid = threadIdx.x;
@@ -181,53 +171,9 @@ gemv_kernel(const GemvParams P) {
 
     uint32_t expert = 0, total_pairs = 0;
     const uint32_t *pair_src = nullptr;  // routed mode: sorted pairs of this expert
-    if constexpr (FUSED) {
-        const uint32_t R = P.R, E = P.num_experts;
-        if (tid < R) ids_s[tid] = __ldg(P.ids + tid);
-        __syncthreads();
-        if (tid < R) {
-            const uint32_t e = ids_s[tid];
-            bool first = e < E;
-            for (uint32_t t = 0; t < tid && first; t++) first = ids_s[t] != e;
-            first_s[tid] = first;
-        }
-        __syncthreads();
-        if (tid < R && first_s[tid]) {
-            const uint32_t e = ids_s[tid];
-            uint32_t rank = 0;
-            for (uint32_t t = 0; t < R; t++) rank += (first_s[t] && ids_s[t] < e);
-            if (rank == blockIdx.y) expert_s = e;
-        }
-        if (tid == 0) {
-            uint32_t D = 0;
-            for (uint32_t t = 0; t < R; t++) D += first_s[t];
-            npairs_s = D;  // temporarily: number of distinct experts
-        }
-        __syncthreads();
-        // Zero the rows of out-of-range pairs (this row block) and flag them.
-        if (blockIdx.y == 0) {
-            for (uint32_t idx = tid; idx < R * GEMV_ROWS; idx += blockDim.x) {
-                const uint32_t p = idx / GEMV_ROWS, r = row0 + idx % GEMV_ROWS;
-                if (ids_s[p] >= E && r < P.n) store_out(P.out, P.out_dtype, (size_t)p * P.n + r, 0.f);
-            }
-            if (blockIdx.x == 0 && tid < R && ids_s[tid] >= E) atomicOr(P.err, ERR_BAD_ID);
-        }
-        if (blockIdx.y >= npairs_s) return;  // uniform
-        expert = expert_s;
-        __syncthreads();
-        if (tid == 0) {
-            uint32_t c = 0;
-            for (uint32_t t = 0; t < R; t++) c += ids_s[t] == expert;
-            npairs_s = c;
-        }
-        __syncthreads();
-        total_pairs = npairs_s;
-    } else {
-        expert = blockIdx.y;
-        total_pairs = __ldg(P.counts + expert);
-        if (total_pairs == 0) return;
-        pair_src = P.sorted_pairs + __ldg(P.offsets + expert);
-    }
+    if (!route_prologue<FUSED>(P, ids_s, first_s, &expert_s, &npairs_s, row0, GEMV_ROWS, expert,
+                               total_pairs, pair_src))
+        return;
 
     if constexpr (KIND == K_CB2 || KIND == K_CB3 || KIND == K_CB4) {
         if (tid < (1u << kind_bits(KIND)))
@@ -261,18 +207,7 @@ gemv_kernel(const GemvParams P) {
     for (uint32_t pb = 0; pb < total_pairs; pb += NPB) {
         const uint32_t np = tmin<uint32_t>(NPB, total_pairs - pb);
         __syncthreads();  // previous batch's x reads are done
-        if (tid == 0) {
-            if constexpr (FUSED) {
-                uint32_t c2 = 0, seen = 0;
-                for (uint32_t t = 0; t < P.R && c2 < np; t++)
-                    if (ids_s[t] == expert) {
-                        if (seen >= pb) pairs_s[c2++] = t;
-                        seen++;
-                    }
-            } else {
-                for (uint32_t q = 0; q < np; q++) pairs_s[q] = __ldg(pair_src + pb + q);
-            }
-        }
+        load_pairs<FUSED>(P, ids_s, expert, pair_src, pb, np, pairs_s);
         __syncthreads();
         // Stage x rows: element j of pair q at xs[q*xstride + j + j/UC] (one pad word per unit).
         const uint32_t span = P.n_units * U::UC;
@@ -328,6 +263,594 @@ gemv_kernel(const GemvParams P) {
                     store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q] * s2);
         }
     }
+}
+
+
+// ----------------------------------------------------------- 4-bit affine, DP4A
+//
+// Exact integer dot products for 4-bit affine weights. For each 32-code unit u
+// of x (one 16-byte load of a weight row), x is written once per CTA as a
+// 24-bit fixed-point integer q_j = rint(x_j * 2^-E_u), E_u chosen from the
+// unit's largest |x| so that |q_j| < 2^23, and split into three byte planes
+// (q = b2*2^16 + b1*2^8 + b0, b0/b1 unsigned, b2 signed). Then
+//     sum_j c_j x_j = 2^E_u * (sum c_j b0_j + 2^8 sum c_j b1_j + 2^16 sum c_j b2_j)
+// where each inner sum is exact in int32 and computed four codes per dp4a. The
+// group factorisation sum_j (c_j s + b) x_j = s * sum_j c_j x_j + b * sum_j x_j
+// needs one fp32 FMA pair per unit. The only roundings are q_j (below 2^-23
+// of the unit's largest |x|) and the fp32 combination of the partial sums.
+// Weight rows are streamed once with 16-byte non-allocating loads issued
+// before the x planes and scales are staged.
+constexpr int DP_UMAX = 12;  // 16-byte units per lane per pass
+constexpr int DP_PW = 28;    // u32 words of x planes per unit (24 used; 28 keeps LDS.128 conflict-free)
+
+__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c) {
+    int32_t d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint4 ldg_stream16(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void sts8(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+template <int NPB>
+__device__ __forceinline__ void dp4a_unit(const uint4 w, const uint32_t *planes_u, uint32_t plane_stride,
+                                          const float *uscale_u, const float *usum_u,
+                                          uint32_t sum_stride, float s, float b, float (&acc)[NPB]) {
+    const uint32_t lo0 = w.x & 0x0F0F0F0Fu, hi0 = (w.x >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo1 = w.y & 0x0F0F0F0Fu, hi1 = (w.y >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo2 = w.z & 0x0F0F0F0Fu, hi2 = (w.z >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo3 = w.w & 0x0F0F0F0Fu, hi3 = (w.w >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+    for (int q = 0; q < NPB; q++) {
+        const uint4 *pl = (const uint4 *)(planes_u + q * plane_stride);
+        const uint4 v0 = pl[0], v1 = pl[1], v2 = pl[2], v3 = pl[3], v4 = pl[4], v5 = pl[5];
+        // plane words per unit: [word][plane][lo/hi]
+        uint32_t a0 = dp4a_uu(lo0, v0.x, 0u);
+        a0 = dp4a_uu(hi0, v0.y, a0);
+        uint32_t a1 = dp4a_uu(lo0, v0.z, 0u);
+        a1 = dp4a_uu(hi0, v0.w, a1);
+        int32_t a2 = dp4a_us(lo0, v1.x, 0);
+        a2 = dp4a_us(hi0, v1.y, a2);
+        a0 = dp4a_uu(lo1, v1.z, a0);
+        a0 = dp4a_uu(hi1, v1.w, a0);
+        a1 = dp4a_uu(lo1, v2.x, a1);
+        a1 = dp4a_uu(hi1, v2.y, a1);
+        a2 = dp4a_us(lo1, v2.z, a2);
+        a2 = dp4a_us(hi1, v2.w, a2);
+        a0 = dp4a_uu(lo2, v3.x, a0);
+        a0 = dp4a_uu(hi2, v3.y, a0);
+        a1 = dp4a_uu(lo2, v3.z, a1);
+        a1 = dp4a_uu(hi2, v3.w, a1);
+        a2 = dp4a_us(lo2, v4.x, a2);
+        a2 = dp4a_us(hi2, v4.y, a2);
+        a0 = dp4a_uu(lo3, v4.z, a0);
+        a0 = dp4a_uu(hi3, v4.w, a0);
+        a1 = dp4a_uu(lo3, v5.x, a1);
+        a1 = dp4a_uu(hi3, v5.y, a1);
+        a2 = dp4a_us(lo3, v5.z, a2);
+        a2 = dp4a_us(hi3, v5.w, a2);
+        const float d = fmaf((float)a2, 65536.f, fmaf((float)a1, 256.f, (float)a0));
+        acc[q] = fmaf(s, d * uscale_u[q * sum_stride], fmaf(b, usum_u[q * sum_stride], acc[q]));
+    }
+}
+
+template <int NPB, bool FUSED>
+__global__ void __launch_bounds__(GEMV_THREADS)
+gemv_aff4_dp4a(const GemvParams P) {
+    extern __shared__ __align__(16) uint32_t dsm[];
+    __shared__ uint32_t ids_s[FUSED_MAX_R];
+    __shared__ uint32_t first_s[FUSED_MAX_R];
+    __shared__ uint32_t pairs_s[NPB];
+    __shared__ uint32_t expert_s, npairs_s;
+
+    const uint32_t tid = threadIdx.x;
+    const uint32_t row0 = blockIdx.x * GEMV_ROWS;
+    uint32_t expert = 0, total_pairs = 0;
+    const uint32_t *pair_src = nullptr;
+    if (!route_prologue<FUSED>(P, ids_s, first_s, &expert_s, &npairs_s, row0, GEMV_ROWS, expert,
+                               total_pairs, pair_src))
+        return;
+
+    const uint32_t nu = P.n_units;  // 16-byte units (32 codes) per row
+    const uint32_t G = P.groups;
+    uint32_t *planes = dsm;                                          // [NPB][nu][DP_PW]
+    float *uscale = (float *)(planes + (size_t)NPB * nu * DP_PW);    // [NPB][nu]
+    float *usum = uscale + NPB * nu;                                 // [NPB][nu]
+    uint32_t *sb = (uint32_t *)(usum + NPB * nu);                    // [GEMV_ROWS][G]
+
+    const uint32_t warp = tid >> 5, lane = tid & 31u;
+    const uint32_t rsub = lane / GEMV_LPR, l8 = lane % GEMV_LPR;
+    const uint32_t rloc = warp * (32 / GEMV_LPR) + rsub;
+    const uint32_t row = row0 + rloc;
+    const bool row_ok = row < P.n;
+    const size_t row_index = (size_t)expert * P.n + (row_ok ? row : P.n - 1);
+    const uint8_t *rowp = P.packed + row_index * P.row_bytes;
+    const uint32_t upg = P.gs / 32u;  // units per group
+
+    for (uint32_t pb = 0; pb < total_pairs; pb += NPB) {
+        const uint32_t np = tmin<uint32_t>(NPB, total_pairs - pb);
+        float acc[NPB];
+#pragma unroll
+        for (int q = 0; q < NPB; q++) acc[q] = 0.f;
+        for (uint32_t base = 0; base < nu; base += GEMV_LPR * DP_UMAX) {
+            uint4 w[DP_UMAX];
+#pragma unroll
+            for (int i = 0; i < DP_UMAX; i++) {
+                const uint32_t u = base + l8 + GEMV_LPR * i;
+                w[i] = u < nu ? ldg_stream16(rowp + 16u * u) : make_uint4(0, 0, 0, 0);
+            }
+            if (base == 0) {
+                __syncthreads();  // previous batch's planes are no longer read
+                load_pairs<FUSED>(P, ids_s, expert, pair_src, pb, np, pairs_s);
+                if (pb == 0) {
+                    // scales and biases of this CTA's rows, packed (bf16 scale | bf16 bias << 16)
+                    const size_t sbase = ((size_t)expert * P.n + row0) * G;
+                    const uint32_t nrows = tmin<uint32_t>(GEMV_ROWS, P.n - row0);
+                    const unsigned short *sc = (const unsigned short *)P.scales + sbase;
+                    const unsigned short *bi = (const unsigned short *)P.aux + sbase;
+                    for (uint32_t idx = tid; idx < nrows * G; idx += blockDim.x)
+                        sb[idx] = (uint32_t)__ldg(sc + idx) | ((uint32_t)__ldg(bi + idx) << 16);
+                }
+                __syncthreads();
+                // x planes, one warp per (pair, unit), lane = code within the unit
+                const uint32_t plane_base = ptx_smem_addr(planes);
+                for (uint32_t idx = warp; idx < NPB * nu; idx += GEMV_THREADS / 32) {
+                    const uint32_t q = idx / nu, u = idx - q * nu;
+                    const uint32_t j = u * 32u + lane;
+                    float x = 0.f;
+                    if (q < np && j < P.k) {
+                        const uint32_t t = pairs_s[q] / P.n_expert_used;
+                        x = load_x(P.x, P.x_dtype, (size_t)t * P.k + j);
+                    }
+                    const uint32_t eb = (__float_as_uint(x) >> 23) & 0xFFu;
+                    const uint32_t emax = __reduce_max_sync(0xFFFFFFFFu, eb);
+                    int E = (int)emax - 149;
+                    E = E < -126 ? -126 : E;
+                    const float inv = __uint_as_float((uint32_t)(127 - E) << 23);  // 2^-E
+                    const int qv = __float2int_rn(x * inv);
+                    const uint32_t wd = lane >> 3, nib = lane & 7u;
+                    const uint32_t off = plane_base + (idx * DP_PW) * 4u +
+                                         ((wd * 3u) * 2u + (nib & 1u)) * 4u + (nib >> 1);
+                    sts8(off, (uint32_t)qv & 0xFFu);
+                    sts8(off + 8u, ((uint32_t)qv >> 8) & 0xFFu);
+                    sts8(off + 16u, ((uint32_t)qv >> 16) & 0xFFu);
+                    float sum = x;
+#pragma unroll
+                    for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, d);
+                    if (lane == 0) {
+                        uscale[idx] = __uint_as_float((uint32_t)(127 + E) << 23);  // 2^E
+                        usum[idx] = sum;
+                    }
+                }
+                __syncthreads();
+            }
+#pragma unroll
+            for (int i = 0; i < DP_UMAX; i++) {
+                const uint32_t u = base + l8 + GEMV_LPR * i;
+                if (u < nu) {
+                    const uint32_t g = tmin<uint32_t>(u / upg, G - 1u);
+                    const uint32_t sbv = sb[rloc * G + g];
+                    dp4a_unit<NPB>(w[i], planes + u * DP_PW, nu * DP_PW, uscale + u, usum + u, nu,
+                                   bf16_bits_to_f32(sbv & 0xFFFFu), bf16_bits_to_f32(sbv >> 16),
+                                   acc);
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NPB; q++) {
+#pragma unroll
+            for (int d = GEMV_LPR / 2; d > 0; d >>= 1) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], d);
+        }
+        if (l8 == 0 && row_ok) {
+#pragma unroll
+            for (int q = 0; q < NPB; q++)
+                if ((uint32_t)q < np) store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q]);
+        }
+    }
+}
+
+size_t dp4a_smem(const GemvParams &P, int npb) {
+    return (size_t)npb * P.n_units * (DP_PW + 2) * 4 + (size_t)GEMV_ROWS * P.groups * 4;
+}
+
+template <int NPB, bool FUSED>
+cudaError_t launch_dp4a_one(const GemvParams &P, dim3 grid, cudaStream_t st) {
+    const size_t smem = dp4a_smem(P, NPB);
+    auto kern = gemv_aff4_dp4a<NPB, FUSED>;
+    if (smem > 48 * 1024) {
+        static int smem_set[64];
+        cudaError_t e = ensure_dyn_smem(kern, smem, smem_set);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<grid, GEMV_THREADS, smem, st>>>(P);
+    return cudaGetLastError();
+}
+
+template <bool FUSED>
+cudaError_t launch_dp4a(const GemvParams &P, uint32_t npb, dim3 grid, cudaStream_t st) {
+    while (npb > 1 && dp4a_smem(P, (int)npb) > GEMV_SMEM_BUDGET) npb >>= 1;
+    if (npb <= 1) return launch_dp4a_one<1, FUSED>(P, grid, st);
+    if (npb <= 2) return launch_dp4a_one<2, FUSED>(P, grid, st);
+    if (npb <= 4) return launch_dp4a_one<4, FUSED>(P, grid, st);
+    return launch_dp4a_one<8, FUSED>(P, grid, st);
+}
+
+// The DP4A kernel covers 4-bit affine rows of whole 16-byte units with groups of
+// whole 32-code units.
+bool dp4a_ok(const QmmArgs &a) {
+    return a.kind == K_AFF4 && a.group_size % 32 == 0 && a.row_bytes % 16 == 0 &&
+           (uintptr_t)a.packed % 16 == 0 &&
+           (size_t)GEMV_ROWS * a.groups * 4 + (size_t)(a.row_bytes / 16) * (DP_PW + 2) * 4 <= GEMV_SMEM_BUDGET;
+}
+
+
+// ------------------------------------------ 4-bit affine, DP4A, TMA-staged rows
+//
+// Same arithmetic as gemv_aff4_dp4a, but each warp's weight rows (contiguous
+// in memory: rows of one expert are adjacent) arrive by one bulk TMA copy into
+// shared memory, signalled on that warp's mbarrier, and x arrives the same way
+// (for calls with few tokens, before the expert is even known). 512 threads per
+// CTA; LPR lanes per row, so a CTA holds 512/LPR rows and each lane a handful of
+// 16-byte units, which keeps a decode call's CTAs resident in one wave.
+// Modes: PAIR (one CTA column per pair, no deduplication: the m = 1 case),
+// FUSED (distinct experts ranked in the CTA, R <= 64), ROUTED (routing prologue).
+enum { MODE_PAIR = 0, MODE_FUSED = 1, MODE_ROUTED = 2 };
+constexpr int TMA_THREADS = 512;
+constexpr int TMA_WARPS = TMA_THREADS / 32;
+
+struct TmaLayout {
+    uint32_t w, xraw, planes, uscale, usum, sc, bi, total;
+};
+
+__host__ __device__ inline uint32_t al16u(uint32_t v) { return (v + 15u) & ~15u; }
+
+__host__ __device__ inline TmaLayout tma_layout(uint32_t rb, uint32_t row_bytes, uint32_t xraw_bytes,
+                                                uint32_t npb, uint32_t nu, uint32_t G) {
+    TmaLayout L;
+    L.w = 0;
+    L.xraw = al16u(rb * row_bytes);
+    L.planes = al16u(L.xraw + xraw_bytes);
+    L.uscale = L.planes + npb * nu * DP_PW * 4u;
+    L.usum = L.uscale + npb * nu * 4u;
+    L.sc = al16u(L.usum + npb * nu * 4u);
+    L.bi = al16u(L.sc + rb * G * 2u);
+    L.total = al16u(L.bi + rb * G * 2u);
+    return L;
+}
+
+// Eight consecutive x values (16-byte aligned) from a shared-memory row.
+__device__ __forceinline__ void smem_x8(const uint8_t *xr, int dt, uint32_t idx, float (&v)[8]) {
+    if (dt == DT_F32) {
+        const float4 a = *(const float4 *)(xr + 4u * idx), b = *(const float4 *)(xr + 4u * idx + 16u);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        const uint4 h = *(const uint4 *)(xr + 2u * idx);
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            if (dt == DT_BF16) {
+                v[2 * i] = __uint_as_float(hw[i] << 16);
+                v[2 * i + 1] = __uint_as_float(hw[i] & 0xFFFF0000u);
+            } else {
+                v[2 * i] = f16_bits_to_f32(hw[i] & 0xFFFFu);
+                v[2 * i + 1] = f16_bits_to_f32(hw[i] >> 16);
+            }
+        }
+    }
+}
+
+// Build the x planes of one 8-code word (lanes 4k..4k+3 of a warp hold the four
+// words of one unit). All 32 lanes must call it.
+__device__ __forceinline__ void plane_word(const float (&v)[8], uint32_t *unit_planes, uint32_t wd,
+                                           float *uscale_u, float *usum_u, bool store) {
+    uint32_t eb = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) eb = max(eb, (__float_as_uint(v[i]) >> 23) & 0xFFu);
+    eb = max(eb, __shfl_xor_sync(0xFFFFFFFFu, eb, 1));
+    eb = max(eb, __shfl_xor_sync(0xFFFFFFFFu, eb, 2));
+    int E = (int)eb - 149;
+    E = E < -126 ? -126 : E;
+    const float inv = __uint_as_float((uint32_t)(127 - E) << 23);  // 2^-E, |x * 2^-E| < 2^23
+    int q[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) q[i] = __float2int_rn(v[i] * inv);
+    uint32_t pw[6];
+#pragma unroll
+    for (int p = 0; p < 3; p++) {
+        // lo word: bytes p of q0, q2, q4, q6; hi word: bytes p of q1, q3, q5, q7
+        const uint32_t sel = (uint32_t)p | ((uint32_t)(4 + p) << 4);
+        const uint32_t l01 = __byte_perm((uint32_t)q[0], (uint32_t)q[2], sel);
+        const uint32_t l23 = __byte_perm((uint32_t)q[4], (uint32_t)q[6], sel);
+        const uint32_t h01 = __byte_perm((uint32_t)q[1], (uint32_t)q[3], sel);
+        const uint32_t h23 = __byte_perm((uint32_t)q[5], (uint32_t)q[7], sel);
+        pw[2 * p] = __byte_perm(l01, l23, 0x5410);
+        pw[2 * p + 1] = __byte_perm(h01, h23, 0x5410);
+    }
+    if (store) {
+        uint2 *dst = (uint2 *)(unit_planes + wd * 6u);  // [word][plane][lo/hi]
+        dst[0] = make_uint2(pw[0], pw[1]);
+        dst[1] = make_uint2(pw[2], pw[3]);
+        dst[2] = make_uint2(pw[4], pw[5]);
+    }
+    float sum = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+    if (store && wd == 0) {
+        *uscale_u = __uint_as_float((uint32_t)(127 + E) << 23);  // 2^E
+        *usum_u = sum;
+    }
+}
+
+template <int NPB, int MODE, int LPR>
+__global__ void __launch_bounds__(TMA_THREADS)
+gemv_aff4_tma(const GemvParams P) {
+    constexpr uint32_t RB = TMA_THREADS / LPR;  // rows per CTA
+    constexpr uint32_t RPW = 32 / LPR;          // rows per warp
+    constexpr uint64_t WAIT = 1000000000ull;
+    extern __shared__ __align__(128) uint8_t dsm8[];
+    __shared__ uint32_t ids_s[FUSED_MAX_R];
+    __shared__ uint32_t first_s[FUSED_MAX_R];
+    __shared__ uint32_t pairs_s[NPB];
+    __shared__ uint32_t expert_s, npairs_s;
+    __shared__ __align__(8) uint64_t bar_w[TMA_WARPS];
+    __shared__ __align__(8) uint64_t bar_x, bar_s;
+    __shared__ int abort_s;
+
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const uint32_t row0 = blockIdx.x * RB;
+    const uint32_t nu = P.n_units, G = P.groups, rbytes = P.row_bytes;
+    const uint32_t xsz = P.x_dtype == DT_F32 ? 4u : 2u;
+    const uint32_t xrow = P.k * xsz;
+    const bool spec = MODE != MODE_ROUTED && P.x_spec;  // all m x rows staged up front
+    const TmaLayout L = tma_layout(RB, rbytes, spec ? P.m * xrow : NPB * xrow, NPB, nu, G);
+    const uint32_t sbase = ptx::smem_u32(dsm8);
+    volatile int *abort_flag = &abort_s;
+
+    if (tid == 0) {
+        for (int i = 0; i < TMA_WARPS; i++) ptx::mbar_init(ptx::smem_u32(&bar_w[i]), 1);
+        ptx::mbar_init(ptx::smem_u32(&bar_x), 1);
+        ptx::mbar_init(ptx::smem_u32(&bar_s), 1);
+        ptx::fence_mbar_init();
+        abort_s = 0;
+    }
+    __syncthreads();
+    const uint32_t bx = ptx::smem_u32(&bar_x), bs = ptx::smem_u32(&bar_s);
+    if (spec && tid == 0) {
+        ptx::mbar_arrive_expect_tx(bx, P.m * xrow);
+        ptx::bulk_g2s(sbase + L.xraw, P.x, P.m * xrow, bx);
+    }
+
+    uint32_t expert = 0, total_pairs = 0;
+    const uint32_t *pair_src = nullptr;
+    bool work;
+    if constexpr (MODE == MODE_PAIR) {
+        const uint32_t p = blockIdx.y;
+        expert = __ldg(P.ids + p);
+        work = expert < P.num_experts;
+        total_pairs = 1;
+        if (!work) {
+            // out-of-range id: zero this pair's rows of the block
+            for (uint32_t r = row0 + tid; r < tmin<uint32_t>(row0 + RB, P.n); r += blockDim.x)
+                store_out(P.out, P.out_dtype, (size_t)p * P.n + r, 0.f);
+            if (blockIdx.x == 0 && tid == 0) atomicOr(P.err, ERR_BAD_ID);
+        }
+    } else {
+        work = route_prologue<MODE == MODE_FUSED>(P, ids_s, first_s, &expert_s, &npairs_s, row0, RB,
+                                                  expert, total_pairs, pair_src);
+    }
+    if (!work) {
+        if (spec) ptx::mbar_wait_bounded(bx, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);  // drain the copy
+        return;
+    }
+
+    // scales and biases of the CTA's rows (bf16), by bulk copy when aligned
+    const uint32_t nrows = tmin<uint32_t>(RB, P.n - row0);
+    const size_t soff = ((size_t)expert * P.n + row0) * G;
+    const uint32_t sbytes = nrows * G * 2u;
+    const bool s_bulk = (soff * 2u) % 16u == 0 && sbytes % 16u == 0 &&
+                        (uintptr_t)P.scales % 16u == 0 && (uintptr_t)P.aux % 16u == 0;
+    if (s_bulk) {
+        if (tid == 0) {
+            ptx::mbar_arrive_expect_tx(bs, 2u * sbytes);
+            ptx::bulk_g2s(sbase + L.sc, (const unsigned short *)P.scales + soff, sbytes, bs);
+            ptx::bulk_g2s(sbase + L.bi, (const unsigned short *)P.aux + soff, sbytes, bs);
+        }
+    } else {
+        unsigned short *sc = (unsigned short *)(dsm8 + L.sc), *bi = (unsigned short *)(dsm8 + L.bi);
+        for (uint32_t idx = tid; idx < nrows * G; idx += blockDim.x) {
+            sc[idx] = __ldg((const unsigned short *)P.scales + soff + idx);
+            bi[idx] = __ldg((const unsigned short *)P.aux + soff + idx);
+        }
+    }
+
+    // weight rows of this warp: one bulk copy
+    if (lane == 0) {
+        const uint32_t rb0 = row0 + warp * RPW;
+        const uint32_t nr = rb0 < P.n ? tmin<uint32_t>(RPW, P.n - rb0) : 0u;
+        const uint32_t bw = ptx::smem_u32(&bar_w[warp]);
+        if (nr) {
+            ptx::mbar_arrive_expect_tx(bw, nr * rbytes);
+            ptx::bulk_g2s(sbase + L.w + warp * RPW * rbytes,
+                          P.packed + ((size_t)expert * P.n + rb0) * rbytes, nr * rbytes, bw);
+        } else {
+            ptx::mbar_arrive(bw);
+        }
+    }
+    uint32_t *planes = (uint32_t *)(dsm8 + L.planes);
+    float *uscale = (float *)(dsm8 + L.uscale);
+    float *usum = (float *)(dsm8 + L.usum);
+    const unsigned short *sc = (const unsigned short *)(dsm8 + L.sc);
+    const unsigned short *bi = (const unsigned short *)(dsm8 + L.bi);
+    const uint32_t rloc = warp * RPW + lane / LPR, l = lane % LPR;
+    const uint32_t row = row0 + rloc;
+    const uint8_t *wrow = dsm8 + L.w + rloc * rbytes;
+    const uint32_t upg = P.gs / 32u;
+    const uint32_t nwords = nu * 4u;  // 8-code words per x row
+    uint32_t batch = 0;
+
+    for (uint32_t pb = 0; pb < total_pairs; pb += NPB, batch++) {
+        const uint32_t np = tmin<uint32_t>(NPB, total_pairs - pb);
+        if (pb > 0) __syncthreads();  // planes of the previous batch are no longer read
+        if constexpr (MODE == MODE_PAIR) {
+            if (tid == 0) pairs_s[0] = blockIdx.y;
+        } else {
+            load_pairs<MODE == MODE_FUSED>(P, ids_s, expert, pair_src, pb, np, pairs_s);
+        }
+        __syncthreads();
+        if (!spec && tid == 0) {
+            ptx::mbar_arrive_expect_tx(bx, np * xrow);
+            for (uint32_t q = 0; q < np; q++)
+                ptx::bulk_g2s(sbase + L.xraw + q * xrow,
+                              (const uint8_t *)P.x + (size_t)(pairs_s[q] / P.n_expert_used) * xrow,
+                              xrow, bx);
+        }
+        const bool x_ok = ptx::mbar_wait_bounded(bx, spec ? 0u : (batch & 1u), abort_flag, P.err,
+                                                 ERR_TIMEOUT, WAIT);
+        // x planes: one thread per (pair, 8-code word); 4 consecutive lanes hold a unit
+        if (__all_sync(0xFFFFFFFFu, x_ok)) {
+            for (uint32_t base = warp * 32u; base < NPB * nwords; base += TMA_THREADS) {
+                const uint32_t idx = base + lane;
+                float v[8];
+                const uint32_t q = idx / nwords, r = idx - q * nwords;
+                const uint32_t u = r >> 2, wd = r & 3u;
+                const uint32_t j = u * 32u + wd * 8u;
+                const bool valid = idx < NPB * nwords;
+                if (valid && q < np && j < P.k) {
+                    const uint32_t xr = spec ? pairs_s[q] / P.n_expert_used : q;
+                    smem_x8(dsm8 + L.xraw, P.x_dtype, xr * P.k + j, v);
+#pragma unroll
+                    for (int i = 0; i < 8; i++)
+                        if (j + i >= P.k) v[i] = 0.f;  // codes past k meet x = 0
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; i++) v[i] = 0.f;
+                }
+                const uint32_t uidx = valid ? q * nu + u : 0u;
+                plane_word(v, planes + uidx * DP_PW, wd, uscale + uidx, usum + uidx, valid);
+            }
+        }
+        bool s_ok = true;
+        if (pb == 0 && s_bulk) s_ok = ptx::mbar_wait_bounded(bs, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
+        __syncthreads();
+        bool w_ok = true;
+        if (pb == 0)
+            w_ok = ptx::mbar_wait_bounded(ptx::smem_u32(&bar_w[warp]), 0, abort_flag, P.err,
+                                          ERR_TIMEOUT, WAIT);
+        // a wait that gave up has flagged ERR_TIMEOUT; the warp then skips its work but
+        // keeps the block's barrier sequence
+        if (!__all_sync(0xFFFFFFFFu, x_ok && s_ok && w_ok && !*abort_flag)) continue;
+
+        float acc[NPB], acc2[NPB];
+#pragma unroll
+        for (int q = 0; q < NPB; q++) acc[q] = acc2[q] = 0.f;
+        uint32_t u = l;
+        for (; u + LPR < nu; u += 2 * LPR) {  // two independent units per step
+            const uint4 w0 = *(const uint4 *)(wrow + 16u * u);
+            const uint4 w1 = *(const uint4 *)(wrow + 16u * (u + LPR));
+            const uint32_t si0 = rloc * G + tmin<uint32_t>(u / upg, G - 1u);
+            const uint32_t si1 = rloc * G + tmin<uint32_t>((u + LPR) / upg, G - 1u);
+            dp4a_unit<NPB>(w0, planes + u * DP_PW, nu * DP_PW, uscale + u, usum + u, nu,
+                           bf16_bits_to_f32(sc[si0]), bf16_bits_to_f32(bi[si0]), acc);
+            dp4a_unit<NPB>(w1, planes + (u + LPR) * DP_PW, nu * DP_PW, uscale + u + LPR,
+                           usum + u + LPR, nu, bf16_bits_to_f32(sc[si1]), bf16_bits_to_f32(bi[si1]),
+                           acc2);
+        }
+        if (u < nu) {
+            const uint4 w0 = *(const uint4 *)(wrow + 16u * u);
+            const uint32_t si0 = rloc * G + tmin<uint32_t>(u / upg, G - 1u);
+            dp4a_unit<NPB>(w0, planes + u * DP_PW, nu * DP_PW, uscale + u, usum + u, nu,
+                           bf16_bits_to_f32(sc[si0]), bf16_bits_to_f32(bi[si0]), acc);
+        }
+#pragma unroll
+        for (int q = 0; q < NPB; q++) {
+            acc[q] += acc2[q];
+#pragma unroll
+            for (int d = LPR / 2; d > 0; d >>= 1) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], d);
+        }
+        if (l == 0 && row < P.n) {
+#pragma unroll
+            for (int q = 0; q < NPB; q++)
+                if ((uint32_t)q < np) store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q]);
+        }
+    }
+    if (*abort_flag) {
+        // a wait gave up: let this CTA's copies land before its shared memory is released
+        ptx::mbar_wait_bounded(ptx::smem_u32(&bar_w[warp]), 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
+        ptx::mbar_wait_bounded(bx, spec ? 0u : ((batch - 1u) & 1u), nullptr, P.err, ERR_TIMEOUT, WAIT);
+        if (s_bulk) ptx::mbar_wait_bounded(bs, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
+    }
+}
+
+int tma_lpr(uint32_t nu) {
+    // lanes per row: about 3 to 6 16-byte units per lane
+    if (nu <= 24) return 4;
+    if (nu <= 48) return 8;
+    if (nu <= 96) return 16;
+    return 32;
+}
+
+template <int NPB, int MODE, int LPR>
+cudaError_t launch_tma_one(const GemvParams &P, uint32_t ycount, cudaStream_t st) {
+    constexpr uint32_t RB = TMA_THREADS / LPR;
+    const uint32_t xsz = P.x_dtype == DT_F32 ? 4u : 2u;
+    const bool spec = MODE != MODE_ROUTED && P.x_spec;
+    const TmaLayout L = tma_layout(RB, P.row_bytes, spec ? P.m * P.k * xsz : NPB * P.k * xsz, NPB,
+                                   P.n_units, P.groups);
+    auto kern = gemv_aff4_tma<NPB, MODE, LPR>;
+    if (L.total > 48 * 1024) {
+        static int smem_set[64];
+        cudaError_t e = ensure_dyn_smem(kern, L.total, smem_set);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((P.n + RB - 1) / RB, ycount);
+    kern<<<grid, TMA_THREADS, L.total, st>>>(P);
+    return cudaGetLastError();
+}
+
+template <int MODE, int LPR>
+cudaError_t launch_tma_npb(const GemvParams &P, uint32_t npb, uint32_t ycount, cudaStream_t st) {
+    if (npb <= 1) return launch_tma_one<1, MODE, LPR>(P, ycount, st);
+    if (npb <= 2) return launch_tma_one<2, MODE, LPR>(P, ycount, st);
+    if (npb <= 4) return launch_tma_one<4, MODE, LPR>(P, ycount, st);
+    return launch_tma_one<8, MODE, LPR>(P, ycount, st);
+}
+
+template <int MODE>
+cudaError_t launch_tma(const GemvParams &P, uint32_t npb, uint32_t ycount, cudaStream_t st) {
+    switch (tma_lpr(P.n_units)) {
+        case 4: return launch_tma_npb<MODE, 4>(P, npb, ycount, st);
+        case 8: return launch_tma_npb<MODE, 8>(P, npb, ycount, st);
+        case 16: return launch_tma_npb<MODE, 16>(P, npb, ycount, st);
+        default: return launch_tma_npb<MODE, 32>(P, npb, ycount, st);
+    }
+}
+
+// The TMA kernel needs the DP4A conditions, 16-byte aligned x rows, and its
+// shared-memory layout within budget for the largest pair batch.
+bool tma_ok(const QmmArgs &a, uint32_t npb, bool spec) {
+    if (!dp4a_ok(a)) return false;
+    const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
+    if ((a.k * xsz) % 16u != 0 || (uintptr_t)a.x % 16u != 0) return false;
+    const uint32_t nu = a.row_bytes / 16u;
+    const uint32_t rb = TMA_THREADS / (uint32_t)tma_lpr(nu);
+    const TmaLayout L = tma_layout(rb, a.row_bytes, spec ? a.m * a.k * xsz : npb * a.k * xsz, npb, nu,
+                                   a.groups);
+    return L.total <= 100u * 1024u;
 }
 
 template <int KIND, int NPB, bool FUSED>
@@ -388,6 +911,7 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     P.x = a.x; P.ids = a.ids; P.packed = a.packed; P.scales = a.scales; P.aux = a.aux;
     P.out = a.out; P.err = err;
     P.R = a.m * a.n_expert_used;
+    P.m = a.m;
     P.k = a.k; P.n = a.n; P.gs = a.group_size; P.groups = a.groups;
     P.n_expert_used = a.n_expert_used; P.num_experts = a.num_experts; P.row_bytes = a.row_bytes;
     const uint32_t uc = (uint32_t)unit_codes(a.kind), ub = (uint32_t)unit_bytes(a.kind);
@@ -410,6 +934,17 @@ cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st) 
     dim3 grid((a.n + GEMV_ROWS - 1) / GEMV_ROWS, distinct_max);
     // pairs of one expert come from distinct tokens unless ids repeat inside a token
     const uint32_t npb = tmin<uint32_t>(a.m, 8u);
+    const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
+    const bool spec = (uint64_t)a.m * a.k * xsz <= 32768u;
+    if (a.m == 1 && tma_ok(a, 1, spec)) {
+        P.x_spec = spec;
+        return launch_tma<MODE_PAIR>(P, 1, P.R, st);
+    }
+    if (tma_ok(a, npb, spec)) {
+        P.x_spec = spec;
+        return launch_tma<MODE_FUSED>(P, npb, distinct_max, st);
+    }
+    if (dp4a_ok(a)) return launch_dp4a<true>(P, npb, grid, st);
     return launch_kind<true>(P, a.kind, npb, grid, st);
 }
 
@@ -418,6 +953,8 @@ cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const u
     GemvParams P = make_params(a, err);
     P.counts = counts; P.offsets = offsets; P.sorted_pairs = sorted_pairs;
     dim3 grid((a.n + GEMV_ROWS - 1) / GEMV_ROWS, a.num_experts);
+    if (tma_ok(a, 8u, false)) return launch_tma<MODE_ROUTED>(P, 8u, a.num_experts, st);
+    if (dp4a_ok(a)) return launch_dp4a<false>(P, 8u, grid, st);
     return launch_kind<false>(P, a.kind, 8u, grid, st);
 }
 

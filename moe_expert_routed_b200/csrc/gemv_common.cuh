@@ -1,0 +1,116 @@
+// gemv_common.cuh -- pieces shared by the decode-path kernels: launch
+// parameters and the routing prologue of one CTA (fused or routed).
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int GEMV_THREADS = 256;
+constexpr int GEMV_LPR = 8;                         // lanes per row
+constexpr int GEMV_ROWS = GEMV_THREADS / GEMV_LPR;  // 32 rows per CTA
+constexpr uint32_t FUSED_MAX_R = 64;
+constexpr size_t GEMV_SMEM_BUDGET = 200 * 1024;
+
+struct GemvParams {
+    const void *x;
+    const uint32_t *ids;
+    const uint8_t *packed;
+    const void *scales;
+    const void *aux;
+    void *out;
+    uint32_t *err;
+    const uint32_t *counts, *offsets, *sorted_pairs;  // routed mode
+    uint32_t R, m, k, n, gs, groups, n_expert_used, num_experts, row_bytes, n_units, xstride;
+    int x_dtype, out_dtype, load_mode;
+    int x_spec;        // TMA kernels: stage all m x rows before routing
+    uint32_t kstages;  // integer-MMA kernel: k stages of the weight copies
+};
+
+// Which expert this CTA serves and how many pairs it has. Fused mode: all ids
+// are read into shared memory, distinct valid experts are ranked in ascending
+// order and blockIdx.y picks one; CTAs with blockIdx.y == 0 also zero the rows
+// of out-of-range pairs for their row block. Routed mode: blockIdx.y is the
+// expert and its pairs come from the routing prologue. Returns false (for the
+// whole CTA) when there is no work. Contains __syncthreads: call uniformly.
+template <bool FUSED>
+__device__ __forceinline__ bool route_prologue(const GemvParams &P, uint32_t *ids_s,
+                                               uint32_t *first_s, uint32_t *expert_s,
+                                               uint32_t *count_s, uint32_t row0, uint32_t rows,
+                                               uint32_t &expert, uint32_t &total_pairs,
+                                               const uint32_t *&pair_src) {
+    const uint32_t tid = threadIdx.x;
+    if constexpr (FUSED) {
+        const uint32_t R = P.R, E = P.num_experts;
+        if (tid < R) ids_s[tid] = __ldg(P.ids + tid);
+        __syncthreads();
+        if (tid < R) {
+            const uint32_t e = ids_s[tid];
+            bool first = e < E;
+            for (uint32_t t = 0; t < tid && first; t++) first = ids_s[t] != e;
+            first_s[tid] = first;
+        }
+        __syncthreads();
+        if (tid < R && first_s[tid]) {
+            const uint32_t e = ids_s[tid];
+            uint32_t rank = 0;
+            for (uint32_t t = 0; t < R; t++) rank += (first_s[t] && ids_s[t] < e);
+            if (rank == blockIdx.y) *expert_s = e;
+        }
+        if (tid == 0) {
+            uint32_t D = 0;
+            for (uint32_t t = 0; t < R; t++) D += first_s[t];
+            *count_s = D;  // number of distinct valid experts
+        }
+        __syncthreads();
+        if (blockIdx.y == 0) {
+            for (uint32_t idx = tid; idx < R * rows; idx += blockDim.x) {
+                const uint32_t p = idx / rows, r = row0 + idx % rows;
+                if (ids_s[p] >= E && r < P.n) store_out(P.out, P.out_dtype, (size_t)p * P.n + r, 0.f);
+            }
+            if (blockIdx.x == 0 && tid < R && ids_s[tid] >= E) atomicOr(P.err, ERR_BAD_ID);
+        }
+        if (blockIdx.y >= *count_s) return false;  // uniform
+        expert = *expert_s;
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t c = 0;
+            for (uint32_t t = 0; t < R; t++) c += ids_s[t] == expert;
+            *count_s = c;
+        }
+        __syncthreads();
+        total_pairs = *count_s;
+        return true;
+    } else {
+        expert = blockIdx.y;
+        total_pairs = __ldg(P.counts + expert);
+        if (total_pairs == 0) return false;
+        pair_src = P.sorted_pairs + __ldg(P.offsets + expert);
+        return true;
+    }
+}
+
+// Pairs [pb, pb+np) of this CTA's expert into pairs_s (thread 0).
+template <bool FUSED>
+__device__ __forceinline__ void load_pairs(const GemvParams &P, const uint32_t *ids_s,
+                                           uint32_t expert, const uint32_t *pair_src, uint32_t pb,
+                                           uint32_t np, uint32_t *pairs_s) {
+    if (threadIdx.x == 0) {
+        if constexpr (FUSED) {
+            uint32_t c2 = 0, seen = 0;
+            for (uint32_t t = 0; t < P.R && c2 < np; t++)
+                if (ids_s[t] == expert) {
+                    if (seen >= pb) pairs_s[c2++] = t;
+                    seen++;
+                }
+        } else {
+            for (uint32_t q = 0; q < np; q++) pairs_s[q] = __ldg(pair_src + pb + q);
+        }
+    }
+}
+
+
+}  // namespace
+}  // namespace moe

@@ -35,6 +35,25 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
         : "memory");
 }
 
+// Arrive on the mbarrier and add `bytes` to the transaction count its current
+// phase waits for (completed by cp.async.bulk ... complete_tx::bytes).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+        "r"(bytes)
+        : "memory");
+}
+
+// Bulk (TMA, non-tensor) copy global -> shared of `bytes` (multiple of 16; both
+// addresses 16-byte aligned), signalled on the mbarrier. No multicast.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
