@@ -151,6 +151,45 @@ moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_u
                             uint32_t *tile_count, void *workspace, size_t workspace_bytes,
                             moe_stream_t stream);
 
+/*
+ * moe_qmm_id_noalloc -- moe_qmm_id for callers that cannot allocate device memory.
+ * (No counterpart on the pages: their operations allocate their own output and
+ * parameter buffers.)
+ *
+ * Who needs it: a service that reserves all device memory at start-up and allows
+ * no allocation on its request path, a plug-in running under another framework's
+ * caching allocator (a raw cudaMalloc bypasses that allocator and can fail when
+ * its pool holds nearly all memory), or a caller that only has the operation's
+ * own inputs and outputs. Instead of a caller-provided workspace, the routing
+ * prologue uses a MOE_NOALLOC_SCRATCH_BYTES array in device memory that belongs
+ * to this library; every GPU that loads the library holds that array until the
+ * process exits. This entry point calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * Same arguments, layouts and results as moe_qmm_id, minus the workspace. The
+ * caller still owns and passes x, ids, the weights and out.
+ *   * Sizes whose workspace (moe_qmm_id_workspace_bytes(m, n_expert_used,
+ *     num_experts)) exceeds MOE_NOALLOC_SCRATCH_BYTES return
+ *     MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing. At num_experts <= 256 that
+ *     admits m * n_expert_used up to about 200,000 routings.
+ *   * The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; a failure returns
+ *     MOE_ERR_CUDA. Make that first call before capturing a stream that uses it.
+ *   * All calls on a device share the one array and it keeps the last call's
+ *     contents. Nothing in it needs to start at zero (every call writes the
+ *     buffers it later reads), but calls that overlap on the GPU (different
+ *     streams without ordering between them) race on it: order them.
+ *   * The array's device error word is not readable through this entry point:
+ *     out-of-range ids still give zero output rows; use moe_qmm_id with a
+ *     workspace to observe MOE_ERR_BAD_EXPERT_ID or MOE_ERR_TIMEOUT.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+moe_status moe_qmm_id_noalloc(const void *x, const uint32_t *ids, const void *packed,
+                              const void *scales, const void *aux, void *out, uint32_t m, uint32_t k,
+                              uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                              uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                              moe_dtype out_dtype, moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the device error word of `workspace`.
  * Returns MOE_OK, MOE_ERR_BAD_EXPERT_ID (some id was >= num_experts),
  * MOE_ERR_TIMEOUT (a bounded wait inside a kernel gave up; its outputs are not

@@ -89,6 +89,21 @@ static moe_status validate(const void *x, const uint32_t *ids, const void *packe
     return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace moe {
+// The scalar checks moe_qmm_id runs first, for other entry points of the library.
+moe_status validate_call(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                         const void *aux, const void *out, uint32_t m, uint32_t k, uint32_t n,
+                         uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
+                         uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype) {
+    return validate(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt, n_expert_used,
+                    num_experts, x_dtype, out_dtype);
+}
+}  // namespace moe
+
+extern "C" {
+
 moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packed,
                            const void *scales, const void *aux, void *out, uint32_t m, uint32_t k,
                            uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,

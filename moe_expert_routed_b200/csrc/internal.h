@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include "moe_qmm.h"
 #include <stddef.h>
 #include <stdint.h>
 
@@ -77,5 +79,11 @@ uint32_t gemm_tile_rows(const QmmArgs &a);
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
                         uint32_t *err, cudaStream_t st);
+
+// moe_qmm_id's scalar validation (MOE_OK or the status moe_qmm_id would return).
+moe_status validate_call(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                         const void *aux, const void *out, uint32_t m, uint32_t k, uint32_t n,
+                         uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
+                         uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype);
 
 }  // namespace moe
