@@ -41,6 +41,9 @@ sys.path.insert(0, ROOT)
 METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
 N_LAYERS = 16
 GRAPH_STEPS = 1000
+# dram__bytes_read.sum + dram__bytes_write.sum of one gate/up launch of the decode
+# kernel (ncu, cold L2): profiles/decode_gate_up_gemv_aff4_tma.md
+GATE_UP_DRAM_BYTES = 17871616
 
 
 def peaks():
@@ -386,11 +389,16 @@ def run_ours(args, dist: Dist):
         del gp
 
     pk = peaks()
-    achieved = W.bytes() * replays / secs / 1e9
+    # dominant kernel: the gate/up launch (about 57% of the step); timed alone from a
+    # graph of gate/up calls only. DRAM traffic per launch from one ncu capture of
+    # this kernel (profiles/decode_gate_up_gemv_aff4_tma.md).
+    achieved = per_call["gate_up"]["GB_per_s"]
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
-                "kernel": "gemv_kernel<AFF4, NPB=1, fused> (gate/up and down launches)"}
+                "frac": achieved / pk["hbm_gbs"], "traffic": GATE_UP_DRAM_BYTES,
+                "algorithmic_bytes": W.bytes((0,)) / W.G,
+                "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+                "kernel": "gemv_aff4_tma (one CTA column per pair), gate/up launch",
+                "step_frac": W.bytes() * replays / secs / 1e9 / pk["hbm_gbs"]}
     e2e_steps = min(max(K // 10, 50), 2000)
     e_secs, per_step_bytes, h2d, d2h = e2e_decode(W, e2e_steps)
     e_secs = dist.max(e_secs)
@@ -424,6 +432,130 @@ def run_ours(args, dist: Dist):
     del g
 
 
+def run_grouped(args, dist: Dist):
+    """One call of the named grouped-path workload per step (routing prologue +
+    tcgen05 grouped GEMM), inputs resident in HBM, CUDA graph of G calls."""
+    import moe_expert_routed_b200 as M
+    from workloads import config_problem
+    from workloads.torch_io import to_device
+
+    M.lib()
+    dev_i = dist.local if dist.world > 1 else 0
+    torch.cuda.set_device(dev_i)
+    P = config_problem(args.config)
+    d = to_device(P)
+    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    out_dt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float16}[P.out_dtype]
+    out = torch.empty((P.m, P.n_expert_used, P.n), dtype=out_dt, device="cuda")
+
+    def call():
+        M.qmm_id(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], n=P.n, group_size=P.group_size,
+                 bits=P.bits, fmt=P.fmt, num_experts=P.num_experts, out=out, workspace=ws)
+
+    def route_only():
+        M.route(d["ids"], P.num_experts, 256 if P.R >= 96 * P.num_experts else 64, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    assert M.poll_error(ws) == 0
+    G = max(1, min(args.steps, 20))
+    graphs = []
+    for fn in (call,):
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            fn()
+        torch.cuda.current_stream().wait_stream(st)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for _ in range(G):
+                fn()
+        graphs.append(g)
+    replays = max(1, args.steps // G)
+    graphs[0].replay()
+    sampler = clocks_sampler(dev_i) if dist.rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    dist.barrier()
+    torch.cuda.synchronize()
+    secs = time_graph(graphs[0], replays)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = clocks_summary(sampler) if dist.rank == 0 else None
+    calls = replays * G
+    # routing prologue alone (outside the timed region): share of a call
+    for _ in range(3):
+        route_only()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(50):
+        route_only()
+    b.record()
+    b.synchronize()
+    route_us = a.elapsed_time(b) / 50 * 1e3
+    secs_max = dist.max(secs)
+    ids = P.ids.reshape(-1)
+    valid = int((ids < P.num_experts).sum())
+    flops = 2.0 * valid * P.n * P.k
+    nbytes = alg_bytes(P, ids)
+    us = secs_max / calls * 1e6
+    tflops = dist.sum(flops * calls) / secs_max / 1e12
+    gbs = dist.sum(nbytes * calls) / secs_max / 1e9
+    pk = peaks()
+    gemm_us = max(us - route_us, 1e-9)
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": dist.world, "steps": calls,
+        "warmup": max(args.warmup, 3), "ms_per_step": us / 1e3, "us_per_call": us,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": {0: "f32", 1: "bf16", 2: "f16"}[P.x_dtype] + " x / fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": f"{args.config}: E{P.num_experts} top{P.n_expert_used} m{P.m} k{P.k} n{P.n} "
+                               f"fmt{P.fmt} bits{P.bits} g{P.group_size}",
+                   "l2": f"weights {P.packed.nbytes / 1e6:.0f} MB (> L2 126 MB), one call per step",
+                   "timing": f"CUDA graph of {G} calls replayed {replays}x, CUDA events"},
+        "effective_GB_per_s": gbs,
+        "route_us": route_us,
+        "gemm_us_estimate": gemm_us,
+        "roofline": {"tensor": {"achieved": flops / gemm_us / 1e6, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": flops / gemm_us / 1e6 / pk["bf16_tflops"]},
+                     "hbm": {"achieved": nbytes / gemm_us / 1e3, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": nbytes / gemm_us / 1e3 / pk["hbm_gbs"]},
+                     "kernel": "grouped_gemm_kernel (tcgen05), time = call - routing prologue"},
+        "gpu_launches": 4 * calls,
+        "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_probe(args):
+    """A few untimed calls of one workload (for profiler captures): decode runs the
+    gate/up projection `reps` times, then the down projection `reps` times; the
+    grouped configs run one full call `reps` times."""
+    import moe_expert_routed_b200 as M
+    from workloads import config_problem
+    from workloads.torch_io import to_device
+
+    M.lib()
+    names = ["decode_gate_up", "decode_down"] if args.probe == "decode" else [args.probe]
+    for name in names:
+        P = config_problem(name)
+        d = to_device(P)
+        ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+        out_dt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float16}[P.out_dtype]
+        out = torch.empty((P.m, P.n_expert_used, P.n), dtype=out_dt, device="cuda")
+        for _ in range(args.reps):
+            M.qmm_id(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], n=P.n, group_size=P.group_size,
+                     bits=P.bits, fmt=P.fmt, num_experts=P.num_experts, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        if M.poll_error(ws) != 0:
+            raise SystemExit(f"{name}: device error word set")
+    print(json.dumps({"probe": args.probe, "reps": args.reps, "status": "ok"}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -432,12 +564,21 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--config", default="decode", choices=["decode", "canvas", "prefill", "skewed"])
+    ap.add_argument("--probe", choices=["decode", "canvas", "prefill", "skewed"],
+                    help="run a few untimed calls (for profiler captures) and exit")
+    ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.probe:
+        run_probe(args)
+        return
     dist = Dist(args.gpus)
     try:
         if args.impl == "reference":
             run_reference(args, dist)
+        elif args.config != "decode":
+            run_grouped(args, dist)
         else:
             run_ours(args, dist)
     finally:

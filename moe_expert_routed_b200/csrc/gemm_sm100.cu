@@ -11,18 +11,25 @@
 // GEMM fed by expert_offsets / sorted_token_ids (metrale helpers_b.rs,
 // launch_grouped_gemm).
 //
-// Warp roles (288 threads):
-//   warps 0-7  producers: per 64-wide k-tile, dequantise 128 rows x 64 codes to
-//              16-bit values in the 128-byte-swizzled K-major layout and gather
-//              the pairs' x rows (cp.async, or f32 loads split into two bf16
-//              halves); then the epilogue: TMEM -> registers (tcgen05.ld),
-//              times scale2 for NVFP4, rounded once to the output type, stored to
-//              row p of out (the scatter back to [token][slot] order).
-//   warp 8     TMEM allocation; one lane issues tcgen05.mma (kind::f16, fp32
-//              accumulation in TMEM) and tcgen05.commit.
-// Stages are handed over with mbarriers (full: 256 producer arrivals; empty and
-// accumulator-ready: tcgen05.commit). Every wait is bounded (1 s); a wait that
-// gives up sets ERR_TIMEOUT, the CTA drains its in-flight MMAs and copies,
+// Warp roles (416 threads), each running through the k-tiles on its own:
+//   warps 0-7   dequantisers: per 64-wide k-tile, turn the staged codes of 128
+//               rows x 64 codes into 16-bit values in the 128-byte-swizzled
+//               K-major layout (and split f32 x into two bf16 halves); then the
+//               epilogue: TMEM -> registers (tcgen05.ld), times scale2 for
+//               NVFP4, rounded once to the output type, stored to row p of out
+//               (the scatter back to [token][slot] order).
+//   warps 8-11  loaders: cp.async the pairs' x rows straight into the B operand
+//               tile and the packed codes and scale words into a staging area,
+//               up to S k-tiles ahead of the tensor core; each loader's
+//               completion is signalled on the stage's mbarrier by the copy
+//               engine (cp.async.mbarrier.arrive), so loaders never block on
+//               their own copies.
+//   warp 12     TMEM allocation; one lane issues tcgen05.mma (kind::f16, fp32
+//               accumulation in TMEM) and tcgen05.commit.
+// Per stage: loaded (loader copies landed) -> full (dequantised) -> empty (the
+// MMAs that read it completed). Dequantisation of k-tile kt overlaps the MMAs
+// of kt-1 and the copies of kt+1 .. kt+S-1. Every wait is bounded (1 s); a wait
+// that gives up sets ERR_TIMEOUT, the CTA drains its in-flight MMAs and copies,
 // frees TMEM and exits.
 //
 // Exactness: products must stay exact so that the fp32 accumulation is the
@@ -40,11 +47,14 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128;
-constexpr int KT = 64;  // k per tile: one 128-byte swizzle atom of 16-bit values
-constexpr int NPROD = 256;
-constexpr int GEMM_THREADS = NPROD + 32;
-constexpr int MMA_WARP = NPROD / 32;
-constexpr int A_TILE = BM * KT * 2;  // bytes per A term per stage
+constexpr int KT = 64;                          // k per tile: one 128-byte swizzle atom of 16-bit values
+constexpr int NDQ = 256;                        // dequantising threads (warps 0-7)
+constexpr int NLD = 128;                        // loader threads (warps 8-11)
+constexpr int GEMM_THREADS = NDQ + NLD + 32;    // + the MMA warp
+constexpr int LD_WARP0 = NDQ / 32;
+constexpr int MMA_WARP = (NDQ + NLD) / 32;
+constexpr int MAX_STAGES = 6;
+constexpr int A_TILE = BM * KT * 2;             // bytes per A term per stage
 constexpr uint64_t WAIT_NS = 1000000000ull;
 
 struct GemmParams {
@@ -56,6 +66,8 @@ struct GemmParams {
     void *out;
     uint32_t *err;
     uint32_t k, n, lg_gs, groups, n_expert_used, row_bytes, ktiles, stages;
+    uint32_t scale_words;  // rows of scales (and biases) 4-byte aligned: staged by the loaders
+    uint32_t raw16;        // rows of codes 16-byte aligned: staged in 16-byte copies (else 8)
     int out_dtype;
     uint64_t timeout_ns;
 };
@@ -90,12 +102,7 @@ __device__ __forceinline__ float round16(float v) {
     else return __bfloat162float(__float2bfloat16_rn(v));
 }
 
-__device__ __forceinline__ uint2 ldg64_guard(const uint8_t *row, uint32_t off, uint32_t row_bytes) {
-    if (off + 8u <= row_bytes) return __ldg((const uint2 *)(row + off));
-    return make_uint2(0u, 0u);
-}
-
-// Raw words holding codes [j0, j0+32) of one row (j0 a multiple of 32).
+// Packed words holding one thread's 32 codes (j0 a multiple of 32).
 template <int KIND> struct Raw;
 template <> struct Raw<K_AFF4> { static constexpr int W = 4; };
 template <> struct Raw<K_CB4> { static constexpr int W = 4; };
@@ -103,127 +110,190 @@ template <> struct Raw<K_NVFP4> { static constexpr int W = 4; };
 template <> struct Raw<K_AFF8> { static constexpr int W = 8; };
 template <> struct Raw<K_AFF6> { static constexpr int W = 6; };
 template <> struct Raw<K_CB2> { static constexpr int W = 2; };
-template <> struct Raw<K_CB3> { static constexpr int W = 5; };
+template <> struct Raw<K_CB3> { static constexpr int W = 4; };  // codes SUB .. SUB+31, SUB <= 8
 
-template <int KIND>
-__device__ __forceinline__ void load_raw(const uint8_t *row, uint32_t j0, uint32_t row_bytes,
-                                         uint32_t (&w)[Raw<KIND>::W], uint32_t &sub) {
-    sub = 0;
-    if constexpr (KIND == K_CB3) {
-        const uint32_t w0 = j0 / 10u;
-        sub = j0 - 10u * w0;
-#pragma unroll
-        for (int i = 0; i < 5; i++) {
-            const uint32_t off = (w0 + i) * 4u;
-            w[i] = (off + 4u <= row_bytes) ? __ldg((const uint32_t *)(row + off)) : 0u;
-        }
-    } else {
-        constexpr int BITS = kind_bits(KIND);
-        const uint32_t off = j0 * BITS / 8u;  // multiple of 8 bytes
-#pragma unroll
-        for (int i = 0; i < Raw<KIND>::W / 2; i++) {
-            uint2 v = ldg64_guard(row, off + 8u * i, row_bytes);
-            w[2 * i] = v.x;
-            w[2 * i + 1] = v.y;
-        }
-    }
-}
-
-template <int KIND, int I>
-__device__ __forceinline__ uint32_t raw_code(const uint32_t (&w)[Raw<KIND>::W], uint32_t sub) {
-    if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
-        return (w[I / 8] >> (4 * (I % 8))) & 15u;
-    } else if constexpr (KIND == K_AFF8) {
-        return (w[I / 4] >> (8 * (I % 4))) & 255u;
-    } else if constexpr (KIND == K_CB2) {
-        return (w[I / 16] >> (2 * (I % 16))) & 3u;
-    } else if constexpr (KIND == K_AFF6) {
-        constexpr int b = 6 * I, wi = b / 32, sh = b % 32;
-        if constexpr (sh <= 26) return (w[wi] >> sh) & 63u;
-        else return __funnelshift_r(w[wi], w[wi + 1], sh) & 63u;
-    } else {  // K_CB3: code (sub + I) of the 5 loaded words, 10 codes per word
-        const uint32_t idx = sub + I;
-        const uint32_t wi = (idx * 205u) >> 11;  // idx / 10 for idx < 1029
-        const uint32_t sh = 3u * (idx - 10u * wi);
-        const uint32_t word = wi == 0 ? w[0] : wi == 1 ? w[1] : wi == 2 ? w[2] : wi == 3 ? w[3] : w[4];
-        return (word >> sh) & 7u;
-    }
-}
-
-template <int KIND, int I>
-struct DeqLoop {
-    static __device__ __forceinline__ void run(const uint32_t (&w)[Raw<KIND>::W], uint32_t sub,
-                                               float s0, float b0, float s1, float b1,
-                                               bool two_groups, const float *cb, float (&v)[32]) {
-        if constexpr (I < 32) {
-            const uint32_t code = raw_code<KIND, I>(w, sub);
-            const float s = (I >= 16 && two_groups) ? s1 : s0;
-            const float b = (I >= 16 && two_groups) ? b1 : b0;
-            if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) v[I] = fmaf((float)code, s, b);
-            else if constexpr (KIND == K_NVFP4) v[I] = e2m1_to_f32(code) * s;
-            else v[I] = cb[code] * s;
-            DeqLoop<KIND, I + 1>::run(w, sub, s0, b0, s1, b1, two_groups, cb, v);
-        }
-    }
+// Staging area of one k-tile: one row per weight row,
+//   bytes [0, RB)         the k-tile's packed codes (3-bit codebook: the 8 words
+//                         from word floor(j0/10), which hold codes j0 .. j0+63)
+//   bytes [RB, RB+8)      the 4-byte-aligned scale word(s) holding the k-tile's groups
+//   bytes [RB+8, RB+16)   the same words of the biases (affine)
+// Rows are an odd number of 16-byte units apart, so 8 consecutive rows read
+// with 16-byte loads touch all 32 banks once.
+template <int KIND> struct RawLayout {
+    static constexpr uint32_t RB = KIND == K_CB3 ? 32u : 8u * kind_bits(KIND);
+    static constexpr uint32_t SC = RB, BI = RB + 8u;
+    static constexpr uint32_t STRIDE = ((RB + 16u) / 16u) % 2u ? RB + 16u : RB + 32u;
+    static constexpr uint32_t TILE = BM * STRIDE;
 };
 
-// Dequantise the thread's 32 codes and store them as 4 chunks of 8 16-bit values
-// (hi term, and lo term when present) at chunk positions c0 .. c0+3 of row r.
-template <int KIND, bool F16>
-__device__ __forceinline__ void dequant_store(const uint32_t (&w)[Raw<KIND>::W], uint32_t sub,
-                                              float s0, float b0, float s1, float b1, bool two_groups,
-                                              const float *cb, uint32_t a_hi, uint32_t a_lo,
-                                              uint32_t r, uint32_t c0) {
-    float v[32];
-    DeqLoop<KIND, 0>::run(w, sub, s0, b0, s1, b1, two_groups, cb, v);
+template <int KIND, int SUB>
+__device__ __forceinline__ uint32_t raw_code(const uint32_t (&w)[Raw<KIND>::W], int i) {
+    // i is a compile-time constant after unrolling
+    if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
+        return (w[i / 8] >> (4 * (i % 8))) & 15u;
+    } else if constexpr (KIND == K_AFF8) {
+        return (w[i / 4] >> (8 * (i % 4))) & 255u;
+    } else if constexpr (KIND == K_CB2) {
+        return (w[i / 16] >> (2 * (i % 16))) & 3u;
+    } else if constexpr (KIND == K_AFF6) {
+        const int b = 6 * i, wi = b / 32, sh = b % 32;
+        return sh <= 26 ? (w[wi] >> sh) & 63u : __funnelshift_r(w[wi], w[wi + 1 < 6 ? wi + 1 : wi], sh) & 63u;
+    } else {  // K_CB3: code (SUB + i) of the loaded words, 10 codes per word
+        return (w[(SUB + i) / 10] >> (3 * ((SUB + i) % 10))) & 7u;
+    }
+}
+
+template <int KIND, int SUB>
+__device__ __forceinline__ void dequant32(const uint32_t (&w)[Raw<KIND>::W], float s0, float b0,
+                                          float s1, float b1, bool two_groups, const float *cb,
+                                          float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        const uint32_t code = raw_code<KIND, SUB>(w, i);
+        const float s = (i >= 16 && two_groups) ? s1 : s0;
+        const float b = (i >= 16 && two_groups) ? b1 : b0;
+        if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) v[i] = fmaf((float)code, s, b);
+        else v[i] = cb[code] * s;
+    }
+}
+
+// Store 32 fp32 weights as 4 chunks of 8 16-bit values at chunk positions
+// c0..c0+3 of row r: the 16-bit rounding (hi) and, for two-term formats, the
+// 16-bit rounding of the remainder (lo).
+template <bool F16, bool TWO>
+__device__ __forceinline__ void store_a(const float (&v)[32], uint32_t a_hi, uint32_t a_lo, uint32_t r,
+                                        uint32_t c0) {
 #pragma unroll
     for (int cc = 0; cc < 4; cc++) {
-        uint32_t h[4], l[4];
+        uint32_t hh[4], ll[4];
 #pragma unroll
         for (int e = 0; e < 4; e++) {
             const float x0 = v[cc * 8 + 2 * e], x1 = v[cc * 8 + 2 * e + 1];
-            h[e] = pack2<F16>(x0, x1);
-            if constexpr (a_terms<KIND>() == 2)
-                l[e] = pack2<F16>(x0 - round16<F16>(x0), x1 - round16<F16>(x1));
+            hh[e] = pack2<F16>(x0, x1);
+            if constexpr (TWO) ll[e] = pack2<F16>(x0 - round16<F16>(x0), x1 - round16<F16>(x1));
         }
         const uint32_t off = swz(r, c0 + cc);
-        sts128(a_hi + off, h[0], h[1], h[2], h[3]);
-        if constexpr (a_terms<KIND>() == 2) sts128(a_lo + off, l[0], l[1], l[2], l[3]);
+        sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
+        if constexpr (TWO) sts128(a_lo + off, ll[0], ll[1], ll[2], ll[3]);
     }
 }
 
-template <int KIND>
-__device__ __forceinline__ void load_scales(const GemmParams &P, size_t row_index, uint32_t g,
-                                            float &s, float &b) {
-    g = min(g, P.groups - 1u);
-    const size_t i = row_index * P.groups + g;
-    if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) {
-        s = bf16_bits_to_f32(__ldg((const unsigned short *)P.scales + i));
-        b = bf16_bits_to_f32(__ldg((const unsigned short *)P.aux + i));
-    } else if constexpr (KIND == K_NVFP4) {
-        s = e4m3_to_f32(__ldg((const uint8_t *)P.scales + i));
-        b = 0.f;
+// NVFP4: e2m1 pairs to f16x2 by the hardware conversion, times the E4M3 block
+// scale (exact: at most 6 significant bits), stored as f16 or bf16 (exact).
+template <bool F16>
+__device__ __forceinline__ void nvfp4_store(const uint32_t (&w)[4], float s0, float s1, bool two_groups,
+                                            uint32_t a_hi, uint32_t r, uint32_t c0) {
+#pragma unroll
+    for (int cc = 0; cc < 4; cc++) {  // word cc holds codes 8cc .. 8cc+7
+        uint32_t h[4];
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+            "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+            : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+            : "r"(w[cc]));
+        const float s = (cc >= 2 && two_groups) ? s1 : s0;
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[e]));
+            o[e] = pack2<F16>(f.x * s, f.y * s);
+        }
+        sts128(a_hi + swz(r, c0 + cc), o[0], o[1], o[2], o[3]);
+    }
+}
+
+template <int KIND, bool F16>
+__device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], uint32_t sub, float s0,
+                                             float b0, float s1, float b1, bool two_groups,
+                                             const float *cb, uint32_t a_hi, uint32_t a_lo, uint32_t r,
+                                             uint32_t c0) {
+    if constexpr (KIND == K_NVFP4) {
+        nvfp4_store<F16>(w, s0, s1, two_groups, a_hi, r, c0);
     } else {
-        s = f16_bits_to_f32(__ldg((const unsigned short *)P.scales + i));
+        float v[32];
+        if constexpr (KIND == K_CB3) {
+            switch (sub) {  // first code's position in word 0: 0, 2, 4, 6 or 8
+                case 0: dequant32<KIND, 0>(w, s0, b0, s1, b1, two_groups, cb, v); break;
+                case 2: dequant32<KIND, 2>(w, s0, b0, s1, b1, two_groups, cb, v); break;
+                case 4: dequant32<KIND, 4>(w, s0, b0, s1, b1, two_groups, cb, v); break;
+                case 6: dequant32<KIND, 6>(w, s0, b0, s1, b1, two_groups, cb, v); break;
+                default: dequant32<KIND, 8>(w, s0, b0, s1, b1, two_groups, cb, v); break;
+            }
+        } else {
+            dequant32<KIND, 0>(w, s0, b0, s1, b1, two_groups, cb, v);
+        }
+        store_a<F16, true>(v, a_hi, a_lo, r, c0);
+    }
+}
+
+// Scale (and bias) whose first byte lies `rel` bytes after the start of the
+// staged scale words sw / bias words bw.
+template <int KIND>
+__device__ __forceinline__ void staged_scale(const uint32_t (&sw)[2], const uint32_t (&bw)[2], uint32_t rel,
+                                             float &s, float &b) {
+    const uint32_t wi = rel >> 2, sh = (rel & 3u) * 8u;
+    const uint32_t sv = (wi ? sw[1] : sw[0]) >> sh;
+    if constexpr (KIND == K_NVFP4) {
+        s = e4m3_to_f32(sv & 0xFFu);
         b = 0.f;
+    } else if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) {
+        s = bf16_bits_to_f32(sv & 0xFFFFu);
+        b = bf16_bits_to_f32(((wi ? bw[1] : bw[0]) >> sh) & 0xFFFFu);
+    } else {
+        s = f16_bits_to_f32(sv & 0xFFFFu);
+        b = 0.f;
+    }
+}
+
+// Scale (and bias) of group g read from global memory (rows of scales that are
+// not 4-byte aligned); groups past the row's end read as 0.
+template <int KIND>
+__device__ __forceinline__ void global_scale(const uint8_t *srow, const uint8_t *brow, uint32_t g,
+                                             uint32_t groups, float &s, float &b) {
+    s = 0.f;
+    b = 0.f;
+    if (g >= groups) return;
+    if constexpr (KIND == K_NVFP4) {
+        s = e4m3_to_f32(__ldg(srow + g));
+    } else {
+        const uint32_t sv = (uint32_t)__ldg(srow + 2 * g) | ((uint32_t)__ldg(srow + 2 * g + 1) << 8);
+        if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) {
+            s = bf16_bits_to_f32(sv);
+            b = bf16_bits_to_f32((uint32_t)__ldg(brow + 2 * g) | ((uint32_t)__ldg(brow + 2 * g + 1) << 8));
+        } else {
+            s = f16_bits_to_f32(sv);
+        }
     }
 }
 
 template <int KIND, int XT, int BN>
+struct GemmCfg {
+    static constexpr int AT = a_terms<KIND>();
+    static constexpr int BT = (XT == DT_F32) ? 2 : 1;
+    static constexpr int B_TILE = BN * KT * 2;
+    static constexpr uint32_t STAGE = AT * A_TILE + BT * B_TILE + RawLayout<KIND>::TILE;
+};
+
+template <int KIND, int XT, int BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const GemmParams P) {
-    constexpr int AT = a_terms<KIND>();
-    constexpr int BT = (XT == DT_F32) ? 2 : 1;
+    using C = GemmCfg<KIND, XT, BN>;
+    constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
+    constexpr uint32_t STAGE = C::STAGE;
+    constexpr uint32_t B_OFF = AT * A_TILE, RAW_OFF = AT * A_TILE + BT * B_TILE;
     constexpr bool F16 = (XT == DT_F16);
-    constexpr int B_TILE = BN * KT * 2;
-    constexpr int STAGE = AT * A_TILE + BT * B_TILE;
+    constexpr uint32_t ES = (KIND == K_NVFP4) ? 1u : 2u;  // bytes per scale
+    constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
+    using RL = RawLayout<KIND>;
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bars[2 * 8 + 1];
+    __shared__ uint64_t bars[3 * MAX_STAGES + 1];
     __shared__ uint32_t tmem_s;
     __shared__ int abort_s;
     __shared__ uint32_t pairs_s[BN];
-    __shared__ uint32_t tok_s[BN];
     __shared__ float cb_s[16];
 
     const uint32_t tile = blockIdx.y;
@@ -238,25 +308,25 @@ grouped_gemm_kernel(const GemmParams P) {
     const uint32_t S = P.stages;
 
     const uint32_t base = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *const base_ptr = smem_raw + (base - ptx::smem_u32(smem_raw));
     const uint32_t full0 = ptx::smem_u32(&bars[0]);
-    const uint32_t empty0 = ptx::smem_u32(&bars[8]);
-    const uint32_t accb = ptx::smem_u32(&bars[16]);
+    const uint32_t loaded0 = ptx::smem_u32(&bars[MAX_STAGES]);
+    const uint32_t empty0 = ptx::smem_u32(&bars[2 * MAX_STAGES]);
+    const uint32_t accb = ptx::smem_u32(&bars[3 * MAX_STAGES]);
     volatile int *abort_flag = &abort_s;
 
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
-            ptx::mbar_init(full0 + 8 * s, NPROD);
+            ptx::mbar_init(full0 + 8 * s, NDQ);
+            ptx::mbar_init(loaded0 + 8 * s, NLD);
             ptx::mbar_init(empty0 + 8 * s, 1);
         }
         ptx::mbar_init(accb, 1);
         ptx::fence_mbar_init();
         abort_s = 0;
     }
-    for (uint32_t i = tid; i < BN; i += blockDim.x) {
-        const uint32_t p = i < nt ? __ldg(P.sorted_pairs + off + r0 + i) : 0u;
-        pairs_s[i] = p;
-        tok_s[i] = p / P.n_expert_used;
-    }
+    for (uint32_t i = tid; i < BN; i += blockDim.x)
+        pairs_s[i] = i < nt ? __ldg(P.sorted_pairs + off + r0 + i) : 0u;
     if constexpr (KIND == K_CB2 || KIND == K_CB3 || KIND == K_CB4) {
         if (tid < (1u << kind_bits(KIND)))
             cb_s[tid] = f16_bits_to_f32(__ldg((const unsigned short *)P.aux + tid));
@@ -269,46 +339,35 @@ grouped_gemm_kernel(const GemmParams P) {
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_s;
+    const bool gs16 = (P.lg_gs == 4);
 
-    if (warp < MMA_WARP) {
-        // ------------------------------------------------------------ producers
+    if (warp < LD_WARP0) {
+        // -------------------------------------------------------- dequantisers
         const uint32_t r = tid & (BM - 1), h = tid >> 7;
-        const uint32_t grow = row0 + r;
-        const uint32_t growc = grow < P.n ? grow : P.n - 1;
-        const size_t row_index = (size_t)e * P.n + growc;
-        const uint8_t *rowp = P.packed + row_index * P.row_bytes;
-        const bool gs16 = (P.lg_gs == 4);
+        const size_t row_index = (size_t)e * P.n + tmin<uint32_t>(row0 + r, P.n - 1);
+        const uint8_t *srow = (const uint8_t *)P.scales + row_index * P.groups * ES;
+        const uint8_t *brow = (const uint8_t *)P.aux + row_index * P.groups * 2u;
         bool ok = true;
         for (uint32_t kt = 0; kt < P.ktiles; kt++) {
-            const uint32_t s = kt % S, use = kt / S;
-            if (use > 0 && !ptx::mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1u, abort_flag,
-                                                   P.err, ERR_TIMEOUT, P.timeout_ns)) {
+            const uint32_t s = kt % S;
+            if (!ptx::mbar_wait_bounded(loaded0 + 8 * s, (kt / S) & 1u, abort_flag, P.err, ERR_TIMEOUT,
+                                        P.timeout_ns)) {
                 ok = false;
                 break;
             }
             const uint32_t st = base + s * STAGE;
-            const uint32_t b_hi = st + AT * A_TILE;
-            // gather x rows of the pairs: token i, 16-byte chunk c of this k-tile
-            if constexpr (BT == 1) {
-                for (uint32_t q = tid; q < nt_pad * 8u; q += NPROD) {
-                    const uint32_t i = q >> 3, c = q & 7u;
-                    const uint32_t kk = kt * KT + c * 8u;
-                    const bool in = i < nt && kk < P.k;
-                    const uint16_t *src = (const uint16_t *)P.x + (in ? (size_t)tok_s[i] * P.k + kk : 0);
-                    ptx::cp_async_16(b_hi + swz(i, c), src, in ? 16u : 0u);
-                }
-                ptx::cp_async_commit();
-            } else {
-                const uint32_t b_lo = b_hi + B_TILE;
-                for (uint32_t q = tid; q < nt_pad * 8u; q += NPROD) {
-                    const uint32_t i = q >> 3, c = q & 7u;
-                    const uint32_t kk = kt * KT + c * 8u;
-                    float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-                    if (i < nt && kk < P.k) {
-                        const float4 *src = (const float4 *)((const float *)P.x + (size_t)tok_s[i] * P.k + kk);
-                        v0 = __ldg(src);
-                        v1 = __ldg(src + 1);
-                    }
+            const uint8_t *stp = base_ptr + s * STAGE;
+            if constexpr (BT == 2) {
+                // f32 x: elements 0-3 of a chunk landed in the hi tile's slot, 4-7 in the
+                // lo tile's slot; rewrite both as the bf16 hi and lo halves
+                const uint32_t cc = tid & 7u;
+#pragma unroll
+                for (int j = 0; j < BN / 32; j++) {
+                    const uint32_t i = (tid >> 3) + 32u * j;
+                    if (i >= nt_pad) continue;
+                    const uint32_t o = swz(i, cc);
+                    const float4 v0 = *(const float4 *)(stp + B_OFF + o);
+                    const float4 v1 = *(const float4 *)(stp + B_OFF + B_TILE + o);
                     const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     uint32_t hi[4], lo[4];
 #pragma unroll
@@ -317,28 +376,51 @@ grouped_gemm_kernel(const GemmParams P) {
                         lo[t] = pack2<false>(f[2 * t] - round16<false>(f[2 * t]),
                                              f[2 * t + 1] - round16<false>(f[2 * t + 1]));
                     }
-                    const uint32_t o = swz(i, c);
-                    sts128(b_hi + o, hi[0], hi[1], hi[2], hi[3]);
-                    sts128(b_lo + o, lo[0], lo[1], lo[2], lo[3]);
+                    sts128(st + B_OFF + o, hi[0], hi[1], hi[2], hi[3]);
+                    sts128(st + B_OFF + B_TILE + o, lo[0], lo[1], lo[2], lo[3]);
                 }
             }
-            // dequantise this thread's 32 codes of row r
-            {
-                const uint32_t j0 = kt * KT + h * 32u;
-                uint32_t w[Raw<KIND>::W];
-                uint32_t sub;
-                load_raw<KIND>(rowp, j0, P.row_bytes, w, sub);
-                float s0, b0, s1 = 0.f, b1 = 0.f;
-                load_scales<KIND>(P, row_index, j0 >> P.lg_gs, s0, b0);
-                if (gs16) load_scales<KIND>(P, row_index, (j0 >> 4) + 1u, s1, b1);
-                dequant_store<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r,
-                                         h * 4u);
+            const uint8_t *rr = stp + RAW_OFF + r * RL::STRIDE;
+            uint32_t w[Raw<KIND>::W];
+            uint32_t sub = 0;
+            if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
+                const uint4 q = *(const uint4 *)(rr + 16u * h);
+                w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
+            } else if constexpr (KIND == K_AFF8) {
+                const uint4 q0 = *(const uint4 *)(rr + 32u * h), q1 = *(const uint4 *)(rr + 32u * h + 16u);
+                w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
+                w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
+            } else if constexpr (KIND == K_AFF6) {
+#pragma unroll
+                for (int i = 0; i < 3; i++) {
+                    const uint2 q = *(const uint2 *)(rr + 24u * h + 8u * i);
+                    w[2 * i] = q.x; w[2 * i + 1] = q.y;
+                }
+            } else if constexpr (KIND == K_CB2) {
+                const uint2 q = *(const uint2 *)(rr + 8u * h);
+                w[0] = q.x; w[1] = q.y;
+            } else {  // K_CB3: codes from (kt*KT) % 10 + 32h of the window
+                const uint32_t c0 = (kt * KT) % 10u + 32u * h, wb = c0 / 10u;
+                sub = c0 - 10u * wb;
+#pragma unroll
+                for (int i = 0; i < 4; i++) w[i] = *(const uint32_t *)(rr + 4u * (wb + i));
             }
-            if constexpr (BT == 1) ptx::cp_async_wait_all();
+            const uint32_t j0 = kt * KT, gh = (j0 + 32u * h) >> P.lg_gs;
+            float s0, b0, s1 = 0.f, b1 = 0.f;
+            if (P.scale_words) {
+                const uint4 q = *(const uint4 *)(rr + RL::SC);
+                const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
+                const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
+                staged_scale<KIND>(sw, bw, gh * ES - base_b, s0, b0);
+                if (gs16) staged_scale<KIND>(sw, bw, (gh + 1u) * ES - base_b, s1, b1);
+            } else {
+                global_scale<KIND>(srow, brow, gh, P.groups, s0, b0);
+                if (gs16) global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, b1);
+            }
+            dequant_tile<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(full0 + 8 * s);
         }
-        if (!ok) ptx::cp_async_wait_all();
         // ------------------------------------------------------------- epilogue
         if (ok && ptx::mbar_wait_bounded(accb, 0, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns)) {
             ptx::tc_fence_after();
@@ -362,6 +444,98 @@ grouped_gemm_kernel(const GemmParams P) {
             }
         }
         ptx::tc_fence_before();
+    } else if (warp < MMA_WARP) {
+        // ------------------------------------------------------------- loaders
+        const uint32_t lt = tid - NDQ;
+        // x: thread lt copies 16-byte chunk lt % 8 of pair rows lt / 8 + 16 j
+        constexpr int NXL = BN * 8 / NLD;
+        constexpr uint32_t XS = (BT == 2) ? 4u : 2u;  // bytes per x element
+        const uint32_t xc = lt & 7u, xi0 = lt >> 3;
+        const uint8_t *xrow[NXL];
+#pragma unroll
+        for (int j = 0; j < NXL; j++) {
+            const uint32_t i = xi0 + 16u * j;
+            xrow[j] = i < nt ? (const uint8_t *)P.x + (size_t)(pairs_s[i] / P.n_expert_used) * P.k * XS
+                             : nullptr;
+        }
+        const uint32_t xdst0 = B_OFF + swz(xi0, xc);  // + 2048 j: 16 rows further down
+        const uint8_t *ebase = P.packed + (size_t)e * P.n * P.row_bytes;
+        const uint32_t nlast = P.n - 1;
+        // scale words: thread lt stages those of weight row lt
+        const size_t srow_index = (size_t)e * P.n + tmin<uint32_t>(row0 + lt, nlast);
+        const uint8_t *srow = (const uint8_t *)P.scales + srow_index * P.groups * ES;
+        const uint8_t *brow = (const uint8_t *)P.aux + srow_index * P.groups * 2u;
+        const uint32_t srow_bytes = P.groups * ES;
+        const uint32_t nsw = (gs16 && ES == 2u) ? 2u : 1u;
+
+        for (uint32_t kt = 0; kt < P.ktiles; kt++) {
+            const uint32_t s = kt % S;
+            if (kt >= S && !ptx::mbar_wait_bounded(empty0 + 8 * s, ((kt / S) - 1u) & 1u, abort_flag, P.err,
+                                                   ERR_TIMEOUT, P.timeout_ns))
+                break;
+            const uint32_t st = base + s * STAGE;
+            // x rows of the pairs, straight into the B operand tile (zero past k and nt)
+            const uint32_t kk = kt * KT + xc * 8u;
+#pragma unroll
+            for (int j = 0; j < NXL; j++) {
+                if (xi0 + 16u * j < nt_pad) {
+                    const bool in = xrow[j] != nullptr && kk < P.k;
+                    const uint8_t *src = in ? xrow[j] + (size_t)kk * XS : (const uint8_t *)P.x;
+                    const uint32_t dst = st + xdst0 + 2048u * j;
+                    ptx::cp_async_16(dst, src, in ? 16u : 0u);
+                    if constexpr (BT == 2) ptx::cp_async_16(dst + B_TILE, in ? src + 16 : src, in ? 16u : 0u);
+                }
+            }
+            // packed codes of the 128 rows (rows past n repeat row n-1; bytes past a row read as 0)
+            const uint32_t raw = st + RAW_OFF;
+            if constexpr (KIND == K_CB3) {
+                const uint32_t w0 = (kt * KT) / 10u;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const uint32_t q = lt + NLD * i, row = q >> 3, c = q & 7u;
+                    const uint8_t *rp = ebase + (size_t)tmin<uint32_t>(row0 + row, nlast) * P.row_bytes;
+                    const uint32_t o = (w0 + c) * 4u;
+                    const bool in = o + 4u <= P.row_bytes;
+                    ptx::cp_async_4(raw + row * RL::STRIDE + 4u * c, rp + (in ? o : 0u), in ? 4u : 0u);
+                }
+            } else {
+                constexpr uint32_t RB = RL::RB;
+                if (P.raw16) {
+                    constexpr uint32_t NC = RB / 16u;
+#pragma unroll
+                    for (uint32_t i = 0; i < NC; i++) {
+                        const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
+                        const uint8_t *rp = ebase + (size_t)tmin<uint32_t>(row0 + row, nlast) * P.row_bytes;
+                        const uint32_t o = kt * RB + 16u * c;
+                        const bool in = o < P.row_bytes;
+                        ptx::cp_async_16(raw + row * RL::STRIDE + 16u * c, rp + (in ? o : 0u), in ? 16u : 0u);
+                    }
+                } else {
+                    constexpr uint32_t NC = RB / 8u;
+#pragma unroll
+                    for (uint32_t i = 0; i < NC; i++) {
+                        const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
+                        const uint8_t *rp = ebase + (size_t)tmin<uint32_t>(row0 + row, nlast) * P.row_bytes;
+                        const uint32_t o = kt * RB + 8u * c;
+                        const bool in = o < P.row_bytes;
+                        ptx::cp_async_8(raw + row * RL::STRIDE + 8u * c, rp + (in ? o : 0u), in ? 8u : 0u);
+                    }
+                }
+            }
+            if (P.scale_words) {
+                const uint32_t base_b = ((kt * KT >> P.lg_gs) * ES) & ~3u;
+                for (uint32_t i = 0; i < nsw; i++) {
+                    const uint32_t o = base_b + 4u * i;
+                    const bool in = o + 4u <= srow_bytes;
+                    ptx::cp_async_4(raw + lt * RL::STRIDE + RL::SC + 4u * i, srow + (in ? o : 0u), in ? 4u : 0u);
+                    if constexpr (AFF)
+                        ptx::cp_async_4(raw + lt * RL::STRIDE + RL::BI + 4u * i, brow + (in ? o : 0u),
+                                        in ? 4u : 0u);
+                }
+            }
+            ptx::cp_async_mbar_arrive(loaded0 + 8 * s);
+        }
+        ptx::cp_async_wait_all();
     } else if (lane == 0) {
         // --------------------------------------------------------------- MMA issue
         const uint32_t idesc = ptx::idesc_f16(F16 ? 0u : 1u, nt_pad);
@@ -377,7 +551,7 @@ grouped_gemm_kernel(const GemmParams P) {
             ptx::tc_fence_after();
             const uint32_t st = base + s * STAGE;
             const uint32_t a_hi = st, a_lo = st + A_TILE;
-            const uint32_t b_hi = st + AT * A_TILE, b_lo = b_hi + B_TILE;
+            const uint32_t b_hi = st + B_OFF, b_lo = b_hi + B_TILE;
 #pragma unroll
             for (int ks = 0; ks < KT / 16; ks++) {
                 const uint32_t ko = ks * 32u;
@@ -398,51 +572,92 @@ grouped_gemm_kernel(const GemmParams P) {
     }
     __syncthreads();
     if (warp == MMA_WARP) {
+        __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, BN);
     }
 }
 
-template <int KIND, int XT, int BN>
-cudaError_t launch_t(const GemmParams &P0, uint32_t n_mtiles, uint32_t max_tiles, cudaStream_t st) {
-    constexpr int AT = a_terms<KIND>();
-    constexpr int BT = (XT == DT_F32) ? 2 : 1;
-    constexpr int STAGE = AT * A_TILE + BT * BN * KT * 2;
-    const int budget = BN >= 256 ? 200 * 1024 : 96 * 1024;
-    int S = budget / STAGE;
-    S = S < 2 ? 2 : (S > 6 ? 6 : S);
-    GemmParams P = P0;
-    P.stages = (uint32_t)S;
-    const size_t smem = (size_t)S * STAGE + 1024;
-    auto kern = grouped_gemm_kernel<KIND, XT, BN>;
-    static int smem_set[64];
-    cudaError_t e = ensure_dyn_smem(kern, smem, smem_set);
-    if (e != cudaSuccess) return e;
-    dim3 grid(n_mtiles, max_tiles);
-    kern<<<grid, GEMM_THREADS, smem, st>>>(P);
-    return cudaGetLastError();
-}
+// Dynamic shared memory per CTA (stages + 1 KB for aligning them), leaving room
+// for the kernel's static shared memory within the 227 KB a CTA may use.
+constexpr size_t GEMM_SMEM_BUDGET = 229000;
 
-template <int KIND, int BN>
-cudaError_t launch_x(const GemmParams &P, int x_dtype, uint32_t nm, uint32_t mt, cudaStream_t st) {
-    switch (x_dtype) {
-        case DT_F32: return launch_t<KIND, DT_F32, BN>(P, nm, mt, st);
-        case DT_BF16: return launch_t<KIND, DT_BF16, BN>(P, nm, mt, st);
-        default: return launch_t<KIND, DT_F16, BN>(P, nm, mt, st);
+struct GemmPlan {
+    uint32_t bn;
+    int stages;
+    size_t smem;
+};
+
+uint32_t raw_tile(int kind) {
+    switch (kind) {
+        case K_AFF4: return RawLayout<K_AFF4>::TILE;
+        case K_AFF6: return RawLayout<K_AFF6>::TILE;
+        case K_AFF8: return RawLayout<K_AFF8>::TILE;
+        case K_CB2: return RawLayout<K_CB2>::TILE;
+        case K_CB3: return RawLayout<K_CB3>::TILE;
+        case K_CB4: return RawLayout<K_CB4>::TILE;
+        default: return RawLayout<K_NVFP4>::TILE;
     }
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmParams &P, int kind, int x_dtype, uint32_t nm, uint32_t mt,
-                      cudaStream_t st) {
+// Tile width and pipeline depth: 256 pairs per tile when experts hold ~100 or
+// more pairs on average (128 with f32 x, whose operand tiles are twice as
+// large), 64 otherwise; as many stages (2..6) as fit.
+bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
+    const uint64_t R = (uint64_t)a.m * a.n_expert_used;
+    const bool big = R >= 96ull * a.num_experts;
+    const bool f32x = a.x_dtype == DT_F32;
+    const uint32_t bn = big ? (f32x ? 128u : 256u) : 64u;
+    const uint32_t at = a.kind == K_NVFP4 ? 1u : 2u, bt = f32x ? 2u : 1u;
+    const size_t stage = (size_t)at * A_TILE + (size_t)bt * bn * KT * 2 + raw_tile(a.kind);
+    if (2 * stage + 1024 > GEMM_SMEM_BUDGET) return false;
+    int S = (int)((GEMM_SMEM_BUDGET - 1024) / stage);
+    S = S > MAX_STAGES ? MAX_STAGES : S;
+    pl->bn = bn;
+    pl->stages = S;
+    pl->smem = (size_t)S * stage + 1024;
+    return true;
+}
+
+template <int KIND, int XT, int BN>
+cudaError_t launch_t(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
+                     cudaStream_t st) {
+    GemmParams P = P0;
+    P.stages = (uint32_t)pl.stages;
+    auto kern = grouped_gemm_kernel<KIND, XT, BN>;
+    static int smem_set[64];
+    cudaError_t e = ensure_dyn_smem(kern, pl.smem, smem_set);
+    if (e != cudaSuccess) return e;
+    dim3 grid(n_mtiles, max_tiles);
+    kern<<<grid, GEMM_THREADS, pl.smem, st>>>(P);
+    return cudaGetLastError();
+}
+
+template <int KIND>
+cudaError_t launch_k(const GemmParams &P, const GemmPlan &pl, int x_dtype, uint32_t nm, uint32_t mt,
+                     cudaStream_t st) {
+    if (x_dtype == DT_F32) {
+        if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, pl, nm, mt, st);
+        return launch_t<KIND, DT_F32, 64>(P, pl, nm, mt, st);
+    }
+    if (x_dtype == DT_BF16) {
+        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, pl, nm, mt, st);
+        return launch_t<KIND, DT_BF16, 64>(P, pl, nm, mt, st);
+    }
+    if (pl.bn == 256) return launch_t<KIND, DT_F16, 256>(P, pl, nm, mt, st);
+    return launch_t<KIND, DT_F16, 64>(P, pl, nm, mt, st);
+}
+
+cudaError_t launch_kind(const GemmParams &P, const GemmPlan &pl, int kind, int x_dtype, uint32_t nm,
+                        uint32_t mt, cudaStream_t st) {
     switch (kind) {
-        case K_AFF4: return launch_x<K_AFF4, BN>(P, x_dtype, nm, mt, st);
-        case K_AFF6: return launch_x<K_AFF6, BN>(P, x_dtype, nm, mt, st);
-        case K_AFF8: return launch_x<K_AFF8, BN>(P, x_dtype, nm, mt, st);
-        case K_CB2: return launch_x<K_CB2, BN>(P, x_dtype, nm, mt, st);
-        case K_CB3: return launch_x<K_CB3, BN>(P, x_dtype, nm, mt, st);
-        case K_CB4: return launch_x<K_CB4, BN>(P, x_dtype, nm, mt, st);
-        case K_NVFP4: return launch_x<K_NVFP4, BN>(P, x_dtype, nm, mt, st);
+        case K_AFF4: return launch_k<K_AFF4>(P, pl, x_dtype, nm, mt, st);
+        case K_AFF6: return launch_k<K_AFF6>(P, pl, x_dtype, nm, mt, st);
+        case K_AFF8: return launch_k<K_AFF8>(P, pl, x_dtype, nm, mt, st);
+        case K_CB2: return launch_k<K_CB2>(P, pl, x_dtype, nm, mt, st);
+        case K_CB3: return launch_k<K_CB3>(P, pl, x_dtype, nm, mt, st);
+        case K_CB4: return launch_k<K_CB4>(P, pl, x_dtype, nm, mt, st);
+        case K_NVFP4: return launch_k<K_NVFP4>(P, pl, x_dtype, nm, mt, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -453,21 +668,24 @@ bool gemm_supported(const QmmArgs &a) {
     const uint32_t gs = a.group_size;
     if (gs < 16 || (gs & (gs - 1)) != 0) return false;
     if (a.k % 8 != 0 || a.k % gs != 0) return false;
-    // packed codes are read with 8-byte loads (4-byte word loads for 3-bit codebook rows)
+    // packed codes are staged with 8- or 16-byte copies (4-byte words for 3-bit codebook rows)
     if (a.row_bytes % (a.kind == K_CB3 ? 4u : 8u) != 0) return false;
     if ((uintptr_t)a.packed % 16 != 0 || (uintptr_t)a.x % 16 != 0) return false;
     if (a.num_experts > ROUTE_MAX_E) return false;
-    return true;
+    GemmPlan pl;
+    return gemm_plan(a, &pl);
 }
 
 uint32_t gemm_tile_rows(const QmmArgs &a) {
-    const uint64_t R = (uint64_t)a.m * a.n_expert_used;
-    return (R >= 96ull * a.num_experts) ? 256u : 64u;
+    GemmPlan pl;
+    return gemm_plan(a, &pl) ? pl.bn : 64u;
 }
 
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
                         uint32_t *err, cudaStream_t st) {
+    GemmPlan pl;
+    if (!gemm_plan(a, &pl)) return cudaErrorNotSupported;
     GemmParams P{};
     P.x = a.x; P.offsets = offsets; P.sorted_pairs = sorted_pairs; P.tiles = tiles;
     P.tile_count = tile_count; P.packed = a.packed; P.scales = a.scales; P.aux = a.aux;
@@ -478,11 +696,14 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.lg_gs = lg;
     P.groups = a.groups; P.n_expert_used = a.n_expert_used; P.row_bytes = a.row_bytes;
     P.ktiles = (a.k + KT - 1) / KT;
+    const uint32_t es = a.kind == K_NVFP4 ? 1u : 2u;
+    P.scale_words = (a.groups * es) % 4u == 0 && (uintptr_t)a.scales % 4u == 0 &&
+                    (a.fmt != FMT_AFFINE || (uintptr_t)a.aux % 4u == 0);
+    P.raw16 = a.kind != K_CB3 && a.row_bytes % 16u == 0;
     P.out_dtype = a.out_dtype;
     P.timeout_ns = WAIT_NS;
     const uint32_t nm = (a.n + BM - 1) / BM;
-    if (gemm_tile_rows(a) == 256u) return launch_bn<256>(P, a.kind, a.x_dtype, nm, max_tiles, st);
-    return launch_bn<64>(P, a.kind, a.x_dtype, nm, max_tiles, st);
+    return launch_kind(P, pl, a.kind, a.x_dtype, nm, max_tiles, st);
 }
 
 }  // namespace moe

@@ -66,22 +66,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended for up to `hint_ns` while
+// the phase is incomplete (it resumes as soon as the phase completes), so that
+// waiting warps do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete. Gives up after
 // `timeout_ns` of wall time (or ~2^31 polls), or as soon as another thread of
 // the CTA has raised *abort_flag (not checked when abort_flag is null); on
 // timeout raises *abort_flag and sets `err_bit` in *err. Returns true if the
-// phase completed.
+// phase completed. Each poll may suspend the thread for up to 20 us.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int *abort_flag, uint32_t *err,
                                                   uint32_t err_bit, uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1; it < 0x80000000u; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u) {
-            if (abort_flag && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > timeout_ns) break;
-        }
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (abort_flag && *abort_flag) return false;
+        if (globaltimer_ns() - t0 > timeout_ns) break;
     }
     if (abort_flag) *abort_flag = 1;
     atomicOr(err, err_bit);
@@ -103,6 +116,22 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                  "r"(src_bytes)
                  : "memory");
+}
+
+// 4- and 8-byte copies (through L1); same zero-fill rule.
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// Arrive on the mbarrier once all cp.async copies this thread has issued so far
+// have landed. The arrival is one of the barrier's expected arrivals (.noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit() {
