@@ -796,6 +796,357 @@ gemv_aff4_tma(const GemvParams P) {
     }
 }
 
+// -------------------- 4-bit affine, one token: x planes held in registers
+//
+// With a single token every (token, slot) pair multiplies the same x row, so a
+// lane can keep the x planes of its own slice of k in registers for every
+// weight row it meets, and shared memory only carries the weight rows (each
+// byte read once). Rows of all pairs are numbered globally (pair p's column c
+// is row p*n + c) and split into equal contiguous ranges, two CTAs per SM, so
+// every SM streams the same number of bytes whatever the experts. A group of
+// LPR lanes owns one row at a time; lane l of the group holds 32-code units
+// l, l+LPR, ..., UPL of them. Each warp's rows arrive by bulk copies (one per
+// pair the range touches) on the warp's own mbarrier; scales, biases and x
+// by bulk copies issued before the planes are built.
+constexpr int ROWS_THREADS = 256;
+constexpr int ROWS_WARPS = ROWS_THREADS / 32;
+constexpr uint32_t ROWS_MAX_PAIRS = 64;
+
+struct RowsLayout {
+    uint32_t w, xraw, planes, uscale, usum, sc, bi, total;
+};
+
+__host__ __device__ inline RowsLayout rows_layout(uint32_t rb, uint32_t row_bytes, uint32_t x_bytes,
+                                                  uint32_t nu, uint32_t G) {
+    RowsLayout L;
+    L.w = 0;
+    L.xraw = al16u(rb * row_bytes);
+    L.planes = al16u(L.xraw + x_bytes);
+    L.uscale = L.planes + nu * DP_PW * 4u;
+    L.usum = L.uscale + nu * 4u;
+    L.sc = al16u(L.usum + nu * 4u);
+    L.bi = al16u(L.sc + rb * G * 2u);
+    L.total = al16u(L.bi + rb * G * 2u);
+    return L;
+}
+
+// Exact integer dot product of one 32-code unit with x planes held in registers
+// (same arithmetic as dp4a_unit).
+__device__ __forceinline__ float dp4a_unit_reg(const uint4 w, const uint4 (&v)[6], float usc, float usm,
+                                               float s, float b, float acc) {
+    const uint32_t lo0 = w.x & 0x0F0F0F0Fu, hi0 = (w.x >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo1 = w.y & 0x0F0F0F0Fu, hi1 = (w.y >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo2 = w.z & 0x0F0F0F0Fu, hi2 = (w.z >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo3 = w.w & 0x0F0F0F0Fu, hi3 = (w.w >> 4) & 0x0F0F0F0Fu;
+    uint32_t a0 = dp4a_uu(lo0, v[0].x, 0u);
+    a0 = dp4a_uu(hi0, v[0].y, a0);
+    uint32_t a1 = dp4a_uu(lo0, v[0].z, 0u);
+    a1 = dp4a_uu(hi0, v[0].w, a1);
+    int32_t a2 = dp4a_us(lo0, v[1].x, 0);
+    a2 = dp4a_us(hi0, v[1].y, a2);
+    a0 = dp4a_uu(lo1, v[1].z, a0);
+    a0 = dp4a_uu(hi1, v[1].w, a0);
+    a1 = dp4a_uu(lo1, v[2].x, a1);
+    a1 = dp4a_uu(hi1, v[2].y, a1);
+    a2 = dp4a_us(lo1, v[2].z, a2);
+    a2 = dp4a_us(hi1, v[2].w, a2);
+    a0 = dp4a_uu(lo2, v[3].x, a0);
+    a0 = dp4a_uu(hi2, v[3].y, a0);
+    a1 = dp4a_uu(lo2, v[3].z, a1);
+    a1 = dp4a_uu(hi2, v[3].w, a1);
+    a2 = dp4a_us(lo2, v[4].x, a2);
+    a2 = dp4a_us(hi2, v[4].y, a2);
+    a0 = dp4a_uu(lo3, v[4].z, a0);
+    a0 = dp4a_uu(hi3, v[4].w, a0);
+    a1 = dp4a_uu(lo3, v[5].x, a1);
+    a1 = dp4a_uu(hi3, v[5].y, a1);
+    a2 = dp4a_us(lo3, v[5].z, a2);
+    a2 = dp4a_us(hi3, v[5].w, a2);
+    // a0 + 256 a1 < 2^26 (each plane sum is below 2^17): exact in int32
+    const float d = fmaf((float)a2, 65536.f, (float)(int32_t)(a0 + (a1 << 8)));
+    return fmaf(s, d * usc, fmaf(b, usm, acc));
+}
+
+template <int LPR, int UPL>
+__global__ void __launch_bounds__(ROWS_THREADS, 2)
+gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
+    constexpr uint32_t RPI = 32 / LPR;  // rows a warp works on at once
+    constexpr uint64_t WAIT = 1000000000ull;
+    extern __shared__ __align__(128) uint8_t dsm8[];
+    __shared__ uint32_t ex_s[ROWS_MAX_PAIRS];
+    __shared__ __align__(8) uint64_t bar_w[ROWS_WARPS];
+    __shared__ __align__(8) uint64_t bar_x, bar_s;
+    __shared__ int abort_s;
+
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const uint32_t n = P.n, nu = P.n_units, G = P.groups, rbytes = P.row_bytes;
+    const uint32_t total_rows = P.R * n;
+    const uint32_t g0 = blockIdx.x * rows_per_cta;
+    const uint32_t nrows = tmin<uint32_t>(rows_per_cta, total_rows - g0);
+    const uint32_t p_first = g0 / n, p_last = (g0 + nrows - 1u) / n;
+    const uint32_t xsz = P.x_dtype == DT_F32 ? 4u : 2u;
+    const RowsLayout L = rows_layout(rows_per_cta, rbytes, P.k * xsz, nu, G);
+    const uint32_t sbase = ptx::smem_u32(dsm8);
+    volatile int *abort_flag = &abort_s;
+
+    // experts of the pairs this CTA touches (loads in flight across the barrier)
+    if (tid <= p_last - p_first) ex_s[tid] = __ldg(P.ids + p_first + tid);
+    if (tid == 0) {
+        for (int i = 0; i < ROWS_WARPS; i++) ptx::mbar_init(ptx::smem_u32(&bar_w[i]), 1);
+        ptx::mbar_init(ptx::smem_u32(&bar_x), 1);
+        ptx::mbar_init(ptx::smem_u32(&bar_s), 1);
+        ptx::fence_mbar_init();
+        abort_s = 0;
+    }
+    __syncthreads();
+    const uint32_t bx = ptx::smem_u32(&bar_x), bs = ptx::smem_u32(&bar_s);
+    const uint32_t bw = ptx::smem_u32(&bar_w[warp]);
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(bx, P.k * xsz);
+        ptx::bulk_g2s(sbase + L.xraw, P.x, P.k * xsz, bx);
+    }
+    // scales and biases of the CTA's rows: one bulk copy of each per pair when aligned
+    const bool s_bulk = P.s_bulk != 0;
+    if (s_bulk) {
+        if (tid == 0) {
+            uint32_t bytes = 0;
+            for (uint32_t p = p_first; p <= p_last; p++) {
+                const uint32_t lo = p == p_first ? g0 - p * n : 0u;
+                const uint32_t hi = p == p_last ? g0 + nrows - p * n : n;
+                if (ex_s[p - p_first] < P.num_experts) bytes += 2u * (hi - lo) * G * 2u;
+            }
+            ptx::mbar_arrive_expect_tx(bs, bytes);
+            for (uint32_t p = p_first; p <= p_last; p++) {
+                const uint32_t lo = p == p_first ? g0 - p * n : 0u;
+                const uint32_t hi = p == p_last ? g0 + nrows - p * n : n;
+                const uint32_t e = ex_s[p - p_first];
+                if (e >= P.num_experts) continue;
+                const uint32_t dst = (p * n + lo - g0) * G * 2u;
+                const size_t src = ((size_t)e * n + lo) * G;
+                ptx::bulk_g2s(sbase + L.sc + dst, (const unsigned short *)P.scales + src, (hi - lo) * G * 2u, bs);
+                ptx::bulk_g2s(sbase + L.bi + dst, (const unsigned short *)P.aux + src, (hi - lo) * G * 2u, bs);
+            }
+        }
+    } else {
+        unsigned short *sc = (unsigned short *)(dsm8 + L.sc), *bi = (unsigned short *)(dsm8 + L.bi);
+        for (uint32_t idx = tid; idx < nrows * G; idx += blockDim.x) {
+            const uint32_t r = idx / G, gi = idx - r * G;
+            const uint32_t g = g0 + r, p = g / n, c = g - p * n;
+            const uint32_t e = ex_s[p - p_first];
+            const size_t src = ((size_t)(e < P.num_experts ? e : 0u) * n + c) * G + gi;
+            sc[idx] = __ldg((const unsigned short *)P.scales + src);
+            bi[idx] = __ldg((const unsigned short *)P.aux + src);
+        }
+    }
+
+    // this warp's rows [a, b) of the CTA's range, one bulk copy per pair they touch
+    const uint32_t rpw = (nrows + ROWS_WARPS - 1) / ROWS_WARPS;
+    const uint32_t a = tmin<uint32_t>(warp * rpw, nrows), b = tmin<uint32_t>(a + rpw, nrows);
+    if (lane == 0) {
+        uint32_t bytes = 0;
+        for (uint32_t r = a; r < b;) {
+            const uint32_t g = g0 + r, p = g / n, c0 = g - p * n;
+            const uint32_t cnt = tmin<uint32_t>(b - r, n - c0);
+            const uint32_t e = ex_s[p - p_first];
+            if (e < P.num_experts) bytes += cnt * rbytes;
+            r += cnt;
+        }
+        ptx::mbar_arrive_expect_tx(bw, bytes);
+        for (uint32_t r = a; r < b;) {
+            const uint32_t g = g0 + r, p = g / n, c0 = g - p * n;
+            const uint32_t cnt = tmin<uint32_t>(b - r, n - c0);
+            const uint32_t e = ex_s[p - p_first];
+            if (e < P.num_experts)
+                ptx::bulk_g2s(sbase + L.w + r * rbytes, P.packed + ((size_t)e * n + c0) * rbytes,
+                              cnt * rbytes, bw);
+            else if (c0 == 0)
+                atomicOr(P.err, ERR_BAD_ID);
+            r += cnt;
+        }
+    }
+    // x planes, once per CTA: one thread per 8-code word, 4 consecutive lanes per unit
+    uint32_t *planes = (uint32_t *)(dsm8 + L.planes);
+    float *uscale = (float *)(dsm8 + L.uscale);
+    float *usum = (float *)(dsm8 + L.usum);
+    const bool x_ok = ptx::mbar_wait_bounded(bx, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
+    if (__all_sync(0xFFFFFFFFu, x_ok)) {
+        const uint32_t nwords = nu * 4u;
+        for (uint32_t base = warp * 32u; base < nwords; base += ROWS_THREADS) {
+            const uint32_t idx = base + lane;
+            const bool valid = idx < nwords;
+            const uint32_t u = valid ? idx >> 2 : 0u, wd = idx & 3u;
+            const uint32_t j = u * 32u + wd * 8u;
+            float v[8];
+            if (valid && j < P.k) {
+                smem_x8(dsm8 + L.xraw, P.x_dtype, j, v);
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    if (j + i >= P.k) v[i] = 0.f;  // codes past k meet x = 0
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; i++) v[i] = 0.f;
+            }
+            plane_word(v, planes + u * DP_PW, wd, uscale + u, usum + u, valid);
+        }
+    }
+    __syncthreads();
+
+    // this lane's units and their planes, in registers for all its rows
+    const uint32_t gi = lane / LPR, l = lane % LPR;
+    const uint32_t upg = P.gs / 32u;
+    uint4 pv[UPL][6];
+    float usc[UPL], usm[UPL];
+    uint32_t grp[UPL];
+#pragma unroll
+    for (int i = 0; i < UPL; i++) {
+        const uint32_t u = tmin<uint32_t>(l + (uint32_t)i * LPR, nu - 1u);
+        const uint4 *pl = (const uint4 *)(planes + u * DP_PW);
+#pragma unroll
+        for (int t = 0; t < 6; t++) pv[i][t] = pl[t];
+        usc[i] = uscale[u];
+        usm[i] = usum[u];
+        grp[i] = tmin<uint32_t>(u / upg, G - 1u);
+    }
+    bool s_ok = true;
+    if (s_bulk) s_ok = ptx::mbar_wait_bounded(bs, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
+    const bool w_ok = ptx::mbar_wait_bounded(bw, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
+    if (!__all_sync(0xFFFFFFFFu, x_ok && s_ok && w_ok && !*abort_flag)) {
+        // a wait gave up: let this warp's copies land before shared memory is released
+        ptx::mbar_wait_bounded(bw, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
+        if (s_bulk) ptx::mbar_wait_bounded(bs, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
+        return;
+    }
+    const unsigned short *sc = (const unsigned short *)(dsm8 + L.sc);
+    const unsigned short *bi = (const unsigned short *)(dsm8 + L.bi);
+
+    // rows a + gi, a + gi + RPI, ...: (pair, column) carried along
+    uint32_t g = g0 + a + gi;
+    uint32_t p = g / n, c = g - p * n;
+    for (uint32_t r = a + gi; r < b + gi; r += RPI) {
+        const bool valid = r < b;
+        const uint32_t e = valid ? ex_s[p - p_first] : 0u;
+        const bool live = valid && e < P.num_experts;
+        float acc = 0.f;
+        if (live) {
+            const uint8_t *wrow = dsm8 + L.w + r * rbytes;
+            const unsigned short *srow = sc + r * G, *brow = bi + r * G;
+#pragma unroll
+            for (int i = 0; i < UPL; i++) {
+                const uint32_t u = l + (uint32_t)i * LPR;
+                if (u < nu) {
+                    const uint4 w = *(const uint4 *)(wrow + 16u * u);
+                    acc = dp4a_unit_reg(w, pv[i], usc[i], usm[i], bf16_bits_to_f32(srow[grp[i]]),
+                                        bf16_bits_to_f32(brow[grp[i]]), acc);
+                }
+            }
+        }
+#pragma unroll
+        for (int d = LPR / 2; d > 0; d >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, d);
+        if (valid && l == 0) store_out(P.out, P.out_dtype, (size_t)p * n + c, acc);
+        c += RPI;
+        if (c >= n) {
+            c -= n;
+            p++;
+        }
+    }
+}
+
+// Lanes per row and units per lane for nu 32-code units: the pair with the
+// fewest idle lanes, at most 3 units per lane (0 when nu is too large: the
+// planes and two rows of units of 4 units per lane do not fit in registers).
+void rows_shape(uint32_t nu, int *lpr, int *upl) {
+    *lpr = 0;
+    *upl = 0;
+    double best = 0.0;
+    for (int L = 32; L >= 4; L >>= 1) {
+        const uint32_t U = (nu + L - 1) / L;
+        if (U > 3 || U == 0) continue;
+        const double eff = (double)nu / (double)(L * U);
+        if (eff > best + 1e-9) {
+            best = eff;
+            *lpr = L;
+            *upl = (int)U;
+        }
+    }
+}
+
+template <int LPR, int UPL>
+cudaError_t launch_rows_t(const GemvParams &P, uint32_t rb, uint32_t ctas, size_t smem, cudaStream_t st) {
+    auto kern = gemv_aff4_rows<LPR, UPL>;
+    if (smem > 48 * 1024) {
+        static int smem_set[64];
+        cudaError_t e = ensure_dyn_smem(kern, smem, smem_set);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<ctas, ROWS_THREADS, smem, st>>>(P, rb);
+    return cudaGetLastError();
+}
+
+template <int LPR>
+cudaError_t launch_rows_l(const GemvParams &P, int upl, uint32_t rb, uint32_t ctas, size_t smem,
+                          cudaStream_t st) {
+    switch (upl) {
+        case 1: return launch_rows_t<LPR, 1>(P, rb, ctas, smem, st);
+        case 2: return launch_rows_t<LPR, 2>(P, rb, ctas, smem, st);
+        default: return launch_rows_t<LPR, 3>(P, rb, ctas, smem, st);
+    }
+}
+
+int sm_count() {
+    static int count[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (count[dev] == 0) {
+        int c = 0;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+        count[dev] = c;
+    }
+    return count[dev];
+}
+
+// Rows per CTA: an even split of all rows over two CTAs per SM, rounded up to
+// 8 rows so that ranges of scale rows start on 16-byte boundaries.
+uint32_t rows_per_cta(uint32_t total_rows) {
+    const uint32_t ctas = 2u * (uint32_t)sm_count();
+    uint32_t rb = (total_rows + ctas - 1) / ctas;
+    return (rb + 7u) & ~7u;
+}
+
+// One token, 4-bit affine rows of whole 16-byte units, groups of whole units,
+// at most 96 units (k <= 3072) per row, and the CTA's shared memory within budget.
+bool rows_ok(const QmmArgs &a) {
+    if (a.m != 1 || a.n_expert_used > ROWS_MAX_PAIRS || !dp4a_ok(a)) return false;
+    const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
+    if ((a.k * xsz) % 16u != 0 || (uintptr_t)a.x % 16u != 0) return false;
+    int lpr, upl;
+    rows_shape(a.row_bytes / 16u, &lpr, &upl);
+    if (lpr == 0) return false;
+    const uint64_t total = (uint64_t)a.n_expert_used * a.n;
+    if (total >= (1ull << 31)) return false;
+    const uint32_t rb = rows_per_cta((uint32_t)total);
+    const RowsLayout L = rows_layout(rb, a.row_bytes, a.k * xsz, a.row_bytes / 16u, a.groups);
+    return L.total <= 110u * 1024u;
+}
+
+cudaError_t launch_rows(GemvParams P, const QmmArgs &a, cudaStream_t st) {
+    int lpr, upl;
+    rows_shape(P.n_units, &lpr, &upl);
+    const uint32_t total = P.R * P.n;
+    const uint32_t rb = rows_per_cta(total);
+    const uint32_t ctas = (total + rb - 1) / rb;
+    const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
+    const RowsLayout L = rows_layout(rb, P.row_bytes, a.k * xsz, P.n_units, P.groups);
+    // with n a multiple of 8, every range a CTA copies starts and ends on a multiple of
+    // 8 rows, and 8 rows of bf16 scales are a whole number of 16-byte units
+    P.s_bulk = (a.n % 8u) == 0 && (uintptr_t)a.scales % 16u == 0 && (uintptr_t)a.aux % 16u == 0;
+    switch (lpr) {
+        case 4: return launch_rows_l<4>(P, upl, rb, ctas, L.total, st);
+        case 8: return launch_rows_l<8>(P, upl, rb, ctas, L.total, st);
+        case 16: return launch_rows_l<16>(P, upl, rb, ctas, L.total, st);
+        default: return launch_rows_l<32>(P, upl, rb, ctas, L.total, st);
+    }
+}
+
 int tma_lpr(uint32_t nu) {
     // lanes per row: about 3 to 6 16-byte units per lane
     if (nu <= 24) return 4;
@@ -936,6 +1287,7 @@ cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st) 
     const uint32_t npb = tmin<uint32_t>(a.m, 8u);
     const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
     const bool spec = (uint64_t)a.m * a.k * xsz <= 32768u;
+    if (rows_ok(a)) return launch_rows(P, a, st);
     if (a.m == 1 && tma_ok(a, 1, spec)) {
         P.x_spec = spec;
         return launch_tma<MODE_PAIR>(P, 1, P.R, st);

@@ -26,6 +26,7 @@ struct GemvParams {
     uint32_t R, m, k, n, gs, groups, n_expert_used, num_experts, row_bytes, n_units, xstride;
     int x_dtype, out_dtype, load_mode;
     int x_spec;        // TMA kernels: stage all m x rows before routing
+    int s_bulk;        // one-token kernel: scale and bias rows staged by bulk copies
     uint32_t kstages;  // integer-MMA kernel: k stages of the weight copies
 };
 

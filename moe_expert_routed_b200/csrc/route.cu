@@ -8,8 +8,8 @@
 //   route_hist    one CTA per chunk of ROUTE_CHUNK ids: shared-memory histogram
 //   route_scan    one CTA: bucket totals, offsets, per-(chunk, bucket) bases,
 //                 tile list
-//   route_scatter one CTA per chunk: stable ranks inside the chunk from warp
-//                 match masks and per-warp counts, then the scatter
+//   route_scatter one CTA per chunk: per-warp bucket counts, their prefix over
+//                 the warps, then stable ranks from warp match masks
 #include "common.cuh"
 #include "internal.h"
 
@@ -17,17 +17,42 @@ namespace moe {
 
 namespace {
 
+constexpr uint32_t ROUTE_WARPS = ROUTE_THREADS / 32;
+constexpr uint32_t ROUTE_PER_WARP = ROUTE_CHUNK / ROUTE_WARPS;  // ids per warp slice
+constexpr uint32_t ROUTE_ROUNDS = ROUTE_PER_WARP / 32;          // ids per lane
+
+// Bucket of each id of this warp's slice of the chunk (ids past R: ~0u), all
+// loads issued before any is used. Lane l holds ids slice + 32 r + l.
+__device__ __forceinline__ void load_buckets(const uint32_t *__restrict__ ids, uint32_t R, uint32_t E,
+                                             uint32_t (&bk)[ROUTE_ROUNDS]) {
+    const uint64_t w0 = (uint64_t)blockIdx.x * ROUTE_CHUNK + (threadIdx.x >> 5) * ROUTE_PER_WARP;
+    const uint32_t lane = threadIdx.x & 31u;
+#pragma unroll
+    for (uint32_t r = 0; r < ROUTE_ROUNDS; r++) {
+        const uint64_t i = w0 + 32u * r + lane;
+        bk[r] = i < R ? __ldg(ids + i) : 0u;
+    }
+#pragma unroll
+    for (uint32_t r = 0; r < ROUTE_ROUNDS; r++) {
+        const uint64_t i = w0 + 32u * r + lane;
+        bk[r] = i < R ? (bk[r] < E ? bk[r] : E) : 0xFFFFFFFFu;
+    }
+}
+
 __global__ void __launch_bounds__(ROUTE_THREADS)
 route_hist(const uint32_t *__restrict__ ids, uint32_t R, uint32_t E, uint32_t *__restrict__ chunk_hist) {
     extern __shared__ uint32_t hist[];
     const uint32_t NB = E + 1;
+    uint32_t bk[ROUTE_ROUNDS];
+    load_buckets(ids, R, E, bk);
     for (uint32_t b = threadIdx.x; b < NB; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    const uint64_t base = (uint64_t)blockIdx.x * ROUTE_CHUNK;
-    const uint64_t end = tmin<uint64_t>(base + ROUTE_CHUNK, R);
-    for (uint64_t i = base + threadIdx.x; i < end; i += blockDim.x) {
-        uint32_t e = __ldg(ids + i);
-        atomicAdd(&hist[e < E ? e : E], 1u);
+    const uint32_t lane = threadIdx.x & 31u;
+#pragma unroll
+    for (uint32_t r = 0; r < ROUTE_ROUNDS; r++) {
+        // one atomic per distinct bucket of the warp's 32 ids
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bk[r]);
+        if (bk[r] <= E && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[bk[r]], (uint32_t)__popc(peers));
     }
     __syncthreads();
     for (uint32_t b = threadIdx.x; b < NB; b += blockDim.x)
@@ -118,63 +143,60 @@ route_scan(const uint32_t *__restrict__ chunk_hist, uint32_t C, uint32_t E, uint
     }
 }
 
+// Stable scatter of one chunk. Each warp owns a contiguous slice of the chunk:
+// pass 1 counts the slice's ids per bucket, then a per-bucket prefix over the
+// warps (from the chunk's base) gives each warp its first position per bucket,
+// and pass 2 walks the slice in order, ranking equal buckets inside each group
+// of 32 ids by their match mask. Two block barriers in all.
 __global__ void __launch_bounds__(ROUTE_THREADS)
 route_scatter(const uint32_t *__restrict__ ids, uint32_t R, uint32_t E,
               const uint32_t *__restrict__ chunk_base, uint32_t *__restrict__ sorted_pairs,
               uint32_t *__restrict__ err, void *out, uint32_t n, int out_dtype) {
-    extern __shared__ uint32_t sm[];
-    constexpr uint32_t NW = ROUTE_THREADS / 32;
+    extern __shared__ uint32_t wbase[];  // [ROUTE_WARPS][E + 1]
     const uint32_t NB = E + 1;
-    uint32_t *running = sm;        // [NB]
-    uint32_t *wcnt = sm + NB;      // [NW][NB]
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
-    for (uint32_t b = tid; b < NB; b += blockDim.x) {
-        running[b] = chunk_base[(size_t)blockIdx.x * NB + b];
-        for (uint32_t w = 0; w < NW; w++) wcnt[w * NB + b] = 0;
+    uint32_t bk[ROUTE_ROUNDS];
+    load_buckets(ids, R, E, bk);
+    for (uint32_t b = tid; b < ROUTE_WARPS * NB; b += blockDim.x) wbase[b] = 0;
+    __syncthreads();
+    uint32_t *mine = wbase + warp * NB;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (uint32_t r = 0; r < ROUTE_ROUNDS; r++) {
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bk[r]);
+        if (bk[r] <= E && (peers & lt_mask) == 0) mine[bk[r]] += (uint32_t)__popc(peers);
+        __syncwarp();
     }
     __syncthreads();
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    const uint64_t base = (uint64_t)blockIdx.x * ROUTE_CHUNK;
-    for (uint32_t r = 0; r < ROUTE_CHUNK / ROUTE_THREADS; r++) {
-        const uint64_t first = base + (uint64_t)r * ROUTE_THREADS;
-        if (first >= R) break;  // uniform across the block
-        const uint64_t i = first + tid;
-        const bool valid = i < R;
-        uint32_t b = 0xFFFFFFFFu;
-        if (valid) {
-            uint32_t e = __ldg(ids + i);
-            b = e < E ? e : E;
+    for (uint32_t b = tid; b < NB; b += blockDim.x) {
+        uint32_t run = chunk_base[(size_t)blockIdx.x * NB + b];
+        for (uint32_t w = 0; w < ROUTE_WARPS; w++) {
+            const uint32_t c = wbase[w * NB + b];
+            wbase[w * NB + b] = run;
+            run += c;
         }
+    }
+    __syncthreads();
+    const uint64_t w0 = (uint64_t)blockIdx.x * ROUTE_CHUNK + warp * ROUTE_PER_WARP;
+#pragma unroll
+    for (uint32_t r = 0; r < ROUTE_ROUNDS; r++) {
+        const uint32_t b = bk[r];
+        const bool valid = b <= E;
         const uint32_t peers = __match_any_sync(0xFFFFFFFFu, b);
-        const uint32_t rank = __popc(peers & lt_mask);
-        const bool leader = valid && rank == 0;
-        if (leader) wcnt[warp * NB + b] = __popc(peers);
-        __syncthreads();
+        const uint32_t i = (uint32_t)(w0 + 32u * r + lane);
         if (valid) {
-            uint32_t pos = running[b] + rank;
-            for (uint32_t w = 0; w < warp; w++) pos += wcnt[w * NB + b];
-            if (pos < R) sorted_pairs[pos] = (uint32_t)i;
+            const uint32_t pos = mine[b] + (uint32_t)__popc(peers & lt_mask);
+            if (pos < R) sorted_pairs[pos] = i;
             else atomicOr(err, ERR_INTERNAL);
             if (b == E) {
                 atomicOr(err, ERR_BAD_ID);
                 if (out)
-                    for (uint32_t col = 0; col < n; col++) store_out(out, out_dtype, i * n + col, 0.f);
+                    for (uint32_t col = 0; col < n; col++) store_out(out, out_dtype, (size_t)i * n + col, 0.f);
             }
         }
-        __syncthreads();
-        if (leader) {
-            bool last = true;
-            uint32_t sum = 0;
-            for (uint32_t w = 0; w < NW; w++) {
-                uint32_t c = wcnt[w * NB + b];
-                sum += c;
-                if (w > warp && c) last = false;
-            }
-            if (last) running[b] += sum;
-        }
-        __syncthreads();
-        if (leader) wcnt[warp * NB + b] = 0;
-        __syncthreads();
+        __syncwarp();
+        if (valid && (peers & lt_mask) == 0) mine[b] += (uint32_t)__popc(peers);
+        __syncwarp();
     }
 }
 
@@ -194,7 +216,7 @@ cudaError_t launch_route(const uint32_t *ids, uint32_t R, uint32_t E, uint32_t t
         max_tiles, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t sc_smem = (size_t)NB * (1 + ROUTE_THREADS / 32) * sizeof(uint32_t);
+    const size_t sc_smem = (size_t)NB * ROUTE_WARPS * sizeof(uint32_t);
     route_scatter<<<chunks, ROUTE_THREADS, sc_smem, st>>>(ids, R, E, chunk_base, sorted_pairs,
                                                            err, out, n, out_dtype);
     return cudaGetLastError();
