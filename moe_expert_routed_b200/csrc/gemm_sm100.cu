@@ -178,11 +178,21 @@ __device__ __forceinline__ void store_a(const float (&v)[32], uint32_t a_hi, uin
     }
 }
 
+// Two E4M3 bytes (low byte first) to f16x2 by the hardware conversion.
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t two) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+    return *reinterpret_cast<__half2 *>(&h);
+}
+
 // NVFP4: e2m1 pairs to f16x2 by the hardware conversion, times the E4M3 block
-// scale (exact: at most 6 significant bits), stored as f16 or bf16 (exact).
+// scales s01 = (s0, s1) as an f16 multiply (exact: at most 6 significant bits,
+// magnitudes in [2^-10, 2688]), stored as f16, or as bf16 through f32 (exact).
+// Codes 0-15 of the thread's 32 belong to the group of s0, codes 16-31 to s1.
 template <bool F16>
-__device__ __forceinline__ void nvfp4_store(const uint32_t (&w)[4], float s0, float s1, bool two_groups,
-                                            uint32_t a_hi, uint32_t r, uint32_t c0) {
+__device__ __forceinline__ void nvfp4_store(const uint32_t (&w)[4], __half2 s01, uint32_t a_hi, uint32_t r,
+                                            uint32_t c0) {
+    const __half2 sa = __low2half2(s01), sb = __high2half2(s01);
 #pragma unroll
     for (int cc = 0; cc < 4; cc++) {  // word cc holds codes 8cc .. 8cc+7
         uint32_t h[4];
@@ -194,12 +204,17 @@ __device__ __forceinline__ void nvfp4_store(const uint32_t (&w)[4], float s0, fl
             "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
             : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
             : "r"(w[cc]));
-        const float s = (cc >= 2 && two_groups) ? s1 : s0;
+        const __half2 sc = cc >= 2 ? sb : sa;
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; e++) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[e]));
-            o[e] = pack2<F16>(f.x * s, f.y * s);
+            const __half2 pr = __hmul2(*reinterpret_cast<const __half2 *>(&h[e]), sc);
+            if constexpr (F16) {
+                o[e] = *reinterpret_cast<const uint32_t *>(&pr);
+            } else {
+                const float2 f = __half22float2(pr);
+                o[e] = pack2<false>(f.x, f.y);
+            }
         }
         sts128(a_hi + swz(r, c0 + cc), o[0], o[1], o[2], o[3]);
     }
@@ -210,9 +225,8 @@ __device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], 
                                              float b0, float s1, float b1, bool two_groups,
                                              const float *cb, uint32_t a_hi, uint32_t a_lo, uint32_t r,
                                              uint32_t c0) {
-    if constexpr (KIND == K_NVFP4) {
-        nvfp4_store<F16>(w, s0, s1, two_groups, a_hi, r, c0);
-    } else {
+    static_assert(KIND != K_NVFP4, "NVFP4 tiles go through nvfp4_store");
+    {
         float v[32];
         if constexpr (KIND == K_CB3) {
             switch (sub) {  // first code's position in word 0: 0, 2, 4, 6 or 8
@@ -288,6 +302,8 @@ grouped_gemm_kernel(const GemmParams P) {
     constexpr uint32_t ES = (KIND == K_NVFP4) ? 1u : 2u;  // bytes per scale
     constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
     using RL = RawLayout<KIND>;
+    // up to 256 pairs: one accumulator of BN columns; more: a second one from column 256
+    constexpr uint32_t TMEM_COLS = BN <= 64 ? 64u : BN <= 128 ? 128u : BN <= 256 ? 256u : 512u;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[3 * MAX_STAGES + 1];
@@ -332,7 +348,7 @@ grouped_gemm_kernel(const GemmParams P) {
             cb_s[tid] = f16_bits_to_f32(__ldg((const unsigned short *)P.aux + tid));
     }
     if (warp == MMA_WARP) {
-        ptx::tmem_alloc(ptx::smem_u32(&tmem_s), BN);
+        ptx::tmem_alloc(ptx::smem_u32(&tmem_s), TMEM_COLS);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -406,18 +422,33 @@ grouped_gemm_kernel(const GemmParams P) {
                 for (int i = 0; i < 4; i++) w[i] = *(const uint32_t *)(rr + 4u * (wb + i));
             }
             const uint32_t j0 = kt * KT, gh = (j0 + 32u * h) >> P.lg_gs;
-            float s0, b0, s1 = 0.f, b1 = 0.f;
-            if (P.scale_words) {
-                const uint4 q = *(const uint4 *)(rr + RL::SC);
-                const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
-                const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
-                staged_scale<KIND>(sw, bw, gh * ES - base_b, s0, b0);
-                if (gs16) staged_scale<KIND>(sw, bw, (gh + 1u) * ES - base_b, s1, b1);
+            if constexpr (KIND == K_NVFP4) {
+                // groups of 16: this half's two E4M3 scales, converted together (exact in f16)
+                __half2 s01;
+                if (P.scale_words) {
+                    // the staged word holds groups 4kt .. 4kt+3; this half's are bytes 2h, 2h+1
+                    s01 = e4m3x2_to_half2((*(const uint32_t *)(rr + RL::SC) >> (16u * h)) & 0xFFFFu);
+                } else {
+                    float s0, s1, unused;
+                    global_scale<KIND>(srow, brow, gh, P.groups, s0, unused);
+                    global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, unused);
+                    s01 = __floats2half2_rn(s0, s1);
+                }
+                nvfp4_store<F16>(w, s01, st, r, h * 4u);
             } else {
-                global_scale<KIND>(srow, brow, gh, P.groups, s0, b0);
-                if (gs16) global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, b1);
+                float s0, b0, s1 = 0.f, b1 = 0.f;
+                if (P.scale_words) {
+                    const uint4 q = *(const uint4 *)(rr + RL::SC);
+                    const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
+                    const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
+                    staged_scale<KIND>(sw, bw, gh * ES - base_b, s0, b0);
+                    if (gs16) staged_scale<KIND>(sw, bw, (gh + 1u) * ES - base_b, s1, b1);
+                } else {
+                    global_scale<KIND>(srow, brow, gh, P.groups, s0, b0);
+                    if (gs16) global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, b1);
+                }
+                dequant_tile<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
             }
-            dequant_tile<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(full0 + 8 * s);
         }
@@ -538,7 +569,9 @@ grouped_gemm_kernel(const GemmParams P) {
         ptx::cp_async_wait_all();
     } else if (lane == 0) {
         // --------------------------------------------------------------- MMA issue
-        const uint32_t idesc = ptx::idesc_f16(F16 ? 0u : 1u, nt_pad);
+        const uint32_t n1 = tmin<uint32_t>(nt_pad, 256u), n2 = nt_pad - n1;
+        const uint32_t idesc = ptx::idesc_f16(F16 ? 0u : 1u, n1);
+        const uint32_t idesc2 = ptx::idesc_f16(F16 ? 0u : 1u, n2 > 0 ? n2 : 16u);
         uint32_t accum = 0;
         bool ok = true;
         for (uint32_t kt = 0; kt < P.ktiles; kt++) {
@@ -556,11 +589,23 @@ grouped_gemm_kernel(const GemmParams P) {
             for (int ks = 0; ks < KT / 16; ks++) {
                 const uint32_t ko = ks * 32u;
                 ptx::mma_f16_ss(tmem, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_hi + ko), idesc, accum);
-                accum = 1;
                 if constexpr (BT == 2)
                     ptx::mma_f16_ss(tmem, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_lo + ko), idesc, 1);
                 if constexpr (AT == 2)
                     ptx::mma_f16_ss(tmem, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b_hi + ko), idesc, 1);
+                if constexpr (BN > 256) {
+                    // pairs 256 .. nt_pad - 1: B rows from 256 (32 KB into the tile), TMEM columns from 256
+                    if (n2 > 0) {
+                        const uint32_t b2 = b_hi + 256u * 128u;
+                        ptx::mma_f16_ss(tmem + 256u, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b2 + ko), idesc2, accum);
+                        if constexpr (BT == 2)
+                            ptx::mma_f16_ss(tmem + 256u, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b2 + B_TILE + ko),
+                                            idesc2, 1);
+                        if constexpr (AT == 2)
+                            ptx::mma_f16_ss(tmem + 256u, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b2 + ko), idesc2, 1);
+                    }
+                }
+                accum = 1;
             }
             ptx::mma_commit(empty0 + 8 * s);
         }
@@ -574,7 +619,7 @@ grouped_gemm_kernel(const GemmParams P) {
     if (warp == MMA_WARP) {
         __syncwarp();
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, BN);
+        ptx::tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -600,14 +645,17 @@ uint32_t raw_tile(int kind) {
     }
 }
 
-// Tile width and pipeline depth: 256 pairs per tile when experts hold ~100 or
-// more pairs on average (128 with f32 x, whose operand tiles are twice as
-// large), 64 otherwise; as many stages (2..6) as fit.
+// Tile width and pipeline depth: when experts hold ~100 or more pairs on
+// average, 256 pairs per tile (128 with f32 x, whose operand tiles are twice
+// as large), and 320 for NVFP4 with 16-bit x, whose single-term weight tile
+// leaves room for it: experts of up to 320 pairs then take one tile, so their
+// weights are dequantised once instead of once for 256 pairs and again for a
+// small remainder. 64 otherwise; as many stages (2..6) as fit.
 bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
     const uint64_t R = (uint64_t)a.m * a.n_expert_used;
     const bool big = R >= 96ull * a.num_experts;
     const bool f32x = a.x_dtype == DT_F32;
-    const uint32_t bn = big ? (f32x ? 128u : 256u) : 64u;
+    const uint32_t bn = big ? (f32x ? 128u : a.kind == K_NVFP4 ? 320u : 256u) : 64u;
     const uint32_t at = a.kind == K_NVFP4 ? 1u : 2u, bt = f32x ? 2u : 1u;
     const size_t stage = (size_t)at * A_TILE + (size_t)bt * bn * KT * 2 + raw_tile(a.kind);
     if (2 * stage + 1024 > GEMM_SMEM_BUDGET) return false;
@@ -639,6 +687,12 @@ cudaError_t launch_k(const GemmParams &P, const GemmPlan &pl, int x_dtype, uint3
     if (x_dtype == DT_F32) {
         if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, pl, nm, mt, st);
         return launch_t<KIND, DT_F32, 64>(P, pl, nm, mt, st);
+    }
+    if constexpr (KIND == K_NVFP4) {
+        if (pl.bn == 320) {
+            if (x_dtype == DT_BF16) return launch_t<KIND, DT_BF16, 320>(P, pl, nm, mt, st);
+            return launch_t<KIND, DT_F16, 320>(P, pl, nm, mt, st);
+        }
     }
     if (x_dtype == DT_BF16) {
         if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, pl, nm, mt, st);

@@ -1,8 +1,9 @@
 """The one-token decode kernel (x planes in registers, rows of all pairs split
 evenly over the SMs) against the oracle, element by element: row ranges that
-straddle pairs, lanes with idle units, the widest rows it takes and the first
-one it does not, every x / out type, scale rows that cannot be bulk-copied,
-and duplicate and out-of-range ids."""
+straddle pairs, lanes with idle units, groups of 32 to 256 codes, odd group
+counts, the widest rows it takes and the first one it does not (handled by
+the TMA-staged decode kernel), every x / out type, scale rows that cannot be
+bulk-copied, and duplicate and out-of-range ids."""
 
 import pytest
 import torch
@@ -23,6 +24,8 @@ CASES = [
     (3072, 64, 128, 8, 16, DT_BF16, DT_F32),  # 96 units: the widest row of the kernel
     (3104, 32, 32, 4, 6, DT_F32, DT_F32),     # 97 units: handled by the other decode kernel
     (2816, 1, 64, 8, 12, DT_BF16, DT_F32),    # one row per pair
+    (1024, 48, 256, 4, 6, DT_BF16, DT_F32),   # groups of 256
+    (4096, 24, 256, 3, 4, DT_F16, DT_F32),    # 128 units: handled by the other decode kernel
 ]
 
 
