@@ -291,8 +291,10 @@ struct GemmCfg {
     static constexpr uint32_t STAGE = AT * A_TILE + BT * B_TILE + RawLayout<KIND>::TILE;
 };
 
+// Tiles of 64 pairs (few pairs per expert, dequantisation-bound) run two CTAs
+// per SM: two pipeline stages each, registers capped for two CTAs.
 template <int KIND, int XT, int BN>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, BN == 64 ? 2 : 1)
 grouped_gemm_kernel(const GemmParams P) {
     using C = GemmCfg<KIND, XT, BN>;
     constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
@@ -661,6 +663,7 @@ bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
     if (2 * stage + 1024 > GEMM_SMEM_BUDGET) return false;
     int S = (int)((GEMM_SMEM_BUDGET - 1024) / stage);
     S = S > MAX_STAGES ? MAX_STAGES : S;
+    if (bn == 64) S = 2;  // two CTAs per SM
     pl->bn = bn;
     pl->stages = S;
     pl->smem = (size_t)S * stage + 1024;
