@@ -96,10 +96,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     }
 }
 
+// The two values of a packed 16-bit pair back as floats (exact).
 template <bool F16>
-__device__ __forceinline__ float round16(float v) {
-    if constexpr (F16) return __half2float(__float2half_rn(v));
-    else return __bfloat162float(__float2bfloat16_rn(v));
+__device__ __forceinline__ float2 unpack2(uint32_t p) {
+    if constexpr (F16) {
+        return __half22float2(*reinterpret_cast<const __half2 *>(&p));
+    } else {
+        return make_float2(__uint_as_float(p << 16), __uint_as_float(p & 0xFFFF0000u));
+    }
 }
 
 // Packed words holding one thread's 32 codes (j0 a multiple of 32).
@@ -170,7 +174,10 @@ __device__ __forceinline__ void store_a(const float (&v)[32], uint32_t a_hi, uin
         for (int e = 0; e < 4; e++) {
             const float x0 = v[cc * 8 + 2 * e], x1 = v[cc * 8 + 2 * e + 1];
             hh[e] = pack2<F16>(x0, x1);
-            if constexpr (TWO) ll[e] = pack2<F16>(x0 - round16<F16>(x0), x1 - round16<F16>(x1));
+            if constexpr (TWO) {
+                const float2 h = unpack2<F16>(hh[e]);
+                ll[e] = pack2<F16>(x0 - h.x, x1 - h.y);
+            }
         }
         const uint32_t off = swz(r, c0 + cc);
         sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
@@ -391,8 +398,8 @@ grouped_gemm_kernel(const GemmParams P) {
 #pragma unroll
                     for (int t = 0; t < 4; t++) {
                         hi[t] = pack2<false>(f[2 * t], f[2 * t + 1]);
-                        lo[t] = pack2<false>(f[2 * t] - round16<false>(f[2 * t]),
-                                             f[2 * t + 1] - round16<false>(f[2 * t + 1]));
+                        const float2 h = unpack2<false>(hi[t]);
+                        lo[t] = pack2<false>(f[2 * t] - h.x, f[2 * t + 1] - h.y);
                     }
                     sts128(st + B_OFF + o, hi[0], hi[1], hi[2], hi[3]);
                     sts128(st + B_OFF + B_TILE + o, lo[0], lo[1], lo[2], lo[3]);
