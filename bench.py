@@ -243,32 +243,44 @@ def time_graph(g, replays: int) -> float:
 
 
 def e2e_decode(W: DecodeWorkload, steps: int):
-    """Through the public API with host buffers: per step, pinned host x and ids are
-    copied in, both projections run, both outputs are copied back."""
+    """Through the public API with host buffers: per step, one copy brings that
+    step's x rows and ids of both projections in from pinned host memory, both
+    projections run, one copy takes both outputs back."""
     M = W.M
-    hx = [W.x[i][: min(steps, W.G)].cpu().pin_memory() for i in range(2)]
-    hid = [W.ids[i][: min(steps, W.G)].cpu().pin_memory() for i in range(2)]
-    hout = [torch.empty((8, P.n), dtype=torch.float32).pin_memory() for P in W.projs]
-    dx = [torch.empty((1, P.k), dtype=torch.bfloat16, device="cuda") for P in W.projs]
-    did = [torch.empty((1, 8), dtype=torch.int32, device="cuda") for _ in W.projs]
-    dout = [torch.empty((1, 8, P.n), dtype=torch.float32, device="cuda") for P in W.projs]
-    n = hx[0].shape[0]
-    h2d = sum(hx[i][0].numel() * 2 + hid[i][0].numel() * 4 for i in range(2))
-    d2h = sum(o.numel() * 4 for o in hout)
+    n = min(steps, W.G)
+    # per-step input block: x of each projection (bf16), then ids of each projection
+    xb = [P.k * 2 for P in W.projs]
+    ib = [W.ids[i][0].numel() * 4 for i in range(2)]
+    offs, o = [], 0
+    for b in xb + ib:
+        offs.append(o)
+        o += (b + 15) // 16 * 16
+    blk = o
+    hin = torch.zeros((n, blk), dtype=torch.uint8).pin_memory()
+    for p in range(2):
+        hin[:, offs[p]:offs[p] + xb[p]] = W.x[p][:n].cpu().contiguous().view(torch.uint8).reshape(n, -1)
+        hin[:, offs[2 + p]:offs[2 + p] + ib[p]] = W.ids[p][:n].cpu().contiguous().view(torch.uint8).reshape(n, -1)
+    din = torch.empty(blk, dtype=torch.uint8, device="cuda")
+    dx = [din[offs[p]:offs[p] + xb[p]].view(torch.bfloat16).view(1, W.projs[p].k) for p in range(2)]
+    did = [din[offs[2 + p]:offs[2 + p] + ib[p]].view(torch.int32).view(1, -1) for p in range(2)]
+    nout = [8 * P.n for P in W.projs]
+    dout_all = torch.empty(sum(nout), dtype=torch.float32, device="cuda")
+    hout = torch.empty(sum(nout), dtype=torch.float32).pin_memory()
+    dout = [dout_all[:nout[0]].view(1, 8, W.projs[0].n), dout_all[nout[0]:].view(1, 8, W.projs[1].n)]
+    h2d = sum(xb) + sum(ib)
+    d2h = sum(nout) * 4
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record()
     for s in range(steps):
-        i = s % n
+        din.copy_(hin[s % n], non_blocking=True)
         for p, P in enumerate(W.projs):
-            dx[p].copy_(hx[p][i:i + 1], non_blocking=True)
-            did[p].copy_(hid[p][i:i + 1], non_blocking=True)
             L = W.layers[p][s % N_LAYERS]
             M.qmm_id(dx[p], did[p], L["packed"], L["scales"], L["aux"], n=P.n,
                      group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
                      out=dout[p], workspace=W.ws[p])
-            hout[p].copy_(dout[p][0], non_blocking=True)
+        hout.copy_(dout_all, non_blocking=True)
     b.record()
     b.synchronize()
     secs = a.elapsed_time(b) / 1e3

@@ -118,6 +118,26 @@ moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packe
                            moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
                            moe_stream_t stream, moe_path path);
 
+/*
+ * moe_qmm_id_bias -- moe_qmm_id followed by a per-expert output bias, added in
+ * the kernels' epilogue: out[t][s][col] = sum_j dequant(W[e][col][j]) x[t][j]
+ * + bias[e][col], e = ids[t * n_expert_used + s] (turboquant
+ * fast_switch_patch.py, the switch layer's output: y + expand_dims(bias[indices], -2)).
+ *   expert_bias  [num_experts, n] in bias_dtype (MOE_F32, MOE_BF16 or MOE_F16),
+ *                device pointer, caller-owned, element-aligned. Required.
+ *   path         as moe_qmm_id_path.
+ * The sum is formed in fp32 and rounded once to out_dtype. Rows of out-of-range
+ * ids stay 0 (no bias), with the error word set as for moe_qmm_id. Other
+ * arguments, ownership and errors as moe_qmm_id; MOE_ERR_INVALID_ARGUMENT also for
+ * a null expert_bias or an unknown bias_dtype.
+ */
+moe_status moe_qmm_id_bias(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                           const void *aux, const void *expert_bias, void *out, uint32_t m, uint32_t k,
+                           uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                           moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace,
+                           size_t workspace_bytes, moe_stream_t stream, moe_path path);
+
 /* Workspace bytes moe_qmm_id needs for these sizes (any path). Returns 0 if the
  * sizes overflow. */
 size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t num_experts);

@@ -16,6 +16,7 @@ tensor is not on a CUDA device, calls raise.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.moe_qmm_id.argtypes = [vp] * 6 + [u32] * 5 + [i32, u32, u32, i32, i32, vp, sz, vp]
         L.moe_qmm_id.restype = i32
         L.moe_qmm_id_path.argtypes = L.moe_qmm_id.argtypes + [i32]
+        L.moe_qmm_id_bias.argtypes = [vp] * 7 + [u32] * 5 + [i32, u32, u32, i32, i32, i32, vp, sz, vp, i32]
+        L.moe_qmm_id_bias.restype = i32
         L.moe_qmm_id_path.restype = i32
         L.moe_qmm_id_workspace_bytes.argtypes = [u32, u32, u32]
         L.moe_qmm_id_workspace_bytes.restype = sz
@@ -78,6 +81,7 @@ def status_str(status: int) -> str:
         return "?"
 
 
+@functools.lru_cache(maxsize=256)
 def packed_row_bytes(fmt: int, bits: int, k: int) -> int:
     return int(lib().moe_packed_row_bytes(fmt, bits, k))
 
@@ -99,6 +103,8 @@ def _stream_ptr(device) -> int:
 
 
 def _check_dev(t: torch.Tensor, name: str, device):
+    if isinstance(t, torch.Tensor) and t.is_cuda and t.device == device and t.is_contiguous():
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"quantized_matmul_id: {name} must be a torch.Tensor")
     if not t.is_cuda:
@@ -116,13 +122,16 @@ def _nbytes(t: torch.Tensor) -> int:
 def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
            aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
            out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
-           workspace: torch.Tensor | None = None, path: str = "auto") -> torch.Tensor:
+           workspace: torch.Tensor | None = None, path: str = "auto",
+           expert_bias: torch.Tensor | None = None) -> torch.Tensor:
     """Expert-routed quantized matmul on the current CUDA stream.
 
     x [m, k] (f32 / bf16 / f16); ids [m, n_expert_used] int32/uint32; packed, scales,
     aux: raw storage tensors (any dtype, byte lengths checked); returns out
     [m, n_expert_used, n]. Buffer-size checks and their messages follow
-    mlx-native quantized_matmul_id.rs (quantized_matmul_id).
+    mlx-native quantized_matmul_id.rs (quantized_matmul_id). expert_bias, if given,
+    is a [num_experts, n] f32 / bf16 / f16 tensor added to every pair's row of its
+    expert (moe_qmm_id_bias).
     """
     device = x.device
     for t, name in ((x, "input"), (ids, "ids"), (packed, "weight"), (scales, "scales"),
@@ -175,11 +184,21 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
         workspace = new_workspace(m, n_expert_used, num_experts, device)
     else:
         _check_dev(workspace, "workspace", device)
-    st = lib().moe_qmm_id_path(
-        x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
-        out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used, num_experts,
-        _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], workspace.data_ptr(), _nbytes(workspace),
-        _stream_ptr(device), _PATHS[path])
+    if expert_bias is None:
+        st = lib().moe_qmm_id_path(
+            x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
+            out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used, num_experts,
+            _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], workspace.data_ptr(), _nbytes(workspace),
+            _stream_ptr(device), _PATHS[path])
+    else:
+        _check_dev(expert_bias, "expert_bias", device)
+        if expert_bias.dtype not in _TORCH_DT or expert_bias.numel() < num_experts * n:
+            raise ValueError("quantized_matmul_id: expert_bias must hold [num_experts, N] f32/bf16/f16")
+        st = lib().moe_qmm_id_bias(
+            x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
+            expert_bias.data_ptr(), out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used,
+            num_experts, _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], _TORCH_DT[expert_bias.dtype],
+            workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), _PATHS[path])
     if st != MOE_OK:
         raise MoeError(st, "moe_qmm_id")
     return out

@@ -102,14 +102,15 @@ moe_status validate_call(const void *x, const uint32_t *ids, const void *packed,
 }
 }  // namespace moe
 
-extern "C" {
+namespace moe {
+namespace {
 
-moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packed,
-                           const void *scales, const void *aux, void *out, uint32_t m, uint32_t k,
-                           uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
-                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
-                           moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
-                           moe_stream_t stream, moe_path path) {
+// moe_qmm_id with an optional per-expert output bias (null: none).
+moe_status run(const void *x, const uint32_t *ids, const void *packed, const void *scales, const void *aux,
+               const void *bias, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
+               uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+               moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace, size_t workspace_bytes,
+               moe_stream_t stream, moe_path path) {
     moe_status v = validate(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt,
                             n_expert_used, num_experts, x_dtype, out_dtype);
     if (v != MOE_OK) return v;
@@ -128,6 +129,8 @@ moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packe
     a.x_dtype = (int)x_dtype; a.out_dtype = (int)out_dtype;
     a.row_bytes = (uint32_t)row_bytes_of((int)fmt, bits, k);
     a.groups = (k + group_size - 1) / group_size;
+    a.bias = bias;
+    a.bias_dtype = (int)bias_dtype;
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);
@@ -173,6 +176,32 @@ moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packe
         }
     }
     return ce == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_qmm_id_path(const void *x, const uint32_t *ids, const void *packed,
+                           const void *scales, const void *aux, void *out, uint32_t m, uint32_t k,
+                           uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                           moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                           moe_stream_t stream, moe_path path) {
+    return run(x, ids, packed, scales, aux, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
+               num_experts, x_dtype, out_dtype, MOE_F32, workspace, workspace_bytes, stream, path);
+}
+
+moe_status moe_qmm_id_bias(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                           const void *aux, const void *expert_bias, void *out, uint32_t m, uint32_t k,
+                           uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                           moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace,
+                           size_t workspace_bytes, moe_stream_t stream, moe_path path) {
+    if (!expert_bias || (int)bias_dtype < 0 || (int)bias_dtype > 2) return MOE_ERR_INVALID_ARGUMENT;
+    return run(x, ids, packed, scales, aux, expert_bias, out, m, k, n, group_size, bits, fmt, n_expert_used,
+               num_experts, x_dtype, out_dtype, bias_dtype, workspace, workspace_bytes, stream, path);
 }
 
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,

@@ -67,6 +67,13 @@ __device__ __forceinline__ float load_x(const void *x, int dt, size_t idx) {
     return dt == DT_BF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
 }
 
+// Per-expert output bias (f32, bf16 or f16) at element idx of [num_experts, n];
+// 0 without a bias.
+__device__ __forceinline__ float load_bias(const void *bias, int dt, size_t idx) {
+    if (!bias) return 0.f;
+    return load_x(bias, dt, idx);
+}
+
 __device__ __forceinline__ void store_out(void *out, int dt, size_t idx, float v) {
     if (dt == DT_F32) {
         ((float *)out)[idx] = v;

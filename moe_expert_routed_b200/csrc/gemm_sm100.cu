@@ -68,6 +68,8 @@ struct GemmParams {
     uint32_t k, n, lg_gs, groups, n_expert_used, row_bytes, ktiles, stages;
     uint32_t scale_words;  // rows of scales (and biases) 4-byte aligned: staged by the loaders
     uint32_t raw16;        // rows of codes 16-byte aligned: staged in 16-byte copies (else 8)
+    const void *bias;      // per-expert output bias [num_experts, n] (bias_dtype), or null
+    int bias_dtype;
     int out_dtype;
     uint64_t timeout_ns;
 };
@@ -467,6 +469,7 @@ grouped_gemm_kernel(const GemmParams P) {
             const uint32_t q = warp & 3u, ch = warp >> 2;
             const uint32_t grow_e = row0 + q * 32u + lane;
             const float s2 = (KIND == K_NVFP4) ? __ldg((const float *)P.aux + e) : 1.f;
+            const float bv = grow_e < P.n ? load_bias(P.bias, P.bias_dtype, (size_t)e * P.n + grow_e) : 0.f;
             const uint32_t c_begin = ch * (BN / 2), c_end = tmin<uint32_t>(c_begin + BN / 2, nt);
             for (uint32_t c0 = c_begin; c0 < c_end; c0 += 16) {
                 uint32_t v[16];
@@ -478,7 +481,7 @@ grouped_gemm_kernel(const GemmParams P) {
                         const uint32_t col = c0 + i;
                         if (col < c_end)
                             store_out(P.out, P.out_dtype, (size_t)pairs_s[col] * P.n + grow_e,
-                                      __uint_as_float(v[i]) * s2);
+                                      __uint_as_float(v[i]) * s2 + bv);
                     }
                 }
             }
@@ -765,6 +768,7 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
                     (a.fmt != FMT_AFFINE || (uintptr_t)a.aux % 4u == 0);
     P.raw16 = a.kind != K_CB3 && a.row_bytes % 16u == 0;
     P.out_dtype = a.out_dtype;
+    P.bias = a.bias; P.bias_dtype = a.bias_dtype;
     P.timeout_ns = WAIT_NS;
     const uint32_t nm = (a.n + BM - 1) / BM;
     return launch_kind(P, pl, a.kind, a.x_dtype, nm, max_tiles, st);

@@ -260,7 +260,8 @@ gemv_kernel(const GemvParams P) {
 #pragma unroll
             for (int q = 0; q < NPB; q++)
                 if ((uint32_t)q < np)
-                    store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q] * s2);
+                    store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row,
+                              acc[q] * s2 + load_bias(P.bias, P.bias_dtype, (size_t)expert * P.n + row));
         }
     }
 }
@@ -457,9 +458,10 @@ gemv_aff4_dp4a(const GemvParams P) {
             for (int d = GEMV_LPR / 2; d > 0; d >>= 1) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], d);
         }
         if (l8 == 0 && row_ok) {
+            const float bv = load_bias(P.bias, P.bias_dtype, (size_t)expert * P.n + row);
 #pragma unroll
             for (int q = 0; q < NPB; q++)
-                if ((uint32_t)q < np) store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q]);
+                if ((uint32_t)q < np) store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q] + bv);
         }
     }
 }
@@ -783,9 +785,10 @@ gemv_aff4_tma(const GemvParams P) {
             for (int d = LPR / 2; d > 0; d >>= 1) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], d);
         }
         if (l == 0 && row < P.n) {
+            const float bv = load_bias(P.bias, P.bias_dtype, (size_t)expert * P.n + row);
 #pragma unroll
             for (int q = 0; q < NPB; q++)
-                if ((uint32_t)q < np) store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q]);
+                if ((uint32_t)q < np) store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q] + bv);
         }
     }
     if (*abort_flag) {
@@ -1042,7 +1045,11 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
         }
 #pragma unroll
         for (int d = LPR / 2; d > 0; d >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, d);
-        if (valid && l == 0) store_out(P.out, P.out_dtype, (size_t)p * n + c, acc);
+        if (valid && l == 0) {
+            const uint32_t e = ex_s[p - p_first];
+            store_out(P.out, P.out_dtype, (size_t)p * n + c,
+                      e < P.num_experts ? acc + load_bias(P.bias, P.bias_dtype, (size_t)e * n + c) : 0.f);
+        }
         c += RPI;
         if (c >= n) {
             c -= n;
@@ -1271,6 +1278,7 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     if ((uint64_t)P.n_units * uc < a.k) P.n_units = (a.k + uc - 1) / uc;
     P.xstride = P.n_units * (uc + 1);
     P.x_dtype = a.x_dtype; P.out_dtype = a.out_dtype;
+    P.bias = a.bias; P.bias_dtype = a.bias_dtype;
     const bool al16 = ((uintptr_t)a.packed % 16 == 0) && (a.row_bytes % 16 == 0);
     const bool al4 = ((uintptr_t)a.packed % 4 == 0) && (a.row_bytes % 4 == 0);
     P.load_mode = al16 ? 16 : al4 ? 4 : 1;

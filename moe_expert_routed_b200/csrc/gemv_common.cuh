@@ -27,7 +27,8 @@ struct GemvParams {
     int x_dtype, out_dtype, load_mode;
     int x_spec;        // TMA kernels: stage all m x rows before routing
     int s_bulk;        // one-token kernel: scale and bias rows staged by bulk copies
-    uint32_t kstages;  // integer-MMA kernel: k stages of the weight copies
+    const void *bias;  // per-expert output bias [num_experts, n] (bias_dtype), or null
+    int bias_dtype;
 };
 
 // Which expert this CTA serves and how many pairs it has. Fused mode: all ids

@@ -65,6 +65,8 @@ struct QmmArgs {
     uint32_t m, k, n, group_size, bits, n_expert_used, num_experts;
     int fmt, kind, x_dtype, out_dtype;
     uint32_t row_bytes, groups;
+    const void *bias;  // per-expert output bias [num_experts, n] (bias_dtype), or null
+    int bias_dtype;
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).

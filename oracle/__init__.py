@@ -64,6 +64,8 @@ def lib():
         L.oracle_expert_max_abs_weight.argtypes = [ctypes.c_void_p] * 3 + [u32, u32, u32, u32,
                                                                             u32, i32, u32]
         L.oracle_expert_max_abs_weight.restype = ctypes.c_double
+        L.oracle_add_expert_bias.argtypes = [ctypes.c_void_p] * 3 + [u64] + [ctypes.c_void_p] * 2 + [i32, u32, u32]
+        L.oracle_add_expert_bias.restype = None
         L.oracle_route.argtypes = [ctypes.c_void_p, u64, u32, u32, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, u64]
         L.oracle_route.restype = ctypes.c_int64
@@ -157,6 +159,21 @@ def qmm_id_sample(P, pairs: np.ndarray, cols: np.ndarray, nthreads: int | None =
                                     nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle rejected the sample")
+    return vals
+
+
+def add_expert_bias(vals: np.ndarray, P, bias: np.ndarray, bias_dtype: int, pairs=None, cols=None):
+    """vals (double, from qmm_id or qmm_id_sample) += bias[ids[p]][col] for valid ids,
+    in place; bias [num_experts, n] raw storage (float32, or uint16 bits of bf16/f16)."""
+    assert vals.dtype == np.float64 and vals.flags["C_CONTIGUOUS"]
+    ids = np.ascontiguousarray(P.ids.reshape(-1), dtype=np.uint32)
+    bias = np.ascontiguousarray(bias)
+    if pairs is not None:
+        pairs = np.ascontiguousarray(pairs, dtype=np.uint32)
+        cols = np.ascontiguousarray(cols, dtype=np.uint32)
+    lib().oracle_add_expert_bias(_ptr(vals), _ptr(pairs) if pairs is not None else None,
+                                 _ptr(cols) if cols is not None else None, vals.size, _ptr(ids),
+                                 _ptr(bias), bias_dtype, P.n, P.num_experts)
     return vals
 
 

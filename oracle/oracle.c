@@ -36,6 +36,11 @@
  *
  * Out-of-range ids (e >= num_experts) produce an all-zero output row and are
  * counted in *bad_ids.
+ *
+ * Per-expert output bias (turboquant fast_switch_patch.py, the switch layer's
+ * "y + mx.expand_dims(bias[indices], -2)"): oracle_add_expert_bias adds
+ * bias[e][col] to the double result of every pair with a valid id, before the
+ * single rounding to the output type; rows of out-of-range ids stay zero.
  */
 #include <math.h>
 #include <pthread.h>
@@ -360,4 +365,18 @@ int64_t oracle_route(const uint32_t *ids, uint64_t R, uint32_t E, uint32_t tile_
             nt++;
         }
     return (int64_t)nt;
+}
+
+/* vals[i] += bias[e][col] for element i = (pair p, column col) with e = ids[p] <
+ * num_experts (bias [num_experts, n], dtype 0 f32, 1 bf16, 2 f16). With pairs and
+ * cols NULL, element i is pair i / n, column i % n. */
+void oracle_add_expert_bias(double *vals, const uint32_t *pairs, const uint32_t *cols, uint64_t count,
+                            const uint32_t *ids, const void *bias, int bias_dtype, uint32_t n,
+                            uint32_t num_experts) {
+    for (uint64_t i = 0; i < count; i++) {
+        const uint64_t p = pairs ? pairs[i] : i / n;
+        const uint64_t col = cols ? cols[i] : i % n;
+        const uint32_t e = ids[p];
+        if (e < num_experts) vals[i] += x_at(bias, bias_dtype, (uint64_t)e * n + col);
+    }
 }

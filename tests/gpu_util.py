@@ -88,3 +88,29 @@ def check_sampled(P, out: torch.Tensor, pairs: np.ndarray, cols: np.ndarray, nth
     ref = oracle.qmm_id_sample(P, pairs, cols, nthreads=nthreads)
     got = out_to_f64(out)[pairs, cols]
     return compare(P, got, ref, pairs, cols)
+
+
+def bias_tensor(bias: np.ndarray, bias_dtype: int) -> torch.Tensor:
+    """Device tensor of a per-expert bias array from workloads.gen.expert_bias."""
+    if bias_dtype == DT_F32:
+        return torch.from_numpy(bias).cuda()
+    t = torch.from_numpy(bias.view(np.int16)).cuda()
+    return t.view(torch.bfloat16 if bias_dtype == DT_BF16 else torch.float16)
+
+
+def run_bias(P, bias: np.ndarray, bias_dtype: int, path="auto", dev=None, out=None, workspace=None):
+    dev = dev or to_device(P)
+    return M.qmm_id(dev["x"], dev["ids"], dev["packed"], dev["scales"], dev["aux"], n=P.n,
+                    group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
+                    out=out, out_dtype=TORCH_OUT[P.out_dtype], workspace=workspace, path=path,
+                    expert_bias=bias_tensor(bias, bias_dtype))
+
+
+def check_full_bias(P, out: torch.Tensor, bias: np.ndarray, bias_dtype: int, nthreads=None):
+    """Full-output comparison with the oracle plus its per-expert bias step."""
+    ref, _ = oracle.qmm_id(P, nthreads=nthreads)
+    ref = oracle.add_expert_bias(ref.reshape(-1).copy(), P, bias, bias_dtype)
+    got = out_to_f64(out)
+    pairs = np.repeat(np.arange(P.R), P.n)
+    cols = np.tile(np.arange(P.n), P.R)
+    return compare(P, got.reshape(-1), ref, pairs, cols)

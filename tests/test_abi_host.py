@@ -79,6 +79,17 @@ def test_unsupported_and_workspace_errors_before_cuda():
     assert _call(wsb=64) == 3                        # workspace too small
 
 
+def test_bias_entry_rejects_before_cuda():
+    L = M.lib()
+
+    def call(bias=16, bdt=0, m=4):
+        return L.moe_qmm_id_bias(16, 16, 16, 16, 16, bias, 16, m, 256, 128, 32, 4, 0, 2, 8, 0, 0, bdt,
+                                 4096, 1 << 20, None, 0)
+    assert call(bias=0) == 1          # null bias
+    assert call(bdt=3) == 1           # unknown bias dtype
+    assert call(m=0) == 1             # the operation's own checks still apply
+
+
 def test_route_invalid_arguments():
     L = M.lib()
     assert L.moe_qmm_id_route(16, 0, 8, 8, 64, 16, 16, 16, 16, 16, 4096, 1 << 20, None) == 1

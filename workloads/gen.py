@@ -151,6 +151,16 @@ class Problem:
         return Problem(**{**self.__dict__, "x": np.ascontiguousarray(x), "m": m})
 
 
+def expert_bias(seed: int, num_experts: int, n: int, dtype: int, sigma: float = 0.05) -> np.ndarray:
+    """Per-expert output bias [num_experts, n], N(0, sigma): float32 for DT_F32, else
+    the bf16 / f16 bit patterns as uint16."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    b = (rng.standard_normal((num_experts, n)) * sigma).astype(np.float32)
+    if dtype == DT_F32:
+        return b
+    return bf16_bits(b) if dtype == DT_BF16 else f16_bits(b)
+
+
 def _draw_x(rng, m, k, x_dtype):
     xf = rng.standard_normal((m, k), dtype=np.float32)
     if x_dtype == DT_F32:
