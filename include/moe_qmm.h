@@ -66,7 +66,8 @@ typedef enum {
     MOE_ERR_WORKSPACE_TOO_SMALL = 3,
     MOE_ERR_CUDA = 4,
     MOE_ERR_BAD_EXPERT_ID = 5,
-    MOE_ERR_TIMEOUT = 6
+    MOE_ERR_TIMEOUT = 6,
+    MOE_ERR_BAD_EXPERT_POINTER = 7
 } moe_status;
 
 /* Which kernel path computes the call. AUTO picks DECODE when
@@ -137,6 +138,34 @@ moe_status moe_qmm_id_bias(const void *x, const uint32_t *ids, const void *packe
                            uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                            moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace,
                            size_t workspace_bytes, moe_stream_t stream, moe_path path);
+
+/*
+ * moe_qmm_id_ptrs -- moe_qmm_id with each expert's weights in its own buffers,
+ * named by device tables of per-expert base addresses (metrale helpers_b.rs,
+ * ExpertPtrTable {packed_ptrs, scale_ptrs, scale2_vals} and launch_grouped_gemm).
+ *   packed_ptrs  [num_experts] u64 device table: expert e's packed rows,
+ *                [n, row_bytes] bytes, any alignment. A null entry means the expert
+ *                is not held by this caller (spark_model helpers_a.rs: a NULL slot
+ *                is skipped, the expert-parallel remote convention): the rows of
+ *                its pairs are left untouched.
+ *   scale_ptrs   [num_experts] u64: expert e's scales [n, ceil(k/gs)] (bf16 affine,
+ *                f16 codebook: 2-byte aligned; u8 E4M3 for NVFP4).
+ *   bias_ptrs    [num_experts] u64: AFFINE expert e's biases [n, ceil(k/gs)] bf16
+ *                (2-byte aligned); ignored otherwise (may be null).
+ *   aux          CODEBOOK: f16 codebook [2^bits]; NVFP4: f32 scale2 [num_experts]
+ *                (the table's scale2_vals); ignored for AFFINE.
+ * The tables and every buffer they name are caller-owned device memory. The
+ * call runs the CUDA-core kernels (path AUTO or DECODE; GROUPED returns
+ * MOE_ERR_UNSUPPORTED). A non-null expert with a null or misaligned scale / bias
+ * buffer is skipped and reported by moe_qmm_id_poll_error as
+ * MOE_ERR_BAD_EXPERT_POINTER. Other arguments and errors as moe_qmm_id;
+ * MOE_ERR_INVALID_ARGUMENT also for null tables.
+ */
+moe_status moe_qmm_id_ptrs(const void *x, const uint32_t *ids, const uint64_t *packed_ptrs,
+                           const uint64_t *scale_ptrs, const uint64_t *bias_ptrs, const void *aux, void *out,
+                           uint32_t m, uint32_t k, uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
+                           void *workspace, size_t workspace_bytes, moe_stream_t stream, moe_path path);
 
 /* Workspace bytes moe_qmm_id needs for these sizes (any path). Returns 0 if the
  * sizes overflow. */
@@ -213,7 +242,8 @@ moe_status moe_qmm_id_noalloc(const void *x, const uint32_t *ids, const void *pa
 /* Synchronise `stream`, read and clear the device error word of `workspace`.
  * Returns MOE_OK, MOE_ERR_BAD_EXPERT_ID (some id was >= num_experts),
  * MOE_ERR_TIMEOUT (a bounded wait inside a kernel gave up; its outputs are not
- * valid) or MOE_ERR_CUDA. */
+ * valid), MOE_ERR_BAD_EXPERT_POINTER (moe_qmm_id_ptrs skipped an expert whose
+ * scale or bias buffer was null or misaligned) or MOE_ERR_CUDA. */
 moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream);
 
 /* Static description of a status code. */

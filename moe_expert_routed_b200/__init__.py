@@ -30,7 +30,7 @@ MOE_OK = 0
 STATUS_NAMES = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED",
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_EXPERT_ID",
-    6: "MOE_ERR_TIMEOUT",
+    6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_BAD_EXPERT_POINTER",
 }
 
 _TORCH_DT = {torch.float32: DT_F32, torch.bfloat16: DT_BF16, torch.float16: DT_F16}
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.moe_qmm_id_path.argtypes = L.moe_qmm_id.argtypes + [i32]
         L.moe_qmm_id_bias.argtypes = [vp] * 7 + [u32] * 5 + [i32, u32, u32, i32, i32, i32, vp, sz, vp, i32]
         L.moe_qmm_id_bias.restype = i32
+        L.moe_qmm_id_ptrs.argtypes = [vp] * 7 + [u32] * 5 + [i32, u32, u32, i32, i32, vp, sz, vp, i32]
+        L.moe_qmm_id_ptrs.restype = i32
         L.moe_qmm_id_path.restype = i32
         L.moe_qmm_id_workspace_bytes.argtypes = [u32, u32, u32]
         L.moe_qmm_id_workspace_bytes.restype = sz
@@ -201,6 +203,36 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
             workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), _PATHS[path])
     if st != MOE_OK:
         raise MoeError(st, "moe_qmm_id")
+    return out
+
+
+def qmm_id_ptrs(x: torch.Tensor, ids: torch.Tensor, packed_ptrs: torch.Tensor, scale_ptrs: torch.Tensor,
+                bias_ptrs: torch.Tensor | None, aux: torch.Tensor | None, *, n: int, group_size: int,
+                bits: int, fmt: int, num_experts: int, out: torch.Tensor,
+                workspace: torch.Tensor | None = None, path: str = "auto") -> torch.Tensor:
+    """moe_qmm_id_ptrs: weights in per-expert buffers named by device tables of
+    addresses (int64 tensors of num_experts entries; a 0 packed entry skips the
+    expert and leaves its pairs' rows of out untouched). aux: codebook (CODEBOOK) or
+    scale2 [num_experts] (NVFP4); bias_ptrs: affine biases."""
+    device = x.device
+    for t, name in ((x, "input"), (ids, "ids"), (packed_ptrs, "packed_ptrs"), (scale_ptrs, "scale_ptrs"),
+                    (out, "out")):
+        _check_dev(t, name, device)
+    for t, name in ((packed_ptrs, "packed_ptrs"), (scale_ptrs, "scale_ptrs"), (bias_ptrs, "bias_ptrs")):
+        if t is not None and (t.element_size() != 8 or t.numel() < num_experts):
+            raise ValueError(f"quantized_matmul_id: {name} must hold num_experts 64-bit addresses")
+    m, k = x.shape
+    n_expert_used = ids.shape[1]
+    if workspace is None:
+        workspace = new_workspace(m, n_expert_used, num_experts, device)
+    st = lib().moe_qmm_id_ptrs(
+        x.data_ptr(), ids.data_ptr(), packed_ptrs.data_ptr(), scale_ptrs.data_ptr(),
+        bias_ptrs.data_ptr() if bias_ptrs is not None else None,
+        aux.data_ptr() if aux is not None else None, out.data_ptr(), m, k, n, group_size, bits, fmt,
+        n_expert_used, num_experts, _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], workspace.data_ptr(),
+        _nbytes(workspace), _stream_ptr(device), _PATHS[path])
+    if st != MOE_OK:
+        raise MoeError(st, "moe_qmm_id_ptrs")
     return out
 
 

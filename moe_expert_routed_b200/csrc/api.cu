@@ -68,6 +68,8 @@ const char *moe_status_str(moe_status s) {
         case MOE_ERR_CUDA: return "CUDA error";
         case MOE_ERR_BAD_EXPERT_ID: return "an expert id was >= num_experts (its output rows are zero)";
         case MOE_ERR_TIMEOUT: return "a bounded device wait gave up; outputs are not valid";
+        case MOE_ERR_BAD_EXPERT_POINTER:
+            return "a pointer-table expert had a null or misaligned scale / bias buffer (its rows are untouched)";
     }
     return "unknown status";
 }
@@ -105,15 +107,27 @@ moe_status validate_call(const void *x, const uint32_t *ids, const void *packed,
 namespace moe {
 namespace {
 
-// moe_qmm_id with an optional per-expert output bias (null: none).
+// Weights held as per-expert buffers (null: contiguous [E, n, ...] arrays).
+struct PtrTables {
+    const uint64_t *packed, *scales, *biases;
+};
+
+// moe_qmm_id with an optional per-expert output bias (null: none) and optional
+// pointer-table weights.
 moe_status run(const void *x, const uint32_t *ids, const void *packed, const void *scales, const void *aux,
                const void *bias, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
                uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace, size_t workspace_bytes,
-               moe_stream_t stream, moe_path path) {
-    moe_status v = validate(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt,
-                            n_expert_used, num_experts, x_dtype, out_dtype);
+               moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}) {
+    moe_status v = validate(x, ids, pt.packed ? (const void *)pt.packed : packed,
+                            pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
+                            fmt, n_expert_used, num_experts, x_dtype, out_dtype);
     if (v != MOE_OK) return v;
+    if (pt.packed) {
+        // pointer-table weights run on the CUDA-core kernels
+        if (path == MOE_PATH_GROUPED) return MOE_ERR_UNSUPPORTED;
+        path = MOE_PATH_DECODE;
+    }
     if ((int)path < 0 || (int)path > 2) return MOE_ERR_INVALID_ARGUMENT;
     if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
     const uint64_t R = (uint64_t)m * n_expert_used;
@@ -131,6 +145,9 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     a.groups = (k + group_size - 1) / group_size;
     a.bias = bias;
     a.bias_dtype = (int)bias_dtype;
+    a.packed_ptrs = pt.packed;
+    a.scale_ptrs = pt.scales;
+    a.bias_ptrs = pt.biases;
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);
@@ -204,6 +221,19 @@ moe_status moe_qmm_id_bias(const void *x, const uint32_t *ids, const void *packe
                num_experts, x_dtype, out_dtype, bias_dtype, workspace, workspace_bytes, stream, path);
 }
 
+moe_status moe_qmm_id_ptrs(const void *x, const uint32_t *ids, const uint64_t *packed_ptrs,
+                           const uint64_t *scale_ptrs, const uint64_t *bias_ptrs, const void *aux, void *out,
+                           uint32_t m, uint32_t k, uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                           uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
+                           void *workspace, size_t workspace_bytes, moe_stream_t stream, moe_path path) {
+    if (!packed_ptrs || !scale_ptrs || (fmt == MOE_FMT_AFFINE && !bias_ptrs)) return MOE_ERR_INVALID_ARGUMENT;
+    // affine biases come from bias_ptrs; aux is the codebook or scale2 table
+    const void *aux_arg = fmt == MOE_FMT_AFFINE ? (const void *)bias_ptrs : aux;
+    return run(x, ids, nullptr, nullptr, aux_arg, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
+               num_experts, x_dtype, out_dtype, MOE_F32, workspace, workspace_bytes, stream, path,
+               PtrTables{packed_ptrs, scale_ptrs, bias_ptrs});
+}
+
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,
                       const void *aux, void *out, uint32_t m, uint32_t k, uint32_t n,
                       uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
@@ -253,6 +283,7 @@ moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream) {
     }
     if (w & ERR_TIMEOUT) return MOE_ERR_TIMEOUT;
     if (w & ERR_BAD_ID) return MOE_ERR_BAD_EXPERT_ID;
+    if (w & ERR_BAD_POINTER) return MOE_ERR_BAD_EXPERT_POINTER;
     if (w & ERR_INTERNAL) return MOE_ERR_CUDA;
     return MOE_OK;
 }

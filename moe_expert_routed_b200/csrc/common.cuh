@@ -19,6 +19,7 @@ enum Kind : int { K_AFF4 = 0, K_AFF6, K_AFF8, K_CB2, K_CB3, K_CB4, K_NVFP4, K_CO
 constexpr uint32_t ERR_BAD_ID = 1u;
 constexpr uint32_t ERR_TIMEOUT = 2u;
 constexpr uint32_t ERR_INTERNAL = 4u;
+constexpr uint32_t ERR_BAD_POINTER = 8u;  // pointer-table weights: missing or misaligned scales / biases
 
 __host__ __device__ inline int kind_of(int fmt, int bits) {
     if (fmt == FMT_AFFINE) return bits == 4 ? K_AFF4 : bits == 6 ? K_AFF6 : bits == 8 ? K_AFF8 : -1;

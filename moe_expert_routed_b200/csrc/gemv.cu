@@ -185,22 +185,44 @@ gemv_kernel(const GemvParams P) {
     const uint32_t row = row0 + warp * (32 / GEMV_LPR) + rsub;
     const bool row_ok = row < P.n;
     const uint32_t row_c = row_ok ? row : P.n - 1;  // clamp: loads stay in bounds
-    const size_t row_index = (size_t)expert * P.n + row_c;
+    constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
+    // the expert's packed rows, scales and (affine) biases: slices of the contiguous
+    // arrays, or the expert's own buffers from the pointer tables
+    const uint8_t *wbase, *sbase, *bbase;
+    size_t row_index = (size_t)expert * P.n + row_c;
+    int load_mode = P.load_mode;
+    if (P.packed_ptrs) {
+        wbase = (const uint8_t *)__ldg(P.packed_ptrs + expert);
+        if (!wbase) return;  // expert held elsewhere: its pairs' rows are not ours to write
+        sbase = (const uint8_t *)__ldg(P.scale_ptrs + expert);
+        bbase = AFF ? (const uint8_t *)__ldg(P.bias_ptrs + expert) : nullptr;
+        const uintptr_t sa = (uintptr_t)sbase | (AFF ? (uintptr_t)bbase : 0u);
+        if (!sbase || (AFF && !bbase) || (KIND != K_NVFP4 && (sa & 1u))) {
+            // scales / biases missing or not 2-byte aligned: skip the expert, flag it
+            if (tid == 0 && blockIdx.x == 0) atomicOr(P.err, ERR_BAD_POINTER);
+            return;
+        }
+        row_index = row_c;
+        const uintptr_t wa = (uintptr_t)wbase;
+        load_mode = (wa % 16u == 0 && P.row_bytes % 16u == 0) ? 16 : (wa % 4u == 0 && P.row_bytes % 4u == 0) ? 4 : 1;
+    } else {
+        wbase = P.packed;
+        sbase = (const uint8_t *)P.scales;
+        bbase = (const uint8_t *)P.aux;
+    }
 
     GemvCtx c;
-    c.row = P.packed + row_index * P.row_bytes;
+    c.row = wbase + row_index * P.row_bytes;
     c.row_bytes = P.row_bytes;
     c.gs = P.gs;
     c.groups = P.groups;
     c.codebook = (const uint16_t *)P.aux;
     if constexpr (KIND == K_NVFP4) {
-        c.scales = (const uint8_t *)P.scales + row_index * P.groups;
+        c.scales = (const uint8_t *)sbase + row_index * P.groups;
         c.biases = nullptr;
     } else {
-        c.scales = (const uint16_t *)P.scales + row_index * P.groups;
-        c.biases = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8)
-                       ? (const void *)((const uint16_t *)P.aux + row_index * P.groups)
-                       : nullptr;
+        c.scales = (const uint16_t *)sbase + row_index * P.groups;
+        c.biases = AFF ? (const void *)((const uint16_t *)bbase + row_index * P.groups) : nullptr;
     }
     const float s2 = (KIND == K_NVFP4) ? __ldg((const float *)P.aux + expert) : 1.f;
 
@@ -231,7 +253,7 @@ gemv_kernel(const GemvParams P) {
             for (int ub = 0; ub < UNITS_PER_BATCH; ub++) {
                 const uint32_t u = u0 + ub * GEMV_LPR;
                 if (u < P.n_units) {
-                    load_unit<U::UW>(c.row, u, c.row_bytes, P.load_mode, w[ub]);
+                    load_unit<U::UW>(c.row, u, c.row_bytes, load_mode, w[ub]);
                 } else {
 #pragma unroll
                     for (int v = 0; v < U::UW; v++) w[ub][v] = 0u;
@@ -1279,6 +1301,7 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     P.xstride = P.n_units * (uc + 1);
     P.x_dtype = a.x_dtype; P.out_dtype = a.out_dtype;
     P.bias = a.bias; P.bias_dtype = a.bias_dtype;
+    P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
     const bool al16 = ((uintptr_t)a.packed % 16 == 0) && (a.row_bytes % 16 == 0);
     const bool al4 = ((uintptr_t)a.packed % 4 == 0) && (a.row_bytes % 4 == 0);
     P.load_mode = al16 ? 16 : al4 ? 4 : 1;
@@ -1295,6 +1318,7 @@ cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st) 
     const uint32_t npb = tmin<uint32_t>(a.m, 8u);
     const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
     const bool spec = (uint64_t)a.m * a.k * xsz <= 32768u;
+    if (a.packed_ptrs) return launch_kind<true>(P, a.kind, npb, grid, st);  // pointer-table weights
     if (rows_ok(a)) return launch_rows(P, a, st);
     if (a.m == 1 && tma_ok(a, 1, spec)) {
         P.x_spec = spec;
@@ -1313,6 +1337,7 @@ cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const u
     GemvParams P = make_params(a, err);
     P.counts = counts; P.offsets = offsets; P.sorted_pairs = sorted_pairs;
     dim3 grid((a.n + GEMV_ROWS - 1) / GEMV_ROWS, a.num_experts);
+    if (a.packed_ptrs) return launch_kind<false>(P, a.kind, 8u, grid, st);  // pointer-table weights
     if (tma_ok(a, 8u, false)) return launch_tma<MODE_ROUTED>(P, 8u, a.num_experts, st);
     if (dp4a_ok(a)) return launch_dp4a<false>(P, 8u, grid, st);
     return launch_kind<false>(P, a.kind, 8u, grid, st);

@@ -29,6 +29,10 @@ struct GemvParams {
     int s_bulk;        // one-token kernel: scale and bias rows staged by bulk copies
     const void *bias;  // per-expert output bias [num_experts, n] (bias_dtype), or null
     int bias_dtype;
+    // pointer-table weights (null: contiguous [E, n, ...] arrays): per-expert base
+    // addresses of the packed rows, scales and affine biases; a null packed pointer
+    // means the expert is not held here and its pairs' rows are left untouched
+    const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;
 };
 
 // Which expert this CTA serves and how many pairs it has. Fused mode: all ids

@@ -67,6 +67,7 @@ struct QmmArgs {
     uint32_t row_bytes, groups;
     const void *bias;  // per-expert output bias [num_experts, n] (bias_dtype), or null
     int bias_dtype;
+    const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;  // pointer-table weights, or null
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).

@@ -90,6 +90,18 @@ def test_bias_entry_rejects_before_cuda():
     assert call(m=0) == 1             # the operation's own checks still apply
 
 
+def test_pointer_table_entry_rejects_before_cuda():
+    L = M.lib()
+
+    def call(packed=16, scales=16, biases=16, fmt=0, bits=4, gs=32, path=0):
+        return L.moe_qmm_id_ptrs(16, 16, packed, scales, biases, 16, 16, 4, 256, 128, gs, bits, fmt, 2, 8,
+                                 0, 0, 4096, 1 << 20, None, path)
+    assert call(packed=0) == 1
+    assert call(scales=0) == 1
+    assert call(biases=0) == 1                    # affine biases come from the table
+    assert call(path=2) == 2                      # the grouped path is not offered
+
+
 def test_route_invalid_arguments():
     L = M.lib()
     assert L.moe_qmm_id_route(16, 0, 8, 8, 64, 16, 16, 16, 16, 16, 4096, 1 << 20, None) == 1
@@ -98,7 +110,7 @@ def test_route_invalid_arguments():
 
 
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert M.status_str(s) and M.status_str(s) != "unknown status"
 
 
