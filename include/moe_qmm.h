@@ -154,12 +154,14 @@ moe_status moe_qmm_id_bias(const void *x, const uint32_t *ids, const void *packe
  *                (2-byte aligned); ignored otherwise (may be null).
  *   aux          CODEBOOK: f16 codebook [2^bits]; NVFP4: f32 scale2 [num_experts]
  *                (the table's scale2_vals); ignored for AFFINE.
- * The tables and every buffer they name are caller-owned device memory. The
- * call runs the CUDA-core kernels (path AUTO or DECODE; GROUPED returns
- * MOE_ERR_UNSUPPORTED). A non-null expert with a null or misaligned scale / bias
- * buffer is skipped and reported by moe_qmm_id_poll_error as
- * MOE_ERR_BAD_EXPERT_POINTER. Other arguments and errors as moe_qmm_id;
- * MOE_ERR_INVALID_ARGUMENT also for null tables.
+ * The tables and every buffer they name are caller-owned device memory. Paths
+ * as moe_qmm_id_path. The CUDA-core path takes code buffers at any alignment;
+ * the grouped GEMM needs 8-byte aligned code buffers (4 for 3-bit codebook
+ * rows). 16-bit scales and biases must be 2-byte aligned on both paths. A
+ * non-null expert whose buffers break these rules, or whose scale / bias entry
+ * is null, is skipped (its rows are untouched) and reported by
+ * moe_qmm_id_poll_error as MOE_ERR_BAD_EXPERT_POINTER. Other arguments and
+ * errors as moe_qmm_id; MOE_ERR_INVALID_ARGUMENT also for null tables.
  */
 moe_status moe_qmm_id_ptrs(const void *x, const uint32_t *ids, const uint64_t *packed_ptrs,
                            const uint64_t *scale_ptrs, const uint64_t *bias_ptrs, const void *aux, void *out,

@@ -123,11 +123,6 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
                             pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
                             fmt, n_expert_used, num_experts, x_dtype, out_dtype);
     if (v != MOE_OK) return v;
-    if (pt.packed) {
-        // pointer-table weights run on the CUDA-core kernels
-        if (path == MOE_PATH_GROUPED) return MOE_ERR_UNSUPPORTED;
-        path = MOE_PATH_DECODE;
-    }
     if ((int)path < 0 || (int)path > 2) return MOE_ERR_INVALID_ARGUMENT;
     if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
     const uint64_t R = (uint64_t)m * n_expert_used;

@@ -70,6 +70,9 @@ struct GemmParams {
     uint32_t raw16;        // rows of codes 16-byte aligned: staged in 16-byte copies (else 8)
     const void *bias;      // per-expert output bias [num_experts, n] (bias_dtype), or null
     int bias_dtype;
+    // pointer-table weights (null: contiguous arrays): per-expert base addresses of
+    // the packed rows, scales and affine biases; a null packed entry skips the expert
+    const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;
     int out_dtype;
     uint64_t timeout_ns;
 };
@@ -334,6 +337,28 @@ grouped_gemm_kernel(const GemmParams P) {
     const uint32_t row0 = blockIdx.x * BM;
     const uint32_t S = P.stages;
 
+    // the expert's packed rows, scales and (affine) biases
+    const uint8_t *wb = P.packed + (size_t)e * P.n * P.row_bytes;
+    const uint8_t *sb = (const uint8_t *)P.scales + (size_t)e * P.n * P.groups * ES;
+    const uint8_t *bb = (const uint8_t *)P.aux + (size_t)e * P.n * P.groups * 2u;
+    bool scale_words = P.scale_words != 0, raw16 = P.raw16 != 0;
+    if (P.packed_ptrs) {
+        wb = (const uint8_t *)__ldg(P.packed_ptrs + e);
+        if (!wb) return;  // expert held elsewhere: its pairs' rows are not ours to write (uniform)
+        sb = (const uint8_t *)__ldg(P.scale_ptrs + e);
+        bb = AFF ? (const uint8_t *)__ldg(P.bias_ptrs + e) : nullptr;
+        // the copies need 8-byte aligned code rows (4 for 3-bit codebook rows) and 2-byte
+        // aligned 16-bit scales / biases; other experts are skipped and flagged (uniform)
+        const uintptr_t wal = KIND == K_CB3 ? 4u : 8u;
+        const uintptr_t sal = (uintptr_t)sb | (AFF ? (uintptr_t)bb : 0u);
+        if (!sb || (AFF && !bb) || ((uintptr_t)wb % wal) != 0 || (KIND != K_NVFP4 && (sal & 1u))) {
+            if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(P.err, ERR_BAD_POINTER);
+            return;
+        }
+        raw16 = raw16 && (uintptr_t)wb % 16u == 0;
+        scale_words = scale_words && sal % 4u == 0 && (uintptr_t)sb % 4u == 0;
+    }
+
     const uint32_t base = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - ptx::smem_u32(smem_raw));
     const uint32_t full0 = ptx::smem_u32(&bars[0]);
@@ -371,9 +396,9 @@ grouped_gemm_kernel(const GemmParams P) {
     if (warp < LD_WARP0) {
         // -------------------------------------------------------- dequantisers
         const uint32_t r = tid & (BM - 1), h = tid >> 7;
-        const size_t row_index = (size_t)e * P.n + tmin<uint32_t>(row0 + r, P.n - 1);
-        const uint8_t *srow = (const uint8_t *)P.scales + row_index * P.groups * ES;
-        const uint8_t *brow = (const uint8_t *)P.aux + row_index * P.groups * 2u;
+        const size_t row_in = tmin<uint32_t>(row0 + r, P.n - 1);  // row within the expert
+        const uint8_t *srow = sb + row_in * P.groups * ES;
+        const uint8_t *brow = bb + row_in * P.groups * 2u;
         bool ok = true;
         for (uint32_t kt = 0; kt < P.ktiles; kt++) {
             const uint32_t s = kt % S;
@@ -436,7 +461,7 @@ grouped_gemm_kernel(const GemmParams P) {
             if constexpr (KIND == K_NVFP4) {
                 // groups of 16: this half's two E4M3 scales, converted together (exact in f16)
                 __half2 s01;
-                if (P.scale_words) {
+                if (scale_words) {
                     // the staged word holds groups 4kt .. 4kt+3; this half's are bytes 2h, 2h+1
                     s01 = e4m3x2_to_half2((*(const uint32_t *)(rr + RL::SC) >> (16u * h)) & 0xFFFFu);
                 } else {
@@ -448,7 +473,7 @@ grouped_gemm_kernel(const GemmParams P) {
                 nvfp4_store<F16>(w, s01, st, r, h * 4u);
             } else {
                 float s0, b0, s1 = 0.f, b1 = 0.f;
-                if (P.scale_words) {
+                if (scale_words) {
                     const uint4 q = *(const uint4 *)(rr + RL::SC);
                     const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
                     const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
@@ -502,12 +527,12 @@ grouped_gemm_kernel(const GemmParams P) {
                              : nullptr;
         }
         const uint32_t xdst0 = B_OFF + swz(xi0, xc);  // + 2048 j: 16 rows further down
-        const uint8_t *ebase = P.packed + (size_t)e * P.n * P.row_bytes;
+        const uint8_t *ebase = wb;
         const uint32_t nlast = P.n - 1;
         // scale words: thread lt stages those of weight row lt
-        const size_t srow_index = (size_t)e * P.n + tmin<uint32_t>(row0 + lt, nlast);
-        const uint8_t *srow = (const uint8_t *)P.scales + srow_index * P.groups * ES;
-        const uint8_t *brow = (const uint8_t *)P.aux + srow_index * P.groups * 2u;
+        const size_t srow_in = tmin<uint32_t>(row0 + lt, nlast);
+        const uint8_t *srow = sb + srow_in * P.groups * ES;
+        const uint8_t *brow = bb + srow_in * P.groups * 2u;
         const uint32_t srow_bytes = P.groups * ES;
         const uint32_t nsw = (gs16 && ES == 2u) ? 2u : 1u;
 
@@ -543,7 +568,7 @@ grouped_gemm_kernel(const GemmParams P) {
                 }
             } else {
                 constexpr uint32_t RB = RL::RB;
-                if (P.raw16) {
+                if (raw16) {
                     constexpr uint32_t NC = RB / 16u;
 #pragma unroll
                     for (uint32_t i = 0; i < NC; i++) {
@@ -565,7 +590,7 @@ grouped_gemm_kernel(const GemmParams P) {
                     }
                 }
             }
-            if (P.scale_words) {
+            if (scale_words) {
                 const uint32_t base_b = ((kt * KT >> P.lg_gs) * ES) & ~3u;
                 for (uint32_t i = 0; i < nsw; i++) {
                     const uint32_t o = base_b + 4u * i;
@@ -769,6 +794,7 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.raw16 = a.kind != K_CB3 && a.row_bytes % 16u == 0;
     P.out_dtype = a.out_dtype;
     P.bias = a.bias; P.bias_dtype = a.bias_dtype;
+    P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
     P.timeout_ns = WAIT_NS;
     const uint32_t nm = (a.n + BM - 1) / BM;
     return launch_kind(P, pl, a.kind, a.x_dtype, nm, max_tiles, st);

@@ -99,7 +99,7 @@ def test_pointer_table_entry_rejects_before_cuda():
     assert call(packed=0) == 1
     assert call(scales=0) == 1
     assert call(biases=0) == 1                    # affine biases come from the table
-    assert call(path=2) == 2                      # the grouped path is not offered
+    assert call(path=7) == 1                      # unknown path
 
 
 def test_route_invalid_arguments():
