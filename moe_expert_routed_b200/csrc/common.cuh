@@ -85,6 +85,5 @@ __device__ __forceinline__ void store_out(void *out, int dt, size_t idx, float v
     }
 }
 
-__device__ __forceinline__ uint32_t out_elem_bytes(int dt) { return dt == DT_F32 ? 4u : 2u; }
 
 }  // namespace moe

@@ -305,7 +305,10 @@ struct GemmCfg {
 
 // Tiles of 64 pairs (few pairs per expert, dequantisation-bound) run two CTAs
 // per SM: two pipeline stages each, registers capped for two CTAs.
-template <int KIND, int XT, int BN>
+// PTRS: weights from the pointer tables (decided at compile time so that the
+// contiguous case keeps its copy-width and scale-staging branches on kernel
+// parameters).
+template <int KIND, int XT, int BN, bool PTRS>
 __global__ void __launch_bounds__(GEMM_THREADS, BN == 64 ? 2 : 1)
 grouped_gemm_kernel(const GemmParams P) {
     using C = GemmCfg<KIND, XT, BN>;
@@ -341,8 +344,8 @@ grouped_gemm_kernel(const GemmParams P) {
     const uint8_t *wb = P.packed + (size_t)e * P.n * P.row_bytes;
     const uint8_t *sb = (const uint8_t *)P.scales + (size_t)e * P.n * P.groups * ES;
     const uint8_t *bb = (const uint8_t *)P.aux + (size_t)e * P.n * P.groups * 2u;
-    bool scale_words = P.scale_words != 0, raw16 = P.raw16 != 0;
-    if (P.packed_ptrs) {
+    bool ptr_scale_words = false, ptr_raw16 = false;
+    if constexpr (PTRS) {
         wb = (const uint8_t *)__ldg(P.packed_ptrs + e);
         if (!wb) return;  // expert held elsewhere: its pairs' rows are not ours to write (uniform)
         sb = (const uint8_t *)__ldg(P.scale_ptrs + e);
@@ -355,8 +358,8 @@ grouped_gemm_kernel(const GemmParams P) {
             if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(P.err, ERR_BAD_POINTER);
             return;
         }
-        raw16 = raw16 && (uintptr_t)wb % 16u == 0;
-        scale_words = scale_words && sal % 4u == 0 && (uintptr_t)sb % 4u == 0;
+        ptr_raw16 = P.raw16 != 0 && (uintptr_t)wb % 16u == 0;
+        ptr_scale_words = P.scale_words != 0 && sal % 4u == 0 && (uintptr_t)sb % 4u == 0;
     }
 
     const uint32_t base = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -461,7 +464,7 @@ grouped_gemm_kernel(const GemmParams P) {
             if constexpr (KIND == K_NVFP4) {
                 // groups of 16: this half's two E4M3 scales, converted together (exact in f16)
                 __half2 s01;
-                if (scale_words) {
+                if (PTRS ? ptr_scale_words : P.scale_words != 0) {
                     // the staged word holds groups 4kt .. 4kt+3; this half's are bytes 2h, 2h+1
                     s01 = e4m3x2_to_half2((*(const uint32_t *)(rr + RL::SC) >> (16u * h)) & 0xFFFFu);
                 } else {
@@ -473,7 +476,7 @@ grouped_gemm_kernel(const GemmParams P) {
                 nvfp4_store<F16>(w, s01, st, r, h * 4u);
             } else {
                 float s0, b0, s1 = 0.f, b1 = 0.f;
-                if (scale_words) {
+                if (PTRS ? ptr_scale_words : P.scale_words != 0) {
                     const uint4 q = *(const uint4 *)(rr + RL::SC);
                     const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
                     const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
@@ -568,7 +571,7 @@ grouped_gemm_kernel(const GemmParams P) {
                 }
             } else {
                 constexpr uint32_t RB = RL::RB;
-                if (raw16) {
+                if (PTRS ? ptr_raw16 : P.raw16 != 0) {
                     constexpr uint32_t NC = RB / 16u;
 #pragma unroll
                     for (uint32_t i = 0; i < NC; i++) {
@@ -590,7 +593,7 @@ grouped_gemm_kernel(const GemmParams P) {
                     }
                 }
             }
-            if (scale_words) {
+            if (PTRS ? ptr_scale_words : P.scale_words != 0) {
                 const uint32_t base_b = ((kt * KT >> P.lg_gs) * ES) & ~3u;
                 for (uint32_t i = 0; i < nsw; i++) {
                     const uint32_t o = base_b + 4u * i;
@@ -705,18 +708,25 @@ bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
     return true;
 }
 
-template <int KIND, int XT, int BN>
-cudaError_t launch_t(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
-                     cudaStream_t st) {
+template <int KIND, int XT, int BN, bool PTRS>
+cudaError_t launch_tp(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
+                      cudaStream_t st) {
     GemmParams P = P0;
     P.stages = (uint32_t)pl.stages;
-    auto kern = grouped_gemm_kernel<KIND, XT, BN>;
+    auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS>;
     static int smem_set[64];
     cudaError_t e = ensure_dyn_smem(kern, pl.smem, smem_set);
     if (e != cudaSuccess) return e;
     dim3 grid(n_mtiles, max_tiles);
     kern<<<grid, GEMM_THREADS, pl.smem, st>>>(P);
     return cudaGetLastError();
+}
+
+template <int KIND, int XT, int BN>
+cudaError_t launch_t(const GemmParams &P, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
+                     cudaStream_t st) {
+    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true>(P, pl, n_mtiles, max_tiles, st);
+    return launch_tp<KIND, XT, BN, false>(P, pl, n_mtiles, max_tiles, st);
 }
 
 template <int KIND>
