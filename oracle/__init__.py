@@ -69,6 +69,10 @@ def lib():
         L.oracle_route.argtypes = [ctypes.c_void_p, u64, u32, u32, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, u64]
         L.oracle_route.restype = ctypes.c_int64
+        L.oracle_act.argtypes = [i32, ctypes.c_double]
+        L.oracle_act.restype = ctypes.c_double
+        L.oracle_glu_elems.argtypes = [ctypes.c_void_p] * 2 + [u64, i32, ctypes.c_void_p]
+        L.oracle_glu_elems.restype = None
         del u8p, u16p, u32p, dp, vp
         _lib = L
     return _lib
@@ -175,6 +179,34 @@ def add_expert_bias(vals: np.ndarray, P, bias: np.ndarray, bias_dtype: int, pair
                                  _ptr(cols) if cols is not None else None, vals.size, _ptr(ids),
                                  _ptr(bias), bias_dtype, P.n, P.num_experts)
     return vals
+
+
+ACT_SILU, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
+
+
+def act(code: int, g: float) -> float:
+    """Activation of the gated output in double (0 SiLU, 1 GELU tanh form, 2 GELU erf form)."""
+    return lib().oracle_act(int(code), float(g))
+
+
+def glu_elems(gate: np.ndarray, up: np.ndarray, code: int) -> np.ndarray:
+    """act(gate) * up elementwise, double."""
+    gate = np.ascontiguousarray(gate, dtype=np.float64)
+    up = np.ascontiguousarray(up, dtype=np.float64)
+    assert gate.shape == up.shape
+    out = np.empty(gate.shape, dtype=np.float64)
+    lib().oracle_glu_elems(_ptr(gate), _ptr(up), gate.size, int(code), _ptr(out))
+    return out
+
+
+def glu(vals: np.ndarray, code: int) -> np.ndarray:
+    """Gated output of full results vals [R, n] (double, bias already added): rows
+    [0, n/2) of an expert are the gate, [n/2, n) the up projection; returns
+    act(gate) * up, [R, n/2] double."""
+    R, n = vals.shape
+    assert n % 2 == 0
+    nh = n // 2
+    return glu_elems(vals[:, :nh], vals[:, nh:], code)
 
 
 def expert_max_abs_weight(P, e: int) -> float:

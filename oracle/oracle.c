@@ -41,6 +41,12 @@
  * "y + mx.expand_dims(bias[indices], -2)"): oracle_add_expert_bias adds
  * bias[e][col] to the double result of every pair with a valid id, before the
  * single rounding to the output type; rows of out-of-range ids stay zero.
+ *
+ * Gated output (spark_model helpers_a.rs, MoeLayer: the fused gate+up kernel
+ * with SiLU, or GELU for GeGLU experts after set_gelu_activation): with rows
+ * [0, n/2) of each expert the gate and rows [n/2, n) the up projection,
+ * oracle_glu_elems forms act(gate) * up in double from the double results
+ * (bias already added), before the single rounding.
  */
 #include <math.h>
 #include <pthread.h>
@@ -379,4 +385,19 @@ void oracle_add_expert_bias(double *vals, const uint32_t *pairs, const uint32_t 
         const uint32_t e = ids[p];
         if (e < num_experts) vals[i] += x_at(bias, bias_dtype, (uint64_t)e * n + col);
     }
+}
+
+/* act(g) in double: 0 SiLU, g / (1 + e^-g); 1 GELU in its tanh form,
+ * g/2 (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))); 2 GELU in its erf form,
+ * g/2 (1 + erf(g / sqrt(2))) = g * Phi(g). Other codes return NAN. */
+double oracle_act(int act, double g) {
+    if (act == 0) return g / (1.0 + exp(-g));
+    if (act == 1) return 0.5 * g * (1.0 + tanh(sqrt(2.0 / 3.14159265358979323846) * (g + 0.044715 * g * g * g)));
+    if (act == 2) return 0.5 * g * (1.0 + erf(g / sqrt(2.0)));
+    return NAN;
+}
+
+/* out[i] = act(gate[i]) * up[i] for i < count. */
+void oracle_glu_elems(const double *gate, const double *up, uint64_t count, int act, double *out) {
+    for (uint64_t i = 0; i < count; i++) out[i] = oracle_act(act, gate[i]) * up[i];
 }
