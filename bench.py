@@ -195,37 +195,40 @@ class DecodeWorkload:
                                    .view(np.int16)).view(torch.bfloat16).cuda() for P in self.projs]
         self.out = [torch.empty((self.G, 8, P.n), dtype=torch.float32, device="cuda")
                     for P in self.projs]
+        # gated gate/up output: act(gate) * up, n/2 columns
+        self.out_glu = torch.empty((self.G, 8, self.projs[0].n // 2), dtype=torch.float32, device="cuda")
         self.ws = [M.new_workspace(1, 8, P.num_experts) for P in self.projs]
         self.step_bytes = [
             [alg_bytes(P, self.ids[i][s].cpu().numpy().view(np.uint32)) for s in range(self.G)]
             for i, P in enumerate(self.projs)]
 
-    def call(self, proj: int, s: int):
+    def call(self, proj: int, s: int, act=None):
         P = self.projs[proj]
         L = self.layers[proj][s % N_LAYERS]
         self.M.qmm_id(self.x[proj][s:s + 1], self.ids[proj][s:s + 1], L["packed"], L["scales"],
                       L["aux"], n=P.n, group_size=P.group_size, bits=P.bits, fmt=P.fmt,
-                      num_experts=P.num_experts, out=self.out[proj][s], workspace=self.ws[proj])
+                      num_experts=P.num_experts, out=self.out_glu[s] if act else self.out[proj][s],
+                      workspace=self.ws[proj], act=act)
 
-    def step(self, s: int, projs=(0, 1)):
+    def step(self, s: int, projs=(0, 1), act=None):
         for p in projs:
-            self.call(p, s)
+            self.call(p, s, act)
 
     def bytes(self, projs=(0, 1)) -> float:
         return sum(sum(self.step_bytes[p]) for p in projs)
 
-    def capture(self, projs=(0, 1)):
+    def capture(self, projs=(0, 1), act=None):
         g = torch.cuda.CUDAGraph()
         st = torch.cuda.Stream()
         st.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(st):
             for s in range(min(self.G, 4)):
-                self.step(s, projs)  # warm the launch path outside capture
+                self.step(s, projs, act)  # warm the launch path outside capture
         torch.cuda.current_stream().wait_stream(st)
         torch.cuda.synchronize()
         with torch.cuda.graph(g):
             for s in range(self.G):
-                self.step(s, projs)
+                self.step(s, projs, act)
         torch.cuda.synchronize()
         return g
 
@@ -399,6 +402,15 @@ def run_ours(args, dist: Dist):
         per_call[name] = {"us_per_call": t / (max(1, replays // 2) * G) * 1e6,
                           "GB_per_s": W.bytes((p,)) * max(1, replays // 2) / t / 1e9}
         del gp
+    # the gate/up projection with its SiLU-gated epilogue (moe_qmm_id_glu): same
+    # weights and x, half the output columns
+    gp = W.capture(projs=(0,), act="silu")
+    gp.replay()
+    t = time_graph(gp, max(1, replays // 2))
+    glu_bytes = W.bytes((0,)) - G * 8 * (W.projs[0].n // 2) * 4
+    per_call["gate_up_silu"] = {"us_per_call": t / (max(1, replays // 2) * G) * 1e6,
+                                "GB_per_s": glu_bytes * max(1, replays // 2) / t / 1e9}
+    del gp
 
     pk = peaks()
     # dominant kernel: the gate/up launch (about 57% of the step); timed alone from a

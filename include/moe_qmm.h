@@ -169,6 +169,40 @@ moe_status moe_qmm_id_ptrs(const void *x, const uint32_t *ids, const uint64_t *p
                            uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
                            void *workspace, size_t workspace_bytes, moe_stream_t stream, moe_path path);
 
+/* Activation of a gated (GLU) output; see moe_qmm_id_glu. */
+typedef enum {
+    MOE_ACT_SILU = 0,      /* act(g) = g / (1 + exp(-g))                                  */
+    MOE_ACT_GELU_TANH = 1, /* act(g) = g/2 (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))      */
+    MOE_ACT_GELU_ERF = 2   /* act(g) = g/2 (1 + erf(g / sqrt(2)))                          */
+} moe_act;
+
+/*
+ * moe_qmm_id_glu -- the fused gate+up projection of a gated MoE MLP: moe_qmm_id
+ * over experts whose n weight rows hold the gate projection in rows [0, n/2) and
+ * the up projection in rows [n/2, n), with the activation applied in the
+ * epilogue (spark_model helpers_a.rs, MoeLayer: the fused gate+up kernel, SiLU
+ * by default and GELU for GeGLU experts via set_gelu_activation):
+ *
+ *     y[p][r]   = sum_j dequant(W[e][r][j]) x[t][j] (+ expert_bias[e][r])
+ *     out[p][c] = act(y[p][c]) * y[p][n/2 + c],   c < n/2
+ *
+ *   n            rows per expert; must be even (MOE_ERR_INVALID_ARGUMENT otherwise).
+ *   out          [m, n_expert_used, n/2] of out_dtype; every element is written
+ *                (zeros for out-of-range ids).
+ *   expert_bias  [num_experts, n] in bias_dtype, or NULL for none; added to gate and
+ *                up before the activation.
+ *   act          a moe_act (MOE_ERR_INVALID_ARGUMENT for other values).
+ * y is the fp32 accumulator; act(gate) * up is formed in fp32 and rounded once to
+ * out_dtype. Storage, other arguments, paths, ownership and errors as
+ * moe_qmm_id_path / moe_qmm_id_bias.
+ */
+moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                          const void *aux, const void *expert_bias, void *out, uint32_t m, uint32_t k,
+                          uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                          uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                          moe_dtype out_dtype, moe_dtype bias_dtype, moe_act act, void *workspace,
+                          size_t workspace_bytes, moe_stream_t stream, moe_path path);
+
 /* Workspace bytes moe_qmm_id needs for these sizes (any path). Returns 0 if the
  * sizes overflow. */
 size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t num_experts);

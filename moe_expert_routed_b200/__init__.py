@@ -25,6 +25,8 @@ FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4 = 0, 1, 2
 DT_F32, DT_BF16, DT_F16 = 0, 1, 2
 PATH_AUTO, PATH_DECODE, PATH_GROUPED = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "grouped": PATH_GROUPED}
+ACT_SILU, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
+ACTS = {"silu": ACT_SILU, "gelu_tanh": ACT_GELU_TANH, "gelu_erf": ACT_GELU_ERF}
 
 MOE_OK = 0
 STATUS_NAMES = {
@@ -61,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.moe_qmm_id_bias.restype = i32
         L.moe_qmm_id_ptrs.argtypes = [vp] * 7 + [u32] * 5 + [i32, u32, u32, i32, i32, vp, sz, vp, i32]
         L.moe_qmm_id_ptrs.restype = i32
+        L.moe_qmm_id_glu.argtypes = [vp] * 7 + [u32] * 5 + [i32, u32, u32, i32, i32, i32, i32, vp, sz, vp, i32]
+        L.moe_qmm_id_glu.restype = i32
         L.moe_qmm_id_path.restype = i32
         L.moe_qmm_id_workspace_bytes.argtypes = [u32, u32, u32]
         L.moe_qmm_id_workspace_bytes.restype = sz
@@ -125,7 +129,7 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
            aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
            out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
            workspace: torch.Tensor | None = None, path: str = "auto",
-           expert_bias: torch.Tensor | None = None) -> torch.Tensor:
+           expert_bias: torch.Tensor | None = None, act: str | None = None) -> torch.Tensor:
     """Expert-routed quantized matmul on the current CUDA stream.
 
     x [m, k] (f32 / bf16 / f16); ids [m, n_expert_used] int32/uint32; packed, scales,
@@ -133,7 +137,10 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
     [m, n_expert_used, n]. Buffer-size checks and their messages follow
     mlx-native quantized_matmul_id.rs (quantized_matmul_id). expert_bias, if given,
     is a [num_experts, n] f32 / bf16 / f16 tensor added to every pair's row of its
-    expert (moe_qmm_id_bias).
+    expert (moe_qmm_id_bias). act ("silu", "gelu_tanh" or "gelu_erf") makes it the
+    fused gate+up projection (moe_qmm_id_glu): rows [0, n/2) of each expert are the
+    gate, rows [n/2, n) the up projection, and out [m, n_expert_used, n/2] holds
+    act(gate) * up.
     """
     device = x.device
     for t, name in ((x, "input"), (ids, "ids"), (packed, "weight"), (scales, "scales"),
@@ -176,26 +183,41 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
     if _nbytes(aux) < aux_need:
         raise ValueError(f"quantized_matmul_id: {aux_name} buffer too small: expected at least "
                          f"{aux_need} bytes, got {_nbytes(aux)}")
+    if act is not None:
+        if act not in ACTS:
+            raise ValueError(f"quantized_matmul_id: unknown activation {act!r} (one of {sorted(ACTS)})")
+        if n % 2:
+            raise ValueError("quantized_matmul_id: a gated output needs an even N (gate and up halves)")
+    out_n = n // 2 if act is not None else n
     if out is None:
-        out = torch.empty((m, n_expert_used, n), dtype=out_dtype, device=device)
+        out = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
     else:
         _check_dev(out, "out", device)
-        if out.dtype not in _TORCH_DT or out.numel() < m * n_expert_used * n:
-            raise ValueError("quantized_matmul_id: out must hold [M, n_expert_used, N] f32/bf16/f16")
+        if out.dtype not in _TORCH_DT or out.numel() < m * n_expert_used * out_n:
+            raise ValueError("quantized_matmul_id: out must hold [M, n_expert_used, N] f32/bf16/f16 "
+                             "(N/2 columns with a gated output)")
     if workspace is None:
         workspace = new_workspace(m, n_expert_used, num_experts, device)
     else:
         _check_dev(workspace, "workspace", device)
-    if expert_bias is None:
+    if expert_bias is not None:
+        _check_dev(expert_bias, "expert_bias", device)
+        if expert_bias.dtype not in _TORCH_DT or expert_bias.numel() < num_experts * n:
+            raise ValueError("quantized_matmul_id: expert_bias must hold [num_experts, N] f32/bf16/f16")
+    if act is not None:
+        st = lib().moe_qmm_id_glu(
+            x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
+            expert_bias.data_ptr() if expert_bias is not None else None, out.data_ptr(), m, k, n,
+            group_size, bits, fmt, n_expert_used, num_experts, _TORCH_DT[x.dtype], _TORCH_DT[out.dtype],
+            _TORCH_DT[expert_bias.dtype] if expert_bias is not None else 0, ACTS[act],
+            workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), _PATHS[path])
+    elif expert_bias is None:
         st = lib().moe_qmm_id_path(
             x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
             out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used, num_experts,
             _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], workspace.data_ptr(), _nbytes(workspace),
             _stream_ptr(device), _PATHS[path])
     else:
-        _check_dev(expert_bias, "expert_bias", device)
-        if expert_bias.dtype not in _TORCH_DT or expert_bias.numel() < num_experts * n:
-            raise ValueError("quantized_matmul_id: expert_bias must hold [num_experts, N] f32/bf16/f16")
         st = lib().moe_qmm_id_bias(
             x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
             expert_bias.data_ptr(), out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used,

@@ -112,13 +112,13 @@ struct PtrTables {
     const uint64_t *packed, *scales, *biases;
 };
 
-// moe_qmm_id with an optional per-expert output bias (null: none) and optional
-// pointer-table weights.
+// moe_qmm_id with an optional per-expert output bias (null: none), optional
+// pointer-table weights and an optional gated output (act >= 0: act(gate) * up).
 moe_status run(const void *x, const uint32_t *ids, const void *packed, const void *scales, const void *aux,
                const void *bias, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
                uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace, size_t workspace_bytes,
-               moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}) {
+               moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}, int act = -1) {
     moe_status v = validate(x, ids, pt.packed ? (const void *)pt.packed : packed,
                             pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
                             fmt, n_expert_used, num_experts, x_dtype, out_dtype);
@@ -143,6 +143,8 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     a.packed_ptrs = pt.packed;
     a.scale_ptrs = pt.scales;
     a.bias_ptrs = pt.biases;
+    a.act = act;
+    a.out_n = act >= 0 ? n / 2u : n;
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);
@@ -178,7 +180,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         const uint32_t max_tiles = (uint32_t)(R / tile_rows + num_experts + 1);
         ce = launch_route(ids, (uint32_t)R, num_experts, tile_rows, counts, offsets, sp, tiles, tc,
                           max_tiles, (uint32_t *)(ws + L.chunk_hist),
-                          (uint32_t *)(ws + L.chunk_base), L.chunks, err, out, n, (int)out_dtype,
+                          (uint32_t *)(ws + L.chunk_base), L.chunks, err, out, a.out_n, (int)out_dtype,
                           st);
         if (ce == cudaSuccess) {
             if (choice == GROUPED)
@@ -227,6 +229,19 @@ moe_status moe_qmm_id_ptrs(const void *x, const uint32_t *ids, const uint64_t *p
     return run(x, ids, nullptr, nullptr, aux_arg, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
                num_experts, x_dtype, out_dtype, MOE_F32, workspace, workspace_bytes, stream, path,
                PtrTables{packed_ptrs, scale_ptrs, bias_ptrs});
+}
+
+moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                          const void *aux, const void *expert_bias, void *out, uint32_t m, uint32_t k,
+                          uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
+                          uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
+                          moe_dtype out_dtype, moe_dtype bias_dtype, moe_act act, void *workspace,
+                          size_t workspace_bytes, moe_stream_t stream, moe_path path) {
+    if ((int)act < 0 || (int)act > 2 || (n & 1u)) return MOE_ERR_INVALID_ARGUMENT;
+    if (expert_bias && ((int)bias_dtype < 0 || (int)bias_dtype > 2)) return MOE_ERR_INVALID_ARGUMENT;
+    return run(x, ids, packed, scales, aux, expert_bias, out, m, k, n, group_size, bits, fmt, n_expert_used,
+               num_experts, x_dtype, out_dtype, expert_bias ? bias_dtype : MOE_F32, workspace, workspace_bytes,
+               stream, path, PtrTables{nullptr, nullptr, nullptr}, (int)act);
 }
 
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,

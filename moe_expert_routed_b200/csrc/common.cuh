@@ -85,5 +85,25 @@ __device__ __forceinline__ void store_out(void *out, int dt, size_t idx, float v
     }
 }
 
+// ------------------------------------------------ gated (GLU) output epilogue
+//
+// The fused gate+up projection (spark_model helpers_a.rs, MoeLayer: the fused
+// gate+up kernel with SiLU, or GELU for GeGLU experts via set_gelu_activation):
+// with n weight rows per expert, rows [0, n/2) are the gate and rows [n/2, n)
+// the up projection, and the output element j of a pair is act(gate_j) * up_j.
+// The kernels walk "logical" rows in which gate and up rows alternate, so that
+// both halves of an output land next to each other: logical row L is weight row
+// L/2 (L even, gate) or n/2 + L/2 (L odd, up). nh = n/2, or 0 without GLU.
+__host__ __device__ __forceinline__ uint32_t glu_row(uint32_t L, uint32_t nh) {
+    return nh ? ((L & 1u) ? nh + (L >> 1) : (L >> 1)) : L;
+}
+
+// act(g) in fp32: 0 SiLU g / (1 + e^-g); 1 GELU, tanh form
+// g/2 (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))); 2 GELU, erf form g/2 (1 + erf(g / sqrt 2)).
+__device__ __forceinline__ float glu_act(int act, float g) {
+    if (act == 0) return g / (1.f + expf(-g));
+    if (act == 1) return 0.5f * g * (1.f + tanhf(0.7978845608f * fmaf(0.044715f * g * g, g, g)));
+    return 0.5f * g * (1.f + erff(g * 0.70710678f));
+}
 
 }  // namespace moe

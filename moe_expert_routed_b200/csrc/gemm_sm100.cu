@@ -75,6 +75,10 @@ struct GemmParams {
     const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;
     int out_dtype;
     uint64_t timeout_ns;
+    // gated output (0: plain): tile rows alternate gate and up weight rows (glu_row),
+    // and the epilogue writes act(gate) * up into rows of glu_nh = n/2 columns
+    uint32_t glu_nh;
+    int act;
 };
 
 template <int KIND> constexpr int a_terms() { return KIND == K_NVFP4 ? 1 : 2; }
@@ -307,8 +311,9 @@ struct GemmCfg {
 // per SM: two pipeline stages each, registers capped for two CTAs.
 // PTRS: weights from the pointer tables (decided at compile time so that the
 // contiguous case keeps its copy-width and scale-staging branches on kernel
-// parameters).
-template <int KIND, int XT, int BN, bool PTRS>
+// parameters). GLU: gated output (glu_row order, act(gate) * up epilogue), also
+// decided at compile time so that the plain kernels carry none of it.
+template <int KIND, int XT, int BN, bool PTRS, bool GLU>
 __global__ void __launch_bounds__(GEMM_THREADS, BN == 64 ? 2 : 1)
 grouped_gemm_kernel(const GemmParams P) {
     using C = GemmCfg<KIND, XT, BN>;
@@ -399,7 +404,7 @@ grouped_gemm_kernel(const GemmParams P) {
     if (warp < LD_WARP0) {
         // -------------------------------------------------------- dequantisers
         const uint32_t r = tid & (BM - 1), h = tid >> 7;
-        const size_t row_in = tmin<uint32_t>(row0 + r, P.n - 1);  // row within the expert
+        const size_t row_in = glu_row(tmin<uint32_t>(row0 + r, P.n - 1), GLU ? P.glu_nh : 0u);  // row within the expert
         const uint8_t *srow = sb + row_in * P.groups * ES;
         const uint8_t *brow = bb + row_in * P.groups * 2u;
         bool ok = true;
@@ -495,15 +500,27 @@ grouped_gemm_kernel(const GemmParams P) {
         if (ok && ptx::mbar_wait_bounded(accb, 0, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns)) {
             ptx::tc_fence_after();
             const uint32_t q = warp & 3u, ch = warp >> 2;
-            const uint32_t grow_e = row0 + q * 32u + lane;
+            const uint32_t grow_e = row0 + q * 32u + lane;  // logical row
+            const uint32_t nh = GLU ? P.glu_nh : 0u;
             const float s2 = (KIND == K_NVFP4) ? __ldg((const float *)P.aux + e) : 1.f;
-            const float bv = grow_e < P.n ? load_bias(P.bias, P.bias_dtype, (size_t)e * P.n + grow_e) : 0.f;
+            const float bv = grow_e < P.n ? load_bias(P.bias, P.bias_dtype, (size_t)e * P.n + glu_row(grow_e, nh)) : 0.f;
             const uint32_t c_begin = ch * (BN / 2), c_end = tmin<uint32_t>(c_begin + BN / 2, nt);
             for (uint32_t c0 = c_begin; c0 < c_end; c0 += 16) {
                 uint32_t v[16];
                 ptx::tmem_ld16(tmem + ((q * 32u) << 16) + c0, v);
                 ptx::tmem_wait_ld();
-                if (grow_e < P.n) {
+                if constexpr (GLU) {
+                    // even lanes hold gate rows, the next lane the matching up row
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const float y = __uint_as_float(v[i]) * s2 + bv;
+                        const float up = __shfl_xor_sync(0xFFFFFFFFu, y, 1);
+                        const uint32_t col = c0 + i;
+                        if (col < c_end && grow_e < P.n && !(lane & 1u))
+                            store_out(P.out, P.out_dtype, (size_t)pairs_s[col] * nh + (grow_e >> 1),
+                                      glu_act(P.act, y) * up);
+                    }
+                } else if (grow_e < P.n) {
 #pragma unroll
                     for (int i = 0; i < 16; i++) {
                         const uint32_t col = c0 + i;
@@ -533,7 +550,7 @@ grouped_gemm_kernel(const GemmParams P) {
         const uint8_t *ebase = wb;
         const uint32_t nlast = P.n - 1;
         // scale words: thread lt stages those of weight row lt
-        const size_t srow_in = tmin<uint32_t>(row0 + lt, nlast);
+        const size_t srow_in = glu_row(tmin<uint32_t>(row0 + lt, nlast), GLU ? P.glu_nh : 0u);
         const uint8_t *srow = sb + srow_in * P.groups * ES;
         const uint8_t *brow = bb + srow_in * P.groups * 2u;
         const uint32_t srow_bytes = P.groups * ES;
@@ -564,7 +581,7 @@ grouped_gemm_kernel(const GemmParams P) {
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
                     const uint32_t q = lt + NLD * i, row = q >> 3, c = q & 7u;
-                    const uint8_t *rp = ebase + (size_t)tmin<uint32_t>(row0 + row, nlast) * P.row_bytes;
+                    const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
                     const uint32_t o = (w0 + c) * 4u;
                     const bool in = o + 4u <= P.row_bytes;
                     ptx::cp_async_4(raw + row * RL::STRIDE + 4u * c, rp + (in ? o : 0u), in ? 4u : 0u);
@@ -576,7 +593,7 @@ grouped_gemm_kernel(const GemmParams P) {
 #pragma unroll
                     for (uint32_t i = 0; i < NC; i++) {
                         const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
-                        const uint8_t *rp = ebase + (size_t)tmin<uint32_t>(row0 + row, nlast) * P.row_bytes;
+                        const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
                         const uint32_t o = kt * RB + 16u * c;
                         const bool in = o < P.row_bytes;
                         ptx::cp_async_16(raw + row * RL::STRIDE + 16u * c, rp + (in ? o : 0u), in ? 16u : 0u);
@@ -586,7 +603,7 @@ grouped_gemm_kernel(const GemmParams P) {
 #pragma unroll
                     for (uint32_t i = 0; i < NC; i++) {
                         const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
-                        const uint8_t *rp = ebase + (size_t)tmin<uint32_t>(row0 + row, nlast) * P.row_bytes;
+                        const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
                         const uint32_t o = kt * RB + 8u * c;
                         const bool in = o < P.row_bytes;
                         ptx::cp_async_8(raw + row * RL::STRIDE + 8u * c, rp + (in ? o : 0u), in ? 8u : 0u);
@@ -708,12 +725,12 @@ bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
     return true;
 }
 
-template <int KIND, int XT, int BN, bool PTRS>
+template <int KIND, int XT, int BN, bool PTRS, bool GLU>
 cudaError_t launch_tp(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
                       cudaStream_t st) {
     GemmParams P = P0;
     P.stages = (uint32_t)pl.stages;
-    auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS>;
+    auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS, GLU>;
     static int smem_set[64];
     cudaError_t e = ensure_dyn_smem(kern, pl.smem, smem_set);
     if (e != cudaSuccess) return e;
@@ -725,8 +742,9 @@ cudaError_t launch_tp(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtile
 template <int KIND, int XT, int BN>
 cudaError_t launch_t(const GemmParams &P, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
                      cudaStream_t st) {
-    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true>(P, pl, n_mtiles, max_tiles, st);
-    return launch_tp<KIND, XT, BN, false>(P, pl, n_mtiles, max_tiles, st);
+    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true, false>(P, pl, n_mtiles, max_tiles, st);
+    if (P.glu_nh) return launch_tp<KIND, XT, BN, false, true>(P, pl, n_mtiles, max_tiles, st);
+    return launch_tp<KIND, XT, BN, false, false>(P, pl, n_mtiles, max_tiles, st);
 }
 
 template <int KIND>
@@ -806,6 +824,8 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.bias = a.bias; P.bias_dtype = a.bias_dtype;
     P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
     P.timeout_ns = WAIT_NS;
+    P.glu_nh = a.act >= 0 ? a.n / 2u : 0u;
+    P.act = a.act;
     const uint32_t nm = (a.n + BM - 1) / BM;
     return launch_kind(P, pl, a.kind, a.x_dtype, nm, max_tiles, st);
 }

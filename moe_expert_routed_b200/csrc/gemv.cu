@@ -182,9 +182,9 @@ gemv_kernel(const GemvParams P) {
 
     const uint32_t warp = tid >> 5, lane = tid & 31u;
     const uint32_t rsub = lane / GEMV_LPR, l8 = lane % GEMV_LPR;
-    const uint32_t row = row0 + warp * (32 / GEMV_LPR) + rsub;
+    const uint32_t row = row0 + warp * (32 / GEMV_LPR) + rsub;  // logical row (glu_row)
     const bool row_ok = row < P.n;
-    const uint32_t row_c = row_ok ? row : P.n - 1;  // clamp: loads stay in bounds
+    const uint32_t row_c = glu_row(row_ok ? row : P.n - 1, P.glu_nh);  // weight row; clamped loads stay in bounds
     constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
     // the expert's packed rows, scales and (affine) biases: slices of the contiguous
     // arrays, or the expert's own buffers from the pointer tables
@@ -278,12 +278,22 @@ gemv_kernel(const GemvParams P) {
 #pragma unroll
             for (int d = GEMV_LPR / 2; d > 0; d >>= 1) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], d);
         }
-        if (l8 == 0 && row_ok) {
+        const float bv = load_bias(P.bias, P.bias_dtype, (size_t)expert * P.n + row_c);
+        if (P.glu_nh) {
+            // gate rows sit in even row slots, the matching up row GEMV_LPR lanes further on
+#pragma unroll
+            for (int q = 0; q < NPB; q++) {
+                const float y = acc[q] * s2 + bv;
+                const float up = __shfl_xor_sync(0xFFFFFFFFu, y, GEMV_LPR);
+                if (l8 == 0 && row_ok && !(rsub & 1u) && (uint32_t)q < np)
+                    store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.glu_nh + (row >> 1),
+                              glu_act(P.act, y) * up);
+            }
+        } else if (l8 == 0 && row_ok) {
 #pragma unroll
             for (int q = 0; q < NPB; q++)
                 if ((uint32_t)q < np)
-                    store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row,
-                              acc[q] * s2 + load_bias(P.bias, P.bias_dtype, (size_t)expert * P.n + row));
+                    store_out(P.out, P.out_dtype, (size_t)pairs_s[q] * P.n + row, acc[q] * s2 + bv);
         }
     }
 }
@@ -892,10 +902,11 @@ __device__ __forceinline__ float dp4a_unit_reg(const uint4 w, const uint4 (&v)[6
     return fmaf(s, d * usc, fmaf(b, usm, acc));
 }
 
-template <int LPR, int UPL>
+template <int LPR, int UPL, bool GLU>
 __global__ void __launch_bounds__(ROWS_THREADS, 2)
 gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     constexpr uint32_t RPI = 32 / LPR;  // rows a warp works on at once
+    constexpr uint32_t AREAS = GLU ? 2u : 1u;
     constexpr uint64_t WAIT = 1000000000ull;
     extern __shared__ __align__(128) uint8_t dsm8[];
     __shared__ uint32_t ex_s[ROWS_MAX_PAIRS];
@@ -904,13 +915,15 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     __shared__ int abort_s;
 
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-    const uint32_t n = P.n, nu = P.n_units, G = P.groups, rbytes = P.row_bytes;
-    const uint32_t total_rows = P.R * n;
+    // nn: rows of the walk per pair (with GLU one row of the walk is an output
+    // element: gate row c in the first shared-memory area, up row n/2 + c in the second)
+    const uint32_t n = P.n, nn = GLU ? P.glu_nh : n, nu = P.n_units, G = P.groups, rbytes = P.row_bytes;
+    const uint32_t total_rows = P.R * nn;
     const uint32_t g0 = blockIdx.x * rows_per_cta;
     const uint32_t nrows = tmin<uint32_t>(rows_per_cta, total_rows - g0);
-    const uint32_t p_first = g0 / n, p_last = (g0 + nrows - 1u) / n;
+    const uint32_t p_first = g0 / nn, p_last = (g0 + nrows - 1u) / nn;
     const uint32_t xsz = P.x_dtype == DT_F32 ? 4u : 2u;
-    const RowsLayout L = rows_layout(rows_per_cta, rbytes, P.k * xsz, nu, G);
+    const RowsLayout L = rows_layout(AREAS * rows_per_cta, rbytes, P.k * xsz, nu, G);
     const uint32_t sbase = ptx::smem_u32(dsm8);
     volatile int *abort_flag = &abort_s;
 
@@ -930,62 +943,68 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
         ptx::mbar_arrive_expect_tx(bx, P.k * xsz);
         ptx::bulk_g2s(sbase + L.xraw, P.x, P.k * xsz, bx);
     }
-    // scales and biases of the CTA's rows: one bulk copy of each per pair when aligned
+    // scales and biases of the CTA's rows: one bulk copy of each per pair and area when aligned
     const bool s_bulk = P.s_bulk != 0;
     if (s_bulk) {
         if (tid == 0) {
             uint32_t bytes = 0;
             for (uint32_t p = p_first; p <= p_last; p++) {
-                const uint32_t lo = p == p_first ? g0 - p * n : 0u;
-                const uint32_t hi = p == p_last ? g0 + nrows - p * n : n;
-                if (ex_s[p - p_first] < P.num_experts) bytes += 2u * (hi - lo) * G * 2u;
+                const uint32_t lo = p == p_first ? g0 - p * nn : 0u;
+                const uint32_t hi = p == p_last ? g0 + nrows - p * nn : nn;
+                if (ex_s[p - p_first] < P.num_experts) bytes += AREAS * 2u * (hi - lo) * G * 2u;
             }
             ptx::mbar_arrive_expect_tx(bs, bytes);
             for (uint32_t p = p_first; p <= p_last; p++) {
-                const uint32_t lo = p == p_first ? g0 - p * n : 0u;
-                const uint32_t hi = p == p_last ? g0 + nrows - p * n : n;
+                const uint32_t lo = p == p_first ? g0 - p * nn : 0u;
+                const uint32_t hi = p == p_last ? g0 + nrows - p * nn : nn;
                 const uint32_t e = ex_s[p - p_first];
                 if (e >= P.num_experts) continue;
-                const uint32_t dst = (p * n + lo - g0) * G * 2u;
-                const size_t src = ((size_t)e * n + lo) * G;
-                ptx::bulk_g2s(sbase + L.sc + dst, (const unsigned short *)P.scales + src, (hi - lo) * G * 2u, bs);
-                ptx::bulk_g2s(sbase + L.bi + dst, (const unsigned short *)P.aux + src, (hi - lo) * G * 2u, bs);
+                for (uint32_t h = 0; h < AREAS; h++) {
+                    const uint32_t dst = (h * rows_per_cta + p * nn + lo - g0) * G * 2u;
+                    const size_t src = ((size_t)e * n + h * nn + lo) * G;
+                    ptx::bulk_g2s(sbase + L.sc + dst, (const unsigned short *)P.scales + src, (hi - lo) * G * 2u, bs);
+                    ptx::bulk_g2s(sbase + L.bi + dst, (const unsigned short *)P.aux + src, (hi - lo) * G * 2u, bs);
+                }
             }
         }
     } else {
         unsigned short *sc = (unsigned short *)(dsm8 + L.sc), *bi = (unsigned short *)(dsm8 + L.bi);
-        for (uint32_t idx = tid; idx < nrows * G; idx += blockDim.x) {
-            const uint32_t r = idx / G, gi = idx - r * G;
-            const uint32_t g = g0 + r, p = g / n, c = g - p * n;
-            const uint32_t e = ex_s[p - p_first];
-            const size_t src = ((size_t)(e < P.num_experts ? e : 0u) * n + c) * G + gi;
-            sc[idx] = __ldg((const unsigned short *)P.scales + src);
-            bi[idx] = __ldg((const unsigned short *)P.aux + src);
+        for (uint32_t h = 0; h < AREAS; h++) {
+            for (uint32_t idx = tid; idx < nrows * G; idx += blockDim.x) {
+                const uint32_t r = idx / G, gi = idx - r * G;
+                const uint32_t g = g0 + r, p = g / nn, c = g - p * nn;
+                const uint32_t e = ex_s[p - p_first];
+                const size_t src = ((size_t)(e < P.num_experts ? e : 0u) * n + h * nn + c) * G + gi;
+                sc[h * rows_per_cta * G + idx] = __ldg((const unsigned short *)P.scales + src);
+                bi[h * rows_per_cta * G + idx] = __ldg((const unsigned short *)P.aux + src);
+            }
         }
     }
 
-    // this warp's rows [a, b) of the CTA's range, one bulk copy per pair they touch
+    // this warp's rows [a, b) of the CTA's range, one bulk copy per pair (and area) they touch
     const uint32_t rpw = (nrows + ROWS_WARPS - 1) / ROWS_WARPS;
     const uint32_t a = tmin<uint32_t>(warp * rpw, nrows), b = tmin<uint32_t>(a + rpw, nrows);
     if (lane == 0) {
         uint32_t bytes = 0;
         for (uint32_t r = a; r < b;) {
-            const uint32_t g = g0 + r, p = g / n, c0 = g - p * n;
-            const uint32_t cnt = tmin<uint32_t>(b - r, n - c0);
+            const uint32_t g = g0 + r, p = g / nn, c0 = g - p * nn;
+            const uint32_t cnt = tmin<uint32_t>(b - r, nn - c0);
             const uint32_t e = ex_s[p - p_first];
-            if (e < P.num_experts) bytes += cnt * rbytes;
+            if (e < P.num_experts) bytes += AREAS * cnt * rbytes;
             r += cnt;
         }
         ptx::mbar_arrive_expect_tx(bw, bytes);
         for (uint32_t r = a; r < b;) {
-            const uint32_t g = g0 + r, p = g / n, c0 = g - p * n;
-            const uint32_t cnt = tmin<uint32_t>(b - r, n - c0);
+            const uint32_t g = g0 + r, p = g / nn, c0 = g - p * nn;
+            const uint32_t cnt = tmin<uint32_t>(b - r, nn - c0);
             const uint32_t e = ex_s[p - p_first];
-            if (e < P.num_experts)
-                ptx::bulk_g2s(sbase + L.w + r * rbytes, P.packed + ((size_t)e * n + c0) * rbytes,
-                              cnt * rbytes, bw);
-            else if (c0 == 0)
+            if (e < P.num_experts) {
+                for (uint32_t h = 0; h < AREAS; h++)
+                    ptx::bulk_g2s(sbase + L.w + (h * rows_per_cta + r) * rbytes,
+                                  P.packed + ((size_t)e * n + h * nn + c0) * rbytes, cnt * rbytes, bw);
+            } else if (c0 == 0) {
                 atomicOr(P.err, ERR_BAD_ID);
+            }
             r += cnt;
         }
     }
@@ -1046,35 +1065,44 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
 
     // rows a + gi, a + gi + RPI, ...: (pair, column) carried along
     uint32_t g = g0 + a + gi;
-    uint32_t p = g / n, c = g - p * n;
+    uint32_t p = g / nn, c = g - p * nn;
     for (uint32_t r = a + gi; r < b + gi; r += RPI) {
         const bool valid = r < b;
         const uint32_t e = valid ? ex_s[p - p_first] : 0u;
         const bool live = valid && e < P.num_experts;
-        float acc = 0.f;
-        if (live) {
-            const uint8_t *wrow = dsm8 + L.w + r * rbytes;
-            const unsigned short *srow = sc + r * G, *brow = bi + r * G;
+        float acc[AREAS];
 #pragma unroll
-            for (int i = 0; i < UPL; i++) {
-                const uint32_t u = l + (uint32_t)i * LPR;
-                if (u < nu) {
-                    const uint4 w = *(const uint4 *)(wrow + 16u * u);
-                    acc = dp4a_unit_reg(w, pv[i], usc[i], usm[i], bf16_bits_to_f32(srow[grp[i]]),
-                                        bf16_bits_to_f32(brow[grp[i]]), acc);
+        for (uint32_t h = 0; h < AREAS; h++) {
+            acc[h] = 0.f;
+            if (live) {
+                const uint32_t rr = h * rows_per_cta + r;
+                const uint8_t *wrow = dsm8 + L.w + rr * rbytes;
+                const unsigned short *srow = sc + rr * G, *brow = bi + rr * G;
+#pragma unroll
+                for (int i = 0; i < UPL; i++) {
+                    const uint32_t u = l + (uint32_t)i * LPR;
+                    if (u < nu) {
+                        const uint4 w = *(const uint4 *)(wrow + 16u * u);
+                        acc[h] = dp4a_unit_reg(w, pv[i], usc[i], usm[i], bf16_bits_to_f32(srow[grp[i]]),
+                                               bf16_bits_to_f32(brow[grp[i]]), acc[h]);
+                    }
                 }
             }
-        }
 #pragma unroll
-        for (int d = LPR / 2; d > 0; d >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, d);
+            for (int d = LPR / 2; d > 0; d >>= 1) acc[h] += __shfl_xor_sync(0xFFFFFFFFu, acc[h], d);
+        }
         if (valid && l == 0) {
-            const uint32_t e = ex_s[p - p_first];
-            store_out(P.out, P.out_dtype, (size_t)p * n + c,
-                      e < P.num_experts ? acc + load_bias(P.bias, P.bias_dtype, (size_t)e * n + c) : 0.f);
+            float v = 0.f;
+            if (e < P.num_experts) {
+                const size_t bb = (size_t)e * n + c;
+                v = acc[0] + load_bias(P.bias, P.bias_dtype, bb);
+                if constexpr (GLU) v = glu_act(P.act, v) * (acc[1] + load_bias(P.bias, P.bias_dtype, bb + nn));
+            }
+            store_out(P.out, P.out_dtype, (size_t)p * nn + c, v);
         }
         c += RPI;
-        if (c >= n) {
-            c -= n;
+        if (c >= nn) {
+            c -= nn;
             p++;
         }
     }
@@ -1099,9 +1127,9 @@ void rows_shape(uint32_t nu, int *lpr, int *upl) {
     }
 }
 
-template <int LPR, int UPL>
+template <int LPR, int UPL, bool GLU>
 cudaError_t launch_rows_t(const GemvParams &P, uint32_t rb, uint32_t ctas, size_t smem, cudaStream_t st) {
-    auto kern = gemv_aff4_rows<LPR, UPL>;
+    auto kern = gemv_aff4_rows<LPR, UPL, GLU>;
     if (smem > 48 * 1024) {
         static int smem_set[64];
         cudaError_t e = ensure_dyn_smem(kern, smem, smem_set);
@@ -1114,10 +1142,17 @@ cudaError_t launch_rows_t(const GemvParams &P, uint32_t rb, uint32_t ctas, size_
 template <int LPR>
 cudaError_t launch_rows_l(const GemvParams &P, int upl, uint32_t rb, uint32_t ctas, size_t smem,
                           cudaStream_t st) {
+    if (P.glu_nh) {
+        switch (upl) {
+            case 1: return launch_rows_t<LPR, 1, true>(P, rb, ctas, smem, st);
+            case 2: return launch_rows_t<LPR, 2, true>(P, rb, ctas, smem, st);
+            default: return launch_rows_t<LPR, 3, true>(P, rb, ctas, smem, st);
+        }
+    }
     switch (upl) {
-        case 1: return launch_rows_t<LPR, 1>(P, rb, ctas, smem, st);
-        case 2: return launch_rows_t<LPR, 2>(P, rb, ctas, smem, st);
-        default: return launch_rows_t<LPR, 3>(P, rb, ctas, smem, st);
+        case 1: return launch_rows_t<LPR, 1, false>(P, rb, ctas, smem, st);
+        case 2: return launch_rows_t<LPR, 2, false>(P, rb, ctas, smem, st);
+        default: return launch_rows_t<LPR, 3, false>(P, rb, ctas, smem, st);
     }
 }
 
@@ -1133,12 +1168,19 @@ int sm_count() {
     return count[dev];
 }
 
-// Rows per CTA: an even split of all rows over two CTAs per SM, rounded up to
-// 8 rows so that ranges of scale rows start on 16-byte boundaries.
-uint32_t rows_per_cta(uint32_t total_rows) {
-    const uint32_t ctas = 2u * (uint32_t)sm_count();
-    uint32_t rb = (total_rows + ctas - 1) / ctas;
-    return (rb + 7u) & ~7u;
+// Fewest rows whose bf16 scales (G per row) fill whole 16-byte units: 8, 4, 2 or 1.
+uint32_t rows_unit(uint32_t G) {
+    uint32_t u = 8;
+    while (u > 1 && (u / 2u) * G % 8u == 0) u /= 2u;
+    return u;
+}
+
+// Rows per CTA: an even split of all rows over two CTAs per SM, rounded up to a
+// multiple of rows_unit(G) so that ranges of scale rows start on 16-byte boundaries.
+uint32_t rows_per_cta(uint32_t total_rows, uint32_t G) {
+    const uint32_t ctas = 2u * (uint32_t)sm_count(), u = rows_unit(G);
+    const uint32_t rb = (total_rows + ctas - 1) / ctas;
+    return (rb + u - 1) / u * u;
 }
 
 // One token, 4-bit affine rows of whole 16-byte units, groups of whole units,
@@ -1150,24 +1192,28 @@ bool rows_ok(const QmmArgs &a) {
     int lpr, upl;
     rows_shape(a.row_bytes / 16u, &lpr, &upl);
     if (lpr == 0) return false;
-    const uint64_t total = (uint64_t)a.n_expert_used * a.n;
+    const uint64_t total = (uint64_t)a.n_expert_used * a.out_n;  // rows of the walk
     if (total >= (1ull << 31)) return false;
-    const uint32_t rb = rows_per_cta((uint32_t)total);
-    const RowsLayout L = rows_layout(rb, a.row_bytes, a.k * xsz, a.row_bytes / 16u, a.groups);
+    const uint32_t rb = rows_per_cta((uint32_t)total, a.groups);
+    const uint32_t areas = a.act >= 0 ? 2u : 1u;
+    const RowsLayout L = rows_layout(areas * rb, a.row_bytes, a.k * xsz, a.row_bytes / 16u, a.groups);
     return L.total <= 110u * 1024u;
 }
 
 cudaError_t launch_rows(GemvParams P, const QmmArgs &a, cudaStream_t st) {
     int lpr, upl;
     rows_shape(P.n_units, &lpr, &upl);
-    const uint32_t total = P.R * P.n;
-    const uint32_t rb = rows_per_cta(total);
+    const uint32_t total = P.R * P.out_n;  // rows of the walk: output elements of a pair
+    const uint32_t rb = rows_per_cta(total, P.groups);
     const uint32_t ctas = (total + rb - 1) / rb;
     const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
-    const RowsLayout L = rows_layout(rb, P.row_bytes, a.k * xsz, P.n_units, P.groups);
-    // with n a multiple of 8, every range a CTA copies starts and ends on a multiple of
-    // 8 rows, and 8 rows of bf16 scales are a whole number of 16-byte units
-    P.s_bulk = (a.n % 8u) == 0 && (uintptr_t)a.scales % 16u == 0 && (uintptr_t)a.aux % 16u == 0;
+    const uint32_t areas = P.glu_nh ? 2u : 1u;
+    const RowsLayout L = rows_layout(areas * rb, P.row_bytes, a.k * xsz, P.n_units, P.groups);
+    // with out_n a multiple of u = rows_unit(G), every range a CTA copies (gate and up
+    // halves alike) starts and ends on a multiple of u rows, whose scales fill whole
+    // 16-byte units
+    P.s_bulk = (a.out_n % rows_unit(P.groups)) == 0 && (uintptr_t)a.scales % 16u == 0 &&
+               (uintptr_t)a.aux % 16u == 0;
     switch (lpr) {
         case 4: return launch_rows_l<4>(P, upl, rb, ctas, L.total, st);
         case 8: return launch_rows_l<8>(P, upl, rb, ctas, L.total, st);
@@ -1301,6 +1347,9 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     P.xstride = P.n_units * (uc + 1);
     P.x_dtype = a.x_dtype; P.out_dtype = a.out_dtype;
     P.bias = a.bias; P.bias_dtype = a.bias_dtype;
+    P.glu_nh = a.act >= 0 ? a.n / 2u : 0u;
+    P.out_n = a.out_n;
+    P.act = a.act;
     P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
     const bool al16 = ((uintptr_t)a.packed % 16 == 0) && (a.row_bytes % 16 == 0);
     const bool al4 = ((uintptr_t)a.packed % 4 == 0) && (a.row_bytes % 4 == 0);
@@ -1320,6 +1369,7 @@ cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st) 
     const bool spec = (uint64_t)a.m * a.k * xsz <= 32768u;
     if (a.packed_ptrs) return launch_kind<true>(P, a.kind, npb, grid, st);  // pointer-table weights
     if (rows_ok(a)) return launch_rows(P, a, st);
+    if (a.act >= 0) return launch_kind<true>(P, a.kind, npb, grid, st);  // gated output
     if (a.m == 1 && tma_ok(a, 1, spec)) {
         P.x_spec = spec;
         return launch_tma<MODE_PAIR>(P, 1, P.R, st);
@@ -1337,7 +1387,7 @@ cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const u
     GemvParams P = make_params(a, err);
     P.counts = counts; P.offsets = offsets; P.sorted_pairs = sorted_pairs;
     dim3 grid((a.n + GEMV_ROWS - 1) / GEMV_ROWS, a.num_experts);
-    if (a.packed_ptrs) return launch_kind<false>(P, a.kind, 8u, grid, st);  // pointer-table weights
+    if (a.packed_ptrs || a.act >= 0) return launch_kind<false>(P, a.kind, 8u, grid, st);  // pointer tables, gated output
     if (tma_ok(a, 8u, false)) return launch_tma<MODE_ROUTED>(P, 8u, a.num_experts, st);
     if (dp4a_ok(a)) return launch_dp4a<false>(P, 8u, grid, st);
     return launch_kind<false>(P, a.kind, 8u, grid, st);

@@ -33,6 +33,10 @@ struct GemvParams {
     // addresses of the packed rows, scales and affine biases; a null packed pointer
     // means the expert is not held here and its pairs' rows are left untouched
     const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;
+    // gated output (glu_nh = n/2; 0: plain): rows are walked in the logical order of
+    // glu_row and out rows hold out_n = n/2 values act(gate) * up (else out_n = n)
+    uint32_t glu_nh, out_n;
+    int act;
 };
 
 // Which expert this CTA serves and how many pairs it has. Fused mode: all ids
@@ -72,9 +76,11 @@ __device__ __forceinline__ bool route_prologue(const GemvParams &P, uint32_t *id
         }
         __syncthreads();
         if (blockIdx.y == 0) {
-            for (uint32_t idx = tid; idx < R * rows; idx += blockDim.x) {
-                const uint32_t p = idx / rows, r = row0 + idx % rows;
-                if (ids_s[p] >= E && r < P.n) store_out(P.out, P.out_dtype, (size_t)p * P.n + r, 0.f);
+            // output columns of this row block: half as many with a gated output
+            const uint32_t sh = P.glu_nh ? 1u : 0u, c0 = row0 >> sh, cn = rows >> sh;
+            for (uint32_t idx = tid; idx < R * cn; idx += blockDim.x) {
+                const uint32_t p = idx / cn, c = c0 + idx % cn;
+                if (ids_s[p] >= E && c < P.out_n) store_out(P.out, P.out_dtype, (size_t)p * P.out_n + c, 0.f);
             }
             if (blockIdx.x == 0 && tid < R && ids_s[tid] >= E) atomicOr(P.err, ERR_BAD_ID);
         }

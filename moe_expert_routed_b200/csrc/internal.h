@@ -68,6 +68,8 @@ struct QmmArgs {
     const void *bias;  // per-expert output bias [num_experts, n] (bias_dtype), or null
     int bias_dtype;
     const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;  // pointer-table weights, or null
+    int act;         // gated output: -1 none, else the activation (moe_act) of act(gate) * up
+    uint32_t out_n;  // columns of an output row: n, or n / 2 with a gated output
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).

@@ -114,3 +114,75 @@ def check_full_bias(P, out: torch.Tensor, bias: np.ndarray, bias_dtype: int, nth
     pairs = np.repeat(np.arange(P.R), P.n)
     cols = np.tile(np.arange(P.n), P.R)
     return compare(P, got.reshape(-1), ref, pairs, cols)
+
+
+# ------------------------------------------------------------ gated (GLU) output
+#
+# out[p][c] = act(g) * u with g, u the pair's results in gate row c and up row
+# n/2 + c (bias included). With Bg, Bu the per-element bounds above for g and u
+# (atol_t + 2e-3 |y|), the bound on z = act(g) * u is their first-order
+# propagation through |act'| <= 1.2 (SiLU's slope stays below 1.1, GELU's below
+# 1.13), the second-order term |act''| <= 0.8 (GELU's curvature peaks at
+# 2 * phi(0) = 0.80), the cross term, and the fp32 evaluation of the activation:
+# a few ulp relative, plus an absolute 1e-6 |g| |u| where 1 + tanh(.) or
+# 1 + erf(.) cancels for negative g. 16-bit outputs add one unit in their last
+# place after rounding the oracle's z.
+ACT_CODE = {"silu": 0, "gelu_tanh": 1, "gelu_erf": 2}
+
+
+def run_glu(P, act: str, path="auto", bias=None, bias_dtype=DT_F32, dev=None, out=None, workspace=None):
+    dev = dev or to_device(P)
+    return M.qmm_id(dev["x"], dev["ids"], dev["packed"], dev["scales"], dev["aux"], n=P.n,
+                    group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
+                    out=out, out_dtype=TORCH_OUT[P.out_dtype], workspace=workspace, path=path,
+                    expert_bias=bias_tensor(bias, bias_dtype) if bias is not None else None, act=act)
+
+
+def compare_glu(P, act: str, got: np.ndarray, g_ref: np.ndarray, u_ref: np.ndarray, pairs: np.ndarray):
+    """got/g_ref/u_ref at the same output elements of pairs[i]; refs in double."""
+    ids = P.ids.reshape(-1)[pairs]
+    bad_id = ids >= P.num_experts
+    X = R.x_f64(P)
+    xn = np.linalg.norm(X[pairs // P.n_expert_used], axis=1)
+    wmax = expert_wmax(P, np.unique(ids[~bad_id]))
+    wm = np.array([wmax.get(int(e), 0.0) for e in ids])
+    atol = 1e-2 * xn * wm / np.sqrt(P.k)
+    bg = atol + 2e-3 * np.abs(g_ref)
+    bu = atol + 2e-3 * np.abs(u_ref)
+    code = ACT_CODE[act]
+    z = oracle.glu_elems(g_ref, u_ref, code)
+    ag = np.abs(oracle.glu_elems(g_ref, np.ones_like(g_ref), code))
+    if P.out_dtype == DT_F32:
+        z_ref, slack = z, 0.0
+    else:
+        bits = oracle.round_out(z, P.out_dtype)
+        z_ref = R.bf16_to_f64(bits) if P.out_dtype == DT_BF16 else R.f16_to_f64(bits)
+        slack = ulp16(z_ref, P.out_dtype)
+    au = np.abs(u_ref)
+    bound = (1.2 * au * bg + ag * bu + 1.2 * bg * bu + 0.4 * bg * bg * (au + bu)
+             + 4e-6 * np.abs(z) + 1e-6 * np.abs(g_ref) * au + slack)
+    err = np.abs(got - z_ref)
+    viol = (err > bound) & ~bad_id
+    viol |= bad_id & (got != 0.0)
+    ratio = float(np.max(np.where(bad_id, 0.0, err / np.maximum(bound, 1e-300)))) if got.size else 0.0
+    return int(viol.sum()), ratio, dict(max_abs_err=float(err.max()) if err.size else 0.0)
+
+
+def check_full_glu(P, act: str, out: torch.Tensor, bias=None, bias_dtype=DT_F32, nthreads=None):
+    """Full gated output against the oracle (plus its bias step) and its glu step."""
+    ref, _ = oracle.qmm_id(P, nthreads=nthreads)
+    if bias is not None:
+        oracle.add_expert_bias(ref.reshape(-1), P, bias, bias_dtype)
+    nh = P.n // 2
+    got = out_to_f64(out).reshape(P.R, nh)
+    pairs = np.repeat(np.arange(P.R), nh)
+    return compare_glu(P, act, got.reshape(-1), ref[:, :nh].reshape(-1), ref[:, nh:].reshape(-1), pairs)
+
+
+def check_sampled_glu(P, act: str, out: torch.Tensor, pairs: np.ndarray, cols: np.ndarray, nthreads=None):
+    """Sampled gated outputs (pairs[i], cols[i] < n/2) against the oracle's elements."""
+    nh = P.n // 2
+    g = oracle.qmm_id_sample(P, pairs, cols, nthreads=nthreads)
+    u = oracle.qmm_id_sample(P, pairs, cols + nh, nthreads=nthreads)
+    got = out_to_f64(out).reshape(P.R, nh)[pairs, cols]
+    return compare_glu(P, act, got, g, u, pairs)

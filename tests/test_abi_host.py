@@ -90,6 +90,21 @@ def test_bias_entry_rejects_before_cuda():
     assert call(m=0) == 1             # the operation's own checks still apply
 
 
+def test_glu_entry_rejects_before_cuda():
+    L = M.lib()
+
+    def call(n=128, act=0, bias=16, bdt=0, m=4, path=0):
+        return L.moe_qmm_id_glu(16, 16, 16, 16, 16, bias, 16, m, 256, n, 32, 4, 0, 2, 8, 0, 0, bdt, act,
+                                4096, 1 << 20, None, path)
+    assert call(n=127) == 1           # gate and up halves need an even n
+    assert call(act=3) == 1           # unknown activation
+    assert call(act=-1) == 1
+    assert call(bdt=3) == 1           # unknown bias dtype with a bias
+    assert call(m=0) == 1             # the operation's own checks still apply
+    assert call(path=5) == 1          # unknown path
+    assert call(bias=0, bdt=3, m=0) == 1  # without a bias its dtype is ignored; m=0 still rejected
+
+
 def test_pointer_table_entry_rejects_before_cuda():
     L = M.lib()
 
