@@ -170,7 +170,7 @@ def clocks_summary(proc):
 class DecodeWorkload:
     """gate/up + down projections of one decode token, rotating weight copies."""
 
-    def __init__(self, steps_per_graph: int, seed: int = 2):
+    def __init__(self, steps_per_graph: int, seed: int = 2, pdl: bool = True):
         import moe_expert_routed_b200 as M
         from workloads.torch_io import to_device
         from workloads import config_problem
@@ -178,6 +178,10 @@ class DecodeWorkload:
 
         self.M = M
         self.projs = [config_problem("decode_gate_up"), config_problem("decode_down")]
+        # launch modes of a step: gate/up as a programmatic dependent launch (it waits for
+        # the previous kernel before reading anything); down also streams its weights
+        # early, since its ids were ready before gate/up began
+        self.launch = ("pdl", "early_weights") if pdl else (None, None)
         self.G = steps_per_graph
         rng = np.random.Generator(np.random.PCG64(seed + 100))
         self.layers = []
@@ -202,17 +206,19 @@ class DecodeWorkload:
             [alg_bytes(P, self.ids[i][s].cpu().numpy().view(np.uint32)) for s in range(self.G)]
             for i, P in enumerate(self.projs)]
 
-    def call(self, proj: int, s: int, act=None):
+    def call(self, proj: int, s: int, act=None, launch=None):
         P = self.projs[proj]
         L = self.layers[proj][s % N_LAYERS]
         self.M.qmm_id(self.x[proj][s:s + 1], self.ids[proj][s:s + 1], L["packed"], L["scales"],
                       L["aux"], n=P.n, group_size=P.group_size, bits=P.bits, fmt=P.fmt,
                       num_experts=P.num_experts, out=self.out_glu[s] if act else self.out[proj][s],
-                      workspace=self.ws[proj], act=act)
+                      workspace=self.ws[proj], act=act, launch=launch)
 
     def step(self, s: int, projs=(0, 1), act=None):
+        # the step's launch modes apply to the full gate/up + down sequence only
+        full = tuple(projs) == (0, 1)
         for p in projs:
-            self.call(p, s, act)
+            self.call(p, s, act, self.launch[p] if full else None)
 
     def bytes(self, projs=(0, 1)) -> float:
         return sum(sum(self.step_bytes[p]) for p in projs)
@@ -282,7 +288,7 @@ def e2e_decode(W: DecodeWorkload, steps: int):
             L = W.layers[p][s % N_LAYERS]
             M.qmm_id(dx[p], did[p], L["packed"], L["scales"], L["aux"], n=P.n,
                      group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
-                     out=dout[p], workspace=W.ws[p])
+                     out=dout[p], workspace=W.ws[p], launch=W.launch[p])
         hout.copy_(dout_all, non_blocking=True)
     b.record()
     b.synchronize()
@@ -372,7 +378,7 @@ def run_ours(args, dist: Dist):
     torch.cuda.set_device(dev)
     K, Wm = args.steps, args.warmup
     G = min(GRAPH_STEPS, K)
-    W = DecodeWorkload(G)
+    W = DecodeWorkload(G, pdl=not args.no_pdl)
     g = W.capture()
     replays = max(1, K // G)
     steps_timed = replays * G
@@ -440,6 +446,9 @@ def run_ours(args, dist: Dist):
                    "l2": f"inputs larger than L2: {N_LAYERS} rotated weight copies "
                          f"({N_LAYERS * 0.428:.1f} GB), fresh ids and x every step",
                    "timing": f"CUDA graph of {G} steps replayed {replays}x, CUDA events",
+                   "launch": ("gate/up: programmatic dependent launch; down: PDL with early weight "
+                              "streaming (its ids were ready before gate/up began)")
+                             if not args.no_pdl else "plain stream order",
                    "parallelism": f"replicas x{dist.world}"},
         "per_call": per_call,
         "roofline": roofline,
@@ -587,6 +596,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="decode step without programmatic dependent launch between its calls")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--config", default="decode", choices=["decode", "canvas", "prefill", "skewed"])
     ap.add_argument("--probe", choices=["decode", "canvas", "prefill", "skewed"],

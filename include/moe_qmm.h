@@ -80,6 +80,28 @@ typedef enum {
  * routed GEMV instead. */
 typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_GROUPED = 2 } moe_path;
 
+/* Launch flags, OR-ed into the path argument of the entry points that take one
+ * (for example (moe_path)(MOE_PATH_AUTO | MOE_LAUNCH_PDL)); other bits above the
+ * low byte are MOE_ERR_INVALID_ARGUMENT. They are honoured by the one-token decode
+ * kernel (m = 1, 4-bit affine, k <= 3072) and ignored by the other kernels, which
+ * always start after the previous work on the stream has completed.
+ *   MOE_LAUNCH_PDL            launch as a programmatic dependent of the previous
+ *                             kernel on the stream: the kernel may be scheduled on
+ *                             SMs that kernel frees before it completes, and waits
+ *                             for its completion (griddepcontrol.wait) before it
+ *                             reads any input. Hides the launch gap between
+ *                             back-to-back calls.
+ *   MOE_LAUNCH_EARLY_WEIGHTS  with MOE_LAUNCH_PDL: the caller promises that ids,
+ *                             packed, scales and aux were complete before the
+ *                             previous kernel on the stream began (for example the
+ *                             down projection after the gate+up projection that
+ *                             used the same ids). The kernel then reads ids and
+ *                             starts streaming the experts' weights before that
+ *                             kernel completes; x and the expert bias are read,
+ *                             and out is written, only after it. */
+#define MOE_LAUNCH_PDL 0x100u
+#define MOE_LAUNCH_EARLY_WEIGHTS 0x200u
+
 #define MOE_DECODE_MAX_ROUTINGS 64u
 /* Largest num_experts the routing prologue (and so the grouped path) accepts. */
 #define MOE_ROUTE_MAX_EXPERTS 1024u

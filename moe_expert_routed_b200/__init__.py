@@ -26,6 +26,9 @@ DT_F32, DT_BF16, DT_F16 = 0, 1, 2
 PATH_AUTO, PATH_DECODE, PATH_GROUPED = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "grouped": PATH_GROUPED}
 ACT_SILU, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
+# launch flags OR-ed into the path argument (programmatic dependent launch)
+LAUNCH_PDL, LAUNCH_EARLY_WEIGHTS = 0x100, 0x200
+_LAUNCH = {None: 0, "pdl": LAUNCH_PDL, "early_weights": LAUNCH_PDL | LAUNCH_EARLY_WEIGHTS}
 ACTS = {"silu": ACT_SILU, "gelu_tanh": ACT_GELU_TANH, "gelu_erf": ACT_GELU_ERF}
 
 MOE_OK = 0
@@ -129,7 +132,8 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
            aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
            out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
            workspace: torch.Tensor | None = None, path: str = "auto",
-           expert_bias: torch.Tensor | None = None, act: str | None = None) -> torch.Tensor:
+           expert_bias: torch.Tensor | None = None, act: str | None = None,
+           launch: str | None = None) -> torch.Tensor:
     """Expert-routed quantized matmul on the current CUDA stream.
 
     x [m, k] (f32 / bf16 / f16); ids [m, n_expert_used] int32/uint32; packed, scales,
@@ -140,7 +144,9 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
     expert (moe_qmm_id_bias). act ("silu", "gelu_tanh" or "gelu_erf") makes it the
     fused gate+up projection (moe_qmm_id_glu): rows [0, n/2) of each expert are the
     gate, rows [n/2, n) the up projection, and out [m, n_expert_used, n/2] holds
-    act(gate) * up.
+    act(gate) * up. launch ("pdl" or "early_weights") sets the C ABI's launch flags
+    (MOE_LAUNCH_PDL, plus MOE_LAUNCH_EARLY_WEIGHTS): see include/moe_qmm.h for the
+    promise "early_weights" makes about ids and weights.
     """
     device = x.device
     for t, name in ((x, "input"), (ids, "ids"), (packed, "weight"), (scales, "scales"),
@@ -183,6 +189,9 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
     if _nbytes(aux) < aux_need:
         raise ValueError(f"quantized_matmul_id: {aux_name} buffer too small: expected at least "
                          f"{aux_need} bytes, got {_nbytes(aux)}")
+    if launch not in _LAUNCH:
+        raise ValueError(f"quantized_matmul_id: unknown launch mode {launch!r}")
+    path_arg = _PATHS[path] | _LAUNCH[launch]
     if act is not None:
         if act not in ACTS:
             raise ValueError(f"quantized_matmul_id: unknown activation {act!r} (one of {sorted(ACTS)})")
@@ -210,19 +219,19 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
             expert_bias.data_ptr() if expert_bias is not None else None, out.data_ptr(), m, k, n,
             group_size, bits, fmt, n_expert_used, num_experts, _TORCH_DT[x.dtype], _TORCH_DT[out.dtype],
             _TORCH_DT[expert_bias.dtype] if expert_bias is not None else 0, ACTS[act],
-            workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), _PATHS[path])
+            workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), path_arg)
     elif expert_bias is None:
         st = lib().moe_qmm_id_path(
             x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
             out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used, num_experts,
             _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], workspace.data_ptr(), _nbytes(workspace),
-            _stream_ptr(device), _PATHS[path])
+            _stream_ptr(device), path_arg)
     else:
         st = lib().moe_qmm_id_bias(
             x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
             expert_bias.data_ptr(), out.data_ptr(), m, k, n, group_size, bits, fmt, n_expert_used,
             num_experts, _TORCH_DT[x.dtype], _TORCH_DT[out.dtype], _TORCH_DT[expert_bias.dtype],
-            workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), _PATHS[path])
+            workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), path_arg)
     if st != MOE_OK:
         raise MoeError(st, "moe_qmm_id")
     return out

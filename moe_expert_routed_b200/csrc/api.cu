@@ -123,7 +123,11 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
                             pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
                             fmt, n_expert_used, num_experts, x_dtype, out_dtype);
     if (v != MOE_OK) return v;
-    if ((int)path < 0 || (int)path > 2) return MOE_ERR_INVALID_ARGUMENT;
+    // the low byte is the path, higher bits launch flags
+    const uint32_t launch_flags = (uint32_t)path & ~0xFFu;
+    path = (moe_path)((uint32_t)path & 0xFFu);
+    if ((int)path > 2 || (launch_flags & ~(uint32_t)(MOE_LAUNCH_PDL | MOE_LAUNCH_EARLY_WEIGHTS)))
+        return MOE_ERR_INVALID_ARGUMENT;
     if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
     const uint64_t R = (uint64_t)m * n_expert_used;
     WsLayout L;
@@ -145,6 +149,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     a.bias_ptrs = pt.biases;
     a.act = act;
     a.out_n = act >= 0 ? n / 2u : n;
+    a.launch_flags = launch_flags;
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);

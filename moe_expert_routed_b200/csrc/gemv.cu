@@ -926,6 +926,14 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     const RowsLayout L = rows_layout(AREAS * rows_per_cta, rbytes, P.k * xsz, nu, G);
     const uint32_t sbase = ptx::smem_u32(dsm8);
     volatile int *abort_flag = &abort_s;
+    const bool early = P.early_weights != 0;
+
+    // a kernel launched after this one on the stream may be scheduled as soon as
+    // SMs free up; it waits for this grid itself before touching what it writes
+    ptx::griddep_launch_dependents();
+    // programmatic launch: without early_weights every input may come from the
+    // previous kernel on the stream, so wait for it first (a no-op otherwise)
+    if (!early) ptx::griddep_wait();
 
     // experts of the pairs this CTA touches (loads in flight across the barrier)
     if (tid <= p_last - p_first) ex_s[tid] = __ldg(P.ids + p_first + tid);
@@ -939,7 +947,7 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     __syncthreads();
     const uint32_t bx = ptx::smem_u32(&bar_x), bs = ptx::smem_u32(&bar_s);
     const uint32_t bw = ptx::smem_u32(&bar_w[warp]);
-    if (tid == 0) {
+    if (tid == 0 && !early) {
         ptx::mbar_arrive_expect_tx(bx, P.k * xsz);
         ptx::bulk_g2s(sbase + L.xraw, P.x, P.k * xsz, bx);
     }
@@ -1006,6 +1014,15 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
                 atomicOr(P.err, ERR_BAD_ID);
             }
             r += cnt;
+        }
+    }
+    if (early) {
+        // ids, weights and scales were ready before the previous kernel began (the
+        // caller's promise); x may be its output, and out may still be read by it
+        ptx::griddep_wait();
+        if (tid == 0) {
+            ptx::mbar_arrive_expect_tx(bx, P.k * xsz);
+            ptx::bulk_g2s(sbase + L.xraw, P.x, P.k * xsz, bx);
         }
     }
     // x planes, once per CTA: one thread per 8-code word, 4 consecutive lanes per unit
@@ -1135,8 +1152,23 @@ cudaError_t launch_rows_t(const GemvParams &P, uint32_t rb, uint32_t ctas, size_
         cudaError_t e = ensure_dyn_smem(kern, smem, smem_set);
         if (e != cudaSuccess) return e;
     }
-    kern<<<ctas, ROWS_THREADS, smem, st>>>(P, rb);
-    return cudaGetLastError();
+    if (!P.pdl) {
+        kern<<<ctas, ROWS_THREADS, smem, st>>>(P, rb);
+        return cudaGetLastError();
+    }
+    // programmatic dependent launch: may be scheduled before the previous kernel on
+    // the stream completes; the kernel waits for it (griddepcontrol.wait) itself
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctas);
+    cfg.blockDim = dim3(ROWS_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, P, rb);
 }
 
 template <int LPR>
@@ -1350,6 +1382,8 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     P.glu_nh = a.act >= 0 ? a.n / 2u : 0u;
     P.out_n = a.out_n;
     P.act = a.act;
+    P.pdl = (a.launch_flags & MOE_LAUNCH_PDL) != 0;
+    P.early_weights = (a.launch_flags & MOE_LAUNCH_EARLY_WEIGHTS) != 0;
     P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
     const bool al16 = ((uintptr_t)a.packed % 16 == 0) && (a.row_bytes % 16 == 0);
     const bool al4 = ((uintptr_t)a.packed % 4 == 0) && (a.row_bytes % 4 == 0);

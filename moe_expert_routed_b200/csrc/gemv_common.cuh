@@ -37,6 +37,10 @@ struct GemvParams {
     // glu_row and out rows hold out_n = n/2 values act(gate) * up (else out_n = n)
     uint32_t glu_nh, out_n;
     int act;
+    // programmatic dependent launch (one-token kernel): with early_weights the ids,
+    // weights and scales are read, and the weight copies issued, before waiting for
+    // the previous kernel on the stream; otherwise everything waits for it
+    int pdl, early_weights;
 };
 
 // Which expert this CTA serves and how many pairs it has. Fused mode: all ids

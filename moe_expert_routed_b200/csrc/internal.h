@@ -70,6 +70,7 @@ struct QmmArgs {
     const uint64_t *packed_ptrs, *scale_ptrs, *bias_ptrs;  // pointer-table weights, or null
     int act;         // gated output: -1 none, else the activation (moe_act) of act(gate) * up
     uint32_t out_n;  // columns of an output row: n, or n / 2 with a gated output
+    uint32_t launch_flags;  // MOE_LAUNCH_* bits of the path argument
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).

@@ -101,6 +101,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return false;
 }
 
+// ------------------------------------------- programmatic dependent launch
+
+// Block until the grids this one depends on programmatically (launched with the
+// programmatic stream serialization attribute) have completed and their memory
+// operations are visible; returns at once for a grid launched without it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the grid that depends on this one programmatically be scheduled once every
+// CTA of this grid has issued this or exited (no effect without such a grid).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- fences
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

@@ -115,6 +115,8 @@ def test_pointer_table_entry_rejects_before_cuda():
     assert call(scales=0) == 1
     assert call(biases=0) == 1                    # affine biases come from the table
     assert call(path=7) == 1                      # unknown path
+    assert call(path=0x400) == 1                  # unknown launch flag
+    assert call(path=0x100 | 3) == 1              # unknown path under a known flag
 
 
 def test_route_invalid_arguments():
