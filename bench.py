@@ -254,7 +254,9 @@ def time_graph(g, replays: int) -> float:
 def e2e_decode(W: DecodeWorkload, steps: int):
     """Through the public API with host buffers: per step, one copy brings that
     step's x rows and ids of both projections in from pinned host memory, both
-    projections run, one copy takes both outputs back."""
+    projections run (moe_expert_routed_b200.Plan: one per layer copy and
+    projection, bound before the timed region, the step's launch modes), one copy
+    takes both outputs back."""
     M = W.M
     n = min(steps, W.G)
     # per-step input block: x of each projection (bf16), then ids of each projection
@@ -278,17 +280,20 @@ def e2e_decode(W: DecodeWorkload, steps: int):
     dout = [dout_all[:nout[0]].view(1, 8, W.projs[0].n), dout_all[nout[0]:].view(1, 8, W.projs[1].n)]
     h2d = sum(xb) + sum(ib)
     d2h = sum(nout) * 4
+    plans = [[M.Plan(L["packed"], L["scales"], L["aux"], m=1, k=P.k, n=P.n, group_size=P.group_size,
+                     bits=P.bits, fmt=P.fmt, n_expert_used=8, num_experts=P.num_experts,
+                     x_dtype=torch.bfloat16, out_dtype=torch.float32, workspace=W.ws[p],
+                     launch=W.launch[p]) for L in W.layers[p]] for p, P in enumerate(W.projs)]
+    hrows = [hin[i] for i in range(n)]
+    st = torch.cuda.current_stream()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record()
     for s in range(steps):
-        din.copy_(hin[s % n], non_blocking=True)
-        for p, P in enumerate(W.projs):
-            L = W.layers[p][s % N_LAYERS]
-            M.qmm_id(dx[p], did[p], L["packed"], L["scales"], L["aux"], n=P.n,
-                     group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
-                     out=dout[p], workspace=W.ws[p], launch=W.launch[p])
+        din.copy_(hrows[s % n], non_blocking=True)
+        plans[0][s % N_LAYERS](dx[0], did[0], dout[0], st)
+        plans[1][s % N_LAYERS](dx[1], did[1], dout[1], st)
         hout.copy_(dout_all, non_blocking=True)
     b.record()
     b.synchronize()
@@ -435,7 +440,7 @@ def run_ours(args, dist: Dist):
     e2e = {"value": dist.sum(per_step_bytes * e2e_steps) / e_secs / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "us_per_step": e_secs / e2e_steps * 1e6, "steps": e2e_steps,
-           "path": "moe_expert_routed_b200.qmm_id (Python binding -> C ABI), pinned host buffers"}
+           "path": "moe_expert_routed_b200.Plan (Python binding -> moe_qmm_plan_run), pinned host buffers"}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world, "steps": steps_timed,
         "warmup": warm_replays * G, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,

@@ -297,6 +297,37 @@ moe_status moe_qmm_id_noalloc(const void *x, const uint32_t *ids, const void *pa
                               uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                               moe_dtype out_dtype, moe_stream_t stream);
 
+/*
+ * moe_qmm_plan -- a call with everything but x, ids and out bound once, for
+ * callers that issue the same projection many times (one plan per layer and
+ * projection in a decode loop). The plan lives in caller-owned storage (no
+ * allocation); moe_qmm_plan_init validates the bound arguments once, and
+ * moe_qmm_plan_run takes only the per-call pointers and the stream.
+ *   moe_qmm_plan_init  packed, scales, aux, sizes, formats, types, workspace and path
+ *                      (launch flags included) as moe_qmm_id_path; expert_bias and
+ *                      bias_dtype as moe_qmm_id_bias, or NULL for none; act -1 for a
+ *                      plain output, else a moe_act (the output of moe_qmm_id_glu).
+ *                      Returns the status moe_qmm_id would return for these
+ *                      arguments (x, ids and out are checked by each run).
+ *                      The plan keeps the pointers, not the data: the buffers must
+ *                      outlive it.
+ *   moe_qmm_plan_run   x, ids, out as moe_qmm_id. MOE_ERR_INVALID_ARGUMENT for a
+ *                      plan that was not initialised successfully, or a NULL
+ *                      pointer.
+ */
+typedef struct {
+    uint64_t opaque[24];
+} moe_qmm_plan;
+
+moe_status moe_qmm_plan_init(moe_qmm_plan *plan, const void *packed, const void *scales, const void *aux,
+                             const void *expert_bias, uint32_t m, uint32_t k, uint32_t n,
+                             uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
+                             uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
+                             moe_dtype bias_dtype, int32_t act, void *workspace, size_t workspace_bytes,
+                             moe_path path);
+moe_status moe_qmm_plan_run(const moe_qmm_plan *plan, const void *x, const uint32_t *ids, void *out,
+                            moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the device error word of `workspace`.
  * Returns MOE_OK, MOE_ERR_BAD_EXPERT_ID (some id was >= num_experts),
  * MOE_ERR_TIMEOUT (a bounded wait inside a kernel gave up; its outputs are not

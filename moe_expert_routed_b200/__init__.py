@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.moe_qmm_id_ptrs.restype = i32
         L.moe_qmm_id_glu.argtypes = [vp] * 7 + [u32] * 5 + [i32, u32, u32, i32, i32, i32, i32, vp, sz, vp, i32]
         L.moe_qmm_id_glu.restype = i32
+        L.moe_qmm_plan_init.argtypes = [vp] * 5 + [u32] * 5 + [i32, u32, u32, i32, i32, i32, i32, vp, sz, i32]
+        L.moe_qmm_plan_init.restype = i32
+        L.moe_qmm_plan_run.argtypes = [vp] * 5
+        L.moe_qmm_plan_run.restype = i32
         L.moe_qmm_id_path.restype = i32
         L.moe_qmm_id_workspace_bytes.argtypes = [u32, u32, u32]
         L.moe_qmm_id_workspace_bytes.restype = sz
@@ -128,26 +132,10 @@ def _nbytes(t: torch.Tensor) -> int:
     return t.numel() * t.element_size()
 
 
-def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
-           aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
-           out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
-           workspace: torch.Tensor | None = None, path: str = "auto",
-           expert_bias: torch.Tensor | None = None, act: str | None = None,
-           launch: str | None = None) -> torch.Tensor:
-    """Expert-routed quantized matmul on the current CUDA stream.
-
-    x [m, k] (f32 / bf16 / f16); ids [m, n_expert_used] int32/uint32; packed, scales,
-    aux: raw storage tensors (any dtype, byte lengths checked); returns out
-    [m, n_expert_used, n]. Buffer-size checks and their messages follow
-    mlx-native quantized_matmul_id.rs (quantized_matmul_id). expert_bias, if given,
-    is a [num_experts, n] f32 / bf16 / f16 tensor added to every pair's row of its
-    expert (moe_qmm_id_bias). act ("silu", "gelu_tanh" or "gelu_erf") makes it the
-    fused gate+up projection (moe_qmm_id_glu): rows [0, n/2) of each expert are the
-    gate, rows [n/2, n) the up projection, and out [m, n_expert_used, n/2] holds
-    act(gate) * up. launch ("pdl" or "early_weights") sets the C ABI's launch flags
-    (MOE_LAUNCH_PDL, plus MOE_LAUNCH_EARLY_WEIGHTS): see include/moe_qmm.h for the
-    promise "early_weights" makes about ids and weights.
-    """
+def _validate_only(x, ids, packed, scales, aux, *, n, group_size, bits, fmt, num_experts, out,
+                   expert_bias, act, launch):
+    """qmm_id's argument checks (devices, shapes, dtypes, buffer sizes) without a
+    call; returns (m, k, n_expert_used, out_n). out may be None."""
     device = x.device
     for t, name in ((x, "input"), (ids, "ids"), (packed, "weight"), (scales, "scales"),
                     (aux, "aux")):
@@ -191,28 +179,55 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
                          f"{aux_need} bytes, got {_nbytes(aux)}")
     if launch not in _LAUNCH:
         raise ValueError(f"quantized_matmul_id: unknown launch mode {launch!r}")
-    path_arg = _PATHS[path] | _LAUNCH[launch]
     if act is not None:
         if act not in ACTS:
             raise ValueError(f"quantized_matmul_id: unknown activation {act!r} (one of {sorted(ACTS)})")
         if n % 2:
             raise ValueError("quantized_matmul_id: a gated output needs an even N (gate and up halves)")
     out_n = n // 2 if act is not None else n
-    if out is None:
-        out = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
-    else:
+    if out is not None:
         _check_dev(out, "out", device)
         if out.dtype not in _TORCH_DT or out.numel() < m * n_expert_used * out_n:
             raise ValueError("quantized_matmul_id: out must hold [M, n_expert_used, N] f32/bf16/f16 "
                              "(N/2 columns with a gated output)")
-    if workspace is None:
-        workspace = new_workspace(m, n_expert_used, num_experts, device)
-    else:
-        _check_dev(workspace, "workspace", device)
     if expert_bias is not None:
         _check_dev(expert_bias, "expert_bias", device)
         if expert_bias.dtype not in _TORCH_DT or expert_bias.numel() < num_experts * n:
             raise ValueError("quantized_matmul_id: expert_bias must hold [num_experts, N] f32/bf16/f16")
+    return m, k, n_expert_used, out_n
+
+
+def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+           aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
+           out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
+           workspace: torch.Tensor | None = None, path: str = "auto",
+           expert_bias: torch.Tensor | None = None, act: str | None = None,
+           launch: str | None = None) -> torch.Tensor:
+    """Expert-routed quantized matmul on the current CUDA stream.
+
+    x [m, k] (f32 / bf16 / f16); ids [m, n_expert_used] int32/uint32; packed, scales,
+    aux: raw storage tensors (any dtype, byte lengths checked); returns out
+    [m, n_expert_used, n]. Buffer-size checks and their messages follow
+    mlx-native quantized_matmul_id.rs (quantized_matmul_id). expert_bias, if given,
+    is a [num_experts, n] f32 / bf16 / f16 tensor added to every pair's row of its
+    expert (moe_qmm_id_bias). act ("silu", "gelu_tanh" or "gelu_erf") makes it the
+    fused gate+up projection (moe_qmm_id_glu): rows [0, n/2) of each expert are the
+    gate, rows [n/2, n) the up projection, and out [m, n_expert_used, n/2] holds
+    act(gate) * up. launch ("pdl" or "early_weights") sets the C ABI's launch flags
+    (MOE_LAUNCH_PDL, plus MOE_LAUNCH_EARLY_WEIGHTS): see include/moe_qmm.h for the
+    promise "early_weights" makes about ids and weights.
+    """
+    device = x.device
+    m, k, n_expert_used, out_n = _validate_only(x, ids, packed, scales, aux, n=n, group_size=group_size,
+                                                bits=bits, fmt=fmt, num_experts=num_experts, out=out,
+                                                expert_bias=expert_bias, act=act, launch=launch)
+    path_arg = _PATHS[path] | _LAUNCH[launch]
+    if out is None:
+        out = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
+    if workspace is None:
+        workspace = new_workspace(m, n_expert_used, num_experts, device)
+    else:
+        _check_dev(workspace, "workspace", device)
     if act is not None:
         st = lib().moe_qmm_id_glu(
             x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
@@ -235,6 +250,59 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
     if st != MOE_OK:
         raise MoeError(st, "moe_qmm_id")
     return out
+
+
+class Plan:
+    """moe_qmm_plan: one projection with its weights, sizes, types, workspace, path,
+    launch mode, optional expert bias and optional gated output bound once
+    (validated like qmm_id); each call passes only x, ids and out. For decode
+    loops, where the per-call argument checks of qmm_id cost more host time than
+    the kernel takes on the device.
+
+        plan = Plan(packed, scales, aux, m=1, k=..., n=..., group_size=..., bits=..., fmt=...,
+                    n_expert_used=8, num_experts=128, x_dtype=torch.bfloat16)
+        plan(x, ids, out)          # on the current stream, or stream=<torch.cuda.Stream>
+    """
+
+    def __init__(self, packed: torch.Tensor, scales: torch.Tensor, aux: torch.Tensor, *, m: int, k: int,
+                 n: int, group_size: int, bits: int, fmt: int, n_expert_used: int, num_experts: int,
+                 x_dtype: torch.dtype = torch.bfloat16, out_dtype: torch.dtype = torch.float32,
+                 workspace: torch.Tensor | None = None, path: str = "auto", launch: str | None = None,
+                 expert_bias: torch.Tensor | None = None, act: str | None = None):
+        device = packed.device
+        # the same size checks as qmm_id, on a placeholder x of the bound shape
+        x0 = torch.empty((m, k), dtype=x_dtype, device=device)
+        ids0 = torch.zeros((m, n_expert_used), dtype=torch.int32, device=device)
+        out_n = n // 2 if act is not None else n
+        out0 = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
+        if workspace is None:
+            workspace = new_workspace(m, n_expert_used, num_experts, device)
+        _validate_only(x0, ids0, packed, scales, aux, n=n, group_size=group_size, bits=bits, fmt=fmt,
+                       num_experts=num_experts, out=out0, expert_bias=expert_bias, act=act, launch=launch)
+        self._keep = (packed, scales, aux, workspace, expert_bias)  # buffers the plan points into
+        self._buf = ctypes.create_string_buffer(24 * 8)
+        self.shape = (m, n_expert_used, out_n)
+        self.device = device
+        st = lib().moe_qmm_plan_init(
+            self._buf, packed.data_ptr(), scales.data_ptr(), aux.data_ptr(),
+            expert_bias.data_ptr() if expert_bias is not None else None, m, k, n, group_size, bits, fmt,
+            n_expert_used, num_experts, _TORCH_DT[x_dtype], _TORCH_DT[out_dtype],
+            _TORCH_DT[expert_bias.dtype] if expert_bias is not None else 0,
+            ACTS[act] if act is not None else -1, workspace.data_ptr(), _nbytes(workspace),
+            _PATHS[path] | _LAUNCH[launch])
+        if st != MOE_OK:
+            raise MoeError(st, "moe_qmm_plan_init")
+        self._run = lib().moe_qmm_plan_run
+        self._ref = ctypes.addressof(self._buf)
+
+    def __call__(self, x: torch.Tensor, ids: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+        """x [m, k], ids [m, n_expert_used], out [m, n_expert_used, n (or n/2)]: contiguous
+        tensors on the plan's device of the bound types (not re-checked here)."""
+        s = (stream or torch.cuda.current_stream(self.device)).cuda_stream
+        st = self._run(self._ref, x.data_ptr(), ids.data_ptr(), out.data_ptr(), s)
+        if st != MOE_OK:
+            raise MoeError(st, "moe_qmm_plan_run")
+        return out
 
 
 def qmm_id_ptrs(x: torch.Tensor, ids: torch.Tensor, packed_ptrs: torch.Tensor, scale_ptrs: torch.Tensor,

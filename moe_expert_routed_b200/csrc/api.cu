@@ -259,6 +259,76 @@ moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, co
                            workspace_bytes, stream, MOE_PATH_AUTO);
 }
 
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// What a moe_qmm_plan holds (inside the caller's opaque storage).
+struct PlanData {
+    uint64_t magic;
+    const void *packed, *scales, *aux, *bias;
+    void *workspace;
+    size_t workspace_bytes;
+    uint32_t m, k, n, group_size, bits, n_expert_used, num_experts;
+    int32_t fmt, x_dtype, out_dtype, bias_dtype, act;
+    uint32_t path;
+};
+static_assert(sizeof(PlanData) <= sizeof(moe_qmm_plan), "plan storage too small");
+constexpr uint64_t PLAN_MAGIC = 0x6d6f65706c616e31ull;
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_qmm_plan_init(moe_qmm_plan *plan, const void *packed, const void *scales, const void *aux,
+                             const void *expert_bias, uint32_t m, uint32_t k, uint32_t n,
+                             uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,
+                             uint32_t num_experts, moe_dtype x_dtype, moe_dtype out_dtype,
+                             moe_dtype bias_dtype, int32_t act, void *workspace, size_t workspace_bytes,
+                             moe_path path) {
+    if (!plan) return MOE_ERR_INVALID_ARGUMENT;
+    memset(plan, 0, sizeof(*plan));
+    // the operation's checks, with placeholders for the per-call pointers
+    const void *ph = packed;
+    moe_status v = validate(ph, (const uint32_t *)ph, packed, scales, aux, ph, m, k, n, group_size, bits, fmt,
+                            n_expert_used, num_experts, x_dtype, out_dtype);
+    if (v != MOE_OK) return v;
+    if (act < -1 || act > 2 || (act >= 0 && (n & 1u))) return MOE_ERR_INVALID_ARGUMENT;
+    if (expert_bias && ((int)bias_dtype < 0 || (int)bias_dtype > 2)) return MOE_ERR_INVALID_ARGUMENT;
+    const uint32_t flags = (uint32_t)path & ~0xFFu;
+    if (((uint32_t)path & 0xFFu) > 2 || (flags & ~(uint32_t)(MOE_LAUNCH_PDL | MOE_LAUNCH_EARLY_WEIGHTS)))
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
+    WsLayout L;
+    if (!ws_layout((uint64_t)m * n_expert_used, num_experts, &L)) return MOE_ERR_UNSUPPORTED;
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    PlanData d = {};
+    d.packed = packed; d.scales = scales; d.aux = aux; d.bias = expert_bias;
+    d.workspace = workspace; d.workspace_bytes = workspace_bytes;
+    d.m = m; d.k = k; d.n = n; d.group_size = group_size; d.bits = bits;
+    d.n_expert_used = n_expert_used; d.num_experts = num_experts;
+    d.fmt = (int32_t)fmt; d.x_dtype = (int32_t)x_dtype; d.out_dtype = (int32_t)out_dtype;
+    d.bias_dtype = expert_bias ? (int32_t)bias_dtype : (int32_t)MOE_F32;
+    d.act = act; d.path = (uint32_t)path;
+    d.magic = PLAN_MAGIC;
+    memcpy(plan, &d, sizeof(d));
+    return MOE_OK;
+}
+
+moe_status moe_qmm_plan_run(const moe_qmm_plan *plan, const void *x, const uint32_t *ids, void *out,
+                            moe_stream_t stream) {
+    if (!plan) return MOE_ERR_INVALID_ARGUMENT;
+    PlanData d;
+    memcpy(&d, plan, sizeof(d));
+    if (d.magic != PLAN_MAGIC) return MOE_ERR_INVALID_ARGUMENT;
+    return run(x, ids, d.packed, d.scales, d.aux, d.bias, out, d.m, d.k, d.n, d.group_size, d.bits,
+               (moe_fmt)d.fmt, d.n_expert_used, d.num_experts, (moe_dtype)d.x_dtype, (moe_dtype)d.out_dtype,
+               (moe_dtype)d.bias_dtype, d.workspace, d.workspace_bytes, stream, (moe_path)d.path,
+               PtrTables{nullptr, nullptr, nullptr}, d.act);
+}
+
 moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_used,
                             uint32_t num_experts, uint32_t tile_rows, uint32_t *counts,
                             uint32_t *offsets, uint32_t *sorted_pairs, uint32_t *tiles,

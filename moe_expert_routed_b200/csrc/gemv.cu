@@ -1118,7 +1118,7 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
             store_out(P.out, P.out_dtype, (size_t)p * nn + c, v);
         }
         c += RPI;
-        if (c >= nn) {
+        while (c >= nn) {  // pairs of fewer than RPI rows are stepped over whole
             c -= nn;
             p++;
         }

@@ -105,6 +105,26 @@ def test_glu_entry_rejects_before_cuda():
     assert call(bias=0, bdt=3, m=0) == 1  # without a bias its dtype is ignored; m=0 still rejected
 
 
+def test_plan_validation_before_cuda():
+    import ctypes
+    L = M.lib()
+    buf = ctypes.create_string_buffer(24 * 8)
+
+    def init(m=4, n=128, act=-1, bias=None, bdt=0, path=0, ws=4096, wsb=1 << 20):
+        return L.moe_qmm_plan_init(buf, 16, 16, 16, bias, m, 256, n, 32, 4, 0, 2, 8, 0, 0, bdt, act, ws, wsb, path)
+    assert init(m=0) == 1                 # the operation's own checks
+    assert init(act=3) == 1               # unknown activation
+    assert init(act=0, n=127) == 1        # gated output needs an even n
+    assert init(bias=16, bdt=4) == 1      # unknown bias dtype
+    assert init(path=0x400) == 1          # unknown launch flag
+    assert init(ws=None) == 1             # no workspace
+    assert init(wsb=16) == 3              # workspace too small
+    # a plan that failed to initialise is refused by run (no CUDA call is made)
+    assert L.moe_qmm_plan_run(buf, 16, 16, 16, None) == 1
+    assert L.moe_qmm_plan_run(None, 16, 16, 16, None) == 1
+    assert init() == 0                    # valid: only host-side state is written
+
+
 def test_pointer_table_entry_rejects_before_cuda():
     L = M.lib()
 

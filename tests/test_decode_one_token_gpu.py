@@ -26,6 +26,9 @@ CASES = [
     (2816, 1, 64, 8, 12, DT_BF16, DT_F32),    # one row per pair
     (1024, 48, 256, 4, 6, DT_BF16, DT_F32),   # groups of 256
     (4096, 24, 256, 3, 4, DT_F16, DT_F32),    # 128 units: handled by the other decode kernel
+    (96, 5, 32, 6, 9, DT_BF16, DT_F32),       # 4 lanes per row: 8 rows at once step over whole pairs
+    (224, 3, 32, 8, 10, DT_F16, DT_F32),      # 8 lanes per row, pairs of 3 rows
+    (1408, 7, 64, 8, 12, DT_BF16, DT_F32),    # 32 lanes per row, 4 rows per pass over pairs of 7
 ]
 
 
