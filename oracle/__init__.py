@@ -44,6 +44,8 @@ def lib():
         L.oracle_f16_to_double.restype = ctypes.c_double
         L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_to_double.restype = ctypes.c_double
+        L.oracle_e8m0_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0_to_double.restype = ctypes.c_double
         L.oracle_e2m1_to_double.argtypes = [ctypes.c_uint8]
         L.oracle_e2m1_to_double.restype = ctypes.c_double
         L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
@@ -99,6 +101,10 @@ def f16_to_double(bits: int) -> float:
 
 def e4m3_to_double(b: int) -> float:
     return lib().oracle_e4m3_to_double(int(b))
+
+
+def e8m0_to_double(b: int) -> float:
+    return lib().oracle_e8m0_to_double(int(b))
 
 
 def e2m1_to_double(c: int) -> float:

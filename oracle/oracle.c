@@ -25,7 +25,7 @@
  *   * affine 6-bit: 4 codes per 3-byte triplet read as one little-endian 24-bit
  *     integer, code j at bit 6*(j mod 4) of triplet floor(j/4)
  *     (quantized_matmul_id.rs, expert_weight_bytes: "triplets_per_row");
- *   * NVFP4: two E2M1 codes per byte, element 2i in the low nibble
+ *   * NVFP4 and MXFP4: two E2M1 codes per byte, element 2i in the low nibble
  *     (spark_model helpers_a.rs: routed weights stored [N, K/2]).
  *
  * Dequantisation of code c in group g = floor(j / group_size):
@@ -33,6 +33,9 @@
  *   codebook : codebook[c] * scale[e][col][g]                  (f16; fast_switch_patch.py
  *                                                              "cb[code] * scale")
  *   NVFP4    : e2m1(c) * e4m3(scale[e][col][floor(j/16)]) * scale2[e]
+ *   MXFP4    : e2m1(c) * e8m0(scale[e][col][floor(j/32)])   (spark_model helpers_a.rs:
+ *              native-MXFP4 routed experts carry one E8M0 scale per 32 values,
+ *              [N, K/32]; no second-level scale)
  *
  * Out-of-range ids (e >= num_experts) produce an all-zero output row and are
  * counted in *bad_ids.
@@ -54,7 +57,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { O_FMT_AFFINE = 0, O_FMT_CODEBOOK = 1, O_FMT_NVFP4 = 2 };
+enum { O_FMT_AFFINE = 0, O_FMT_CODEBOOK = 1, O_FMT_NVFP4 = 2, O_FMT_MXFP4 = 3 };
 enum { O_DT_F32 = 0, O_DT_BF16 = 1, O_DT_F16 = 2 };
 
 /* ---------------------------------------------------------------- decoders */
@@ -88,6 +91,12 @@ double oracle_e4m3_to_double(uint8_t b) {
     if (e == 0) mag = ldexp((double)f, -6 - 3);
     else mag = ldexp(1.0 + f / 8.0, e - 7);
     return s ? -mag : mag;
+}
+
+/* OCP Microscaling E8M0 scale: an unsigned biased exponent, 2^(b - 127); 0xFF is NaN. */
+double oracle_e8m0_to_double(uint8_t b) {
+    if (b == 0xFF) return NAN;
+    return ldexp(1.0, (int)b - 127);
 }
 
 /* OCP Microscaling FP4 E2M1: bias 1, no infinities or NaN, exponent field 0
@@ -153,7 +162,7 @@ void oracle_round_out(const double *in, void *out, uint64_t count, int out_dtype
 /* ------------------------------------------------------------ code storage */
 
 uint64_t oracle_row_bytes(int fmt, int bits, uint32_t k) {
-    if (fmt == O_FMT_NVFP4) return (uint64_t)k / 2;
+    if (fmt == O_FMT_NVFP4 || fmt == O_FMT_MXFP4) return (uint64_t)k / 2;
     if (fmt == O_FMT_AFFINE && bits == 6) return ((uint64_t)k + 3) / 4 * 3;
     uint32_t epw = 32u / (uint32_t)bits;
     return ((uint64_t)k + epw - 1) / epw * 4;
@@ -163,7 +172,7 @@ static unsigned bit_at(const uint8_t *row, uint64_t i) { return (row[i >> 3] >> 
 
 /* Start bit of element j inside its packed row. */
 static uint64_t code_start_bit(int fmt, int bits, uint32_t j) {
-    if (fmt == O_FMT_NVFP4) return 4ull * j;
+    if (fmt == O_FMT_NVFP4 || fmt == O_FMT_MXFP4) return 4ull * j;
     if (fmt == O_FMT_AFFINE && bits == 6) return 24ull * (j / 4) + 6ull * (j % 4);
     uint32_t epw = 32u / (uint32_t)bits;
     return 32ull * (j / epw) + (uint64_t)bits * (j % epw);
@@ -205,6 +214,8 @@ static double weight(const problem_t *P, uint32_t e, uint32_t col, uint32_t j) {
         double s = oracle_f16_to_double(((const uint16_t *)P->scales)[sidx]);
         return cb * s;
     }
+    if (P->fmt == O_FMT_MXFP4)
+        return oracle_e2m1_to_double((uint8_t)c) * oracle_e8m0_to_double(((const uint8_t *)P->scales)[sidx]);
     /* NVFP4 */
     double s = oracle_e4m3_to_double(((const uint8_t *)P->scales)[sidx]);
     double s2 = (double)((const float *)P->aux)[e];
@@ -277,7 +288,8 @@ static int make_problem(problem_t *P, const void *x, const uint32_t *ids, const 
     if (fmt == O_FMT_AFFINE && bits != 4 && bits != 6 && bits != 8) return -1;
     if (fmt == O_FMT_CODEBOOK && bits != 2 && bits != 3 && bits != 4) return -1;
     if (fmt == O_FMT_NVFP4 && (bits != 4 || group_size != 16 || (k & 1))) return -1;
-    if (fmt < 0 || fmt > 2 || x_dtype < 0 || x_dtype > 2) return -1;
+    if (fmt == O_FMT_MXFP4 && (bits != 4 || group_size != 32 || (k & 1))) return -1;
+    if (fmt < 0 || fmt > 3 || x_dtype < 0 || x_dtype > 2) return -1;
     P->x = x; P->ids = ids; P->packed = packed; P->scales = scales; P->aux = aux;
     P->m = m; P->k = k; P->n = n; P->group_size = group_size; P->bits = bits;
     P->n_expert_used = n_expert_used; P->num_experts = num_experts;

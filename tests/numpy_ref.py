@@ -3,8 +3,8 @@
 It differs from the oracle in every step that could hide a mistake:
 * codes are unpacked from whole little-endian u32 words / 24-bit triplets with
   array shifts (the word-level form of the packing), not bit by bit;
-* bf16 / f16 / E4M3 are decoded by torch / numpy dtype casts, E2M1 by the
-  OCP table in tests/golden/e2m1_values.txt;
+* bf16 / f16 / E4M3 / E8M0 are decoded by torch / numpy dtype casts, E2M1 by
+  the OCP table in tests/golden/e2m1_values.txt;
 * the contraction is one ``numpy.einsum`` in float64.
 """
 
@@ -15,7 +15,7 @@ import os
 import numpy as np
 import torch
 
-from workloads.gen import FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4, DT_F32, DT_BF16
+from workloads.gen import FMT_AFFINE, FMT_CODEBOOK, FMT_MXFP4, FMT_NVFP4, DT_F32, DT_BF16
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -42,11 +42,16 @@ def e4m3_to_f64(b):
     return t.to(torch.float64).numpy()
 
 
+def e8m0_to_f64(b):
+    t = torch.from_numpy(np.ascontiguousarray(b, dtype=np.uint8)).view(torch.float8_e8m0fnu)
+    return t.to(torch.float64).numpy()
+
+
 def unpack_codes(packed: np.ndarray, fmt: int, bits: int, k: int) -> np.ndarray:
     """packed [..., row_bytes] -> codes [..., k] (int64)."""
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
     lead = packed.shape[:-1]
-    if fmt == FMT_NVFP4:
+    if fmt in (FMT_NVFP4, FMT_MXFP4):
         lo = (packed & 0xF).astype(np.int64)
         hi = (packed >> 4).astype(np.int64)
         codes = np.stack([lo, hi], axis=-1).reshape(*lead, -1)
@@ -67,7 +72,7 @@ def pack_codes(codes: np.ndarray, fmt: int, bits: int) -> np.ndarray:
     """Inverse of unpack_codes for hand-built tests: codes [..., k] -> packed bytes."""
     codes = np.asarray(codes, dtype=np.int64)
     lead, k = codes.shape[:-1], codes.shape[-1]
-    if fmt == FMT_NVFP4:
+    if fmt in (FMT_NVFP4, FMT_MXFP4):
         c = np.zeros((*lead, k + (k & 1)), np.int64)
         c[..., :k] = codes
         c = c.reshape(*lead, -1, 2)
@@ -103,6 +108,8 @@ def dequant_dense(P) -> np.ndarray:
         cb = f16_to_f64(P.aux)
         s = f16_to_f64(P.scales)[..., g]
         return cb[codes] * s
+    if P.fmt == FMT_MXFP4:
+        return E2M1_TABLE[codes] * e8m0_to_f64(P.scales)[..., g]
     s = e4m3_to_f64(P.scales)[..., g]
     s2 = P.aux.astype(np.float64)[:, None, None]
     return E2M1_TABLE[codes] * s * s2

@@ -10,6 +10,7 @@ from .gen import (  # noqa: F401
     FMT_AFFINE,
     FMT_CODEBOOK,
     FMT_NVFP4,
+    FMT_MXFP4,
     DT_F32,
     DT_BF16,
     DT_F16,

@@ -10,9 +10,10 @@ the layout the operation reads:
   are uniformly random codes (padding bits included, which the operation must
   ignore).
 * ``scales``  [E, n, ceil(k/group_size)]: bf16 bits (affine), f16 bits
-  (codebook) or E4M3 bytes (NVFP4, one per 16 values).
+  (codebook), E4M3 bytes (NVFP4, one per 16 values) or E8M0 bytes (MXFP4, one
+  per 32 values).
 * ``aux``     affine: bf16 bias bits [E, n, G]; codebook: f16 centroid bits
-  [2**bits]; NVFP4: float32 scale2 [E].
+  [2**bits]; NVFP4: float32 scale2 [E]; MXFP4: one unused float32.
 
 Conversions of freshly drawn float32 values to bf16 / f16 / E4M3 bit patterns
 use torch/numpy dtype casts (round to nearest even). Nothing here decodes codes
@@ -30,12 +31,13 @@ from scipy.special import ndtr, ndtri
 FMT_AFFINE = 0
 FMT_CODEBOOK = 1
 FMT_NVFP4 = 2
+FMT_MXFP4 = 3
 DT_F32 = 0
 DT_BF16 = 1
 DT_F16 = 2
 
 DT_NAMES = {DT_F32: "f32", DT_BF16: "bf16", DT_F16: "f16"}
-FMT_NAMES = {FMT_AFFINE: "affine", FMT_CODEBOOK: "codebook", FMT_NVFP4: "nvfp4"}
+FMT_NAMES = {FMT_AFFINE: "affine", FMT_CODEBOOK: "codebook", FMT_NVFP4: "nvfp4", FMT_MXFP4: "mxfp4"}
 
 
 def storage_row_bytes(fmt: int, bits: int, k: int) -> int:
@@ -51,7 +53,7 @@ def storage_row_bytes(fmt: int, bits: int, k: int) -> int:
     if fmt in (FMT_AFFINE, FMT_CODEBOOK):
         epw = 32 // bits
         return (k + epw - 1) // epw * 4
-    if fmt == FMT_NVFP4:
+    if fmt in (FMT_NVFP4, FMT_MXFP4):
         return k // 2
     raise ValueError(f"unknown format {fmt}")
 
@@ -190,6 +192,7 @@ def make_problem(
     ids: str = "uniform",
     zipf_s: float = 1.1,
     scale2: float = 1.0 / 448.0,
+    mx_sigma: float = 0.02,
 ) -> Problem:
     """Draw one problem instance. Order of draws: ids, x, packed codes, scales, aux."""
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -225,6 +228,15 @@ def make_problem(
         amax = ndtri(0.5 * (1.0 + u ** (1.0 / 16.0)))
         scales = e4m3_bits((amax / 6.0).astype(np.float32))
         aux = np.full((num_experts,), scale2, dtype=np.float32)
+    elif fmt == FMT_MXFP4:
+        if group_size != 32:
+            raise ValueError("MXFP4 uses 32-value blocks")
+        # OCP MX shared exponent of a block of 32 weights ~ N(0, mx_sigma^2):
+        # floor(log2(amax)) - 2 (E2M1's largest exponent), biased by 127
+        u = rng.random(size=(num_experts, n, G))
+        amax = mx_sigma * ndtri(0.5 * (1.0 + u ** (1.0 / 32.0)))
+        scales = (np.floor(np.log2(amax)) - 2 + 127).clip(0, 254).astype(np.uint8)
+        aux = np.zeros((1,), dtype=np.float32)
     else:
         raise ValueError(fmt)
     return Problem(
