@@ -458,7 +458,10 @@ def run_ours(args, dist: Dist):
     # this kernel.
     achieved = per_call["gate_up"]["GB_per_s"]
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": GATE_UP_DRAM_BYTES,
+                "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "traffic_note": f"{GATE_UP_DRAM_BYTES} B per launch (= the algorithmic bytes) in the last ncu "
+                                "capture, taken before the launch-dependency and gated-output changes to "
+                                "the kernel; null until re-captured",
                 "algorithmic_bytes": W.bytes((0,)) / W.G,
                 "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
                 "kernel": "gemv_aff4_rows (rows of all pairs split evenly over the SMs), gate/up launch",

@@ -44,6 +44,14 @@
  *                    scale E4M3 bytes [E, n, k/16], scale2 f32 [E]
  *                    (spark_model quant_dispatch.rs, w4a16_gemv: B packed,
  *                    B_scale, scale2).
+ *   MOE_FMT_MXFP4    bits 4, group_size 32: E2M1 codes stored as for NVFP4.
+ *                    w = e2m1(code) * 2^(scale - 127), scale E8M0 bytes
+ *                    [E, n, k/32] (0xFF is NaN); no aux array (spark_model
+ *                    helpers_a.rs: native-MXFP4 routed experts, per-32 E8M0
+ *                    scales [N, K/32]). Computed by the CUDA-core decode
+ *                    kernels on every path: MOE_PATH_GROUPED returns
+ *                    MOE_ERR_UNSUPPORTED and MOE_PATH_AUTO uses the routed GEMV
+ *                    for large calls.
  */
 #ifndef MOE_QMM_H
 #define MOE_QMM_H
@@ -57,7 +65,7 @@ extern "C" {
 
 typedef struct CUstream_st *moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
 
-typedef enum { MOE_FMT_AFFINE = 0, MOE_FMT_CODEBOOK = 1, MOE_FMT_NVFP4 = 2 } moe_fmt;
+typedef enum { MOE_FMT_AFFINE = 0, MOE_FMT_CODEBOOK = 1, MOE_FMT_NVFP4 = 2, MOE_FMT_MXFP4 = 3 } moe_fmt;
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_F16 = 2 } moe_dtype;
 typedef enum {
     MOE_OK = 0,
@@ -114,7 +122,8 @@ typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_GROUPED = 2 } mo
  *   scales   [num_experts, n, ceil(k / group_size)]: bf16 (AFFINE), f16 (CODEBOOK),
  *            E4M3 bytes (NVFP4).
  *   aux      AFFINE: biases bf16 [num_experts, n, ceil(k/group_size)];
- *            CODEBOOK: codebook f16 [2^bits]; NVFP4: scale2 f32 [num_experts].
+ *            CODEBOOK: codebook f16 [2^bits]; NVFP4: scale2 f32 [num_experts];
+ *            MXFP4: unused (may be NULL).
  *   out      [m, n_expert_used, n] of out_dtype (f32, bf16 or f16); every
  *            element is written (zeros for out-of-range ids). Results are rounded
  *            once from the fp32 accumulator, to nearest even.

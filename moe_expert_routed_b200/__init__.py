@@ -21,7 +21,7 @@ import os
 
 import torch
 
-FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4 = 0, 1, 2
+FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4, FMT_MXFP4 = 0, 1, 2, 3
 DT_F32, DT_BF16, DT_F16 = 0, 1, 2
 PATH_AUTO, PATH_DECODE, PATH_GROUPED = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "grouped": PATH_GROUPED}
@@ -149,6 +149,8 @@ def _validate_only(x, ids, packed, scales, aux, *, n, group_size, bits, fmt, num
         raise ValueError("quantized_matmul_id: ids must be a [M, n_expert_used] 32-bit integer tensor")
     m, k = x.shape
     n_expert_used = ids.shape[1]
+    if fmt not in (FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4, FMT_MXFP4):
+        raise ValueError(f"quantized_matmul_id: unknown format {fmt}")
     if bits not in ({4, 6, 8} if fmt == FMT_AFFINE else {2, 3, 4} if fmt == FMT_CODEBOOK else {4}):
         raise ValueError(f"quantized_matmul_id: unsupported bits value {bits} for format {fmt}")
     if m == 0 or k == 0 or n == 0:
@@ -167,13 +169,14 @@ def _validate_only(x, ids, packed, scales, aux, *, n, group_size, bits, fmt, num
         raise ValueError(f"quantized_matmul_id: weight buffer too small: expected at least {total_w} "
                          f"bytes for {num_experts} experts, got {_nbytes(packed)}")
     G = (k + group_size - 1) // group_size
-    per_s = {FMT_AFFINE: 2, FMT_CODEBOOK: 2, FMT_NVFP4: 1}[fmt]
+    per_s = {FMT_AFFINE: 2, FMT_CODEBOOK: 2, FMT_NVFP4: 1, FMT_MXFP4: 1}[fmt]
     total_s = num_experts * n * G * per_s
     if _nbytes(scales) < total_s:
         raise ValueError(f"quantized_matmul_id: scales buffer too small: expected at least {total_s} "
                          f"bytes, got {_nbytes(scales)}")
-    aux_need = {FMT_AFFINE: total_s, FMT_CODEBOOK: 2 * (1 << bits), FMT_NVFP4: 4 * num_experts}[fmt]
-    aux_name = {FMT_AFFINE: "biases", FMT_CODEBOOK: "codebook", FMT_NVFP4: "scale2"}[fmt]
+    aux_need = {FMT_AFFINE: total_s, FMT_CODEBOOK: 2 * (1 << bits), FMT_NVFP4: 4 * num_experts,
+                FMT_MXFP4: 0}[fmt]
+    aux_name = {FMT_AFFINE: "biases", FMT_CODEBOOK: "codebook", FMT_NVFP4: "scale2", FMT_MXFP4: "aux"}[fmt]
     if _nbytes(aux) < aux_need:
         raise ValueError(f"quantized_matmul_id: {aux_name} buffer too small: expected at least "
                          f"{aux_need} bytes, got {_nbytes(aux)}")

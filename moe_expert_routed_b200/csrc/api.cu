@@ -35,7 +35,7 @@ bool ws_layout(uint64_t R, uint32_t E, WsLayout *L) {
 }
 
 static uint64_t row_bytes_of(int fmt, uint32_t bits, uint32_t k) {
-    if (fmt == FMT_NVFP4) return k / 2u;
+    if (fmt == FMT_NVFP4 || fmt == FMT_MXFP4) return k / 2u;
     if (fmt == FMT_AFFINE && bits == 6) return ((uint64_t)k + 3) / 4 * 3;
     const uint32_t epw = 32u / bits;
     return ((uint64_t)k + epw - 1) / epw * 4;
@@ -49,7 +49,7 @@ extern "C" {
 
 size_t moe_packed_row_bytes(moe_fmt fmt, uint32_t bits, uint32_t k) {
     if (kind_of((int)fmt, (int)bits) < 0) return 0;
-    if (fmt == MOE_FMT_NVFP4 && (k & 1u)) return 0;
+    if ((fmt == MOE_FMT_NVFP4 || fmt == MOE_FMT_MXFP4) && (k & 1u)) return 0;
     return (size_t)row_bytes_of((int)fmt, bits, k);
 }
 
@@ -83,8 +83,10 @@ static moe_status validate(const void *x, const uint32_t *ids, const void *packe
     if (!m || !k || !n || !group_size || !n_expert_used || !num_experts) return MOE_ERR_INVALID_ARGUMENT;
     if ((int)x_dtype < 0 || (int)x_dtype > 2 || (int)out_dtype < 0 || (int)out_dtype > 2)
         return MOE_ERR_INVALID_ARGUMENT;
-    if (!x || !ids || !packed || !scales || !aux || !out) return MOE_ERR_INVALID_ARGUMENT;
+    if (!x || !ids || !packed || !scales || !out) return MOE_ERR_INVALID_ARGUMENT;
+    if (!aux && fmt != MOE_FMT_MXFP4) return MOE_ERR_INVALID_ARGUMENT;  // MXFP4 has no aux array
     if (fmt == MOE_FMT_NVFP4 && (group_size != 16 || (k & 1u))) return MOE_ERR_INVALID_ARGUMENT;
+    if (fmt == MOE_FMT_MXFP4 && (group_size != 32 || (k & 1u))) return MOE_ERR_INVALID_ARGUMENT;
     if (k % group_size != 0) return MOE_ERR_UNSUPPORTED;
     if ((uint64_t)m * n_expert_used > 0x7FFFFFFFull) return MOE_ERR_UNSUPPORTED;
     if (row_bytes_of((int)fmt, bits, k) > 0xFFFFFFFFull) return MOE_ERR_UNSUPPORTED;

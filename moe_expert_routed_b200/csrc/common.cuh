@@ -9,11 +9,11 @@
 
 namespace moe {
 
-enum Fmt : int { FMT_AFFINE = 0, FMT_CODEBOOK = 1, FMT_NVFP4 = 2 };
+enum Fmt : int { FMT_AFFINE = 0, FMT_CODEBOOK = 1, FMT_NVFP4 = 2, FMT_MXFP4 = 3 };
 enum DType : int { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
 
 // Storage kinds: one per (format, bits) pair the kernels are specialised for.
-enum Kind : int { K_AFF4 = 0, K_AFF6, K_AFF8, K_CB2, K_CB3, K_CB4, K_NVFP4, K_COUNT };
+enum Kind : int { K_AFF4 = 0, K_AFF6, K_AFF8, K_CB2, K_CB3, K_CB4, K_NVFP4, K_MXFP4, K_COUNT };
 
 // Device error word bits (first u32 of the workspace).
 constexpr uint32_t ERR_BAD_ID = 1u;
@@ -25,6 +25,7 @@ __host__ __device__ inline int kind_of(int fmt, int bits) {
     if (fmt == FMT_AFFINE) return bits == 4 ? K_AFF4 : bits == 6 ? K_AFF6 : bits == 8 ? K_AFF8 : -1;
     if (fmt == FMT_CODEBOOK) return bits == 2 ? K_CB2 : bits == 3 ? K_CB3 : bits == 4 ? K_CB4 : -1;
     if (fmt == FMT_NVFP4) return bits == 4 ? K_NVFP4 : -1;
+    if (fmt == FMT_MXFP4) return bits == 4 ? K_MXFP4 : -1;
     return -1;
 }
 
@@ -56,6 +57,12 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
 }
 
 // OCP MX FP4 E2M1: bias 1, exponent field 0 = subnormal m * 0.5, no NaN/Inf.
+// OCP Microscaling E8M0 scale byte: 2^(b - 127); 0xFF is NaN, 0 the subnormal 2^-127.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
+    if (b == 0xFFu) return __uint_as_float(0x7FC00000u);
+    return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
 __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
     uint32_t s = (c >> 3) & 1u, e = (c >> 1) & 3u, m = c & 1u;
     float mag = (e == 0u) ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));

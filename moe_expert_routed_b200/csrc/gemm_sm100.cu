@@ -785,6 +785,7 @@ cudaError_t launch_kind(const GemmParams &P, const GemmPlan &pl, int kind, int x
 }  // namespace
 
 bool gemm_supported(const QmmArgs &a) {
+    if (a.kind == K_MXFP4) return false;  // MXFP4 runs on the CUDA-core paths
     const uint32_t gs = a.group_size;
     if (gs < 16 || (gs & (gs - 1)) != 0) return false;
     if (a.k % 8 != 0 || a.k % gs != 0) return false;

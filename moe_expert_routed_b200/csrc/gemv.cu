@@ -43,11 +43,12 @@ template <> struct UnitShape<K_CB2> { static constexpr int UW = 4, UC = 64; };
 template <> struct UnitShape<K_CB3> { static constexpr int UW = 4, UC = 40; };
 template <> struct UnitShape<K_CB4> { static constexpr int UW = 4, UC = 32; };
 template <> struct UnitShape<K_NVFP4> { static constexpr int UW = 4, UC = 32; };
+template <> struct UnitShape<K_MXFP4> { static constexpr int UW = 4, UC = 32; };
 
 // Code i (compile-time) of a unit held in registers.
 template <int KIND, int I, int UW>
 __device__ __forceinline__ uint32_t unit_code(const uint32_t (&w)[UW]) {
-    if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
+    if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4 || KIND == K_MXFP4) {
         return (w[I / 8] >> (4 * (I % 8))) & 15u;
     } else if constexpr (KIND == K_AFF8) {
         return (w[I / 4] >> (8 * (I % 4))) & 255u;
@@ -114,6 +115,9 @@ __device__ __forceinline__ void load_group(const GemvCtx &c, uint32_t g, float &
     } else if constexpr (KIND == K_NVFP4) {
         s = e4m3_to_f32(__ldg((const uint8_t *)c.scales + g));
         b = 0.f;
+    } else if constexpr (KIND == K_MXFP4) {
+        s = e8m0_to_f32(__ldg((const uint8_t *)c.scales + g));
+        b = 0.f;
     } else {
         s = f16_bits_to_f32(__ldg((const unsigned short *)c.scales + g));
         b = 0.f;
@@ -124,7 +128,7 @@ template <int KIND>
 __device__ __forceinline__ float dequant(uint32_t code, float s, float b, const float *cb) {
     if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) {
         return fmaf((float)code, s, b);
-    } else if constexpr (KIND == K_NVFP4) {
+    } else if constexpr (KIND == K_NVFP4 || KIND == K_MXFP4) {
         return e2m1_to_f32(code) * s;
     } else {
         return cb[code] * s;
@@ -197,7 +201,7 @@ gemv_kernel(const GemvParams P) {
         sbase = (const uint8_t *)__ldg(P.scale_ptrs + expert);
         bbase = AFF ? (const uint8_t *)__ldg(P.bias_ptrs + expert) : nullptr;
         const uintptr_t sa = (uintptr_t)sbase | (AFF ? (uintptr_t)bbase : 0u);
-        if (!sbase || (AFF && !bbase) || (KIND != K_NVFP4 && (sa & 1u))) {
+        if (!sbase || (AFF && !bbase) || (KIND != K_NVFP4 && KIND != K_MXFP4 && (sa & 1u))) {
             // scales / biases missing or not 2-byte aligned: skip the expert, flag it
             if (tid == 0 && blockIdx.x == 0) atomicOr(P.err, ERR_BAD_POINTER);
             return;
@@ -217,7 +221,7 @@ gemv_kernel(const GemvParams P) {
     c.gs = P.gs;
     c.groups = P.groups;
     c.codebook = (const uint16_t *)P.aux;
-    if constexpr (KIND == K_NVFP4) {
+    if constexpr (KIND == K_NVFP4 || KIND == K_MXFP4) {  // byte scales
         c.scales = (const uint8_t *)sbase + row_index * P.groups;
         c.biases = nullptr;
     } else {
@@ -1346,6 +1350,7 @@ cudaError_t launch_kind(const GemvParams &P, int kind, uint32_t npb, dim3 grid, 
         case K_CB3: return launch_npb<K_CB3, FUSED>(P, npb, grid, st);
         case K_CB4: return launch_npb<K_CB4, FUSED>(P, npb, grid, st);
         case K_NVFP4: return launch_npb<K_NVFP4, FUSED>(P, npb, grid, st);
+        case K_MXFP4: return launch_npb<K_MXFP4, FUSED>(P, npb, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1358,6 +1363,7 @@ int unit_codes(int kind) {
         case K_CB2: return UnitShape<K_CB2>::UC;
         case K_CB3: return UnitShape<K_CB3>::UC;
         case K_CB4: return UnitShape<K_CB4>::UC;
+        case K_MXFP4: return UnitShape<K_MXFP4>::UC;
         default: return UnitShape<K_NVFP4>::UC;
     }
 }

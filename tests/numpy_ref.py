@@ -143,4 +143,6 @@ def dequant_expert(P, e: int) -> np.ndarray:
         return codes * bf16_to_f64(P.scales[e])[:, g] + bf16_to_f64(P.aux[e])[:, g]
     if P.fmt == FMT_CODEBOOK:
         return f16_to_f64(P.aux)[codes] * f16_to_f64(P.scales[e])[:, g]
+    if P.fmt == FMT_MXFP4:
+        return E2M1_TABLE[codes] * e8m0_to_f64(P.scales[e])[:, g]
     return E2M1_TABLE[codes] * e4m3_to_f64(P.scales[e])[:, g] * float(P.aux[e])

@@ -42,6 +42,9 @@ def test_row_bytes_match_oracle(fmt, bits, k):
 def test_row_bytes_invalid():
     assert M.packed_row_bytes(FMT_AFFINE, 5, 64) == 0
     assert M.packed_row_bytes(FMT_NVFP4, 4, 63) == 0
+    assert M.packed_row_bytes(3, 4, 63) == 0      # MXFP4: two codes per byte, k even
+    assert M.packed_row_bytes(3, 4, 2816) == 1408
+    assert M.packed_row_bytes(3, 3, 64) == 0
     assert M.packed_row_bytes(FMT_CODEBOOK, 8, 64) == 0
 
 
@@ -63,7 +66,8 @@ def _call(**kw):
 
 
 @pytest.mark.parametrize("kw", [dict(m=0), dict(k=0), dict(n=0), dict(gs=0), dict(topk=0),
-                                dict(E=0), dict(bits=5), dict(bits=3), dict(fmt=3),
+                                dict(E=0), dict(bits=5), dict(bits=3), dict(fmt=4),
+                                dict(fmt=3, gs=16), dict(fmt=3, gs=32, k=255), dict(fmt=3, bits=3),
                                 dict(fmt=2, bits=4, gs=32), dict(fmt=2, bits=4, gs=16, k=255),
                                 dict(fmt=1, bits=8), dict(x=0), dict(ids=0), dict(packed=0),
                                 dict(scales=0), dict(aux=0), dict(out=0), dict(ws=0),
