@@ -38,7 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
+METRIC = "µs/call; effective HBM GB/s (decode) and TFLOP/s (canvas/prefill) vs roofline"
 N_LAYERS = 16
 GRAPH_STEPS = 1000
 # dram__bytes_read.sum + dram__bytes_write.sum of one gate/up launch of the decode
