@@ -180,11 +180,12 @@ moe_status moe_qmm_id_bias(const void *x, const uint32_t *ids, const void *packe
  *                is skipped, the expert-parallel remote convention): the rows of
  *                its pairs are left untouched.
  *   scale_ptrs   [num_experts] u64: expert e's scales [n, ceil(k/gs)] (bf16 affine,
- *                f16 codebook: 2-byte aligned; u8 E4M3 for NVFP4).
+ *                f16 codebook: 2-byte aligned; u8 E4M3 for NVFP4, u8 E8M0 for MXFP4).
  *   bias_ptrs    [num_experts] u64: AFFINE expert e's biases [n, ceil(k/gs)] bf16
  *                (2-byte aligned); ignored otherwise (may be null).
  *   aux          CODEBOOK: f16 codebook [2^bits]; NVFP4: f32 scale2 [num_experts]
- *                (the table's scale2_vals); ignored for AFFINE.
+ *                (the table's scale2_vals); ignored for AFFINE and MXFP4 (may be
+ *                NULL for MXFP4).
  * The tables and every buffer they name are caller-owned device memory. Paths
  * as moe_qmm_id_path. The CUDA-core path takes code buffers at any alignment;
  * the grouped GEMM needs 8-byte aligned code buffers (4 for 3-bit codebook
