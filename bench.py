@@ -602,6 +602,72 @@ def run_grouped(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Decode with m = 1, 2, 4, 8 tokens (top-8 of 128 experts), gate/up and down
+    projections timed separately: a CUDA graph of calls with fresh ids and x each
+    call and 16 rotated weight copies. Effective GB/s counts the distinct experts
+    each call actually touches (E[D] = 8, 15.5, 29.1, 51.6 for uniform ids)."""
+    import types
+
+    import moe_expert_routed_b200 as M
+    from workloads import config_problem
+    from workloads.gen import bf16_bits, distinct_uniform_ids
+    from workloads.torch_io import to_device
+
+    calls = 200
+    rng = np.random.Generator(np.random.PCG64(77))
+    sampler = clocks_sampler(torch.cuda.current_device())
+    pk = peaks()
+    rows = []
+    for name in ("decode_gate_up", "decode_down"):
+        P = config_problem(name)
+        base = to_device(P)
+        layers = [{k: base[k].clone() for k in ("packed", "scales", "aux")} for _ in range(N_LAYERS)]
+        for m in (1, 2, 4, 8):
+            ids = distinct_uniform_ids(rng, m * calls, 8, P.num_experts).reshape(calls, m, 8)
+            x = bf16_bits(rng.standard_normal((calls, m, P.k), dtype=np.float32))
+            d_ids = torch.from_numpy(ids.view(np.int32)).cuda()
+            d_x = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+            out = torch.empty((calls, m, 8, P.n), dtype=torch.float32, device="cuda")
+            ws = M.new_workspace(m, 8, P.num_experts)
+            Pm = types.SimpleNamespace(row_bytes=P.row_bytes, groups=P.groups, fmt=P.fmt, n=P.n, k=P.k,
+                                       bits=P.bits, num_experts=P.num_experts, m=m, R=8 * m,
+                                       x_dtype=P.x_dtype, out_dtype=P.out_dtype)
+            nbytes = sum(alg_bytes(Pm, ids[c]) for c in range(calls))
+            distinct = float(np.mean([np.unique(ids[c]).size for c in range(calls)]))
+
+            def one(c):
+                L = layers[c % N_LAYERS]
+                M.qmm_id(d_x[c], d_ids[c], L["packed"], L["scales"], L["aux"], n=P.n,
+                         group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
+                         out=out[c], workspace=ws)
+
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(st):
+                for c in range(4):
+                    one(c)
+            torch.cuda.current_stream().wait_stream(st)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for c in range(calls):
+                    one(c)
+            time_graph(g, max(3, args.warmup // calls))
+            reps = max(1, args.steps // calls)
+            secs = time_graph(g, reps)
+            del g
+            us = secs / (reps * calls) * 1e6
+            gbs = nbytes * reps / secs / 1e9
+            rows.append({"projection": name.replace("decode_", ""), "m": m, "distinct_experts": distinct,
+                         "us_per_call": us, "GB_per_s": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"]})
+    line = {"sweep": "decode m=1..8 (E128 top8, affine 4-bit g64, bf16 x, f32 out), per projection",
+            "rows": rows, "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": pk["source"],
+            "timing": f"CUDA graph of {calls} calls, fresh ids and x per call, {N_LAYERS} rotated weight copies",
+            "clocks": clocks_summary(sampler)}
+    print(json.dumps(line), flush=True)
+
+
 def run_probe(args):
     """A few untimed calls of one workload (for profiler captures): decode runs the
     gate/up projection `reps` times, then the down projection `reps` times; the
@@ -641,10 +707,15 @@ def main():
     ap.add_argument("--probe", choices=["decode", "canvas", "prefill", "skewed"],
                     help="run a few untimed calls (for profiler captures) and exit")
     ap.add_argument("--reps", type=int, default=4)
+    ap.add_argument("--sweep", action="store_true",
+                    help="decode m = 1, 2, 4, 8 curve (one GPU), one JSON line, instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.probe:
         run_probe(args)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
     dist = Dist(args.gpus)
     try:
