@@ -360,6 +360,28 @@ def oracle_decode_sample(budget_s: float = 12.0):
         f"{secs:.1f} s on {threads} threads")
 
 
+def oracle_single_thread():
+    """The oracle on one host thread: one tiny call and one full decode step."""
+    import oracle
+    from workloads import config_problem
+
+    res = {}
+    P = config_problem("tiny")
+    t0 = time.perf_counter()
+    oracle.qmm_id(P, nthreads=1)
+    res["tiny_ms_per_call"] = (time.perf_counter() - t0) * 1e3
+    secs, nbytes = 0.0, 0.0
+    for name in ("decode_gate_up", "decode_down"):
+        P = config_problem(name)
+        t0 = time.perf_counter()
+        oracle.qmm_id(P, nthreads=1)
+        secs += time.perf_counter() - t0
+        nbytes += alg_bytes(P, P.ids.reshape(-1))
+    res["decode_step_ms"] = secs * 1e3
+    res["decode_step_GB_per_s"] = nbytes / secs / 1e9
+    return res
+
+
 # --------------------------------------------------------------------- main
 
 def run_reference(args, dist: Dist):
@@ -497,7 +519,7 @@ def run_ours(args, dist: Dist):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         v, s, threads, sample = oracle_decode_sample(args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample, "single_thread": oracle_single_thread()}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     del g
