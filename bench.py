@@ -1,25 +1,31 @@
 """Benchmark of the expert-routed quantized matmul on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config decode|canvas|prefill|skewed]
+                    [--config decode|canvas|prefill|skewed] [--sweep] [--no-extras]
 
 Default workload ("decode"): one MoE decode step for one token: the gate/up
 projection (128 experts, top-8, k=2816, n=1408) followed by the down projection
 (k=704, n=2816), both 4-bit affine with group 64, bf16 x, f32 out. Every step
 uses fresh ids (8 distinct uniform experts), fresh x, and the next of 16 copies
 of the expert weights (6.9 GB rotated, far above the 126 MB L2), so no step
-finds its weights in L2. The K timed steps are replayed from CUDA graphs of up
-to 1000 steps (launch overhead of the graph only, no host work).
+finds its weights in L2. W untimed warm-up steps, then exactly K timed steps
+replayed from a CUDA graph (up to 1000 steps per graph).
 
 Metric: effective HBM GB/s = algorithmic bytes / time, algorithmic bytes = the
 touched experts' packed codes + scales + biases read once, plus x and out.
-Also reported: us per call of each projection, the roofline fraction against
-MEASURED_PEAKS.json's copy bandwidth, the end-to-end number through the Python
-API with host buffers, and the CPU oracle on a bounded sample.
+The same JSON line also carries, measured outside the timed region:
+  per_call     each decode projection alone (graphs of 100 calls, median of 5)
+  roofline     the dominant kernel (gate/up) against MEASURED_PEAKS.json
+  e2e          the decode step through the Python API with host buffers
+  per_config   the canvas, prefill and skewed workloads (routing + tcgen05
+               grouped GEMM): us/call, TFLOP/s, GB/s and roofline fractions
+  sweep        decode with m = 1, 2, 4, 8 tokens per projection
+  cpu_baseline the CPU oracle on a bounded sample of the decode step
 
 --impl reference times the CPU oracle (the only reference there is) on a
 bounded sample of the same workload. N > 1: independent replicas, one per GPU
-(the operation has no exchange step), value = total bytes / max time.
+(the operation has no exchange step), value = total bytes / max time; the
+per_config and sweep entries are measured at N = 1 only.
 """
 
 from __future__ import annotations
@@ -40,10 +46,14 @@ sys.path.insert(0, ROOT)
 
 METRIC = "µs/call; effective HBM GB/s (decode) and TFLOP/s (canvas/prefill) vs roofline"
 N_LAYERS = 16
-GRAPH_STEPS = 1000
+GRAPH_STEPS = 1000   # longest graph of timed steps (more steps replay it)
+GRAPH_CALLS = 100    # calls per graph for the per-call figures
+REPEATS = 5          # per-call figures: median of this many graph replays
 # dram__bytes_read.sum + dram__bytes_write.sum of one gate/up launch of the decode
-# kernel, from one ncu capture of it (cold L2)
-GATE_UP_DRAM_BYTES = 17875200
+# kernel, from one ncu capture of it (cold L2); None until captured for the current
+# kernel
+GATE_UP_DRAM_BYTES = None
+GATE_UP_TRAFFIC_NOTE = "not yet captured for the current kernel"
 
 
 def peaks():
@@ -168,9 +178,12 @@ def clocks_summary(proc):
 # ------------------------------------------------------------- our workload
 
 class DecodeWorkload:
-    """gate/up + down projections of one decode token, rotating weight copies."""
+    """gate/up + down projections of one decode token, rotating weight copies.
 
-    def __init__(self, steps_per_graph: int, seed: int = 2, pdl: bool = True):
+    G sets of fresh ids (8 distinct uniform experts) and x rows; step s uses set
+    s % G and weight copy s % N_LAYERS."""
+
+    def __init__(self, G: int, seed: int = 2, pdl: bool = True):
         import moe_expert_routed_b200 as M
         from workloads.torch_io import to_device
         from workloads import config_problem
@@ -182,7 +195,7 @@ class DecodeWorkload:
         # the previous kernel before reading anything); down also streams its weights
         # early, since its ids were ready before gate/up began
         self.launch = ("pdl", "early_weights") if pdl else (None, None)
-        self.G = steps_per_graph
+        self.G = G
         rng = np.random.Generator(np.random.PCG64(seed + 100))
         self.layers = []
         for P in self.projs:
@@ -192,51 +205,92 @@ class DecodeWorkload:
                 copies.append({k: (v.clone() if k in ("packed", "scales", "aux") else v)
                                for k, v in base.items()})
             self.layers.append(copies)
-        # fresh ids and x for every step of the graph
-        self.ids = [torch.from_numpy(distinct_uniform_ids(rng, self.G, 8, P.num_experts)
+        self.ids = [torch.from_numpy(distinct_uniform_ids(rng, G, 8, P.num_experts)
                                      .view(np.int32)).cuda() for P in self.projs]
-        self.x = [torch.from_numpy(bf16_bits(rng.standard_normal((self.G, P.k), dtype=np.float32))
+        self.x = [torch.from_numpy(bf16_bits(rng.standard_normal((G, P.k), dtype=np.float32))
                                    .view(np.int16)).view(torch.bfloat16).cuda() for P in self.projs]
-        self.out = [torch.empty((self.G, 8, P.n), dtype=torch.float32, device="cuda")
-                    for P in self.projs]
+        self.out = [torch.empty((G, 8, P.n), dtype=torch.float32, device="cuda") for P in self.projs]
         # gated gate/up output: act(gate) * up, n/2 columns
-        self.out_glu = torch.empty((self.G, 8, self.projs[0].n // 2), dtype=torch.float32, device="cuda")
+        self.out_glu = torch.empty((G, 8, self.projs[0].n // 2), dtype=torch.float32, device="cuda")
         self.ws = [M.new_workspace(1, 8, P.num_experts) for P in self.projs]
-        self.step_bytes = [
-            [alg_bytes(P, self.ids[i][s].cpu().numpy().view(np.uint32)) for s in range(self.G)]
+        self.set_bytes = [
+            [alg_bytes(P, self.ids[i][s].cpu().numpy().view(np.uint32)) for s in range(G)]
             for i, P in enumerate(self.projs)]
 
     def call(self, proj: int, s: int, act=None, launch=None):
         P = self.projs[proj]
         L = self.layers[proj][s % N_LAYERS]
-        self.M.qmm_id(self.x[proj][s:s + 1], self.ids[proj][s:s + 1], L["packed"], L["scales"],
+        i = s % self.G
+        self.M.qmm_id(self.x[proj][i:i + 1], self.ids[proj][i:i + 1], L["packed"], L["scales"],
                       L["aux"], n=P.n, group_size=P.group_size, bits=P.bits, fmt=P.fmt,
-                      num_experts=P.num_experts, out=self.out_glu[s] if act else self.out[proj][s],
+                      num_experts=P.num_experts, out=self.out_glu[i] if act else self.out[proj][i],
                       workspace=self.ws[proj], act=act, launch=launch)
 
-    def step(self, s: int, projs=(0, 1), act=None):
-        # the step's launch modes apply to the full gate/up + down sequence only
+    def step(self, s: int, projs=(0, 1), act=None, launch=None):
+        """One step: the given projections of set s. launch None: the step's own
+        launch modes for the full gate/up + down sequence, plain stream order for a
+        single projection; otherwise that launch mode for every call."""
         full = tuple(projs) == (0, 1)
         for p in projs:
-            self.call(p, s, act, self.launch[p] if full else None)
+            self.call(p, s, act, launch if launch is not None else (self.launch[p] if full else None))
 
-    def bytes(self, projs=(0, 1)) -> float:
-        return sum(sum(self.step_bytes[p]) for p in projs)
+    def bytes(self, steps: int, projs=(0, 1), act=None) -> float:
+        """Algorithmic bytes of steps 0..steps-1 (a gated output writes n/2 columns)."""
+        b = 0.0
+        for p in projs:
+            b += sum(self.set_bytes[p][s % self.G] for s in range(steps))
+            if act and p == 0:
+                b -= steps * 8 * (self.projs[0].n // 2) * 4
+        return b
 
-    def capture(self, projs=(0, 1), act=None):
-        g = torch.cuda.CUDAGraph()
-        st = torch.cuda.Stream()
-        st.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(st):
-            for s in range(min(self.G, 4)):
-                self.step(s, projs, act)  # warm the launch path outside capture
-        torch.cuda.current_stream().wait_stream(st)
+    def capture(self, steps: int, projs=(0, 1), act=None, launch=None):
+        return capture_graph(lambda s: self.step(s, projs, act, launch), steps)
+
+
+def _cudart():
+    """The CUDA runtime library torch itself uses (for cudaGraphUpload)."""
+    import ctypes
+
+    try:
+        import nvidia.cuda_runtime as cr
+
+        path = os.path.join(list(cr.__path__)[0], "lib", "libcudart.so.12")
+        return ctypes.CDLL(path)
+    except Exception:
+        return ctypes.CDLL("libcudart.so.12")
+
+
+def graph_upload(g) -> bool:
+    """Upload an instantiated graph to the device (cudaGraphUpload) so that its
+    first timed replay does not pay for it. False if the call is not available."""
+    import ctypes
+
+    try:
+        rt = _cudart()
+        rc = rt.cudaGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()),
+                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         torch.cuda.synchronize()
-        with torch.cuda.graph(g):
-            for s in range(self.G):
-                self.step(s, projs, act)
-        torch.cuda.synchronize()
-        return g
+        return rc == 0
+    except Exception:
+        return False
+
+
+def capture_graph(fn, calls: int, warm: int = 2):
+    """CUDA graph of fn(0) .. fn(calls-1) on the current device; fn(0..warm-1) runs
+    eagerly on a side stream first, outside the capture."""
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        for i in range(min(warm, calls)):
+            fn(i)
+    torch.cuda.current_stream().wait_stream(st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(calls):
+            fn(i)
+    torch.cuda.synchronize()
+    return g
 
 
 def time_graph(g, replays: int) -> float:
@@ -251,15 +305,27 @@ def time_graph(g, replays: int) -> float:
     return a.elapsed_time(b) / 1e3
 
 
+def per_call(g, calls: int, repeats: int = REPEATS) -> dict:
+    """Median over `repeats` timed replays of a graph of `calls` calls (after one
+    untimed replay): seconds per call, and every repeat's value."""
+    g.replay()
+    torch.cuda.synchronize()
+    ts = [time_graph(g, 1) / calls for _ in range(repeats)]
+    return {"s": statistics.median(ts), "repeats_us": [t * 1e6 for t in ts]}
+
+
 def e2e_decode(W: DecodeWorkload, steps: int):
-    """Through the public API with host buffers: per step, one copy brings that
-    step's x rows and ids of both projections in from pinned host memory, both
-    projections run (moe_expert_routed_b200.Plan: one per layer copy and
-    projection, bound before the timed region, the step's launch modes), one copy
-    takes both outputs back."""
+    """Through the public API with host buffers, pipelined the way a serving loop
+    would run it: every step copies its own x rows and ids (both projections) in
+    from pinned host memory on an input-copy stream, runs both projections
+    (moe_expert_routed_b200.Plan, one per layer copy and projection, the step's
+    launch modes) on the compute stream, and copies both outputs back to pinned
+    host memory on an output-copy stream. Device buffers are double-buffered, so
+    step s+1's input copy and step s-1's output copy overlap step s's kernels;
+    events order each buffer's reuse. The steps are captured once in a CUDA graph
+    and replayed."""
     M = W.M
-    n = min(steps, W.G)
-    # per-step input block: x of each projection (bf16), then ids of each projection
+    n = min(max(steps, 2), W.G)
     xb = [P.k * 2 for P in W.projs]
     ib = [W.ids[i][0].numel() * 4 for i in range(2)]
     offs, o = [], 0
@@ -271,64 +337,69 @@ def e2e_decode(W: DecodeWorkload, steps: int):
     for p in range(2):
         hin[:, offs[p]:offs[p] + xb[p]] = W.x[p][:n].cpu().contiguous().view(torch.uint8).reshape(n, -1)
         hin[:, offs[2 + p]:offs[2 + p] + ib[p]] = W.ids[p][:n].cpu().contiguous().view(torch.uint8).reshape(n, -1)
-    din = torch.empty(blk, dtype=torch.uint8, device="cuda")
-    dx = [din[offs[p]:offs[p] + xb[p]].view(torch.bfloat16).view(1, W.projs[p].k) for p in range(2)]
-    did = [din[offs[2 + p]:offs[2 + p] + ib[p]].view(torch.int32).view(1, -1) for p in range(2)]
     nout = [8 * P.n for P in W.projs]
-    dout_all = torch.empty(sum(nout), dtype=torch.float32, device="cuda")
-    hout = torch.empty(sum(nout), dtype=torch.float32).pin_memory()
-    dout = [dout_all[:nout[0]].view(1, 8, W.projs[0].n), dout_all[nout[0]:].view(1, 8, W.projs[1].n)]
+    hout = torch.empty((n, sum(nout)), dtype=torch.float32).pin_memory()
+    din = [torch.empty(blk, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    dout_all = [torch.empty(sum(nout), dtype=torch.float32, device="cuda") for _ in range(2)]
+    dx = [[d[offs[p]:offs[p] + xb[p]].view(torch.bfloat16).view(1, W.projs[p].k) for p in range(2)] for d in din]
+    did = [[d[offs[2 + p]:offs[2 + p] + ib[p]].view(torch.int32).view(1, -1) for p in range(2)] for d in din]
+    dout = [[d[:nout[0]].view(1, 8, W.projs[0].n), d[nout[0]:].view(1, 8, W.projs[1].n)] for d in dout_all]
     h2d = sum(xb) + sum(ib)
     d2h = sum(nout) * 4
     plans = [[M.Plan(L["packed"], L["scales"], L["aux"], m=1, k=P.k, n=P.n, group_size=P.group_size,
                      bits=P.bits, fmt=P.fmt, n_expert_used=8, num_experts=P.num_experts,
                      x_dtype=torch.bfloat16, out_dtype=torch.float32, workspace=W.ws[p],
                      launch=W.launch[p]) for L in W.layers[p]] for p, P in enumerate(W.projs)]
-    hrows = [hin[i] for i in range(n)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def run_steps(st, count):
+    def run_steps(count):
+        comp = torch.cuda.current_stream()
+        done = [None] * count
+        copied = [None] * count
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
         for s in range(count):
-            din.copy_(hrows[s % n], non_blocking=True)
-            plans[0][s % N_LAYERS](dx[0], did[0], dout[0], st)
-            plans[1][s % N_LAYERS](dx[1], did[1], dout[1], st)
-            hout.copy_(dout_all, non_blocking=True)
+            b = s % 2
+            with torch.cuda.stream(s_in):
+                if s >= 2:
+                    s_in.wait_event(done[s - 2])      # step s-2's kernels no longer read din[b]
+                din[b].copy_(hin[s % n], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            comp.wait_event(ready)
+            if s >= 2:
+                comp.wait_event(copied[s - 2])        # dout[b] of step s-2 has been copied out
+            plans[0][s % N_LAYERS](dx[b][0], did[b][0], dout[b][0], comp)
+            plans[1][s % N_LAYERS](dx[b][1], did[b][1], dout[b][1], comp)
+            done[s] = torch.cuda.Event()
+            done[s].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[s])
+                hout[s % n].copy_(dout_all[b], non_blocking=True)
+                copied[s] = torch.cuda.Event()
+                copied[s].record(s_out)
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
 
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    # the n steps (copy in, two calls, copy out) captured once in a CUDA graph and
-    # replayed, so that the host's issue cost per call does not set the pace; the
-    # copies still run every step
-    try:
-        g = torch.cuda.CUDAGraph()
-        ws = torch.cuda.Stream()
-        ws.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(ws):
-            run_steps(ws, 2)
-        torch.cuda.current_stream().wait_stream(ws)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g):
-            run_steps(torch.cuda.current_stream(), n)
-        g.replay()
-        torch.cuda.synchronize()
-        reps = max(1, (steps + n - 1) // n)
-        a.record()
-        for _ in range(reps):
-            g.replay()
-        b.record()
-        b.synchronize()
-        done, mode = reps * n, f"CUDA graph of {n} steps (copies and calls) replayed {reps}x"
-        del g
-    except RuntimeError as exc:  # capture refused: time the same steps issued one by one
-        torch.cuda.synchronize()
-        st = torch.cuda.current_stream()
-        a.record()
-        run_steps(st, steps)
-        b.record()
-        b.synchronize()
-        done, mode = steps, f"eager ({type(exc).__name__} in graph capture)"
-    secs = a.elapsed_time(b) / 1e3
-    per_step_bytes = W.bytes() / W.G
-    return secs, done, mode, per_step_bytes, h2d, d2h
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run_steps(2)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_steps(n)
+    torch.cuda.synchronize()
+    reps = max(1, (steps + n - 1) // n)
+    g.replay()
+    torch.cuda.synchronize()
+    secs = time_graph(g, reps)
+    # the last replay's host outputs: the results of steps 0..n-1
+    got = hout.clone()
+    del g
+    per_step_bytes = W.bytes(n) / n
+    return secs, reps * n, f"CUDA graph of {n} pipelined steps replayed {reps}x", per_step_bytes, h2d, d2h, got
 
 
 # ------------------------------------------------------------------- oracle
@@ -424,211 +495,130 @@ def run_reference(args, dist: Dist):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, dist: Dist):
-    import moe_expert_routed_b200 as M
-
-    M.lib()  # fails loudly if the CUDA library is missing
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device for --impl ours")
-    dev = dist.local if dist.world > 1 else 0
-    torch.cuda.set_device(dev)
-    K, Wm = args.steps, args.warmup
-    G = min(GRAPH_STEPS, K)
-    W = DecodeWorkload(G, pdl=not args.no_pdl)
-    g = W.capture()
-    replays = max(1, K // G)
-    steps_timed = replays * G
-    warm_replays = max(1, -(-Wm // G))
-    for _ in range(warm_replays):
-        g.replay()
-    torch.cuda.synchronize()
-    sampler = clocks_sampler(dev) if dist.rank == 0 else None
-    time.sleep(0.3 if sampler else 0)
-    dist.barrier()
-    torch.cuda.synchronize()
-    secs = time_graph(g, replays)
-    torch.cuda.synchronize()
-    dist.barrier()
-    clocks = clocks_summary(sampler) if dist.rank == 0 else None
-    secs_max = dist.max(secs)
-    bytes_total = dist.sum(W.bytes() * replays)
-    value = bytes_total / secs_max / 1e9
-    ms_per_step = secs_max / steps_timed * 1e3
-
-    # per-projection calls (separate graphs, outside the timed region)
-    per_call = {}
-    for p, name in ((0, "gate_up"), (1, "down")):
-        gp = W.capture(projs=(p,))
-        gp.replay()
-        t = time_graph(gp, max(1, replays // 2))
-        per_call[name] = {"us_per_call": t / (max(1, replays // 2) * G) * 1e6,
-                          "GB_per_s": W.bytes((p,)) * max(1, replays // 2) / t / 1e9}
-        del gp
-    # the gate/up projection with its SiLU-gated epilogue (moe_qmm_id_glu): same
-    # weights and x, half the output columns
-    gp = W.capture(projs=(0,), act="silu")
-    gp.replay()
-    t = time_graph(gp, max(1, replays // 2))
-    glu_bytes = W.bytes((0,)) - G * 8 * (W.projs[0].n // 2) * 4
-    per_call["gate_up_silu"] = {"us_per_call": t / (max(1, replays // 2) * G) * 1e6,
-                                "GB_per_s": glu_bytes * max(1, replays // 2) / t / 1e9}
-    del gp
-
-    pk = peaks()
-    # dominant kernel: the gate/up launch (about 57% of the step); timed alone from a
-    # graph of gate/up calls only. DRAM traffic per launch from one ncu capture of
-    # this kernel.
-    achieved = per_call["gate_up"]["GB_per_s"]
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "traffic_note": f"{GATE_UP_DRAM_BYTES} B per launch (= the algorithmic bytes) in the last ncu "
-                                "capture, taken before the launch-dependency and gated-output changes to "
-                                "the kernel; null until re-captured",
-                "algorithmic_bytes": W.bytes((0,)) / W.G,
-                "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
-                "kernel": "gemv_aff4_rows (rows of all pairs split evenly over the SMs), gate/up launch",
-                "step_frac": W.bytes() * replays / secs / 1e9 / pk["hbm_gbs"]}
-    e2e_steps = min(max(K // 10, 50), 2000)
-    e_secs, e2e_steps, e2e_mode, per_step_bytes, h2d, d2h = e2e_decode(W, e2e_steps)
-    e_secs = dist.max(e_secs)
-    e2e = {"value": dist.sum(per_step_bytes * e2e_steps) / e_secs / 1e9, "unit": "GB/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "us_per_step": e_secs / e2e_steps * 1e6, "steps": e2e_steps,
-           "path": "moe_expert_routed_b200.Plan (Python binding -> moe_qmm_plan_run), pinned host buffers",
-           "issue": e2e_mode}
-    line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world, "steps": steps_timed,
-        "warmup": warm_replays * G, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "config": {"workload": "decode step m=1: gate/up (E128 top8 k2816 n1408) + down (k704 n2816), "
-                               "affine 4-bit g64, bf16 x, f32 out",
-                   "l2": f"inputs larger than L2: {N_LAYERS} rotated weight copies "
-                         f"({N_LAYERS * 0.428:.1f} GB), fresh ids and x every step",
-                   "timing": f"CUDA graph of {G} steps replayed {replays}x, CUDA events",
-                   "launch": ("gate/up: programmatic dependent launch; down: PDL with early weight "
-                              "streaming (its ids were ready before gate/up began)")
-                             if not args.no_pdl else "plain stream order",
-                   "parallelism": f"replicas x{dist.world}"},
-        "per_call": per_call,
-        "roofline": roofline,
-        "gpu_launches": 2 * steps_timed,
-        "clocks": clocks,
-        "e2e": e2e,
-    }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        v, s, threads, sample = oracle_decode_sample(args.cpu_budget)
-        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                "sample": sample, "single_thread": oracle_single_thread()}
-    if dist.rank == 0:
-        print(json.dumps(line), flush=True)
-    del g
+def decode_per_call(W: DecodeWorkload) -> dict:
+    """Per-call figures of the decode projections: each from a CUDA graph of
+    GRAPH_CALLS calls (fresh ids and x per call, rotated weight copies), the median
+    of REPEATS timed replays.
+      gate_up, down      one projection, calls in plain stream order (each waits
+                         for the previous call's completion, launch gap included)
+      gate_up_pdl        gate/up calls as programmatic dependents of the previous
+                         call (each still waits for it before reading anything)
+      gate_up_silu       gate/up with the SiLU-gated epilogue (n/2 outputs)
+      step               gate/up + down with the step's launch modes"""
+    res = {}
+    G = GRAPH_CALLS
+    for name, projs, act, launch in (("gate_up", (0,), None, None), ("gate_up_pdl", (0,), None, "pdl"),
+                                     ("down", (1,), None, None), ("down_pdl", (1,), None, "pdl"),
+                                     ("gate_up_silu", (0,), "silu", None), ("step", (0, 1), None, None)):
+        g = W.capture(G, projs, act, launch)
+        r = per_call(g, G)
+        del g
+        b = W.bytes(G, projs, act) / G
+        res[name] = {"us_per_call": r["s"] * 1e6, "GB_per_s": b / r["s"] / 1e9,
+                     "algorithmic_bytes": b, "repeats_us": r["repeats_us"]}
+    return res
 
 
-def run_grouped(args, dist: Dist):
-    """One call of the named grouped-path workload per step (routing prologue +
-    tcgen05 grouped GEMM), inputs resident in HBM, CUDA graph of G calls."""
+def grouped_tile_rows(P) -> int:
+    """Tile height of the grouped GEMM for this call (as the library picks it):
+    256 pairs (128 with f32 x, 320 for NVFP4) when experts hold ~96+ pairs on
+    average, else 64. Only sizes the routing prologue's tile list when the
+    prologue is timed alone."""
+    if P.R >= 96 * P.num_experts:
+        return 128 if P.x_dtype == 0 else (320 if P.fmt == 2 else 256)
+    return 64
+
+
+def grouped_entry(name: str, pk: dict) -> dict:
+    """One grouped-path workload (routing prologue + tcgen05 grouped GEMM), inputs
+    resident in HBM: per-call time from a CUDA graph of GRAPH_CALLS calls (median
+    of REPEATS replays), the routing prologue alone timed the same way, and the
+    GEMM time as their difference."""
+    import ctypes
+
     import moe_expert_routed_b200 as M
     from workloads import config_problem
     from workloads.torch_io import to_device
 
-    M.lib()
-    dev_i = dist.local if dist.world > 1 else 0
-    torch.cuda.set_device(dev_i)
-    P = config_problem(args.config)
+    P = config_problem(name)
     d = to_device(P)
     ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
     out_dt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float16}[P.out_dtype]
     out = torch.empty((P.m, P.n_expert_used, P.n), dtype=out_dt, device="cuda")
 
-    def call():
+    def call(_i):
         M.qmm_id(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], n=P.n, group_size=P.group_size,
                  bits=P.bits, fmt=P.fmt, num_experts=P.num_experts, out=out, workspace=ws)
 
-    def route_only():
-        M.route(d["ids"], P.num_experts, 256 if P.R >= 96 * P.num_experts else 64, workspace=ws)
+    T = grouped_tile_rows(P)
+    R = P.R
+    rbuf = [torch.empty(sz, dtype=torch.int32, device="cuda")
+            for sz in (P.num_experts + 1, P.num_experts + 2, R, 2 * (R // T + P.num_experts + 1), 1)]
+    ws_r = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    L = M.lib()
 
-    for _ in range(max(args.warmup, 3)):
-        call()
+    def route_call(_i):
+        st = L.moe_qmm_id_route(d["ids"].data_ptr(), P.m, P.n_expert_used, P.num_experts, T,
+                                *[b.data_ptr() for b in rbuf], ws_r.data_ptr(), ws_r.numel() * ws_r.element_size(),
+                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(f"moe_qmm_id_route: status {st}")
+
+    call(0)
     torch.cuda.synchronize()
-    assert M.poll_error(ws) == 0
-    G = max(1, min(args.steps, 20))
-    graphs = []
-    for fn in (call,):
-        g = torch.cuda.CUDAGraph()
-        st = torch.cuda.Stream()
-        st.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(st):
-            fn()
-        torch.cuda.current_stream().wait_stream(st)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g):
-            for _ in range(G):
-                fn()
-        graphs.append(g)
-    replays = max(1, args.steps // G)
-    graphs[0].replay()
-    sampler = clocks_sampler(dev_i) if dist.rank == 0 else None
-    time.sleep(0.3 if sampler else 0)
-    dist.barrier()
-    torch.cuda.synchronize()
-    secs = time_graph(graphs[0], replays)
-    torch.cuda.synchronize()
-    dist.barrier()
-    clocks = clocks_summary(sampler) if dist.rank == 0 else None
-    calls = replays * G
-    # routing prologue alone (outside the timed region): share of a call
-    for _ in range(3):
-        route_only()
-    torch.cuda.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(50):
-        route_only()
-    b.record()
-    b.synchronize()
-    route_us = a.elapsed_time(b) / 50 * 1e3
-    secs_max = dist.max(secs)
+    if M.poll_error(ws) != 0:
+        raise RuntimeError(f"{name}: device error word set")
+    gc = capture_graph(call, GRAPH_CALLS)
+    rc = per_call(gc, GRAPH_CALLS)
+    del gc
+    gr = capture_graph(route_call, GRAPH_CALLS)
+    rr = per_call(gr, GRAPH_CALLS)
+    del gr
     ids = P.ids.reshape(-1)
     valid = int((ids < P.num_experts).sum())
     flops = 2.0 * valid * P.n * P.k
     nbytes = alg_bytes(P, ids)
-    us = secs_max / calls * 1e6
-    tflops = dist.sum(flops * calls) / secs_max / 1e12
-    gbs = dist.sum(nbytes * calls) / secs_max / 1e9
-    pk = peaks()
-    gemm_us = max(us - route_us, 1e-9)
-    line = {
-        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": dist.world, "steps": calls,
-        "warmup": max(args.warmup, 3), "ms_per_step": us / 1e3, "us_per_call": us,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": {0: "f32", 1: "bf16", 2: "f16"}[P.x_dtype] + " x / fp32 accumulate",
-        "data": "synthetic",
-        "config": {"workload": f"{args.config}: E{P.num_experts} top{P.n_expert_used} m{P.m} k{P.k} n{P.n} "
-                               f"fmt{P.fmt} bits{P.bits} g{P.group_size}",
-                   "l2": f"weights {P.packed.nbytes / 1e6:.0f} MB (> L2 126 MB), one call per step",
-                   "timing": f"CUDA graph of {G} calls replayed {replays}x, CUDA events"},
-        "effective_GB_per_s": gbs,
-        "route_us": route_us,
-        "gemm_us_estimate": gemm_us,
-        "roofline": {"tensor": {"achieved": flops / gemm_us / 1e6, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                                "frac": flops / gemm_us / 1e6 / pk["bf16_tflops"]},
-                     "hbm": {"achieved": nbytes / gemm_us / 1e3, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                             "frac": nbytes / gemm_us / 1e3 / pk["hbm_gbs"]},
-                     "kernel": "grouped_gemm_kernel (tcgen05), time = call - routing prologue"},
-        "gpu_launches": 4 * calls,
-        "clocks": clocks,
+    us, route_us = rc["s"] * 1e6, rr["s"] * 1e6
+    gemm_us = us - route_us
+    t_tc = flops / (pk["bf16_tflops"] * 1e12) * 1e6
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9) * 1e6
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    tf, gb = flops / us / 1e6, nbytes / us / 1e3
+    tf_g, gb_g = flops / gemm_us / 1e6, nbytes / gemm_us / 1e3
+    ent = {
+        "workload": f"E{P.num_experts} top{P.n_expert_used} m{P.m} (R={P.R}) k{P.k} n{P.n}, "
+                    f"{ {0: 'affine', 1: 'codebook', 2: 'nvfp4', 3: 'mxfp4'}[P.fmt]} {P.bits}-bit "
+                    f"g{P.group_size}, {({0: 'f32', 1: 'bf16', 2: 'f16'})[P.x_dtype]} x, "
+                    f"{({0: 'f32', 1: 'bf16', 2: 'f16'})[P.out_dtype]} out",
+        "us_per_call": us, "TFLOP_per_s": tf, "GB_per_s": gb,
+        "route_us": route_us, "gemm_us": gemm_us,
+        "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+        "ideal_us": {"tensor": t_tc, "hbm": t_hbm},
+        "roofline": {"bound": bound,
+                     "achieved": tf if bound == "tensor" else gb,
+                     "peak": pk["bf16_tflops"] if bound == "tensor" else pk["hbm_gbs"],
+                     "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                     "frac": (tf / pk["bf16_tflops"]) if bound == "tensor" else (gb / pk["hbm_gbs"]),
+                     "tensor_frac": tf / pk["bf16_tflops"], "hbm_frac": gb / pk["hbm_gbs"],
+                     "gemm_tensor_frac": tf_g / pk["bf16_tflops"], "gemm_hbm_frac": gb_g / pk["hbm_gbs"],
+                     "peak_source": pk["source"] + " (bf16_tflops burst, hbm_gbs copy)"},
+        "repeats_us": rc["repeats_us"], "route_repeats_us": rr["repeats_us"],
+        "timing": f"CUDA graph of {GRAPH_CALLS} calls, median of {REPEATS} replays; routing prologue alone "
+                  f"the same way; gemm_us = call - routing",
+        "l2": f"weights {P.packed.nbytes / 1e6:.0f} MB + x {P.x.nbytes / 1e6:.0f} MB (> L2 126 MB)",
+        "gpu_launches_per_call": 4,
     }
-    if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+    del d, out, ws, ws_r, rbuf
+    torch.cuda.empty_cache()
+    return ent
 
 
-def run_sweep(args):
+def decode_sweep(pk: dict) -> list:
     """Decode with m = 1, 2, 4, 8 tokens (top-8 of 128 experts), gate/up and down
-    projections timed separately: a CUDA graph of calls with fresh ids and x each
-    call and 16 rotated weight copies. Effective GB/s counts the distinct experts
-    each call actually touches (E[D] = 8, 15.5, 29.1, 51.6 for uniform ids)."""
+    projections separately: a CUDA graph of GRAPH_CALLS calls with fresh ids and x
+    each call and N_LAYERS rotated weight copies, median of REPEATS replays.
+    Effective GB/s counts the distinct experts each call touches (E[D] = 8, 15.5,
+    29.1, 51.6 for uniform ids)."""
     import types
 
     import moe_expert_routed_b200 as M
@@ -636,10 +626,8 @@ def run_sweep(args):
     from workloads.gen import bf16_bits, distinct_uniform_ids
     from workloads.torch_io import to_device
 
-    calls = 200
+    calls = GRAPH_CALLS
     rng = np.random.Generator(np.random.PCG64(77))
-    sampler = clocks_sampler(torch.cuda.current_device())
-    pk = peaks()
     rows = []
     for name in ("decode_gate_up", "decode_down"):
         P = config_problem(name)
@@ -655,7 +643,7 @@ def run_sweep(args):
             Pm = types.SimpleNamespace(row_bytes=P.row_bytes, groups=P.groups, fmt=P.fmt, n=P.n, k=P.k,
                                        bits=P.bits, num_experts=P.num_experts, m=m, R=8 * m,
                                        x_dtype=P.x_dtype, out_dtype=P.out_dtype)
-            nbytes = sum(alg_bytes(Pm, ids[c]) for c in range(calls))
+            nbytes = sum(alg_bytes(Pm, ids[c]) for c in range(calls)) / calls
             distinct = float(np.mean([np.unique(ids[c]).size for c in range(calls)]))
 
             def one(c):
@@ -664,30 +652,159 @@ def run_sweep(args):
                          group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
                          out=out[c], workspace=ws)
 
-            st = torch.cuda.Stream()
-            st.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(st):
-                for c in range(4):
-                    one(c)
-            torch.cuda.current_stream().wait_stream(st)
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for c in range(calls):
-                    one(c)
-            time_graph(g, max(3, args.warmup // calls))
-            reps = max(1, args.steps // calls)
-            secs = time_graph(g, reps)
+            g = capture_graph(one, calls)
+            r = per_call(g, calls)
             del g
-            us = secs / (reps * calls) * 1e6
-            gbs = nbytes * reps / secs / 1e9
             rows.append({"projection": name.replace("decode_", ""), "m": m, "distinct_experts": distinct,
-                         "us_per_call": us, "GB_per_s": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"]})
-    line = {"sweep": "decode m=1..8 (E128 top8, affine 4-bit g64, bf16 x, f32 out), per projection",
-            "rows": rows, "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": pk["source"],
-            "timing": f"CUDA graph of {calls} calls, fresh ids and x per call, {N_LAYERS} rotated weight copies",
-            "clocks": clocks_summary(sampler)}
-    print(json.dumps(line), flush=True)
+                         "us_per_call": r["s"] * 1e6, "GB_per_s": nbytes / r["s"] / 1e9,
+                         "frac_of_hbm": nbytes / r["s"] / 1e9 / pk["hbm_gbs"],
+                         "TFLOP_per_s": 2.0 * 8 * m * P.n * P.k / r["s"] / 1e12})
+        del base, layers
+        torch.cuda.empty_cache()
+    return rows
+
+
+def run_ours(args, dist: Dist):
+    import moe_expert_routed_b200 as M
+
+    M.lib()  # fails loudly if the CUDA library is missing
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    dev = dist.local if dist.world > 1 else 0
+    torch.cuda.set_device(dev)
+    K, Wm = args.steps, args.warmup
+    Gt = min(GRAPH_STEPS, K)
+    W = DecodeWorkload(max(Gt, GRAPH_CALLS), pdl=not args.no_pdl)
+    # the timed graph holds steps 0..Gt-1; uploaded to the device before warm-up so
+    # that its first replay is a plain replay
+    g = W.capture(Gt)
+    uploaded = graph_upload(g)
+    warm_done = Wm
+    for s in range(Wm):  # W untimed warm-up steps (the step's own calls, issued one by one)
+        W.step(s)
+    if not uploaded:
+        g.replay()
+        warm_done += Gt
+    torch.cuda.synchronize()
+    replays = max(1, K // Gt)
+    steps_timed = replays * Gt
+    sampler = clocks_sampler(dev) if dist.rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    dist.barrier()
+    torch.cuda.synchronize()
+    secs = time_graph(g, replays)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = clocks_summary(sampler) if dist.rank == 0 else None
+    del g
+    secs_max = dist.max(secs)
+    bytes_total = dist.sum(W.bytes(Gt) * replays)
+    value = bytes_total / secs_max / 1e9
+    ms_per_step = secs_max / steps_timed * 1e3
+
+    pk = peaks()
+    pc = decode_per_call(W)
+    # dominant kernel: the gate/up launch, timed alone (graph of gate/up calls, median
+    # of repeats); DRAM traffic per launch from an ncu capture of that kernel
+    achieved = pc["gate_up"]["GB_per_s"]
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": GATE_UP_DRAM_BYTES,
+                "traffic_note": GATE_UP_TRAFFIC_NOTE,
+                "algorithmic_bytes": pc["gate_up"]["algorithmic_bytes"],
+                "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+                "kernel": "gemv_aff4_rows, gate/up launch (plain stream order; "
+                          f"{pc['gate_up_pdl']['us_per_call']:.2f} us as programmatic dependents)",
+                "frac_pdl": pc["gate_up_pdl"]["GB_per_s"] / pk["hbm_gbs"],
+                "step_frac": value / dist.world / pk["hbm_gbs"]}
+    e_secs, e_steps, e_mode, per_step_bytes, h2d, d2h, got = e2e_decode(W, min(max(K, 100), 2000))
+    # the pipelined loop's outputs equal the same steps run on the device directly
+    n_chk = got.shape[0]
+    for s in range(n_chk):
+        W.step(s)
+    torch.cuda.synchronize()
+    ref = torch.cat([W.out[0][:n_chk].reshape(n_chk, -1), W.out[1][:n_chk].reshape(n_chk, -1)], 1).cpu()
+    e2e_ok = bool(torch.equal(got, ref))
+    e_secs = dist.max(e_secs)
+    e2e = {"value": dist.sum(per_step_bytes * e_steps) / e_secs / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "us_per_step": e_secs / e_steps * 1e6, "steps": e_steps,
+           "path": "moe_expert_routed_b200.Plan (Python binding -> moe_qmm_plan_run), pinned host buffers, "
+                   "input and output copies on their own streams, double-buffered device buffers",
+           "issue": e_mode, "outputs_match_device_steps": e2e_ok}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world, "steps": steps_timed,
+        "warmup": warm_done, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "decode step m=1: gate/up (E128 top8 k2816 n1408) + down (k704 n2816), "
+                               "affine 4-bit g64, bf16 x, f32 out",
+                   "l2": f"inputs larger than L2: {N_LAYERS} rotated weight copies "
+                         f"({N_LAYERS * 0.428:.1f} GB), fresh ids and x every step",
+                   "timing": f"CUDA graph of {Gt} steps replayed {replays}x, CUDA events"
+                             + ("" if uploaded else " (graph replayed once more during warm-up)"),
+                   "launch": ("gate/up: programmatic dependent launch; down: PDL with early weight "
+                              "streaming (its ids were ready before gate/up began)")
+                             if not args.no_pdl else "plain stream order",
+                   "parallelism": f"replicas x{dist.world}"},
+        "per_call": pc,
+        "roofline": roofline,
+        "gpu_launches": 2 * steps_timed,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    del W
+    torch.cuda.empty_cache()
+    if dist.world == 1 and not args.no_extras:
+        # the other workloads and the decode m-sweep, on this GPU, outside the timed region
+        sampler = clocks_sampler(dev)
+        line["per_config"] = {name: grouped_entry(name, pk) for name in ("canvas", "prefill", "skewed")}
+        line["sweep"] = decode_sweep(pk)
+        line["per_config_clocks"] = clocks_summary(sampler)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        v, s, threads, sample = oracle_decode_sample(args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": sample, "single_thread": oracle_single_thread()}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_grouped(args, dist: Dist):
+    """One grouped-path workload as the bench line (N independent replicas for N > 1)."""
+    import moe_expert_routed_b200 as M
+
+    M.lib()
+    dev_i = dist.local if dist.world > 1 else 0
+    torch.cuda.set_device(dev_i)
+    pk = peaks()
+    sampler = clocks_sampler(dev_i) if dist.rank == 0 else None
+    dist.barrier()
+    ent = grouped_entry(args.config, pk)
+    dist.barrier()
+    clocks = clocks_summary(sampler) if dist.rank == 0 else None
+    us = dist.max(ent["us_per_call"])
+    tf = dist.sum(ent["algorithmic_flops"]) / us / 1e6
+    line = {
+        "metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": dist.world,
+        "steps": GRAPH_CALLS * REPEATS, "warmup": GRAPH_CALLS + 3, "ms_per_step": us / 1e3, "us_per_call": us,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": ent["workload"].split(", ")[-2], "data": "synthetic",
+        "config": {"workload": f"{args.config}: {ent['workload']}", "l2": ent["l2"], "timing": ent["timing"]},
+        "per_config": {args.config: ent}, "roofline": ent["roofline"],
+        "gpu_launches": 4 * GRAPH_CALLS * REPEATS, "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_sweep(args):
+    pk = peaks()
+    sampler = clocks_sampler(torch.cuda.current_device())
+    rows = decode_sweep(pk)
+    print(json.dumps({"sweep": "decode m=1..8 (E128 top8, affine 4-bit g64, bf16 x, f32 out), per projection",
+                      "rows": rows, "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": pk["source"],
+                      "timing": f"CUDA graph of {GRAPH_CALLS} calls, median of {REPEATS} replays, fresh ids and "
+                                f"x per call, {N_LAYERS} rotated weight copies",
+                      "clocks": clocks_summary(sampler)}), flush=True)
 
 
 def run_probe(args):
@@ -718,8 +835,8 @@ def run_probe(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
-    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pdl", action="store_true",
@@ -729,6 +846,8 @@ def main():
     ap.add_argument("--probe", choices=["decode", "canvas", "prefill", "skewed"],
                     help="run a few untimed calls (for profiler captures) and exit")
     ap.add_argument("--reps", type=int, default=4)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="decode bench line without the grouped workloads and the m-sweep")
     ap.add_argument("--sweep", action="store_true",
                     help="decode m = 1, 2, 4, 8 curve (one GPU), one JSON line, instead of the bench line")
     args = ap.parse_args()

@@ -290,15 +290,18 @@ moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_u
  *     MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing. At num_experts <= 256 that
  *     admits m * n_expert_used up to about 200,000 routings.
  *   * The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; a failure returns
+ *     (cudaGetSymbolAddress) with that device current, and so does the first
+ *     call after the device's current CUDA context changed (cudaDeviceReset, or
+ *     a context the caller created and made current): the array belongs to the
+ *     context's copy of the library's module. A failed lookup returns
  *     MOE_ERR_CUDA. Make that first call before capturing a stream that uses it.
  *   * All calls on a device share the one array and it keeps the last call's
  *     contents. Nothing in it needs to start at zero (every call writes the
  *     buffers it later reads), but calls that overlap on the GPU (different
  *     streams without ordering between them) race on it: order them.
- *   * The array's device error word is not readable through this entry point:
- *     out-of-range ids still give zero output rows; use moe_qmm_id with a
- *     workspace to observe MOE_ERR_BAD_EXPERT_ID or MOE_ERR_TIMEOUT.
+ *   * The array's first word is the device error word of these calls:
+ *     out-of-range ids give zero output rows and set a bit there, which
+ *     moe_qmm_id_noalloc_poll_error() reads and clears.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
 moe_status moe_qmm_id_noalloc(const void *x, const uint32_t *ids, const void *packed,
@@ -306,6 +309,11 @@ moe_status moe_qmm_id_noalloc(const void *x, const uint32_t *ids, const void *pa
                               uint32_t n, uint32_t group_size, uint32_t bits, moe_fmt fmt,
                               uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                               moe_dtype out_dtype, moe_stream_t stream);
+
+/* moe_qmm_id_poll_error for the calls of moe_qmm_id_noalloc on the current device:
+ * synchronise `stream`, read and clear the error word in the library's scratch
+ * array. Same results as moe_qmm_id_poll_error; allocates nothing. */
+moe_status moe_qmm_id_noalloc_poll_error(moe_stream_t stream);
 
 /*
  * moe_qmm_plan -- a call with everything but x, ids and out bound once, for
@@ -344,6 +352,20 @@ moe_status moe_qmm_plan_run(const moe_qmm_plan *plan, const void *x, const uint3
  * valid), MOE_ERR_BAD_EXPERT_POINTER (moe_qmm_id_ptrs skipped an expert whose
  * scale or bias buffer was null or misaligned) or MOE_ERR_CUDA. */
 moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream);
+
+/*
+ * moe_qmm_test_inject_wait_timeout -- failure-detection test hook (no counterpart
+ * on the pages). While limit_ns is non-zero, every call launched afterwards from
+ * this process whose kernel has bounded device waits (the tcgen05 grouped GEMM and
+ * the one-token decode kernel) makes one extra wait per CTA on a barrier that
+ * nothing completes, and gives up after limit_ns nanoseconds: the CTA raises its
+ * abort flag, lets its own copies and MMAs in flight complete (with the normal
+ * 1 s limit, not limit_ns), frees its tensor memory and exits, and the call's
+ * error word reports MOE_ERR_TIMEOUT. Outputs of such calls are not valid.
+ * limit_ns = 0 (the default) turns the hook off. The hook only shortens waits:
+ * it never faults or hangs the GPU. Returns MOE_OK.
+ */
+moe_status moe_qmm_test_inject_wait_timeout(uint64_t limit_ns);
 
 /* Static description of a status code. */
 const char *moe_status_str(moe_status s);

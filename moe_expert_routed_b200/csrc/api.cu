@@ -5,11 +5,16 @@
 // happens before any CUDA call.
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 #include "moe_qmm.h"
 
 namespace moe {
+
+// Wait limit of the failure-detection test hook (0: off).
+static std::atomic<uint64_t> g_fault_wait_ns{0};
 
 static inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -152,6 +157,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     a.act = act;
     a.out_n = act >= 0 ? n / 2u : n;
     a.launch_flags = launch_flags;
+    a.fault_wait_ns = g_fault_wait_ns.load(std::memory_order_relaxed);
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);
@@ -355,6 +361,11 @@ moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_u
                                   L.chunks, (uint32_t *)(ws + L.err), nullptr, 0, 0,
                                   (cudaStream_t)stream);
     return ce == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_qmm_test_inject_wait_timeout(uint64_t limit_ns) {
+    moe::g_fault_wait_ns.store(limit_ns, std::memory_order_relaxed);
+    return MOE_OK;
 }
 
 moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream) {

@@ -56,6 +56,9 @@ constexpr int MMA_WARP = (NDQ + NLD) / 32;
 constexpr int MAX_STAGES = 6;
 constexpr int A_TILE = BM * KT * 2;             // bytes per A term per stage
 constexpr uint64_t WAIT_NS = 1000000000ull;
+// limit of the waits that let a CTA's own copies and MMAs complete after another
+// wait gave up (independent of the pipeline waits' limit)
+constexpr uint64_t DRAIN_NS = 1000000000ull;
 
 struct GemmParams {
     const void *x;
@@ -79,6 +82,9 @@ struct GemmParams {
     // and the epilogue writes act(gate) * up into rows of glu_nh = n/2 columns
     uint32_t glu_nh;
     int act;
+    // failure-detection test hook: non-zero makes the MMA warp first wait this long on
+    // a barrier nothing completes (so the CTA aborts); 0 in normal operation
+    uint64_t fault_ns;
 };
 
 template <int KIND> constexpr int a_terms() { return KIND == K_NVFP4 ? 1 : 2; }
@@ -328,7 +334,7 @@ grouped_gemm_kernel(const GemmParams P) {
     constexpr uint32_t TMEM_COLS = BN <= 64 ? 64u : BN <= 128 ? 128u : BN <= 256 ? 256u : 512u;
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bars[3 * MAX_STAGES + 1];
+    __shared__ uint64_t bars[3 * MAX_STAGES + 2];
     __shared__ uint32_t tmem_s;
     __shared__ int abort_s;
     __shared__ uint32_t pairs_s[BN];
@@ -373,6 +379,7 @@ grouped_gemm_kernel(const GemmParams P) {
     const uint32_t loaded0 = ptx::smem_u32(&bars[MAX_STAGES]);
     const uint32_t empty0 = ptx::smem_u32(&bars[2 * MAX_STAGES]);
     const uint32_t accb = ptx::smem_u32(&bars[3 * MAX_STAGES]);
+    const uint32_t never = ptx::smem_u32(&bars[3 * MAX_STAGES + 1]);  // completed by nothing
     volatile int *abort_flag = &abort_s;
 
     if (tid == 0) {
@@ -382,6 +389,7 @@ grouped_gemm_kernel(const GemmParams P) {
             ptx::mbar_init(empty0 + 8 * s, 1);
         }
         ptx::mbar_init(accb, 1);
+        ptx::mbar_init(never, 1);
         ptx::fence_mbar_init();
         abort_s = 0;
     }
@@ -497,7 +505,8 @@ grouped_gemm_kernel(const GemmParams P) {
             ptx::mbar_arrive(full0 + 8 * s);
         }
         // ------------------------------------------------------------- epilogue
-        if (ok && ptx::mbar_wait_bounded(accb, 0, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns)) {
+        if (ok && ptx::mbar_wait_bounded(accb, 0, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns) &&
+            !*abort_flag) {
             ptx::tc_fence_after();
             const uint32_t q = warp & 3u, ch = warp >> 2;
             const uint32_t grow_e = row0 + q * 32u + lane;  // logical row
@@ -631,7 +640,8 @@ grouped_gemm_kernel(const GemmParams P) {
         const uint32_t idesc2 = ptx::idesc_f16(F16 ? 0u : 1u, n2 > 0 ? n2 : 16u);
         uint32_t accum = 0;
         bool ok = true;
-        for (uint32_t kt = 0; kt < P.ktiles; kt++) {
+        if (P.fault_ns) ok = ptx::mbar_wait_bounded(never, 0, abort_flag, P.err, ERR_TIMEOUT, P.fault_ns);
+        for (uint32_t kt = 0; ok && kt < P.ktiles; kt++) {
             const uint32_t s = kt % S, use = kt / S;
             if (!ptx::mbar_wait_bounded(full0 + 8 * s, use & 1u, abort_flag, P.err, ERR_TIMEOUT,
                                         P.timeout_ns)) {
@@ -668,8 +678,9 @@ grouped_gemm_kernel(const GemmParams P) {
         }
         ptx::mma_commit(accb);
         if (!ok) {
-            // drain: the commit above tracks every MMA issued so far
-            ptx::mbar_wait_bounded(accb, 0, nullptr, P.err, ERR_TIMEOUT, P.timeout_ns);
+            // drain: the commit above tracks every MMA issued so far; TMEM is freed only
+            // after it (its own limit, not the pipeline waits' one)
+            ptx::mbar_wait_bounded(accb, 0, nullptr, P.err, ERR_TIMEOUT, DRAIN_NS);
         }
     }
     __syncthreads();
@@ -825,6 +836,7 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.bias = a.bias; P.bias_dtype = a.bias_dtype;
     P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
     P.timeout_ns = WAIT_NS;
+    P.fault_ns = a.fault_wait_ns;
     P.glu_nh = a.act >= 0 ? a.n / 2u : 0u;
     P.act = a.act;
     const uint32_t nm = (a.n + BM - 1) / BM;

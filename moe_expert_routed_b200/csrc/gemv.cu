@@ -915,7 +915,7 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     extern __shared__ __align__(128) uint8_t dsm8[];
     __shared__ uint32_t ex_s[ROWS_MAX_PAIRS];
     __shared__ __align__(8) uint64_t bar_w[ROWS_WARPS];
-    __shared__ __align__(8) uint64_t bar_x, bar_s;
+    __shared__ __align__(8) uint64_t bar_x, bar_s, bar_never;
     __shared__ int abort_s;
 
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
@@ -945,6 +945,7 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
         for (int i = 0; i < ROWS_WARPS; i++) ptx::mbar_init(ptx::smem_u32(&bar_w[i]), 1);
         ptx::mbar_init(ptx::smem_u32(&bar_x), 1);
         ptx::mbar_init(ptx::smem_u32(&bar_s), 1);
+        ptx::mbar_init(ptx::smem_u32(&bar_never), 1);  // completed by nothing
         ptx::fence_mbar_init();
         abort_s = 0;
     }
@@ -1033,7 +1034,11 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     uint32_t *planes = (uint32_t *)(dsm8 + L.planes);
     float *uscale = (float *)(dsm8 + L.uscale);
     float *usum = (float *)(dsm8 + L.usum);
-    const bool x_ok = ptx::mbar_wait_bounded(bx, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
+    // failure-detection test hook: a wait nothing completes, so that the CTA aborts
+    const bool f_ok = !P.fault_ns || warp != 0 ||
+                      ptx::mbar_wait_bounded(ptx::smem_u32(&bar_never), 0, abort_flag, P.err, ERR_TIMEOUT,
+                                             P.fault_ns);
+    const bool x_ok = f_ok && ptx::mbar_wait_bounded(bx, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
     if (__all_sync(0xFFFFFFFFu, x_ok)) {
         const uint32_t nwords = nu * 4u;
         for (uint32_t base = warp * 32u; base < nwords; base += ROWS_THREADS) {
@@ -1076,9 +1081,11 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     if (s_bulk) s_ok = ptx::mbar_wait_bounded(bs, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
     const bool w_ok = ptx::mbar_wait_bounded(bw, 0, abort_flag, P.err, ERR_TIMEOUT, WAIT);
     if (!__all_sync(0xFFFFFFFFu, x_ok && s_ok && w_ok && !*abort_flag)) {
-        // a wait gave up: let this warp's copies land before shared memory is released
+        // a wait gave up: let this warp's copies, the scale copies and the x copy land
+        // before shared memory is released (each with the full limit)
         ptx::mbar_wait_bounded(bw, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
         if (s_bulk) ptx::mbar_wait_bounded(bs, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
+        ptx::mbar_wait_bounded(bx, 0, nullptr, P.err, ERR_TIMEOUT, WAIT);
         return;
     }
     const unsigned short *sc = (const unsigned short *)(dsm8 + L.sc);
@@ -1391,6 +1398,7 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     P.pdl = (a.launch_flags & MOE_LAUNCH_PDL) != 0;
     P.early_weights = (a.launch_flags & MOE_LAUNCH_EARLY_WEIGHTS) != 0;
     P.packed_ptrs = a.packed_ptrs; P.scale_ptrs = a.scale_ptrs; P.bias_ptrs = a.bias_ptrs;
+    P.fault_ns = a.fault_wait_ns;
     const bool al16 = ((uintptr_t)a.packed % 16 == 0) && (a.row_bytes % 16 == 0);
     const bool al4 = ((uintptr_t)a.packed % 4 == 0) && (a.row_bytes % 4 == 0);
     P.load_mode = al16 ? 16 : al4 ? 4 : 1;

@@ -41,6 +41,9 @@ struct GemvParams {
     // weights and scales are read, and the weight copies issued, before waiting for
     // the previous kernel on the stream; otherwise everything waits for it
     int pdl, early_weights;
+    // failure-detection test hook (one-token kernel): non-zero makes every CTA first
+    // wait this long on a barrier nothing completes, so that it aborts; 0 normally
+    uint64_t fault_ns;
 };
 
 // Which expert this CTA serves and how many pairs it has. Fused mode: all ids

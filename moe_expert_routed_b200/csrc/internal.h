@@ -71,6 +71,10 @@ struct QmmArgs {
     int act;         // gated output: -1 none, else the activation (moe_act) of act(gate) * up
     uint32_t out_n;  // columns of an output row: n, or n / 2 with a gated output
     uint32_t launch_flags;  // MOE_LAUNCH_* bits of the path argument
+    // failure-detection test hook (moe_qmm_test_inject_wait_timeout): when non-zero,
+    // kernels with bounded waits make one wait per CTA on a barrier nothing
+    // completes, giving up after this many ns; 0 in normal operation
+    uint64_t fault_wait_ns;
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).

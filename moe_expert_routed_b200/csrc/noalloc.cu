@@ -20,24 +20,64 @@
 namespace {
 
 // The shared scratch. Its name, used in host code, is only a host-side handle:
-// the device address comes from cudaGetSymbolAddress, once per device.
+// the device address comes from cudaGetSymbolAddress, once per device and context.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_scratch_mutex;
-void *g_scratch_ptr[64];
 
-// Device address of the scratch on the current device (looked up on the first
-// call per device, with that device current).
+// Cached device address of the scratch per device, with the id of the CUDA
+// context it was looked up in: a new context on the device (after
+// cudaDeviceReset, or a caller's own context made current) loads the module
+// again and the array may move, so the address is looked up again then.
+struct ScratchAddr {
+    void *ptr;
+    unsigned long long ctx_id;
+};
+ScratchAddr g_scratch[64];
+
+// cuCtxGetCurrent / cuCtxGetId through the runtime's driver entry points (no
+// link-time dependency on the driver library).
+typedef int (*ctx_get_current_t)(void **ctx);
+typedef int (*ctx_get_id_t)(void *ctx, unsigned long long *id);
+ctx_get_current_t g_ctx_get_current;
+ctx_get_id_t g_ctx_get_id;
+bool g_entry_points_looked_up;
+
+// Unique id of the current context, or 0 when there is none or it cannot be read.
+unsigned long long current_context_id() {
+    if (!g_entry_points_looked_up) {
+        g_entry_points_looked_up = true;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", (void **)&g_ctx_get_current, cudaEnableDefault, &q1) !=
+                cudaSuccess || q1 != cudaDriverEntryPointSuccess)
+            g_ctx_get_current = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", (void **)&g_ctx_get_id, cudaEnableDefault, &q2) !=
+                cudaSuccess || q2 != cudaDriverEntryPointSuccess)
+            g_ctx_get_id = nullptr;
+    }
+    if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+    void *ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_get_current(&ctx) != 0 || !ctx) return 0;
+    if (g_ctx_get_id(ctx, &id) != 0) return 0;
+    return id;
+}
+
+// Device address of the scratch on the current device and context: looked up on
+// the first call per device (and again whenever the current context differs from
+// the one the cached address came from), with that device current.
 moe_status scratch_address(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
+    const unsigned long long id = current_context_id();
+    if (!g_scratch[dev].ptr || id == 0 || id != g_scratch[dev].ctx_id) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
-        g_scratch_ptr[dev] = ptr;
+        g_scratch[dev].ptr = ptr;
+        g_scratch[dev].ctx_id = current_context_id();  // the lookup may have created the context
     }
-    *out = g_scratch_ptr[dev];
+    *out = g_scratch[dev].ptr;
     return MOE_OK;
 }
 
@@ -62,4 +102,12 @@ extern "C" moe_status moe_qmm_id_noalloc(const void *x, const uint32_t *ids, con
     return moe_qmm_id_path(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt,
                            n_expert_used, num_experts, x_dtype, out_dtype, scratch,
                            MOE_NOALLOC_SCRATCH_BYTES, stream, MOE_PATH_AUTO);
+}
+
+extern "C" moe_status moe_qmm_id_noalloc_poll_error(moe_stream_t stream) {
+    void *scratch = nullptr;
+    const moe_status s = scratch_address(&scratch);
+    if (s != MOE_OK) return s;
+    // the error word is the scratch's first word, as in a caller's workspace
+    return moe_qmm_id_poll_error(scratch, stream);
 }

@@ -56,3 +56,62 @@ def test_rerun_bit_identical(problem):
     b = run(P, "auto", dev=dev)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def _tile_class_sample(P):
+    """(pairs, cols) covering each kind of tile the grouped GEMM forms, in full
+    output rows: every pair of the hottest and of the coldest expert (all
+    columns for the coldest; for the hottest, all columns of the pairs at each
+    64-pair boundary inside the expert, 0, 63, 64, 127, 128, ..., and the
+    first, middle and last column of every 128-row block for the others), pairs
+    256..319 of an expert with more than 256 pairs (the second accumulator of
+    320-pair tiles), and the last 128-column block of every pair at a tile
+    boundary. The tile list runs over the experts' pairs in ascending pair index
+    (metrale helpers_b.rs, launch_grouped_gemm: expert_offsets / sorted_token_ids)."""
+    ids = P.ids.reshape(-1).astype(np.int64)
+    order = np.argsort(ids, kind="stable")
+    counts = np.bincount(ids, minlength=P.num_experts)
+    starts = np.concatenate(([0], np.cumsum(counts)))
+    used = np.nonzero(counts)[0]
+    hot = int(used[np.argmax(counts[used])])
+    cold = int(used[np.argmin(counts[used])])
+    pairs, cols = [], []
+
+    def full_rows(ps):
+        ps = np.asarray(ps, dtype=np.int64)
+        pairs.append(np.repeat(ps, P.n))
+        cols.append(np.tile(np.arange(P.n), ps.size))
+
+    def some_cols(ps, cs):
+        ps = np.asarray(ps, dtype=np.int64)
+        pairs.append(np.repeat(ps, cs.size))
+        cols.append(np.tile(cs, ps.size))
+
+    hot_pairs = order[starts[hot]:starts[hot + 1]]
+    cold_pairs = order[starts[cold]:starts[cold + 1]]
+    full_rows(cold_pairs)
+    pos = sorted({q for b in range(0, hot_pairs.size, 64) for q in (b, b + 63) if q < hot_pairs.size}
+                 | {hot_pairs.size - 1})
+    full_rows(hot_pairs[pos])
+    blocks = np.arange(0, P.n, 128)
+    some_cols(hot_pairs, np.unique(np.concatenate([blocks, blocks + 64, np.minimum(blocks + 127, P.n - 1)])))
+    big = np.nonzero(counts > 256)[0]
+    if big.size:
+        e = int(big[0])
+        full_rows(order[starts[e] + 256:starts[e] + min(320, counts[e])])
+    # last column block of the first and last pair of every expert
+    edge = np.unique(np.concatenate([order[starts[used]], order[starts[used + 1] - 1]]))
+    some_cols(edge, np.arange(max(0, P.n - 128), P.n))
+    return np.concatenate(pairs), np.concatenate(cols)
+
+
+@pytest.mark.parametrize("name", ["canvas", "prefill", "skewed"])
+def test_every_tile_class(name):
+    P = config_problem(name)
+    dev = to_device(P)
+    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    out = run(P, "auto", dev=dev, workspace=ws)
+    assert M.poll_error(ws) == 0
+    pairs, cols = _tile_class_sample(P)
+    nviol, ratio, info = check_sampled(P, out, pairs, cols)
+    assert nviol == 0, f"{P.name}: {nviol} of {pairs.size} violations, worst err/bound {ratio:.3g} {info}"
