@@ -807,6 +807,54 @@ def run_sweep(args):
                       "clocks": clocks_summary(sampler)}), flush=True)
 
 
+def run_crossover(args):
+    """The decode / grouped crossover: the decode gate/up and down shapes (E128 top8,
+    affine 4-bit g64, bf16 x) at m = 1 .. 64 tokens (8 .. 512 routings), each call
+    timed on the CUDA-core decode path (path="decode": routing fused for R <= 64,
+    else the routing prologue and the routed GEMV) and on the tcgen05 grouped GEMM
+    (path="grouped"): CUDA graphs of calls with fresh ids and x per call and
+    N_LAYERS rotated weight copies, median of REPEATS replays."""
+    import moe_expert_routed_b200 as M
+    from workloads import config_problem
+    from workloads.gen import bf16_bits, distinct_uniform_ids
+    from workloads.torch_io import to_device
+
+    calls = 40
+    rng = np.random.Generator(np.random.PCG64(91))
+    sampler = clocks_sampler(torch.cuda.current_device())
+    rows = []
+    for name in ("decode_gate_up", "decode_down"):
+        P = config_problem(name)
+        base = to_device(P)
+        layers = [{k: base[k].clone() for k in ("packed", "scales", "aux")} for _ in range(N_LAYERS)]
+        for m in (1, 2, 4, 6, 8, 9, 12, 16, 24, 32, 48, 64):
+            ids = distinct_uniform_ids(rng, m * calls, 8, P.num_experts).reshape(calls, m, 8)
+            x = bf16_bits(rng.standard_normal((calls, m, P.k), dtype=np.float32))
+            d_ids = torch.from_numpy(ids.view(np.int32)).cuda()
+            d_x = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+            out = torch.empty((calls, m, 8, P.n), dtype=torch.float32, device="cuda")
+            ws = M.new_workspace(m, 8, P.num_experts)
+            row = {"projection": name.replace("decode_", ""), "m": m, "routings": 8 * m}
+            for path in ("decode", "grouped"):
+                def one(c, path=path):
+                    L = layers[c % N_LAYERS]
+                    M.qmm_id(d_x[c], d_ids[c], L["packed"], L["scales"], L["aux"], n=P.n,
+                             group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
+                             out=out[c], workspace=ws, path=path)
+                g = capture_graph(one, calls)
+                r = per_call(g, calls)
+                del g
+                row[f"{path}_us"] = r["s"] * 1e6
+            row["faster"] = "decode" if row["decode_us"] <= row["grouped_us"] else "grouped"
+            rows.append(row)
+        del base, layers
+        torch.cuda.empty_cache()
+    print(json.dumps({"crossover": "decode path vs grouped GEMM per call, E128 top8 affine 4-bit g64, bf16 x",
+                      "rows": rows, "timing": f"CUDA graph of {calls} calls, median of {REPEATS} replays",
+                      "threshold_in_library": "MOE_DECODE_MAX_ROUTINGS, MOE_DECODE_MAX_PAIRS_PER_EXPERT",
+                      "clocks": clocks_summary(sampler)}), flush=True)
+
+
 def run_probe(args):
     """A few untimed calls of one workload (for profiler captures): decode runs the
     gate/up projection `reps` times, then the down projection `reps` times; the
@@ -850,8 +898,13 @@ def main():
                     help="decode bench line without the grouped workloads and the m-sweep")
     ap.add_argument("--sweep", action="store_true",
                     help="decode m = 1, 2, 4, 8 curve (one GPU), one JSON line, instead of the bench line")
+    ap.add_argument("--crossover", action="store_true",
+                    help="decode path vs grouped GEMM per call at m = 1 .. 64 tokens (one GPU), one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.crossover:
+        run_crossover(args)
+        return
     if args.probe:
         run_probe(args)
         return

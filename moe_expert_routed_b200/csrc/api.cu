@@ -164,6 +164,9 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     cudaStream_t st = (cudaStream_t)stream;
     const bool routable = num_experts <= ROUTE_MAX_E;
     const bool small = R <= MOE_DECODE_MAX_ROUTINGS;
+    // few pairs per expert: the CUDA-core GEMV reads each expert's rows once for all
+    // of its pairs and is faster than the tensor-core GEMM (measured crossover)
+    const bool sparse = R <= (uint64_t)MOE_DECODE_MAX_PAIRS_PER_EXPERT * num_experts;
 
     enum { FUSED, ROUTED_GEMV, GROUPED } choice;
     if (path == MOE_PATH_GROUPED) {
@@ -175,6 +178,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         else return MOE_ERR_UNSUPPORTED;
     } else {
         if (small) choice = FUSED;
+        else if (routable && sparse) choice = ROUTED_GEMV;
         else if (routable && gemm_supported(a)) choice = GROUPED;
         else if (routable) choice = ROUTED_GEMV;
         else return MOE_ERR_UNSUPPORTED;

@@ -26,6 +26,8 @@
 //               their own copies.
 //   warp 12     TMEM allocation; one lane issues tcgen05.mma (kind::f16, fp32
 //               accumulation in TMEM) and tcgen05.commit.
+//   warp 13     with TMA staging, one lane issues the k-tiles' tensor copies of
+//               the packed codes (no multicast), S k-tiles ahead like the loaders.
 // Per stage: loaded (loader copies landed) -> full (dequantised) -> empty (the
 // MMAs that read it completed). Dequantisation of k-tile kt overlaps the MMAs
 // of kt-1 and the copies of kt+1 .. kt+S-1. Every wait is bounded (1 s); a wait
@@ -38,6 +40,11 @@
 // (cb[c]*s) weights are formed in fp32 and split into a 16-bit high part and
 // the 16-bit rounding of the remainder (two MMAs). f32 x is split the same way
 // into two bf16 halves; the lo*lo product is dropped (below 2^-16 relative).
+#include <string.h>
+
+#include <cuda.h>  // CUtensorMap and its encoding enums (the driver is reached via cudaGetDriverEntryPoint)
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -50,9 +57,10 @@ constexpr int BM = 128;
 constexpr int KT = 64;                          // k per tile: one 128-byte swizzle atom of 16-bit values
 constexpr int NDQ = 256;                        // dequantising threads (warps 0-7)
 constexpr int NLD = 128;                        // loader threads (warps 8-11)
-constexpr int GEMM_THREADS = NDQ + NLD + 32;    // + the MMA warp
+constexpr int GEMM_THREADS = NDQ + NLD + 64;    // + the MMA warp and the tensor-copy warp
 constexpr int LD_WARP0 = NDQ / 32;
 constexpr int MMA_WARP = (NDQ + NLD) / 32;
+constexpr int TMA_WARP = MMA_WARP + 1;
 constexpr int MAX_STAGES = 6;
 constexpr int A_TILE = BM * KT * 2;             // bytes per A term per stage
 constexpr uint64_t WAIT_NS = 1000000000ull;
@@ -85,6 +93,9 @@ struct GemmParams {
     // failure-detection test hook: non-zero makes the MMA warp first wait this long on
     // a barrier nothing completes (so the CTA aborts); 0 in normal operation
     uint64_t fault_ns;
+    // packed codes staged by TMA tensor copies (the kernel's tensor-map argument) instead
+    // of the loaders' cp.async
+    uint32_t tma;
 };
 
 template <int KIND> constexpr int a_terms() { return KIND == K_NVFP4 ? 1 : 2; }
@@ -138,12 +149,34 @@ template <> struct Raw<K_CB3> { static constexpr int W = 4; };  // codes SUB .. 
 //   bytes [RB+8, RB+16)   the same words of the biases (affine)
 // Rows are an odd number of 16-byte units apart, so 8 consecutive rows read
 // with 16-byte loads touch all 32 banks once.
+//
+// With TMA staging (contiguous weights, rows a multiple of 16 bytes, not 3-bit)
+// the same area holds instead
+//   [0, BM*RB)            the codes, BM rows of RB bytes written by two 64-row
+//                         tensor copies; for RB = 32 / 64 the 16-byte chunks of a
+//                         row are swizzled within 32 / 64 bytes (the copies'
+//                         SWIZZLE_32B / 64B mode), so 8 consecutive rows read with
+//                         16-byte loads touch all 32 banks once
+//   [BM*RB, BM*RB+BM*16)  per row: scale words (8 bytes), then bias words (8 bytes)
 template <int KIND> struct RawLayout {
     static constexpr uint32_t RB = KIND == K_CB3 ? 32u : 8u * kind_bits(KIND);
     static constexpr uint32_t SC = RB, BI = RB + 8u;
     static constexpr uint32_t STRIDE = ((RB + 16u) / 16u) % 2u ? RB + 16u : RB + 32u;
     static constexpr uint32_t TILE = BM * STRIDE;
+    static constexpr uint32_t TMA_SC = BM * RB;
+    static_assert(BM * RB + BM * 16u <= TILE, "TMA staging fits the cp.async staging area");
 };
+
+// Byte offset of 16-byte chunk c of staged row sr in the TMA code tile (the
+// swizzle the tensor copies apply: address bit 4 ^= bit 7 for 32-byte rows, bits
+// 4-5 ^= bits 7-8 for 64-byte rows; the tile is 1024-byte aligned).
+template <int KIND>
+__device__ __forceinline__ uint32_t tma_chunk(uint32_t sr, uint32_t c) {
+    constexpr uint32_t RB = RawLayout<KIND>::RB;
+    if constexpr (RB == 32) return sr * 32u + 16u * (c ^ ((sr >> 2) & 1u));
+    else if constexpr (RB == 64) return sr * 64u + 16u * (c ^ ((sr >> 1) & 3u));
+    else return sr * RB + 16u * c;
+}
 
 template <int KIND, int SUB>
 __device__ __forceinline__ uint32_t raw_code(const uint32_t (&w)[Raw<KIND>::W], int i) {
@@ -242,6 +275,45 @@ __device__ __forceinline__ void nvfp4_store(const uint32_t (&w)[4], __half2 s01,
     }
 }
 
+// Codebook weights with f16 x (A in f16): each code pair (2e, 2e+1) of the thread's
+// 32 codes is looked up as one f16x2 (cb[c0], cb[c1]) in a pair table of
+// 2^(2 bits) entries, then w = cb * s is split into hi = f16(cb * s) and
+// lo = f16(cb * s - hi) by an f16x2 multiply and a fused multiply-add. cb and s
+// are f16, so cb * s has at most 22 significant bits and hi + lo holds it to
+// within the f16 subnormal spacing (2^-24). Codes of a pair share a word (pairs
+// start at even positions and a 3-bit word holds 10 codes).
+template <int KIND, int SUB>
+__device__ __forceinline__ void cb_pairs_f16(const uint32_t (&w)[Raw<KIND>::W], __half2 s0, __half2 s1,
+                                             bool two_groups, const uint32_t *lut2, uint32_t a_hi,
+                                             uint32_t a_lo, uint32_t r, uint32_t c0) {
+    constexpr int B = kind_bits(KIND);
+#pragma unroll
+    for (int cc = 0; cc < 4; cc++) {
+        uint32_t hh[4], ll[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int i = cc * 8 + 2 * e;  // first code of the pair (compile-time)
+            uint32_t idx;
+            if constexpr (KIND == K_CB3) {
+                idx = (w[(SUB + i) / 10] >> (3 * ((SUB + i) % 10))) & 63u;
+            } else {
+                constexpr int EPW = 32 / B;
+                idx = (w[i / EPW] >> (B * (i % EPW))) & ((1u << (2 * B)) - 1u);
+            }
+            const uint32_t pr = lut2[idx];
+            const __half2 cbp = *reinterpret_cast<const __half2 *>(&pr);
+            const __half2 sv = (i >= 16 && two_groups) ? s1 : s0;
+            const __half2 hi = __hmul2(cbp, sv);
+            const __half2 lo = __hfma2(cbp, sv, __hneg2(hi));
+            hh[e] = *reinterpret_cast<const uint32_t *>(&hi);
+            ll[e] = *reinterpret_cast<const uint32_t *>(&lo);
+        }
+        const uint32_t off = swz(r, c0 + cc);
+        sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
+        sts128(a_lo + off, ll[0], ll[1], ll[2], ll[3]);
+    }
+}
+
 template <int KIND, bool F16>
 __device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], uint32_t sub, float s0,
                                              float b0, float s1, float b1, bool two_groups,
@@ -321,7 +393,7 @@ struct GemmCfg {
 // decided at compile time so that the plain kernels carry none of it.
 template <int KIND, int XT, int BN, bool PTRS, bool GLU>
 __global__ void __launch_bounds__(GEMM_THREADS, BN == 64 ? 2 : 1)
-grouped_gemm_kernel(const GemmParams P) {
+grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap) {
     using C = GemmCfg<KIND, XT, BN>;
     constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
     constexpr uint32_t STAGE = C::STAGE;
@@ -339,6 +411,9 @@ grouped_gemm_kernel(const GemmParams P) {
     __shared__ int abort_s;
     __shared__ uint32_t pairs_s[BN];
     __shared__ float cb_s[16];
+    // codebook with f16 x: f16x2 table of code pairs (cb[c & mask], cb[c >> bits])
+    constexpr bool CBF16 = (KIND == K_CB2 || KIND == K_CB3 || KIND == K_CB4) && XT == DT_F16;
+    __shared__ uint32_t lut2_s[CBF16 ? (1u << (2 * kind_bits(KIND))) : 1u];
 
     const uint32_t tile = blockIdx.y;
     if (tile >= __ldg(P.tile_count)) return;  // uniform
@@ -382,10 +457,11 @@ grouped_gemm_kernel(const GemmParams P) {
     const uint32_t never = ptx::smem_u32(&bars[3 * MAX_STAGES + 1]);  // completed by nothing
     volatile int *abort_flag = &abort_s;
 
+    const bool tma = !PTRS && KIND != K_CB3 && P.tma != 0;
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
             ptx::mbar_init(full0 + 8 * s, NDQ);
-            ptx::mbar_init(loaded0 + 8 * s, NLD);
+            ptx::mbar_init(loaded0 + 8 * s, NLD + (tma ? 1u : 0u));  // + the TMA issuer's arrival
             ptx::mbar_init(empty0 + 8 * s, 1);
         }
         ptx::mbar_init(accb, 1);
@@ -398,6 +474,14 @@ grouped_gemm_kernel(const GemmParams P) {
     if constexpr (KIND == K_CB2 || KIND == K_CB3 || KIND == K_CB4) {
         if (tid < (1u << kind_bits(KIND)))
             cb_s[tid] = f16_bits_to_f32(__ldg((const unsigned short *)P.aux + tid));
+        if constexpr (CBF16) {
+            constexpr uint32_t NC = 1u << kind_bits(KIND);
+            for (uint32_t i = tid; i < NC * NC; i += blockDim.x) {
+                const uint32_t lo = __ldg((const unsigned short *)P.aux + (i & (NC - 1u)));
+                const uint32_t hi = __ldg((const unsigned short *)P.aux + (i / NC));
+                lut2_s[i] = lo | (hi << 16);
+            }
+        }
     }
     if (warp == MMA_WARP) {
         ptx::tmem_alloc(ptx::smem_u32(&tmem_s), TMEM_COLS);
@@ -448,24 +532,31 @@ grouped_gemm_kernel(const GemmParams P) {
                     sts128(st + B_OFF + B_TILE + o, lo[0], lo[1], lo[2], lo[3]);
                 }
             }
+            // this row's codes and scale words: the strided cp.async rows, or the TMA tile
+            // (GLU: staged rows 0-63 hold the gate rows, 64-127 the up rows)
             const uint8_t *rr = stp + RAW_OFF + r * RL::STRIDE;
+            const uint8_t *ct = stp + RAW_OFF;
+            const uint32_t sr = GLU ? ((r & 1u) ? 64u + (r >> 1) : (r >> 1)) : r;
+            const uint8_t *sw_row = tma ? ct + RL::TMA_SC + 16u * r : rr + RL::SC;
             uint32_t w[Raw<KIND>::W];
             uint32_t sub = 0;
             if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
-                const uint4 q = *(const uint4 *)(rr + 16u * h);
+                const uint4 q = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, h) : rr + 16u * h);
                 w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
             } else if constexpr (KIND == K_AFF8) {
-                const uint4 q0 = *(const uint4 *)(rr + 32u * h), q1 = *(const uint4 *)(rr + 32u * h + 16u);
+                const uint4 q0 = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, 2u * h) : rr + 32u * h);
+                const uint4 q1 = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, 2u * h + 1u) : rr + 32u * h + 16u);
                 w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
                 w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
             } else if constexpr (KIND == K_AFF6) {
+                const uint8_t *cr = tma ? ct + sr * RL::RB : rr;
 #pragma unroll
                 for (int i = 0; i < 3; i++) {
-                    const uint2 q = *(const uint2 *)(rr + 24u * h + 8u * i);
+                    const uint2 q = *(const uint2 *)(cr + 24u * h + 8u * i);
                     w[2 * i] = q.x; w[2 * i + 1] = q.y;
                 }
             } else if constexpr (KIND == K_CB2) {
-                const uint2 q = *(const uint2 *)(rr + 8u * h);
+                const uint2 q = *(const uint2 *)((tma ? ct + sr * RL::RB : rr) + 8u * h);
                 w[0] = q.x; w[1] = q.y;
             } else {  // K_CB3: codes from (kt*KT) % 10 + 32h of the window
                 const uint32_t c0 = (kt * KT) % 10u + 32u * h, wb = c0 / 10u;
@@ -479,7 +570,7 @@ grouped_gemm_kernel(const GemmParams P) {
                 __half2 s01;
                 if (PTRS ? ptr_scale_words : P.scale_words != 0) {
                     // the staged word holds groups 4kt .. 4kt+3; this half's are bytes 2h, 2h+1
-                    s01 = e4m3x2_to_half2((*(const uint32_t *)(rr + RL::SC) >> (16u * h)) & 0xFFFFu);
+                    s01 = e4m3x2_to_half2((*(const uint32_t *)sw_row >> (16u * h)) & 0xFFFFu);
                 } else {
                     float s0, s1, unused;
                     global_scale<KIND>(srow, brow, gh, P.groups, s0, unused);
@@ -490,7 +581,7 @@ grouped_gemm_kernel(const GemmParams P) {
             } else {
                 float s0, b0, s1 = 0.f, b1 = 0.f;
                 if (PTRS ? ptr_scale_words : P.scale_words != 0) {
-                    const uint4 q = *(const uint4 *)(rr + RL::SC);
+                    const uint4 q = *(const uint4 *)sw_row;
                     const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
                     const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
                     staged_scale<KIND>(sw, bw, gh * ES - base_b, s0, b0);
@@ -499,7 +590,22 @@ grouped_gemm_kernel(const GemmParams P) {
                     global_scale<KIND>(srow, brow, gh, P.groups, s0, b0);
                     if (gs16) global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, b1);
                 }
-                dequant_tile<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
+                if constexpr (CBF16) {
+                    const __half2 h0 = __float2half2_rn(s0), h1 = __float2half2_rn(s1);  // exact: f16 scales
+                    if constexpr (KIND == K_CB3) {
+                        switch (sub) {  // first code's position in word 0: 0, 2, 4, 6 or 8
+                            case 0: cb_pairs_f16<KIND, 0>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                            case 2: cb_pairs_f16<KIND, 2>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                            case 4: cb_pairs_f16<KIND, 4>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                            case 6: cb_pairs_f16<KIND, 6>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                            default: cb_pairs_f16<KIND, 8>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                        }
+                    } else {
+                        cb_pairs_f16<KIND, 0>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u);
+                    }
+                } else {
+                    dequant_tile<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
+                }
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(full0 + 8 * s);
@@ -585,7 +691,9 @@ grouped_gemm_kernel(const GemmParams P) {
             }
             // packed codes of the 128 rows (rows past n repeat row n-1; bytes past a row read as 0)
             const uint32_t raw = st + RAW_OFF;
-            if constexpr (KIND == K_CB3) {
+            if (tma) {
+                // the codes come by tensor copy from the tensor-copy warp
+            } else if constexpr (KIND == K_CB3) {
                 const uint32_t w0 = (kt * KT) / 10u;
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
@@ -621,18 +729,46 @@ grouped_gemm_kernel(const GemmParams P) {
             }
             if (PTRS ? ptr_scale_words : P.scale_words != 0) {
                 const uint32_t base_b = ((kt * KT >> P.lg_gs) * ES) & ~3u;
+                const uint32_t sdst = tma ? raw + RL::TMA_SC + 16u * lt : raw + lt * RL::STRIDE + RL::SC;
                 for (uint32_t i = 0; i < nsw; i++) {
                     const uint32_t o = base_b + 4u * i;
                     const bool in = o + 4u <= srow_bytes;
-                    ptx::cp_async_4(raw + lt * RL::STRIDE + RL::SC + 4u * i, srow + (in ? o : 0u), in ? 4u : 0u);
-                    if constexpr (AFF)
-                        ptx::cp_async_4(raw + lt * RL::STRIDE + RL::BI + 4u * i, brow + (in ? o : 0u),
-                                        in ? 4u : 0u);
+                    ptx::cp_async_4(sdst + 4u * i, srow + (in ? o : 0u), in ? 4u : 0u);
+                    if constexpr (AFF) ptx::cp_async_4(sdst + 8u + 4u * i, brow + (in ? o : 0u), in ? 4u : 0u);
                 }
             }
             ptx::cp_async_mbar_arrive(loaded0 + 8 * s);
         }
         ptx::cp_async_wait_all();
+    } else if (warp == TMA_WARP) {
+        // ------------------------------------------------------ code tensor copies
+        if (tma && lane == 0) {
+            // per k-tile two 64-row copies of RB bytes per row (GLU: the 64 gate rows,
+            // then the 64 up rows); rows past the expert's last read a neighbour's rows or
+            // zeros and are never stored. The arrival (with the byte count) is one of the
+            // stage's loaded arrivals.
+            constexpr uint32_t RB = RL::RB;
+            ptx::prefetch_tensormap(&tmap);
+            const int32_t y0 = (int32_t)(e * P.n + (GLU ? row0 / 2u : row0));
+            const int32_t y1 = GLU ? (int32_t)(e * P.n + P.glu_nh + row0 / 2u) : y0 + 64;
+            uint32_t last_s = 0, last_par = 0;
+            bool any = false;
+            for (uint32_t kt = 0; kt < P.ktiles; kt++) {
+                const uint32_t s = kt % S;
+                if (kt >= S && !ptx::mbar_wait_bounded(empty0 + 8 * s, ((kt / S) - 1u) & 1u, abort_flag, P.err,
+                                                       ERR_TIMEOUT, P.timeout_ns))
+                    break;
+                const uint32_t bar = loaded0 + 8 * s, raw = base + s * STAGE + RAW_OFF;
+                ptx::mbar_arrive_expect_tx(bar, 2u * 64u * RB);
+                ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
+                ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
+                last_s = s;
+                last_par = (kt / S) & 1u;
+                any = true;
+            }
+            // copies still in flight after a wait gave up land before the CTA exits
+            if (any) ptx::mbar_wait_bounded(loaded0 + 8 * last_s, last_par, nullptr, P.err, ERR_TIMEOUT, DRAIN_NS);
+        }
     } else if (lane == 0) {
         // --------------------------------------------------------------- MMA issue
         const uint32_t n1 = tmin<uint32_t>(nt_pad, 256u), n2 = nt_pad - n1;
@@ -737,8 +873,8 @@ bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
 }
 
 template <int KIND, int XT, int BN, bool PTRS, bool GLU>
-cudaError_t launch_tp(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
-                      cudaStream_t st) {
+cudaError_t launch_tp(const GemmParams &P0, const CUtensorMap &tmap, const GemmPlan &pl, uint32_t n_mtiles,
+                      uint32_t max_tiles, cudaStream_t st) {
     GemmParams P = P0;
     P.stages = (uint32_t)pl.stages;
     auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS, GLU>;
@@ -746,51 +882,99 @@ cudaError_t launch_tp(const GemmParams &P0, const GemmPlan &pl, uint32_t n_mtile
     cudaError_t e = ensure_dyn_smem(kern, pl.smem, smem_set);
     if (e != cudaSuccess) return e;
     dim3 grid(n_mtiles, max_tiles);
-    kern<<<grid, GEMM_THREADS, pl.smem, st>>>(P);
+    kern<<<grid, GEMM_THREADS, pl.smem, st>>>(P, tmap);
     return cudaGetLastError();
 }
 
 template <int KIND, int XT, int BN>
-cudaError_t launch_t(const GemmParams &P, const GemmPlan &pl, uint32_t n_mtiles, uint32_t max_tiles,
-                     cudaStream_t st) {
-    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true, false>(P, pl, n_mtiles, max_tiles, st);
-    if (P.glu_nh) return launch_tp<KIND, XT, BN, false, true>(P, pl, n_mtiles, max_tiles, st);
-    return launch_tp<KIND, XT, BN, false, false>(P, pl, n_mtiles, max_tiles, st);
+cudaError_t launch_t(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, uint32_t n_mtiles,
+                     uint32_t max_tiles, cudaStream_t st) {
+    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true, false>(P, tm, pl, n_mtiles, max_tiles, st);
+    if (P.glu_nh) return launch_tp<KIND, XT, BN, false, true>(P, tm, pl, n_mtiles, max_tiles, st);
+    return launch_tp<KIND, XT, BN, false, false>(P, tm, pl, n_mtiles, max_tiles, st);
 }
 
 template <int KIND>
-cudaError_t launch_k(const GemmParams &P, const GemmPlan &pl, int x_dtype, uint32_t nm, uint32_t mt,
-                     cudaStream_t st) {
+cudaError_t launch_k(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, int x_dtype, uint32_t nm,
+                     uint32_t mt, cudaStream_t st) {
     if (x_dtype == DT_F32) {
-        if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, pl, nm, mt, st);
-        return launch_t<KIND, DT_F32, 64>(P, pl, nm, mt, st);
+        if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, tm, pl, nm, mt, st);
+        return launch_t<KIND, DT_F32, 64>(P, tm, pl, nm, mt, st);
     }
     if constexpr (KIND == K_NVFP4) {
         if (pl.bn == 320) {
-            if (x_dtype == DT_BF16) return launch_t<KIND, DT_BF16, 320>(P, pl, nm, mt, st);
-            return launch_t<KIND, DT_F16, 320>(P, pl, nm, mt, st);
+            if (x_dtype == DT_BF16) return launch_t<KIND, DT_BF16, 320>(P, tm, pl, nm, mt, st);
+            return launch_t<KIND, DT_F16, 320>(P, tm, pl, nm, mt, st);
         }
     }
     if (x_dtype == DT_BF16) {
-        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, pl, nm, mt, st);
-        return launch_t<KIND, DT_BF16, 64>(P, pl, nm, mt, st);
+        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, pl, nm, mt, st);
+        return launch_t<KIND, DT_BF16, 64>(P, tm, pl, nm, mt, st);
     }
-    if (pl.bn == 256) return launch_t<KIND, DT_F16, 256>(P, pl, nm, mt, st);
-    return launch_t<KIND, DT_F16, 64>(P, pl, nm, mt, st);
+    if (pl.bn == 256) return launch_t<KIND, DT_F16, 256>(P, tm, pl, nm, mt, st);
+    return launch_t<KIND, DT_F16, 64>(P, tm, pl, nm, mt, st);
 }
 
-cudaError_t launch_kind(const GemmParams &P, const GemmPlan &pl, int kind, int x_dtype, uint32_t nm,
-                        uint32_t mt, cudaStream_t st) {
+cudaError_t launch_kind(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, int kind, int x_dtype,
+                        uint32_t nm, uint32_t mt, cudaStream_t st) {
     switch (kind) {
-        case K_AFF4: return launch_k<K_AFF4>(P, pl, x_dtype, nm, mt, st);
-        case K_AFF6: return launch_k<K_AFF6>(P, pl, x_dtype, nm, mt, st);
-        case K_AFF8: return launch_k<K_AFF8>(P, pl, x_dtype, nm, mt, st);
-        case K_CB2: return launch_k<K_CB2>(P, pl, x_dtype, nm, mt, st);
-        case K_CB3: return launch_k<K_CB3>(P, pl, x_dtype, nm, mt, st);
-        case K_CB4: return launch_k<K_CB4>(P, pl, x_dtype, nm, mt, st);
-        case K_NVFP4: return launch_k<K_NVFP4>(P, pl, x_dtype, nm, mt, st);
+        case K_AFF4: return launch_k<K_AFF4>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_AFF6: return launch_k<K_AFF6>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_AFF8: return launch_k<K_AFF8>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_CB2: return launch_k<K_CB2>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_CB3: return launch_k<K_CB3>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_CB4: return launch_k<K_CB4>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_NVFP4: return launch_k<K_NVFP4>(P, tm, pl, x_dtype, nm, mt, st);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (null if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return (PFN_cuTensorMapEncodeTiled_v12000)f;
+    }();
+    return fn;
+}
+
+// Bytes of one k-tile of one packed row (the staging's RB) for each storage kind.
+uint32_t ktile_row_bytes(int kind) {
+    switch (kind) {
+        case K_AFF4: return RawLayout<K_AFF4>::RB;
+        case K_AFF6: return RawLayout<K_AFF6>::RB;
+        case K_AFF8: return RawLayout<K_AFF8>::RB;
+        case K_CB2: return RawLayout<K_CB2>::RB;
+        case K_CB4: return RawLayout<K_CB4>::RB;
+        case K_NVFP4: return RawLayout<K_NVFP4>::RB;
+        default: return 0;
+    }
+}
+
+// Tensor map of the packed codes as a [num_experts * n, row_bytes] byte matrix with
+// 64-row x RB-byte boxes, swizzled as tma_chunk expects. False when the codes
+// cannot be staged this way (pointer tables, 3-bit rows, rows not a multiple of
+// 16 bytes, or no driver entry point).
+bool code_tensor_map(const QmmArgs &a, CUtensorMap *m) {
+    const uint32_t rb = ktile_row_bytes(a.kind);
+    if (!rb || a.packed_ptrs || a.row_bytes % 16u != 0 || (uintptr_t)a.packed % 16u != 0) return false;
+    const uint64_t rows = (uint64_t)a.num_experts * a.n;
+    if (rows >= (1ull << 31)) return false;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {a.row_bytes, rows};
+    const cuuint64_t strides[1] = {a.row_bytes};
+    const cuuint32_t box[2] = {rb, 64u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUtensorMapSwizzle sw = rb == 32u ? CU_TENSOR_MAP_SWIZZLE_32B
+                                : rb == 64u ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void *)a.packed, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -839,8 +1023,11 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.fault_ns = a.fault_wait_ns;
     P.glu_nh = a.act >= 0 ? a.n / 2u : 0u;
     P.act = a.act;
+    CUtensorMap tmap;
+    memset(&tmap, 0, sizeof(tmap));
+    P.tma = code_tensor_map(a, &tmap) ? 1u : 0u;
     const uint32_t nm = (a.n + BM - 1) / BM;
-    return launch_kind(P, pl, a.kind, a.x_dtype, nm, max_tiles, st);
+    return launch_kind(P, tmap, pl, a.kind, a.x_dtype, nm, max_tiles, st);
 }
 
 }  // namespace moe

@@ -1405,6 +1405,18 @@ GemvParams make_params(const QmmArgs &a, uint32_t *err) {
     return P;
 }
 
+// Pairs per pass of a decode CTA over its expert's rows: the smallest power of two
+// at or above the mean pairs per expert, ceil(R / num_experts), at most min(m, 8).
+// Every pass computes NPB pair slots, so a batch much larger than an expert's
+// pairs computes mostly empty slots; experts with more pairs take several passes.
+uint32_t pairs_per_pass(const QmmArgs &a) {
+    const uint64_t R = (uint64_t)a.m * a.n_expert_used;
+    const uint64_t mean = (R + a.num_experts - 1) / a.num_experts;
+    uint32_t npb = 1;
+    while (npb < mean && npb < 8u) npb <<= 1;
+    return tmin<uint32_t>(npb, tmin<uint32_t>(a.m, 8u));
+}
+
 }  // namespace
 
 cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st) {
@@ -1412,7 +1424,7 @@ cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st) 
     const uint32_t distinct_max = min(P.R, a.num_experts);
     dim3 grid((a.n + GEMV_ROWS - 1) / GEMV_ROWS, distinct_max);
     // pairs of one expert come from distinct tokens unless ids repeat inside a token
-    const uint32_t npb = tmin<uint32_t>(a.m, 8u);
+    const uint32_t npb = pairs_per_pass(a);
     const uint32_t xsz = a.x_dtype == DT_F32 ? 4u : 2u;
     const bool spec = (uint64_t)a.m * a.k * xsz <= 32768u;
     if (a.packed_ptrs) return launch_kind<true>(P, a.kind, npb, grid, st);  // pointer-table weights
@@ -1435,10 +1447,11 @@ cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const u
     GemvParams P = make_params(a, err);
     P.counts = counts; P.offsets = offsets; P.sorted_pairs = sorted_pairs;
     dim3 grid((a.n + GEMV_ROWS - 1) / GEMV_ROWS, a.num_experts);
-    if (a.packed_ptrs || a.act >= 0) return launch_kind<false>(P, a.kind, 8u, grid, st);  // pointer tables, gated output
-    if (tma_ok(a, 8u, false)) return launch_tma<MODE_ROUTED>(P, 8u, a.num_experts, st);
-    if (dp4a_ok(a)) return launch_dp4a<false>(P, 8u, grid, st);
-    return launch_kind<false>(P, a.kind, 8u, grid, st);
+    const uint32_t npb = pairs_per_pass(a);
+    if (a.packed_ptrs || a.act >= 0) return launch_kind<false>(P, a.kind, npb, grid, st);  // pointer tables, gated output
+    if (tma_ok(a, npb, false)) return launch_tma<MODE_ROUTED>(P, npb, a.num_experts, st);
+    if (dp4a_ok(a)) return launch_dp4a<false>(P, npb, grid, st);
+    return launch_kind<false>(P, a.kind, npb, grid, st);
 }
 
 }  // namespace moe
