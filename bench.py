@@ -521,11 +521,10 @@ def decode_per_call(W: DecodeWorkload) -> dict:
 
 def grouped_tile_rows(P) -> int:
     """Tile height of the grouped GEMM for this call (as the library picks it):
-    256 pairs (128 with f32 x, 320 for NVFP4) when experts hold ~96+ pairs on
-    average, else 64. Only sizes the routing prologue's tile list when the
-    prologue is timed alone."""
+    256 pairs (128 with f32 x) when experts hold ~96+ pairs on average, else 64.
+    Only sizes the routing prologue's tile list when the prologue is timed alone."""
     if P.R >= 96 * P.num_experts:
-        return 128 if P.x_dtype == 0 else (320 if P.fmt == 2 else 256)
+        return 128 if P.x_dtype == 0 else 256
     return 64
 
 
@@ -676,8 +675,21 @@ def run_ours(args, dist: Dist):
     Gt = min(GRAPH_STEPS, K)
     W = DecodeWorkload(max(Gt, GRAPH_CALLS), pdl=not args.no_pdl)
     # the timed graph holds steps 0..Gt-1; uploaded to the device before warm-up so
-    # that its first replay is a plain replay
-    g = W.capture(Gt)
+    # that its first replay is a plain replay. When the K steps fit one graph, the
+    # timing events are event nodes inside it, right before the first step's kernel
+    # and after the last step's, so the timed region is the K steps on the device
+    # without the host's graph-launch latency.
+    ev0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev1 = torch.cuda.Event(enable_timing=True, external=True)
+
+    def timed_step(s):
+        if s == 0:
+            ev0.record()
+        W.step(s)
+        if s == Gt - 1:
+            ev1.record()
+
+    g = capture_graph(timed_step, Gt)
     uploaded = graph_upload(g)
     warm_done = Wm
     for s in range(Wm):  # W untimed warm-up steps (the step's own calls, issued one by one)
@@ -694,6 +706,9 @@ def run_ours(args, dist: Dist):
     torch.cuda.synchronize()
     secs = time_graph(g, replays)
     torch.cuda.synchronize()
+    in_graph = replays == 1
+    if in_graph:
+        secs = ev0.elapsed_time(ev1) / 1e3
     dist.barrier()
     clocks = clocks_summary(sampler) if dist.rank == 0 else None
     del g
@@ -740,7 +755,9 @@ def run_ours(args, dist: Dist):
                                "affine 4-bit g64, bf16 x, f32 out",
                    "l2": f"inputs larger than L2: {N_LAYERS} rotated weight copies "
                          f"({N_LAYERS * 0.428:.1f} GB), fresh ids and x every step",
-                   "timing": f"CUDA graph of {Gt} steps replayed {replays}x, CUDA events"
+                   "timing": (f"CUDA graph of {Gt} steps, CUDA events recorded as nodes of the graph "
+                              "before the first and after the last step" if in_graph else
+                              f"CUDA graph of {Gt} steps replayed {replays}x, CUDA events around the replays")
                              + ("" if uploaded else " (graph replayed once more during warm-up)"),
                    "launch": ("gate/up: programmatic dependent launch; down: PDL with early weight "
                               "streaming (its ids were ready before gate/up began)")

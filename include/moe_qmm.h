@@ -48,10 +48,10 @@
  *                    w = e2m1(code) * 2^(scale - 127), scale E8M0 bytes
  *                    [E, n, k/32] (0xFF is NaN); no aux array (spark_model
  *                    helpers_a.rs: native-MXFP4 routed experts, per-32 E8M0
- *                    scales [N, K/32]). Computed by the CUDA-core decode
- *                    kernels on every path: MOE_PATH_GROUPED returns
- *                    MOE_ERR_UNSUPPORTED and MOE_PATH_AUTO uses the routed GEMV
- *                    for large calls.
+ *                    scales [N, K/32]). The grouped GEMM takes bf16 and f32 x
+ *                    (e2m1 * 2^e is exact in bf16 within its exponent range);
+ *                    with f16 x, MOE_PATH_GROUPED returns MOE_ERR_UNSUPPORTED
+ *                    and MOE_PATH_AUTO uses the routed CUDA-core GEMV.
  */
 #ifndef MOE_QMM_H
 #define MOE_QMM_H

@@ -23,6 +23,7 @@ bool ws_layout(uint64_t R, uint32_t E, WsLayout *L) {
     size_t off = 0;
     L->err = 0;
     L->tile_count = 4;
+    L->work_counter = 8;
     off = 256;
     L->counts = off; off += al256(4ull * (E + 1ull));
     L->offsets = off; off += al256(4ull * (E + 2ull));
@@ -195,13 +196,14 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         uint32_t *tc = (uint32_t *)(ws + L.tile_count);
         const uint32_t tile_rows = choice == GROUPED ? gemm_tile_rows(a) : MIN_TILE_ROWS;
         const uint32_t max_tiles = (uint32_t)(R / tile_rows + num_experts + 1);
+        uint32_t *wc = (uint32_t *)(ws + L.work_counter);
         ce = launch_route(ids, (uint32_t)R, num_experts, tile_rows, counts, offsets, sp, tiles, tc,
                           max_tiles, (uint32_t *)(ws + L.chunk_hist),
                           (uint32_t *)(ws + L.chunk_base), L.chunks, err, out, a.out_n, (int)out_dtype,
-                          st);
+                          st, wc);
         if (ce == cudaSuccess) {
             if (choice == GROUPED)
-                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, st);
+                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, st);
             else
                 ce = launch_gemv_routed(a, counts, offsets, sp, err, st);
         }

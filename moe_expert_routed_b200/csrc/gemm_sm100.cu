@@ -1,8 +1,9 @@
 // gemm_sm100.cu -- expert-grouped GEMM on the 5th-generation tensor cores (tcgen05).
 //
-// One CTA computes a 128 x BN tile of one expert: 128 consecutive weight rows
-// (output columns) of expert e against up to BN of the (token, slot) pairs
-// routed to e (a tile of the routing prologue's tile list). Operands are
+// A persistent grid (one CTA per SM) walks work items: a 128 x BN tile of one
+// expert, 128 consecutive weight rows (output columns) of expert e against up to
+// BN of the (token, slot) pairs routed to e (a tile of the routing prologue's
+// tile list). Operands are
 // swapped relative to out = x * W^T: the dequantised weight tile is the MMA's
 // A operand (M = 128) and the gathered token rows are B (N = pairs in the tile,
 // rounded up to 16), so each weight tile is dequantised once per tile of pairs.
@@ -11,23 +12,30 @@
 // GEMM fed by expert_offsets / sorted_token_ids (metrale helpers_b.rs,
 // launch_grouped_gemm).
 //
-// Warp roles (416 threads), each running through the k-tiles on its own:
+// Warp roles (736 threads), each running through the CTA's items and their
+// k-tiles on its own; the stage ring continues from one item to the next:
 //   warps 0-7   dequantisers: per 64-wide k-tile, turn the staged codes of 128
 //               rows x 64 codes into 16-bit values in the 128-byte-swizzled
-//               K-major layout (and split f32 x into two bf16 halves); then the
-//               epilogue: TMEM -> registers (tcgen05.ld), times scale2 for
-//               NVFP4, rounded once to the output type, stored to row p of out
-//               (the scatter back to [token][slot] order).
-//   warps 8-11  loaders: cp.async the pairs' x rows straight into the B operand
+//               K-major layout (and split f32 x into two bf16 halves).
+//   warps 8-15  loaders: cp.async the pairs' x rows straight into the B operand
 //               tile and the packed codes and scale words into a staging area,
 //               up to S k-tiles ahead of the tensor core; each loader's
 //               completion is signalled on the stage's mbarrier by the copy
 //               engine (cp.async.mbarrier.arrive), so loaders never block on
 //               their own copies.
-//   warp 12     TMEM allocation; one lane issues tcgen05.mma (kind::f16, fp32
+//   warp 16     TMEM allocation; one lane issues tcgen05.mma (kind::f16, fp32
 //               accumulation in TMEM) and tcgen05.commit.
-//   warp 13     with TMA staging, one lane issues the k-tiles' tensor copies of
+//   warp 17     with TMA staging, one lane issues the k-tiles' tensor copies of
 //               the packed codes (no multicast), S k-tiles ahead like the loaders.
+//   warps 18-21 epilogue: TMEM -> registers (tcgen05.ld), times scale2 for
+//               NVFP4, rounded once to the output type, stored to row p of out
+//               (the scatter back to [token][slot] order). Two TMEM accumulators
+//               alternate between items, so an item's epilogue overlaps the next
+//               item's MMAs.
+//   warp 22     scheduler: one lane claims work items (each CTA's first is its
+//               block index, the rest come from an atomic counter, so that CTAs
+//               that finish early take more) and publishes them to the other
+//               roles through a 4-slot ring in shared memory.
 // Per stage: loaded (loader copies landed) -> full (dequantised) -> empty (the
 // MMAs that read it completed). Dequantisation of k-tile kt overlaps the MMAs
 // of kt-1 and the copies of kt+1 .. kt+S-1. Every wait is bounded (1 s); a wait
@@ -56,11 +64,18 @@ namespace {
 constexpr int BM = 128;
 constexpr int KT = 64;                          // k per tile: one 128-byte swizzle atom of 16-bit values
 constexpr int NDQ = 256;                        // dequantising threads (warps 0-7)
-constexpr int NLD = 128;                        // loader threads (warps 8-11)
-constexpr int GEMM_THREADS = NDQ + NLD + 64;    // + the MMA warp and the tensor-copy warp
+constexpr int NLD = 256;                        // loader threads (warps 8-15)
+constexpr int NEP = 128;                        // epilogue threads (warps 18-21)
+constexpr int GEMM_THREADS = NDQ + NLD + 64 + NEP + 32;  // + the MMA, tensor-copy and scheduler warps
 constexpr int LD_WARP0 = NDQ / 32;
 constexpr int MMA_WARP = (NDQ + NLD) / 32;
 constexpr int TMA_WARP = MMA_WARP + 1;
+constexpr int EPI_WARP0 = TMA_WARP + 1;
+constexpr int SCHED_WARP = EPI_WARP0 + NEP / 32;
+constexpr uint32_t RING = 4;                    // work items the scheduler may publish ahead
+// arrivals that release a ring slot: one per dequantiser, loader and epilogue warp,
+// plus the tensor-copy and MMA lanes
+constexpr uint32_t RING_READERS = NDQ / 32 + NLD / 32 + NEP / 32 + 2;
 constexpr int MAX_STAGES = 6;
 constexpr int A_TILE = BM * KT * 2;             // bytes per A term per stage
 constexpr uint64_t WAIT_NS = 1000000000ull;
@@ -90,6 +105,8 @@ struct GemmParams {
     // and the epilogue writes act(gate) * up into rows of glu_nh = n/2 columns
     uint32_t glu_nh;
     int act;
+    uint32_t n_mtiles;      // 128-row blocks per expert (work items per tile)
+    uint32_t *work_counter; // items claimed beyond each CTA's first (zeroed by the routing prologue)
     // failure-detection test hook: non-zero makes the MMA warp first wait this long on
     // a barrier nothing completes (so the CTA aborts); 0 in normal operation
     uint64_t fault_ns;
@@ -98,7 +115,9 @@ struct GemmParams {
     uint32_t tma;
 };
 
-template <int KIND> constexpr int a_terms() { return KIND == K_NVFP4 ? 1 : 2; }
+// 16-bit terms of the A operand: NVFP4 e2m1 * e4m3 and MXFP4 e2m1 * 2^e are exact in
+// one bf16 (or f16) value; affine and codebook weights take a hi and a lo term.
+template <int KIND> constexpr int a_terms() { return (KIND == K_NVFP4 || KIND == K_MXFP4) ? 1 : 2; }
 
 // Byte offset of 16-byte chunk c (0..7) of row r inside a swizzled K-major tile.
 __device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c) {
@@ -137,6 +156,7 @@ template <int KIND> struct Raw;
 template <> struct Raw<K_AFF4> { static constexpr int W = 4; };
 template <> struct Raw<K_CB4> { static constexpr int W = 4; };
 template <> struct Raw<K_NVFP4> { static constexpr int W = 4; };
+template <> struct Raw<K_MXFP4> { static constexpr int W = 4; };
 template <> struct Raw<K_AFF8> { static constexpr int W = 8; };
 template <> struct Raw<K_AFF6> { static constexpr int W = 6; };
 template <> struct Raw<K_CB2> { static constexpr int W = 2; };
@@ -160,7 +180,7 @@ template <> struct Raw<K_CB3> { static constexpr int W = 4; };  // codes SUB .. 
 //   [BM*RB, BM*RB+BM*16)  per row: scale words (8 bytes), then bias words (8 bytes)
 template <int KIND> struct RawLayout {
     static constexpr uint32_t RB = KIND == K_CB3 ? 32u : 8u * kind_bits(KIND);
-    static constexpr uint32_t SC = RB, BI = RB + 8u;
+    static constexpr uint32_t SC = RB;  // scale words at SC, bias words at SC + 8
     static constexpr uint32_t STRIDE = ((RB + 16u) / 16u) % 2u ? RB + 16u : RB + 32u;
     static constexpr uint32_t TILE = BM * STRIDE;
     static constexpr uint32_t TMA_SC = BM * RB;
@@ -181,7 +201,7 @@ __device__ __forceinline__ uint32_t tma_chunk(uint32_t sr, uint32_t c) {
 template <int KIND, int SUB>
 __device__ __forceinline__ uint32_t raw_code(const uint32_t (&w)[Raw<KIND>::W], int i) {
     // i is a compile-time constant after unrolling
-    if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
+    if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4 || KIND == K_MXFP4) {
         return (w[i / 8] >> (4 * (i % 8))) & 15u;
     } else if constexpr (KIND == K_AFF8) {
         return (w[i / 4] >> (8 * (i % 4))) & 255u;
@@ -205,6 +225,7 @@ __device__ __forceinline__ void dequant32(const uint32_t (&w)[Raw<KIND>::W], flo
         const float s = (i >= 16 && two_groups) ? s1 : s0;
         const float b = (i >= 16 && two_groups) ? b1 : b0;
         if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) v[i] = fmaf((float)code, s, b);
+        else if constexpr (KIND == K_MXFP4) v[i] = e2m1_to_f32(code) * s;  // s = 2^(e - 127): exact
         else v[i] = cb[code] * s;
     }
 }
@@ -320,6 +341,7 @@ __device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], 
                                              const float *cb, uint32_t a_hi, uint32_t a_lo, uint32_t r,
                                              uint32_t c0) {
     static_assert(KIND != K_NVFP4, "NVFP4 tiles go through nvfp4_store");
+    constexpr bool TWO = a_terms<KIND>() == 2;
     {
         float v[32];
         if constexpr (KIND == K_CB3) {
@@ -333,7 +355,7 @@ __device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], 
         } else {
             dequant32<KIND, 0>(w, s0, b0, s1, b1, two_groups, cb, v);
         }
-        store_a<F16, true>(v, a_hi, a_lo, r, c0);
+        store_a<F16, TWO>(v, a_hi, a_lo, r, c0);
     }
 }
 
@@ -346,6 +368,9 @@ __device__ __forceinline__ void staged_scale(const uint32_t (&sw)[2], const uint
     const uint32_t sv = (wi ? sw[1] : sw[0]) >> sh;
     if constexpr (KIND == K_NVFP4) {
         s = e4m3_to_f32(sv & 0xFFu);
+        b = 0.f;
+    } else if constexpr (KIND == K_MXFP4) {
+        s = e8m0_to_f32(sv & 0xFFu);
         b = 0.f;
     } else if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) {
         s = bf16_bits_to_f32(sv & 0xFFFFu);
@@ -366,6 +391,8 @@ __device__ __forceinline__ void global_scale(const uint8_t *srow, const uint8_t 
     if (g >= groups) return;
     if constexpr (KIND == K_NVFP4) {
         s = e4m3_to_f32(__ldg(srow + g));
+    } else if constexpr (KIND == K_MXFP4) {
+        s = e8m0_to_f32(__ldg(srow + g));
     } else {
         const uint32_t sv = (uint32_t)__ldg(srow + 2 * g) | ((uint32_t)__ldg(srow + 2 * g + 1) << 8);
         if constexpr (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8) {
@@ -385,92 +412,137 @@ struct GemmCfg {
     static constexpr uint32_t STAGE = AT * A_TILE + BT * B_TILE + RawLayout<KIND>::TILE;
 };
 
-// Tiles of 64 pairs (few pairs per expert, dequantisation-bound) run two CTAs
-// per SM: two pipeline stages each, registers capped for two CTAs.
-// PTRS: weights from the pointer tables (decided at compile time so that the
-// contiguous case keeps its copy-width and scale-staging branches on kernel
-// parameters). GLU: gated output (glu_row order, act(gate) * up epilogue), also
-// decided at compile time so that the plain kernels carry none of it.
+// Work item w of the persistent grid: tile w / n_mtiles of the routing prologue's
+// tile list (expert e, first pair r0 of the expert's pairs) and 128-row block
+// w % n_mtiles of the expert's weight rows. Every role of a CTA walks the same
+// items (read from the scheduler's ring) and evaluates the same item set-up, so
+// they agree on which items are skipped.
+template <int KIND, bool PTRS>
+struct Item {
+    uint32_t e, r0, off, nt, nt_pad, row0;
+    const uint8_t *wb, *sb, *bb;
+    bool ptr_scale_words, ptr_raw16;
+
+    // false when the item is skipped (pointer-table expert not held here, or with
+    // unusable buffers: flagged once per item by block 0 of the column blocks)
+    __device__ __forceinline__ bool load(const GemmParams &P, uint32_t t, uint32_t nb, uint32_t bn) {
+        constexpr uint32_t ES = (KIND == K_NVFP4 || KIND == K_MXFP4) ? 1u : 2u;
+        constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
+        e = __ldg(P.tiles + 2 * t);
+        r0 = __ldg(P.tiles + 2 * t + 1);
+        off = __ldg(P.offsets + e);
+        const uint32_t cnt = __ldg(P.offsets + e + 1) - off;
+        nt = tmin<uint32_t>(bn, cnt - r0);
+        nt_pad = (nt + 15u) & ~15u;
+        row0 = nb * BM;
+        wb = P.packed + (size_t)e * P.n * P.row_bytes;
+        sb = (const uint8_t *)P.scales + (size_t)e * P.n * P.groups * ES;
+        bb = (const uint8_t *)P.aux + (size_t)e * P.n * P.groups * 2u;
+        ptr_scale_words = false;
+        ptr_raw16 = false;
+        if constexpr (PTRS) {
+            wb = (const uint8_t *)__ldg(P.packed_ptrs + e);
+            if (!wb) return false;  // expert held elsewhere: its pairs' rows are not ours to write
+            sb = (const uint8_t *)__ldg(P.scale_ptrs + e);
+            bb = AFF ? (const uint8_t *)__ldg(P.bias_ptrs + e) : nullptr;
+            // the copies need 8-byte aligned code rows (4 for 3-bit codebook rows) and 2-byte
+            // aligned 16-bit scales / biases; other experts are skipped and flagged
+            const uintptr_t wal = KIND == K_CB3 ? 4u : 8u;
+            const uintptr_t sal = (uintptr_t)sb | (AFF ? (uintptr_t)bb : 0u);
+            if (!sb || (AFF && !bb) || ((uintptr_t)wb % wal) != 0 || (ES == 2u && (sal & 1u))) {
+                if (nb == 0 && threadIdx.x == 0) atomicOr(P.err, ERR_BAD_POINTER);
+                return false;
+            }
+            ptr_raw16 = P.raw16 != 0 && (uintptr_t)wb % 16u == 0;
+            ptr_scale_words = P.scale_words != 0 && sal % 4u == 0 && (uintptr_t)sb % 4u == 0;
+        }
+        return true;
+    }
+};
+
+// Persistent grid, one CTA per SM. PTRS: weights from the pointer tables (decided at
+// compile time so that the contiguous case keeps its copy-width and scale-staging
+// branches on kernel parameters). GLU: gated output (glu_row order, act(gate) * up
+// epilogue), also decided at compile time so that the plain kernels carry none of it.
 template <int KIND, int XT, int BN, bool PTRS, bool GLU>
-__global__ void __launch_bounds__(GEMM_THREADS, BN == 64 ? 2 : 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap) {
     using C = GemmCfg<KIND, XT, BN>;
     constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
     constexpr uint32_t STAGE = C::STAGE;
     constexpr uint32_t B_OFF = AT * A_TILE, RAW_OFF = AT * A_TILE + BT * B_TILE;
     constexpr bool F16 = (XT == DT_F16);
-    constexpr uint32_t ES = (KIND == K_NVFP4) ? 1u : 2u;  // bytes per scale
+    constexpr uint32_t ES = (KIND == K_NVFP4 || KIND == K_MXFP4) ? 1u : 2u;  // bytes per scale
     constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
     using RL = RawLayout<KIND>;
-    // up to 256 pairs: one accumulator of BN columns; more: a second one from column 256
-    constexpr uint32_t TMEM_COLS = BN <= 64 ? 64u : BN <= 128 ? 128u : BN <= 256 ? 256u : 512u;
+    // two TMEM accumulators of BN columns: the epilogue drains one while the MMAs fill
+    // the other
+    static_assert(BN == 64 || BN == 128 || BN == 256, "tile widths");
+    constexpr uint32_t NACC = 2u;
+    constexpr uint32_t TMEM_COLS = 2u * BN;
+    constexpr uint32_t ACC_STRIDE = BN;
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bars[3 * MAX_STAGES + 2];
+    __shared__ uint64_t bars[3 * MAX_STAGES + 6 + 2 * RING];
+    __shared__ uint32_t ring_s[RING];
     __shared__ uint32_t tmem_s;
     __shared__ int abort_s;
-    __shared__ uint32_t pairs_s[BN];
     __shared__ float cb_s[16];
     // codebook with f16 x: f16x2 table of code pairs (cb[c & mask], cb[c >> bits])
     constexpr bool CBF16 = (KIND == K_CB2 || KIND == K_CB3 || KIND == K_CB4) && XT == DT_F16;
     __shared__ uint32_t lut2_s[CBF16 ? (1u << (2 * kind_bits(KIND))) : 1u];
 
-    const uint32_t tile = blockIdx.y;
-    if (tile >= __ldg(P.tile_count)) return;  // uniform
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-    const uint32_t e = __ldg(P.tiles + 2 * tile), r0 = __ldg(P.tiles + 2 * tile + 1);
-    const uint32_t off = __ldg(P.offsets + e);
-    const uint32_t cnt = __ldg(P.offsets + e + 1) - off;
-    const uint32_t nt = tmin<uint32_t>(BN, cnt - r0);
-    const uint32_t nt_pad = (nt + 15u) & ~15u;
-    const uint32_t row0 = blockIdx.x * BM;
     const uint32_t S = P.stages;
-
-    // the expert's packed rows, scales and (affine) biases
-    const uint8_t *wb = P.packed + (size_t)e * P.n * P.row_bytes;
-    const uint8_t *sb = (const uint8_t *)P.scales + (size_t)e * P.n * P.groups * ES;
-    const uint8_t *bb = (const uint8_t *)P.aux + (size_t)e * P.n * P.groups * 2u;
-    bool ptr_scale_words = false, ptr_raw16 = false;
-    if constexpr (PTRS) {
-        wb = (const uint8_t *)__ldg(P.packed_ptrs + e);
-        if (!wb) return;  // expert held elsewhere: its pairs' rows are not ours to write (uniform)
-        sb = (const uint8_t *)__ldg(P.scale_ptrs + e);
-        bb = AFF ? (const uint8_t *)__ldg(P.bias_ptrs + e) : nullptr;
-        // the copies need 8-byte aligned code rows (4 for 3-bit codebook rows) and 2-byte
-        // aligned 16-bit scales / biases; other experts are skipped and flagged (uniform)
-        const uintptr_t wal = KIND == K_CB3 ? 4u : 8u;
-        const uintptr_t sal = (uintptr_t)sb | (AFF ? (uintptr_t)bb : 0u);
-        if (!sb || (AFF && !bb) || ((uintptr_t)wb % wal) != 0 || (KIND != K_NVFP4 && (sal & 1u))) {
-            if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(P.err, ERR_BAD_POINTER);
-            return;
-        }
-        ptr_raw16 = P.raw16 != 0 && (uintptr_t)wb % 16u == 0;
-        ptr_scale_words = P.scale_words != 0 && sal % 4u == 0 && (uintptr_t)sb % 4u == 0;
-    }
+    const uint32_t n_items = __ldg(P.tile_count) * P.n_mtiles;
 
     const uint32_t base = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - ptx::smem_u32(smem_raw));
     const uint32_t full0 = ptx::smem_u32(&bars[0]);
     const uint32_t loaded0 = ptx::smem_u32(&bars[MAX_STAGES]);
     const uint32_t empty0 = ptx::smem_u32(&bars[2 * MAX_STAGES]);
-    const uint32_t accb = ptx::smem_u32(&bars[3 * MAX_STAGES]);
-    const uint32_t never = ptx::smem_u32(&bars[3 * MAX_STAGES + 1]);  // completed by nothing
+    const uint32_t accfull0 = ptx::smem_u32(&bars[3 * MAX_STAGES]);       // [2]: MMAs of an item done
+    const uint32_t accempty0 = ptx::smem_u32(&bars[3 * MAX_STAGES + 2]);  // [2]: epilogue done reading
+    const uint32_t drainb = ptx::smem_u32(&bars[3 * MAX_STAGES + 4]);
+    const uint32_t never = ptx::smem_u32(&bars[3 * MAX_STAGES + 5]);  // completed by nothing
+    const uint32_t ringfull0 = ptx::smem_u32(&bars[3 * MAX_STAGES + 6]);          // [RING]
+    const uint32_t ringempty0 = ptx::smem_u32(&bars[3 * MAX_STAGES + 6 + RING]);  // [RING]
     volatile int *abort_flag = &abort_s;
+    volatile uint32_t *ring = ring_s;
+    // The i-th work item of the CTA from the scheduler's ring (n_items: none left);
+    // the slot is released by one arrival per reading warp (lane 0, after the whole
+    // warp has read it) or single reading lane. False if the wait gave up.
+    auto next_item = [&](uint32_t i, bool whole_warp, uint32_t &w) -> bool {
+        const uint32_t slot = i % RING;
+        if (!ptx::mbar_wait_bounded(ringfull0 + 8 * slot, (i / RING) & 1u, abort_flag, P.err, ERR_TIMEOUT,
+                                    P.timeout_ns))
+            return false;
+        w = ring[slot];
+        if (whole_warp) __syncwarp();
+        if (!whole_warp || lane == 0) ptx::mbar_arrive(ringempty0 + 8 * slot);
+        return true;
+    };
 
     const bool tma = !PTRS && KIND != K_CB3 && P.tma != 0;
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
             ptx::mbar_init(full0 + 8 * s, NDQ);
-            ptx::mbar_init(loaded0 + 8 * s, NLD + (tma ? 1u : 0u));  // + the TMA issuer's arrival
+            ptx::mbar_init(loaded0 + 8 * s, NLD + (tma ? 1u : 0u));  // + the tensor-copy warp's arrival
             ptx::mbar_init(empty0 + 8 * s, 1);
         }
-        ptx::mbar_init(accb, 1);
+        for (uint32_t b = 0; b < 2; b++) {
+            ptx::mbar_init(accfull0 + 8 * b, 1);
+            ptx::mbar_init(accempty0 + 8 * b, NEP / 32);  // one arrival per epilogue warp
+        }
+        ptx::mbar_init(drainb, 1);
         ptx::mbar_init(never, 1);
+        for (uint32_t b = 0; b < RING; b++) {
+            ptx::mbar_init(ringfull0 + 8 * b, 1);
+            ptx::mbar_init(ringempty0 + 8 * b, RING_READERS);
+        }
         ptx::fence_mbar_init();
         abort_s = 0;
     }
-    for (uint32_t i = tid; i < BN; i += blockDim.x)
-        pairs_s[i] = i < nt ? __ldg(P.sorted_pairs + off + r0 + i) : 0u;
     if constexpr (KIND == K_CB2 || KIND == K_CB3 || KIND == K_CB4) {
         if (tid < (1u << kind_bits(KIND)))
             cb_s[tid] = f16_bits_to_f32(__ldg((const unsigned short *)P.aux + tid));
@@ -492,137 +564,381 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_s;
     const bool gs16 = (P.lg_gs == 4);
+    const uint32_t nm = P.n_mtiles;
+    Item<KIND, PTRS> it;
 
     if (warp < LD_WARP0) {
         // -------------------------------------------------------- dequantisers
         const uint32_t r = tid & (BM - 1), h = tid >> 7;
-        const size_t row_in = glu_row(tmin<uint32_t>(row0 + r, P.n - 1), GLU ? P.glu_nh : 0u);  // row within the expert
-        const uint8_t *srow = sb + row_in * P.groups * ES;
-        const uint8_t *brow = bb + row_in * P.groups * 2u;
-        bool ok = true;
-        for (uint32_t kt = 0; kt < P.ktiles; kt++) {
-            const uint32_t s = kt % S;
-            if (!ptx::mbar_wait_bounded(loaded0 + 8 * s, (kt / S) & 1u, abort_flag, P.err, ERR_TIMEOUT,
-                                        P.timeout_ns)) {
-                ok = false;
-                break;
-            }
-            const uint32_t st = base + s * STAGE;
-            const uint8_t *stp = base_ptr + s * STAGE;
-            if constexpr (BT == 2) {
-                // f32 x: elements 0-3 of a chunk landed in the hi tile's slot, 4-7 in the
-                // lo tile's slot; rewrite both as the bf16 hi and lo halves
-                const uint32_t cc = tid & 7u;
+        uint32_t g = 0;  // k-tiles of the CTA's earlier items: stage g % S, phase (g / S) & 1
+        for (uint32_t i = 0;; i++) {
+            uint32_t w;
+            if (!next_item(i, true, w) || w >= n_items) break;
+            if (!it.load(P, w / nm, w % nm, BN)) continue;
+            const size_t row_in = glu_row(tmin<uint32_t>(it.row0 + r, P.n - 1), GLU ? P.glu_nh : 0u);
+            const uint8_t *srow = it.sb + row_in * P.groups * ES;
+            const uint8_t *brow = it.bb + row_in * P.groups * 2u;
+            const bool swords = PTRS ? it.ptr_scale_words : P.scale_words != 0;
+            bool ok = true;
+            for (uint32_t kt = 0; kt < P.ktiles; kt++, g++) {
+                const uint32_t s = g % S;
+                if (!ptx::mbar_wait_bounded(loaded0 + 8 * s, (g / S) & 1u, abort_flag, P.err, ERR_TIMEOUT,
+                                            P.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t st = base + s * STAGE;
+                const uint8_t *stp = base_ptr + s * STAGE;
+                if constexpr (BT == 2) {
+                    // f32 x: elements 0-3 of a chunk landed in the hi tile's slot, 4-7 in the
+                    // lo tile's slot; rewrite both as the bf16 hi and lo halves
+                    const uint32_t cc = tid & 7u;
 #pragma unroll
-                for (int j = 0; j < BN / 32; j++) {
-                    const uint32_t i = (tid >> 3) + 32u * j;
-                    if (i >= nt_pad) continue;
-                    const uint32_t o = swz(i, cc);
-                    const float4 v0 = *(const float4 *)(stp + B_OFF + o);
-                    const float4 v1 = *(const float4 *)(stp + B_OFF + B_TILE + o);
-                    const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                    uint32_t hi[4], lo[4];
+                    for (int j = 0; j < BN / 32; j++) {
+                        const uint32_t i = (tid >> 3) + 32u * j;
+                        if (i >= it.nt_pad) continue;
+                        const uint32_t o = swz(i, cc);
+                        const float4 v0 = *(const float4 *)(stp + B_OFF + o);
+                        const float4 v1 = *(const float4 *)(stp + B_OFF + B_TILE + o);
+                        const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        uint32_t hi[4], lo[4];
 #pragma unroll
-                    for (int t = 0; t < 4; t++) {
-                        hi[t] = pack2<false>(f[2 * t], f[2 * t + 1]);
-                        const float2 h = unpack2<false>(hi[t]);
-                        lo[t] = pack2<false>(f[2 * t] - h.x, f[2 * t + 1] - h.y);
+                        for (int t = 0; t < 4; t++) {
+                            hi[t] = pack2<false>(f[2 * t], f[2 * t + 1]);
+                            const float2 hh = unpack2<false>(hi[t]);
+                            lo[t] = pack2<false>(f[2 * t] - hh.x, f[2 * t + 1] - hh.y);
+                        }
+                        sts128(st + B_OFF + o, hi[0], hi[1], hi[2], hi[3]);
+                        sts128(st + B_OFF + B_TILE + o, lo[0], lo[1], lo[2], lo[3]);
                     }
-                    sts128(st + B_OFF + o, hi[0], hi[1], hi[2], hi[3]);
-                    sts128(st + B_OFF + B_TILE + o, lo[0], lo[1], lo[2], lo[3]);
                 }
-            }
-            // this row's codes and scale words: the strided cp.async rows, or the TMA tile
-            // (GLU: staged rows 0-63 hold the gate rows, 64-127 the up rows)
-            const uint8_t *rr = stp + RAW_OFF + r * RL::STRIDE;
-            const uint8_t *ct = stp + RAW_OFF;
-            const uint32_t sr = GLU ? ((r & 1u) ? 64u + (r >> 1) : (r >> 1)) : r;
-            const uint8_t *sw_row = tma ? ct + RL::TMA_SC + 16u * r : rr + RL::SC;
-            uint32_t w[Raw<KIND>::W];
-            uint32_t sub = 0;
-            if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4) {
-                const uint4 q = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, h) : rr + 16u * h);
-                w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
-            } else if constexpr (KIND == K_AFF8) {
-                const uint4 q0 = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, 2u * h) : rr + 32u * h);
-                const uint4 q1 = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, 2u * h + 1u) : rr + 32u * h + 16u);
-                w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
-                w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
-            } else if constexpr (KIND == K_AFF6) {
-                const uint8_t *cr = tma ? ct + sr * RL::RB : rr;
+                // this row's codes and scale words: the strided cp.async rows, or the TMA tile
+                // (GLU: staged rows 0-63 hold the gate rows, 64-127 the up rows)
+                const uint8_t *rr = stp + RAW_OFF + r * RL::STRIDE;
+                const uint8_t *ct = stp + RAW_OFF;
+                const uint32_t sr = GLU ? ((r & 1u) ? 64u + (r >> 1) : (r >> 1)) : r;
+                const uint8_t *sw_row = tma ? ct + RL::TMA_SC + 16u * r : rr + RL::SC;
+                uint32_t wv[Raw<KIND>::W];
+                uint32_t sub = 0;
+                if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4 || KIND == K_MXFP4) {
+                    const uint4 q = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, h) : rr + 16u * h);
+                    wv[0] = q.x; wv[1] = q.y; wv[2] = q.z; wv[3] = q.w;
+                } else if constexpr (KIND == K_AFF8) {
+                    const uint4 q0 = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, 2u * h) : rr + 32u * h);
+                    const uint4 q1 = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, 2u * h + 1u) : rr + 32u * h + 16u);
+                    wv[0] = q0.x; wv[1] = q0.y; wv[2] = q0.z; wv[3] = q0.w;
+                    wv[4] = q1.x; wv[5] = q1.y; wv[6] = q1.z; wv[7] = q1.w;
+                } else if constexpr (KIND == K_AFF6) {
+                    const uint8_t *cr = tma ? ct + sr * RL::RB : rr;
 #pragma unroll
-                for (int i = 0; i < 3; i++) {
-                    const uint2 q = *(const uint2 *)(cr + 24u * h + 8u * i);
-                    w[2 * i] = q.x; w[2 * i + 1] = q.y;
-                }
-            } else if constexpr (KIND == K_CB2) {
-                const uint2 q = *(const uint2 *)((tma ? ct + sr * RL::RB : rr) + 8u * h);
-                w[0] = q.x; w[1] = q.y;
-            } else {  // K_CB3: codes from (kt*KT) % 10 + 32h of the window
-                const uint32_t c0 = (kt * KT) % 10u + 32u * h, wb = c0 / 10u;
-                sub = c0 - 10u * wb;
+                    for (int i = 0; i < 3; i++) {
+                        const uint2 q = *(const uint2 *)(cr + 24u * h + 8u * i);
+                        wv[2 * i] = q.x; wv[2 * i + 1] = q.y;
+                    }
+                } else if constexpr (KIND == K_CB2) {
+                    const uint2 q = *(const uint2 *)((tma ? ct + sr * RL::RB : rr) + 8u * h);
+                    wv[0] = q.x; wv[1] = q.y;
+                } else {  // K_CB3: codes from (kt*KT) % 10 + 32h of the window
+                    const uint32_t c0 = (kt * KT) % 10u + 32u * h, wi = c0 / 10u;
+                    sub = c0 - 10u * wi;
 #pragma unroll
-                for (int i = 0; i < 4; i++) w[i] = *(const uint32_t *)(rr + 4u * (wb + i));
-            }
-            const uint32_t j0 = kt * KT, gh = (j0 + 32u * h) >> P.lg_gs;
-            if constexpr (KIND == K_NVFP4) {
-                // groups of 16: this half's two E4M3 scales, converted together (exact in f16)
-                __half2 s01;
-                if (PTRS ? ptr_scale_words : P.scale_words != 0) {
-                    // the staged word holds groups 4kt .. 4kt+3; this half's are bytes 2h, 2h+1
-                    s01 = e4m3x2_to_half2((*(const uint32_t *)sw_row >> (16u * h)) & 0xFFFFu);
-                } else {
-                    float s0, s1, unused;
-                    global_scale<KIND>(srow, brow, gh, P.groups, s0, unused);
-                    global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, unused);
-                    s01 = __floats2half2_rn(s0, s1);
+                    for (int i = 0; i < 4; i++) wv[i] = *(const uint32_t *)(rr + 4u * (wi + i));
                 }
-                nvfp4_store<F16>(w, s01, st, r, h * 4u);
-            } else {
-                float s0, b0, s1 = 0.f, b1 = 0.f;
-                if (PTRS ? ptr_scale_words : P.scale_words != 0) {
-                    const uint4 q = *(const uint4 *)sw_row;
-                    const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
-                    const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
-                    staged_scale<KIND>(sw, bw, gh * ES - base_b, s0, b0);
-                    if (gs16) staged_scale<KIND>(sw, bw, (gh + 1u) * ES - base_b, s1, b1);
+                const uint32_t j0 = kt * KT, gh = (j0 + 32u * h) >> P.lg_gs;
+                if constexpr (KIND == K_NVFP4) {
+                    // groups of 16: this half's two E4M3 scales, converted together (exact in f16)
+                    __half2 s01;
+                    if (swords) {
+                        // the staged word holds groups 4kt .. 4kt+3; this half's are bytes 2h, 2h+1
+                        s01 = e4m3x2_to_half2((*(const uint32_t *)sw_row >> (16u * h)) & 0xFFFFu);
+                    } else {
+                        float s0, s1, unused;
+                        global_scale<KIND>(srow, brow, gh, P.groups, s0, unused);
+                        global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, unused);
+                        s01 = __floats2half2_rn(s0, s1);
+                    }
+                    nvfp4_store<F16>(wv, s01, st, r, h * 4u);
                 } else {
-                    global_scale<KIND>(srow, brow, gh, P.groups, s0, b0);
-                    if (gs16) global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, b1);
-                }
-                if constexpr (CBF16) {
-                    const __half2 h0 = __float2half2_rn(s0), h1 = __float2half2_rn(s1);  // exact: f16 scales
-                    if constexpr (KIND == K_CB3) {
-                        switch (sub) {  // first code's position in word 0: 0, 2, 4, 6 or 8
-                            case 0: cb_pairs_f16<KIND, 0>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                            case 2: cb_pairs_f16<KIND, 2>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                            case 4: cb_pairs_f16<KIND, 4>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                            case 6: cb_pairs_f16<KIND, 6>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                            default: cb_pairs_f16<KIND, 8>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                    float s0, b0, s1 = 0.f, b1 = 0.f;
+                    if (swords) {
+                        const uint4 q = *(const uint4 *)sw_row;
+                        const uint32_t sw[2] = {q.x, q.y}, bw[2] = {q.z, q.w};
+                        const uint32_t base_b = ((j0 >> P.lg_gs) * ES) & ~3u;
+                        staged_scale<KIND>(sw, bw, gh * ES - base_b, s0, b0);
+                        if (gs16) staged_scale<KIND>(sw, bw, (gh + 1u) * ES - base_b, s1, b1);
+                    } else {
+                        global_scale<KIND>(srow, brow, gh, P.groups, s0, b0);
+                        if (gs16) global_scale<KIND>(srow, brow, gh + 1u, P.groups, s1, b1);
+                    }
+                    if constexpr (CBF16) {
+                        const __half2 h0 = __float2half2_rn(s0), h1 = __float2half2_rn(s1);  // exact: f16 scales
+                        if constexpr (KIND == K_CB3) {
+                            switch (sub) {  // first code's position in word 0: 0, 2, 4, 6 or 8
+                                case 0: cb_pairs_f16<KIND, 0>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                                case 2: cb_pairs_f16<KIND, 2>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                                case 4: cb_pairs_f16<KIND, 4>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                                case 6: cb_pairs_f16<KIND, 6>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                                default: cb_pairs_f16<KIND, 8>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                            }
+                        } else {
+                            cb_pairs_f16<KIND, 0>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u);
                         }
                     } else {
-                        cb_pairs_f16<KIND, 0>(w, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u);
+                        dequant_tile<KIND, F16>(wv, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(full0 + 8 * s);
+            }
+            if (!ok) break;
+        }
+    } else if (warp < MMA_WARP) {
+        // ------------------------------------------------------------- loaders
+        const uint32_t lt = tid - NDQ;
+        // x: thread lt copies 16-byte chunk lt % 8 of pair rows lt / 8 + XR j
+        constexpr int NXL = BN * 8 / NLD;
+        constexpr uint32_t XR = NLD / 8;  // pair rows per pass of the loaders
+        constexpr uint32_t XS = (BT == 2) ? 4u : 2u;  // bytes per x element
+        const uint32_t xc = lt & 7u, xi0 = lt >> 3;
+        const uint32_t xdst0 = B_OFF + swz(xi0, xc);  // + XR * 128 j: XR rows further down
+        const uint32_t nlast = P.n - 1;
+        const uint32_t srow_bytes = P.groups * ES;
+        const uint32_t nsw = (gs16 && ES == 2u) ? 2u : 1u;
+        uint32_t g = 0;
+        bool ok = true;
+        for (uint32_t i = 0; ok; i++) {
+            uint32_t w;
+            if (!next_item(i, true, w) || w >= n_items) break;
+            if (!it.load(P, w / nm, w % nm, BN)) continue;
+            const uint8_t *xrow[NXL];
+#pragma unroll
+            for (int j = 0; j < NXL; j++) {
+                const uint32_t i = xi0 + XR * j;
+                xrow[j] = i < it.nt ? (const uint8_t *)P.x +
+                                          (size_t)(__ldg(P.sorted_pairs + it.off + it.r0 + i) / P.n_expert_used) *
+                                              P.k * XS
+                                    : nullptr;
+            }
+            const uint8_t *ebase = it.wb;
+            const uint32_t row0 = it.row0;
+            // scale words: thread lt < BM stages those of weight row lt
+            const size_t srow_in = glu_row(tmin<uint32_t>(row0 + (lt & (BM - 1)), nlast), GLU ? P.glu_nh : 0u);
+            const uint8_t *srow = it.sb + srow_in * P.groups * ES;
+            const uint8_t *brow = it.bb + srow_in * P.groups * 2u;
+            const bool swords = PTRS ? it.ptr_scale_words : P.scale_words != 0;
+            const bool raw16 = PTRS ? it.ptr_raw16 : P.raw16 != 0;
+            for (uint32_t kt = 0; kt < P.ktiles; kt++, g++) {
+                const uint32_t s = g % S;
+                if (g >= S && !ptx::mbar_wait_bounded(empty0 + 8 * s, ((g / S) - 1u) & 1u, abort_flag, P.err,
+                                                      ERR_TIMEOUT, P.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t st = base + s * STAGE;
+                // x rows of the pairs, straight into the B operand tile (zero past k and nt)
+                const uint32_t kk = kt * KT + xc * 8u;
+#pragma unroll
+                for (int j = 0; j < NXL; j++) {
+                    if (xi0 + XR * j < it.nt_pad) {
+                        const bool in = xrow[j] != nullptr && kk < P.k;
+                        const uint8_t *src = in ? xrow[j] + (size_t)kk * XS : (const uint8_t *)P.x;
+                        const uint32_t dst = st + xdst0 + XR * 128u * j;
+                        ptx::cp_async_16(dst, src, in ? 16u : 0u);
+                        if constexpr (BT == 2) ptx::cp_async_16(dst + B_TILE, in ? src + 16 : src, in ? 16u : 0u);
+                    }
+                }
+                // packed codes of the 128 rows (rows past n repeat row n-1; bytes past a row read as 0)
+                const uint32_t raw = st + RAW_OFF;
+                if (tma) {
+                    // the codes come by tensor copy from the tensor-copy warp
+                } else if constexpr (KIND == K_CB3) {
+                    const uint32_t w0 = (kt * KT) / 10u;
+#pragma unroll
+                    for (int i = 0; i < BM * 8 / NLD; i++) {
+                        const uint32_t q = lt + NLD * i, row = q >> 3, c = q & 7u;
+                        const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
+                        const uint32_t o = (w0 + c) * 4u;
+                        const bool in = o + 4u <= P.row_bytes;
+                        ptx::cp_async_4(raw + row * RL::STRIDE + 4u * c, rp + (in ? o : 0u), in ? 4u : 0u);
                     }
                 } else {
-                    dequant_tile<KIND, F16>(w, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
+                    constexpr uint32_t RB = RL::RB;
+                    if (raw16) {
+                        constexpr uint32_t NC = RB / 16u;
+#pragma unroll
+                        for (uint32_t i = 0; i < (BM * NC + NLD - 1) / NLD; i++) {
+                            const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
+                            if (row >= BM) break;
+                            const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
+                            const uint32_t o = kt * RB + 16u * c;
+                            const bool in = o < P.row_bytes;
+                            ptx::cp_async_16(raw + row * RL::STRIDE + 16u * c, rp + (in ? o : 0u), in ? 16u : 0u);
+                        }
+                    } else {
+                        constexpr uint32_t NC = RB / 8u;
+#pragma unroll
+                        for (uint32_t i = 0; i < (BM * NC + NLD - 1) / NLD; i++) {
+                            const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
+                            if (row >= BM) break;
+                            const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
+                            const uint32_t o = kt * RB + 8u * c;
+                            const bool in = o < P.row_bytes;
+                            ptx::cp_async_8(raw + row * RL::STRIDE + 8u * c, rp + (in ? o : 0u), in ? 8u : 0u);
+                        }
+                    }
+                }
+                if (swords && lt < BM) {
+                    const uint32_t base_b = ((kt * KT >> P.lg_gs) * ES) & ~3u;
+                    const uint32_t sdst = tma ? raw + RL::TMA_SC + 16u * lt : raw + lt * RL::STRIDE + RL::SC;
+                    for (uint32_t i = 0; i < nsw; i++) {
+                        const uint32_t o = base_b + 4u * i;
+                        const bool in = o + 4u <= srow_bytes;
+                        ptx::cp_async_4(sdst + 4u * i, srow + (in ? o : 0u), in ? 4u : 0u);
+                        if constexpr (AFF) ptx::cp_async_4(sdst + 8u + 4u * i, brow + (in ? o : 0u), in ? 4u : 0u);
+                    }
+                }
+                ptx::cp_async_mbar_arrive(loaded0 + 8 * s);
+            }
+        }
+        ptx::cp_async_wait_all();
+    } else if (warp == TMA_WARP) {
+        // ------------------------------------------------------ code tensor copies
+        if (lane == 0) {
+            // per k-tile two 64-row copies of RB bytes per row (GLU: the 64 gate rows,
+            // then the 64 up rows); rows past the expert's last read a neighbour's rows or
+            // zeros and are never stored. The arrival (with the byte count) is one of the
+            // stage's loaded arrivals. Without TMA staging the lane only reads the ring.
+            constexpr uint32_t RB = RL::RB;
+            if (tma) ptx::prefetch_tensormap(&tmap);
+            uint32_t g = 0, last_s = 0, last_par = 0;
+            bool any = false, ok = true;
+            for (uint32_t i = 0; ok; i++) {
+                uint32_t w;
+                if (!next_item(i, false, w) || w >= n_items) break;
+                if (!tma || !it.load(P, w / nm, w % nm, BN)) continue;
+                const int32_t y0 = (int32_t)(it.e * P.n + (GLU ? it.row0 / 2u : it.row0));
+                const int32_t y1 = GLU ? (int32_t)(it.e * P.n + P.glu_nh + it.row0 / 2u) : y0 + 64;
+                for (uint32_t kt = 0; kt < P.ktiles; kt++, g++) {
+                    const uint32_t s = g % S;
+                    if (g >= S && !ptx::mbar_wait_bounded(empty0 + 8 * s, ((g / S) - 1u) & 1u, abort_flag, P.err,
+                                                          ERR_TIMEOUT, P.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = loaded0 + 8 * s, raw = base + s * STAGE + RAW_OFF;
+                    ptx::mbar_arrive_expect_tx(bar, 2u * 64u * RB);
+                    ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
+                    ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
+                    last_s = s;
+                    last_par = (g / S) & 1u;
+                    any = true;
                 }
             }
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(full0 + 8 * s);
+            // copies still in flight after a wait gave up land before the CTA exits
+            if (any) ptx::mbar_wait_bounded(loaded0 + 8 * last_s, last_par, nullptr, P.err, ERR_TIMEOUT, DRAIN_NS);
         }
+    } else if (warp == MMA_WARP) {
+        // --------------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            bool ok = true;
+            if (P.fault_ns) ok = ptx::mbar_wait_bounded(never, 0, abort_flag, P.err, ERR_TIMEOUT, P.fault_ns);
+            uint32_t g = 0, done = 0;  // k-tiles consumed; items computed
+            for (uint32_t i = 0; ok; i++) {
+                uint32_t w;
+                if (!next_item(i, false, w)) {
+                    ok = false;
+                    break;
+                }
+                if (w >= n_items) break;
+                if (!it.load(P, w / nm, w % nm, BN)) continue;
+                const uint32_t buf = done % NACC, use = done / NACC;
+                // the epilogue has read this accumulator's previous item (a fresh barrier's
+                // preceding phase counts as complete, so the first two items do not wait)
+                if (!ptx::mbar_wait_bounded(accempty0 + 8 * buf, (use & 1u) ^ 1u, abort_flag, P.err, ERR_TIMEOUT,
+                                            P.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d = tmem + buf * ACC_STRIDE;
+                const uint32_t idesc = ptx::idesc_f16(F16 ? 0u : 1u, it.nt_pad);
+                uint32_t accum = 0;
+                for (uint32_t kt = 0; kt < P.ktiles; kt++, g++) {
+                    const uint32_t s = g % S;
+                    if (!ptx::mbar_wait_bounded(full0 + 8 * s, (g / S) & 1u, abort_flag, P.err, ERR_TIMEOUT,
+                                                P.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t st = base + s * STAGE;
+                    const uint32_t a_hi = st, a_lo = st + A_TILE;
+                    const uint32_t b_hi = st + B_OFF, b_lo = b_hi + B_TILE;
+#pragma unroll
+                    for (int ks = 0; ks < KT / 16; ks++) {
+                        const uint32_t ko = ks * 32u;
+                        ptx::mma_f16_ss(d, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_hi + ko), idesc, accum);
+                        if constexpr (BT == 2)
+                            ptx::mma_f16_ss(d, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_lo + ko), idesc, 1);
+                        if constexpr (AT == 2)
+                            ptx::mma_f16_ss(d, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b_hi + ko), idesc, 1);
+                        accum = 1;
+                    }
+                    ptx::mma_commit(empty0 + 8 * s);
+                }
+                if (!ok) break;
+                ptx::mma_commit(accfull0 + 8 * buf);
+                done++;
+            }
+            // every MMA issued has completed before TMEM is freed (its own limit, not the
+            // pipeline waits' one)
+            ptx::mma_commit(drainb);
+            ptx::mbar_wait_bounded(drainb, 0, nullptr, P.err, ERR_TIMEOUT, DRAIN_NS);
+        }
+        __syncwarp();
+    } else if (warp == SCHED_WARP) {
+        // ------------------------------------------------------------- scheduler
+        if (lane == 0) {
+            for (uint32_t i = 0;; i++) {
+                const uint32_t slot = i % RING;
+                // every reader has taken the item published in this slot RING items ago
+                if (i >= RING && !ptx::mbar_wait_bounded(ringempty0 + 8 * slot, ((i / RING) - 1u) & 1u, abort_flag,
+                                                         P.err, ERR_TIMEOUT, P.timeout_ns))
+                    break;
+                uint32_t w = i == 0 ? blockIdx.x : gridDim.x + atomicAdd(P.work_counter, 1u);
+                if (w > n_items) w = n_items;  // n_items: no more work
+                ring[slot] = w;
+                ptx::mbar_arrive(ringfull0 + 8 * slot);  // release: the item is visible to the readers
+                if (w >= n_items) break;
+            }
+        }
+    } else {
         // ------------------------------------------------------------- epilogue
-        if (ok && ptx::mbar_wait_bounded(accb, 0, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns) &&
-            !*abort_flag) {
+        // TMEM -> registers (tcgen05.ld), times scale2 for NVFP4, plus the expert bias,
+        // rounded once to the output type, stored to row p of out (the scatter back to
+        // [token][slot] order). Warp w reads TMEM lanes 32 (w % 4) .. + 31.
+        const uint32_t q = warp & 3u;
+        uint32_t done = 0;
+        for (uint32_t i = 0;; i++) {
+            uint32_t w;
+            if (!next_item(i, true, w) || w >= n_items) break;
+            if (!it.load(P, w / nm, w % nm, BN)) continue;
+            const uint32_t buf = done % NACC, use = done / NACC;
+            if (!ptx::mbar_wait_bounded(accfull0 + 8 * buf, use & 1u, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns))
+                break;
             ptx::tc_fence_after();
-            const uint32_t q = warp & 3u, ch = warp >> 2;
-            const uint32_t grow_e = row0 + q * 32u + lane;  // logical row
+            const uint32_t d = tmem + buf * ACC_STRIDE;
+            const uint32_t grow_e = it.row0 + q * 32u + lane;  // logical row
             const uint32_t nh = GLU ? P.glu_nh : 0u;
-            const float s2 = (KIND == K_NVFP4) ? __ldg((const float *)P.aux + e) : 1.f;
-            const float bv = grow_e < P.n ? load_bias(P.bias, P.bias_dtype, (size_t)e * P.n + glu_row(grow_e, nh)) : 0.f;
-            const uint32_t c_begin = ch * (BN / 2), c_end = tmin<uint32_t>(c_begin + BN / 2, nt);
-            for (uint32_t c0 = c_begin; c0 < c_end; c0 += 16) {
-                uint32_t v[16];
-                ptx::tmem_ld16(tmem + ((q * 32u) << 16) + c0, v);
+            const float s2 = (KIND == K_NVFP4) ? __ldg((const float *)P.aux + it.e) : 1.f;
+            const float bv =
+                grow_e < P.n ? load_bias(P.bias, P.bias_dtype, (size_t)it.e * P.n + glu_row(grow_e, nh)) : 0.f;
+            const uint32_t *pairs = P.sorted_pairs + it.off + it.r0;
+            for (uint32_t c0 = 0; c0 < it.nt; c0 += 16) {
+                uint32_t v[16], pr[16];
+                ptx::tmem_ld16(d + ((q * 32u) << 16) + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; i++) pr[i] = c0 + i < it.nt ? __ldg(pairs + c0 + i) : 0u;
                 ptx::tmem_wait_ld();
                 if constexpr (GLU) {
                     // even lanes hold gate rows, the next lane the matching up row
@@ -631,194 +947,25 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                         const float y = __uint_as_float(v[i]) * s2 + bv;
                         const float up = __shfl_xor_sync(0xFFFFFFFFu, y, 1);
                         const uint32_t col = c0 + i;
-                        if (col < c_end && grow_e < P.n && !(lane & 1u))
-                            store_out(P.out, P.out_dtype, (size_t)pairs_s[col] * nh + (grow_e >> 1),
-                                      glu_act(P.act, y) * up);
+                        if (col < it.nt && grow_e < P.n && !(lane & 1u))
+                            store_out(P.out, P.out_dtype, (size_t)pr[i] * nh + (grow_e >> 1), glu_act(P.act, y) * up);
                     }
                 } else if (grow_e < P.n) {
 #pragma unroll
                     for (int i = 0; i < 16; i++) {
                         const uint32_t col = c0 + i;
-                        if (col < c_end)
-                            store_out(P.out, P.out_dtype, (size_t)pairs_s[col] * P.n + grow_e,
-                                      __uint_as_float(v[i]) * s2 + bv);
+                        if (col < it.nt)
+                            store_out(P.out, P.out_dtype, (size_t)pr[i] * P.n + grow_e, __uint_as_float(v[i]) * s2 + bv);
                     }
                 }
             }
-        }
-        ptx::tc_fence_before();
-    } else if (warp < MMA_WARP) {
-        // ------------------------------------------------------------- loaders
-        const uint32_t lt = tid - NDQ;
-        // x: thread lt copies 16-byte chunk lt % 8 of pair rows lt / 8 + 16 j
-        constexpr int NXL = BN * 8 / NLD;
-        constexpr uint32_t XS = (BT == 2) ? 4u : 2u;  // bytes per x element
-        const uint32_t xc = lt & 7u, xi0 = lt >> 3;
-        const uint8_t *xrow[NXL];
-#pragma unroll
-        for (int j = 0; j < NXL; j++) {
-            const uint32_t i = xi0 + 16u * j;
-            xrow[j] = i < nt ? (const uint8_t *)P.x + (size_t)(pairs_s[i] / P.n_expert_used) * P.k * XS
-                             : nullptr;
-        }
-        const uint32_t xdst0 = B_OFF + swz(xi0, xc);  // + 2048 j: 16 rows further down
-        const uint8_t *ebase = wb;
-        const uint32_t nlast = P.n - 1;
-        // scale words: thread lt stages those of weight row lt
-        const size_t srow_in = glu_row(tmin<uint32_t>(row0 + lt, nlast), GLU ? P.glu_nh : 0u);
-        const uint8_t *srow = sb + srow_in * P.groups * ES;
-        const uint8_t *brow = bb + srow_in * P.groups * 2u;
-        const uint32_t srow_bytes = P.groups * ES;
-        const uint32_t nsw = (gs16 && ES == 2u) ? 2u : 1u;
-
-        for (uint32_t kt = 0; kt < P.ktiles; kt++) {
-            const uint32_t s = kt % S;
-            if (kt >= S && !ptx::mbar_wait_bounded(empty0 + 8 * s, ((kt / S) - 1u) & 1u, abort_flag, P.err,
-                                                   ERR_TIMEOUT, P.timeout_ns))
-                break;
-            const uint32_t st = base + s * STAGE;
-            // x rows of the pairs, straight into the B operand tile (zero past k and nt)
-            const uint32_t kk = kt * KT + xc * 8u;
-#pragma unroll
-            for (int j = 0; j < NXL; j++) {
-                if (xi0 + 16u * j < nt_pad) {
-                    const bool in = xrow[j] != nullptr && kk < P.k;
-                    const uint8_t *src = in ? xrow[j] + (size_t)kk * XS : (const uint8_t *)P.x;
-                    const uint32_t dst = st + xdst0 + 2048u * j;
-                    ptx::cp_async_16(dst, src, in ? 16u : 0u);
-                    if constexpr (BT == 2) ptx::cp_async_16(dst + B_TILE, in ? src + 16 : src, in ? 16u : 0u);
-                }
-            }
-            // packed codes of the 128 rows (rows past n repeat row n-1; bytes past a row read as 0)
-            const uint32_t raw = st + RAW_OFF;
-            if (tma) {
-                // the codes come by tensor copy from the tensor-copy warp
-            } else if constexpr (KIND == K_CB3) {
-                const uint32_t w0 = (kt * KT) / 10u;
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const uint32_t q = lt + NLD * i, row = q >> 3, c = q & 7u;
-                    const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
-                    const uint32_t o = (w0 + c) * 4u;
-                    const bool in = o + 4u <= P.row_bytes;
-                    ptx::cp_async_4(raw + row * RL::STRIDE + 4u * c, rp + (in ? o : 0u), in ? 4u : 0u);
-                }
-            } else {
-                constexpr uint32_t RB = RL::RB;
-                if (PTRS ? ptr_raw16 : P.raw16 != 0) {
-                    constexpr uint32_t NC = RB / 16u;
-#pragma unroll
-                    for (uint32_t i = 0; i < NC; i++) {
-                        const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
-                        const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
-                        const uint32_t o = kt * RB + 16u * c;
-                        const bool in = o < P.row_bytes;
-                        ptx::cp_async_16(raw + row * RL::STRIDE + 16u * c, rp + (in ? o : 0u), in ? 16u : 0u);
-                    }
-                } else {
-                    constexpr uint32_t NC = RB / 8u;
-#pragma unroll
-                    for (uint32_t i = 0; i < NC; i++) {
-                        const uint32_t q = lt + NLD * i, row = q / NC, c = q % NC;
-                        const uint8_t *rp = ebase + (size_t)glu_row(tmin<uint32_t>(row0 + row, nlast), GLU ? P.glu_nh : 0u) * P.row_bytes;
-                        const uint32_t o = kt * RB + 8u * c;
-                        const bool in = o < P.row_bytes;
-                        ptx::cp_async_8(raw + row * RL::STRIDE + 8u * c, rp + (in ? o : 0u), in ? 8u : 0u);
-                    }
-                }
-            }
-            if (PTRS ? ptr_scale_words : P.scale_words != 0) {
-                const uint32_t base_b = ((kt * KT >> P.lg_gs) * ES) & ~3u;
-                const uint32_t sdst = tma ? raw + RL::TMA_SC + 16u * lt : raw + lt * RL::STRIDE + RL::SC;
-                for (uint32_t i = 0; i < nsw; i++) {
-                    const uint32_t o = base_b + 4u * i;
-                    const bool in = o + 4u <= srow_bytes;
-                    ptx::cp_async_4(sdst + 4u * i, srow + (in ? o : 0u), in ? 4u : 0u);
-                    if constexpr (AFF) ptx::cp_async_4(sdst + 8u + 4u * i, brow + (in ? o : 0u), in ? 4u : 0u);
-                }
-            }
-            ptx::cp_async_mbar_arrive(loaded0 + 8 * s);
-        }
-        ptx::cp_async_wait_all();
-    } else if (warp == TMA_WARP) {
-        // ------------------------------------------------------ code tensor copies
-        if (tma && lane == 0) {
-            // per k-tile two 64-row copies of RB bytes per row (GLU: the 64 gate rows,
-            // then the 64 up rows); rows past the expert's last read a neighbour's rows or
-            // zeros and are never stored. The arrival (with the byte count) is one of the
-            // stage's loaded arrivals.
-            constexpr uint32_t RB = RL::RB;
-            ptx::prefetch_tensormap(&tmap);
-            const int32_t y0 = (int32_t)(e * P.n + (GLU ? row0 / 2u : row0));
-            const int32_t y1 = GLU ? (int32_t)(e * P.n + P.glu_nh + row0 / 2u) : y0 + 64;
-            uint32_t last_s = 0, last_par = 0;
-            bool any = false;
-            for (uint32_t kt = 0; kt < P.ktiles; kt++) {
-                const uint32_t s = kt % S;
-                if (kt >= S && !ptx::mbar_wait_bounded(empty0 + 8 * s, ((kt / S) - 1u) & 1u, abort_flag, P.err,
-                                                       ERR_TIMEOUT, P.timeout_ns))
-                    break;
-                const uint32_t bar = loaded0 + 8 * s, raw = base + s * STAGE + RAW_OFF;
-                ptx::mbar_arrive_expect_tx(bar, 2u * 64u * RB);
-                ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
-                ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
-                last_s = s;
-                last_par = (kt / S) & 1u;
-                any = true;
-            }
-            // copies still in flight after a wait gave up land before the CTA exits
-            if (any) ptx::mbar_wait_bounded(loaded0 + 8 * last_s, last_par, nullptr, P.err, ERR_TIMEOUT, DRAIN_NS);
-        }
-    } else if (lane == 0) {
-        // --------------------------------------------------------------- MMA issue
-        const uint32_t n1 = tmin<uint32_t>(nt_pad, 256u), n2 = nt_pad - n1;
-        const uint32_t idesc = ptx::idesc_f16(F16 ? 0u : 1u, n1);
-        const uint32_t idesc2 = ptx::idesc_f16(F16 ? 0u : 1u, n2 > 0 ? n2 : 16u);
-        uint32_t accum = 0;
-        bool ok = true;
-        if (P.fault_ns) ok = ptx::mbar_wait_bounded(never, 0, abort_flag, P.err, ERR_TIMEOUT, P.fault_ns);
-        for (uint32_t kt = 0; ok && kt < P.ktiles; kt++) {
-            const uint32_t s = kt % S, use = kt / S;
-            if (!ptx::mbar_wait_bounded(full0 + 8 * s, use & 1u, abort_flag, P.err, ERR_TIMEOUT,
-                                        P.timeout_ns)) {
-                ok = false;
-                break;
-            }
-            ptx::tc_fence_after();
-            const uint32_t st = base + s * STAGE;
-            const uint32_t a_hi = st, a_lo = st + A_TILE;
-            const uint32_t b_hi = st + B_OFF, b_lo = b_hi + B_TILE;
-#pragma unroll
-            for (int ks = 0; ks < KT / 16; ks++) {
-                const uint32_t ko = ks * 32u;
-                ptx::mma_f16_ss(tmem, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_hi + ko), idesc, accum);
-                if constexpr (BT == 2)
-                    ptx::mma_f16_ss(tmem, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_lo + ko), idesc, 1);
-                if constexpr (AT == 2)
-                    ptx::mma_f16_ss(tmem, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b_hi + ko), idesc, 1);
-                if constexpr (BN > 256) {
-                    // pairs 256 .. nt_pad - 1: B rows from 256 (32 KB into the tile), TMEM columns from 256
-                    if (n2 > 0) {
-                        const uint32_t b2 = b_hi + 256u * 128u;
-                        ptx::mma_f16_ss(tmem + 256u, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b2 + ko), idesc2, accum);
-                        if constexpr (BT == 2)
-                            ptx::mma_f16_ss(tmem + 256u, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b2 + B_TILE + ko),
-                                            idesc2, 1);
-                        if constexpr (AT == 2)
-                            ptx::mma_f16_ss(tmem + 256u, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b2 + ko), idesc2, 1);
-                    }
-                }
-                accum = 1;
-            }
-            ptx::mma_commit(empty0 + 8 * s);
-        }
-        ptx::mma_commit(accb);
-        if (!ok) {
-            // drain: the commit above tracks every MMA issued so far; TMEM is freed only
-            // after it (its own limit, not the pipeline waits' one)
-            ptx::mbar_wait_bounded(accb, 0, nullptr, P.err, ERR_TIMEOUT, DRAIN_NS);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(accempty0 + 8 * buf);
+            done++;
         }
     }
+    ptx::tc_fence_before();
     __syncthreads();
     if (warp == MMA_WARP) {
         __syncwarp();
@@ -845,31 +992,44 @@ uint32_t raw_tile(int kind) {
         case K_CB2: return RawLayout<K_CB2>::TILE;
         case K_CB3: return RawLayout<K_CB3>::TILE;
         case K_CB4: return RawLayout<K_CB4>::TILE;
+        case K_MXFP4: return RawLayout<K_MXFP4>::TILE;
         default: return RawLayout<K_NVFP4>::TILE;
     }
 }
 
 // Tile width and pipeline depth: when experts hold ~100 or more pairs on
 // average, 256 pairs per tile (128 with f32 x, whose operand tiles are twice
-// as large), and 320 for NVFP4 with 16-bit x, whose single-term weight tile
-// leaves room for it: experts of up to 320 pairs then take one tile, so their
-// weights are dequantised once instead of once for 256 pairs and again for a
-// small remainder. 64 otherwise; as many stages (2..6) as fit.
+// as large), so that two TMEM accumulators of the tile width fit the 512 columns
+// and an item's epilogue overlaps the next item's MMAs; 64 otherwise. As many
+// stages (2..6) as fit in one CTA per SM.
 bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
     const uint64_t R = (uint64_t)a.m * a.n_expert_used;
     const bool big = R >= 96ull * a.num_experts;
     const bool f32x = a.x_dtype == DT_F32;
-    const uint32_t bn = big ? (f32x ? 128u : a.kind == K_NVFP4 ? 320u : 256u) : 64u;
-    const uint32_t at = a.kind == K_NVFP4 ? 1u : 2u, bt = f32x ? 2u : 1u;
+    const bool fp4 = a.kind == K_NVFP4 || a.kind == K_MXFP4;  // single-term A
+    const uint32_t bn = big ? (f32x ? 128u : 256u) : 64u;
+    const uint32_t at = fp4 ? 1u : 2u, bt = f32x ? 2u : 1u;
     const size_t stage = (size_t)at * A_TILE + (size_t)bt * bn * KT * 2 + raw_tile(a.kind);
     if (2 * stage + 1024 > GEMM_SMEM_BUDGET) return false;
     int S = (int)((GEMM_SMEM_BUDGET - 1024) / stage);
     S = S > MAX_STAGES ? MAX_STAGES : S;
-    if (bn == 64) S = 2;  // two CTAs per SM
     pl->bn = bn;
     pl->stages = S;
     pl->smem = (size_t)S * stage + 1024;
     return true;
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+uint32_t sm_count_gemm() {
+    static int count[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148u;
+    if (count[dev] == 0) {
+        int c = 0;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+        count[dev] = c;
+    }
+    return (uint32_t)count[dev];
 }
 
 template <int KIND, int XT, int BN, bool PTRS, bool GLU>
@@ -881,8 +1041,10 @@ cudaError_t launch_tp(const GemmParams &P0, const CUtensorMap &tmap, const GemmP
     static int smem_set[64];
     cudaError_t e = ensure_dyn_smem(kern, pl.smem, smem_set);
     if (e != cudaSuccess) return e;
-    dim3 grid(n_mtiles, max_tiles);
-    kern<<<grid, GEMM_THREADS, pl.smem, st>>>(P, tmap);
+    // persistent: one CTA per SM, or fewer when there are fewer work items
+    const uint64_t items = (uint64_t)n_mtiles * max_tiles;
+    const uint32_t ctas = (uint32_t)(items < (uint64_t)sm_count_gemm() ? items : (uint64_t)sm_count_gemm());
+    kern<<<ctas, GEMM_THREADS, pl.smem, st>>>(P, tmap);
     return cudaGetLastError();
 }
 
@@ -901,18 +1063,19 @@ cudaError_t launch_k(const GemmParams &P, const CUtensorMap &tm, const GemmPlan 
         if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, tm, pl, nm, mt, st);
         return launch_t<KIND, DT_F32, 64>(P, tm, pl, nm, mt, st);
     }
-    if constexpr (KIND == K_NVFP4) {
-        if (pl.bn == 320) {
-            if (x_dtype == DT_BF16) return launch_t<KIND, DT_BF16, 320>(P, tm, pl, nm, mt, st);
-            return launch_t<KIND, DT_F16, 320>(P, tm, pl, nm, mt, st);
-        }
-    }
+    if constexpr (KIND == K_MXFP4) {
+        // e2m1 * 2^e can leave the f16 range: only bf16 (and f32, as bf16 halves) x here
+        if (x_dtype != DT_BF16) return cudaErrorNotSupported;
+        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, pl, nm, mt, st);
+        return launch_t<KIND, DT_BF16, 64>(P, tm, pl, nm, mt, st);
+    } else {
     if (x_dtype == DT_BF16) {
         if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, pl, nm, mt, st);
         return launch_t<KIND, DT_BF16, 64>(P, tm, pl, nm, mt, st);
     }
     if (pl.bn == 256) return launch_t<KIND, DT_F16, 256>(P, tm, pl, nm, mt, st);
     return launch_t<KIND, DT_F16, 64>(P, tm, pl, nm, mt, st);
+    }
 }
 
 cudaError_t launch_kind(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, int kind, int x_dtype,
@@ -925,6 +1088,7 @@ cudaError_t launch_kind(const GemmParams &P, const CUtensorMap &tm, const GemmPl
         case K_CB3: return launch_k<K_CB3>(P, tm, pl, x_dtype, nm, mt, st);
         case K_CB4: return launch_k<K_CB4>(P, tm, pl, x_dtype, nm, mt, st);
         case K_NVFP4: return launch_k<K_NVFP4>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_MXFP4: return launch_k<K_MXFP4>(P, tm, pl, x_dtype, nm, mt, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -951,6 +1115,7 @@ uint32_t ktile_row_bytes(int kind) {
         case K_CB2: return RawLayout<K_CB2>::RB;
         case K_CB4: return RawLayout<K_CB4>::RB;
         case K_NVFP4: return RawLayout<K_NVFP4>::RB;
+        case K_MXFP4: return RawLayout<K_MXFP4>::RB;
         default: return 0;
     }
 }
@@ -980,7 +1145,9 @@ bool code_tensor_map(const QmmArgs &a, CUtensorMap *m) {
 }  // namespace
 
 bool gemm_supported(const QmmArgs &a) {
-    if (a.kind == K_MXFP4) return false;  // MXFP4 runs on the CUDA-core paths
+    // MXFP4 weights e2m1 * 2^e are exact in bf16 but can leave the f16 range: f16 x
+    // stays on the CUDA-core paths
+    if (a.kind == K_MXFP4 && a.x_dtype == DT_F16) return false;
     const uint32_t gs = a.group_size;
     if (gs < 16 || (gs & (gs - 1)) != 0) return false;
     if (a.k % 8 != 0 || a.k % gs != 0) return false;
@@ -999,7 +1166,7 @@ uint32_t gemm_tile_rows(const QmmArgs &a) {
 
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
-                        uint32_t *err, cudaStream_t st) {
+                        uint32_t *err, uint32_t *work_counter, cudaStream_t st) {
     GemmPlan pl;
     if (!gemm_plan(a, &pl)) return cudaErrorNotSupported;
     GemmParams P{};
@@ -1012,7 +1179,7 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.lg_gs = lg;
     P.groups = a.groups; P.n_expert_used = a.n_expert_used; P.row_bytes = a.row_bytes;
     P.ktiles = (a.k + KT - 1) / KT;
-    const uint32_t es = a.kind == K_NVFP4 ? 1u : 2u;
+    const uint32_t es = (a.kind == K_NVFP4 || a.kind == K_MXFP4) ? 1u : 2u;
     P.scale_words = (a.groups * es) % 4u == 0 && (uintptr_t)a.scales % 4u == 0 &&
                     (a.fmt != FMT_AFFINE || (uintptr_t)a.aux % 4u == 0);
     P.raw16 = a.kind != K_CB3 && a.row_bytes % 16u == 0;
@@ -1027,6 +1194,8 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     memset(&tmap, 0, sizeof(tmap));
     P.tma = code_tensor_map(a, &tmap) ? 1u : 0u;
     const uint32_t nm = (a.n + BM - 1) / BM;
+    P.n_mtiles = nm;
+    P.work_counter = work_counter;
     return launch_kind(P, tmap, pl, a.kind, a.x_dtype, nm, max_tiles, st);
 }
 

@@ -459,7 +459,8 @@ gemv_aff4_dp4a(const GemvParams P) {
                     int E = (int)emax - 149;
                     E = E < -126 ? -126 : E;
                     const float inv = __uint_as_float((uint32_t)(127 - E) << 23);  // 2^-E
-                    const int qv = __float2int_rn(x * inv);
+                    // |x * 2^-E| < 2^23; the clamp keeps a value rounded up to 2^23 in the planes
+                    const int qv = max(-0x7FFFFF, min(0x7FFFFF, __float2int_rn(x * inv)));
                     const uint32_t wd = lane >> 3, nib = lane & 7u;
                     const uint32_t off = plane_base + (idx * DP_PW) * 4u +
                                          ((wd * 3u) * 2u + (nib & 1u)) * 4u + (nib >> 1);
@@ -606,7 +607,7 @@ __device__ __forceinline__ void plane_word(const float (&v)[8], uint32_t *unit_p
     const float inv = __uint_as_float((uint32_t)(127 - E) << 23);  // 2^-E, |x * 2^-E| < 2^23
     int q[8];
 #pragma unroll
-    for (int i = 0; i < 8; i++) q[i] = __float2int_rn(v[i] * inv);
+    for (int i = 0; i < 8; i++) q[i] = max(-0x7FFFFF, min(0x7FFFFF, __float2int_rn(v[i] * inv)));  // < 2^23
     uint32_t pw[6];
 #pragma unroll
     for (int p = 0; p < 3; p++) {
@@ -835,6 +836,49 @@ gemv_aff4_tma(const GemvParams P) {
     }
 }
 
+// Two-plane variant for the one-token kernel: x of a unit as 16-bit fixed point,
+// q_j = rint(x_j * 2^-E_u) with |q_j| < 2^15 (clamped), split into an unsigned low
+// byte plane and a signed high byte plane: q = b1 * 2^8 + b0. For bf16 and f16 x
+// this is exact (x * 2^-E_u is then a multiple of 2^7 (bf16) or 2^4 (f16) below
+// 2^15); for f32 x the rounding is below 2^-15 of the unit's largest |x|. Per word
+// wd of the unit four plane words are stored: plane 0 lo, plane 0 hi, plane 1 lo,
+// plane 1 hi (lo: bytes of codes 0, 2, 4, 6 of the word, hi: codes 1, 3, 5, 7).
+constexpr int DP_PW2 = 20;  // u32 words per unit (16 used; 20 spreads the banks of per-lane loads)
+
+__device__ __forceinline__ void plane_word2(const float (&v)[8], uint32_t *unit_planes, uint32_t wd,
+                                            float *uscale_u, float *usum_u, bool store) {
+    uint32_t eb = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) eb = max(eb, (__float_as_uint(v[i]) >> 23) & 0xFFu);
+    eb = max(eb, __shfl_xor_sync(0xFFFFFFFFu, eb, 1));
+    eb = max(eb, __shfl_xor_sync(0xFFFFFFFFu, eb, 2));
+    int E = (int)eb - 141;
+    E = E < -126 ? -126 : E;
+    const float inv = __uint_as_float((uint32_t)(127 - E) << 23);  // 2^-E, |x * 2^-E| < 2^15
+    int q[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) q[i] = max(-0x7FFF, min(0x7FFF, __float2int_rn(v[i] * inv)));
+    uint32_t pw[4];
+#pragma unroll
+    for (int p = 0; p < 2; p++) {
+        const uint32_t sel = (uint32_t)p | ((uint32_t)(4 + p) << 4);
+        const uint32_t l01 = __byte_perm((uint32_t)q[0], (uint32_t)q[2], sel);
+        const uint32_t l23 = __byte_perm((uint32_t)q[4], (uint32_t)q[6], sel);
+        const uint32_t h01 = __byte_perm((uint32_t)q[1], (uint32_t)q[3], sel);
+        const uint32_t h23 = __byte_perm((uint32_t)q[5], (uint32_t)q[7], sel);
+        pw[2 * p] = __byte_perm(l01, l23, 0x5410);
+        pw[2 * p + 1] = __byte_perm(h01, h23, 0x5410);
+    }
+    if (store) *(uint4 *)(unit_planes + wd * 4u) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+    float sum = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+    if (store && wd == 0) {
+        *uscale_u = __uint_as_float((uint32_t)(127 + E) << 23);  // 2^E
+        *usum_u = sum;
+    }
+}
+
 // -------------------- 4-bit affine, one token: x planes held in registers
 //
 // With a single token every (token, slot) pair multiplies the same x row, so a
@@ -844,9 +888,11 @@ gemv_aff4_tma(const GemvParams P) {
 // is row p*n + c) and split into equal contiguous ranges, two CTAs per SM, so
 // every SM streams the same number of bytes whatever the experts. A group of
 // LPR lanes owns one row at a time; lane l of the group holds 32-code units
-// l, l+LPR, ..., UPL of them. Each warp's rows arrive by bulk copies (one per
-// pair the range touches) on the warp's own mbarrier; scales, biases and x
-// by bulk copies issued before the planes are built.
+// l, l+LPR, ..., UPL of them, as two byte planes of 16-bit fixed point
+// (plane_word2, exact for bf16 and f16 x), so a 32-code unit takes 16 DP4A.
+// Each warp's rows arrive by bulk copies (one per pair the range touches) on the
+// warp's own mbarrier; scales, biases and x by bulk copies issued before the
+// planes are built.
 constexpr int ROWS_THREADS = 256;
 constexpr int ROWS_WARPS = ROWS_THREADS / 32;
 constexpr uint32_t ROWS_MAX_PAIRS = 64;
@@ -861,7 +907,7 @@ __host__ __device__ inline RowsLayout rows_layout(uint32_t rb, uint32_t row_byte
     L.w = 0;
     L.xraw = al16u(rb * row_bytes);
     L.planes = al16u(L.xraw + x_bytes);
-    L.uscale = L.planes + nu * DP_PW * 4u;
+    L.uscale = L.planes + nu * DP_PW2 * 4u;
     L.usum = L.uscale + nu * 4u;
     L.sc = al16u(L.usum + nu * 4u);
     L.bi = al16u(L.sc + rb * G * 2u);
@@ -869,40 +915,24 @@ __host__ __device__ inline RowsLayout rows_layout(uint32_t rb, uint32_t row_byte
     return L;
 }
 
-// Exact integer dot product of one 32-code unit with x planes held in registers
-// (same arithmetic as dp4a_unit).
-__device__ __forceinline__ float dp4a_unit_reg(const uint4 w, const uint4 (&v)[6], float usc, float usm,
-                                               float s, float b, float acc) {
-    const uint32_t lo0 = w.x & 0x0F0F0F0Fu, hi0 = (w.x >> 4) & 0x0F0F0F0Fu;
-    const uint32_t lo1 = w.y & 0x0F0F0F0Fu, hi1 = (w.y >> 4) & 0x0F0F0F0Fu;
-    const uint32_t lo2 = w.z & 0x0F0F0F0Fu, hi2 = (w.z >> 4) & 0x0F0F0F0Fu;
-    const uint32_t lo3 = w.w & 0x0F0F0F0Fu, hi3 = (w.w >> 4) & 0x0F0F0F0Fu;
-    uint32_t a0 = dp4a_uu(lo0, v[0].x, 0u);
-    a0 = dp4a_uu(hi0, v[0].y, a0);
-    uint32_t a1 = dp4a_uu(lo0, v[0].z, 0u);
-    a1 = dp4a_uu(hi0, v[0].w, a1);
-    int32_t a2 = dp4a_us(lo0, v[1].x, 0);
-    a2 = dp4a_us(hi0, v[1].y, a2);
-    a0 = dp4a_uu(lo1, v[1].z, a0);
-    a0 = dp4a_uu(hi1, v[1].w, a0);
-    a1 = dp4a_uu(lo1, v[2].x, a1);
-    a1 = dp4a_uu(hi1, v[2].y, a1);
-    a2 = dp4a_us(lo1, v[2].z, a2);
-    a2 = dp4a_us(hi1, v[2].w, a2);
-    a0 = dp4a_uu(lo2, v[3].x, a0);
-    a0 = dp4a_uu(hi2, v[3].y, a0);
-    a1 = dp4a_uu(lo2, v[3].z, a1);
-    a1 = dp4a_uu(hi2, v[3].w, a1);
-    a2 = dp4a_us(lo2, v[4].x, a2);
-    a2 = dp4a_us(hi2, v[4].y, a2);
-    a0 = dp4a_uu(lo3, v[4].z, a0);
-    a0 = dp4a_uu(hi3, v[4].w, a0);
-    a1 = dp4a_uu(lo3, v[5].x, a1);
-    a1 = dp4a_uu(hi3, v[5].y, a1);
-    a2 = dp4a_us(lo3, v[5].z, a2);
-    a2 = dp4a_us(hi3, v[5].w, a2);
-    // a0 + 256 a1 < 2^26 (each plane sum is below 2^17): exact in int32
-    const float d = fmaf((float)a2, 65536.f, (float)(int32_t)(a0 + (a1 << 8)));
+// Integer dot product of one 32-code unit with two x planes held in registers
+// (v[wd] = plane 0 lo, plane 0 hi, plane 1 lo, plane 1 hi of word wd): 16 DP4A in
+// four chains. Each plane sum is below 2^17 in magnitude, so d = a0 + 2^8 a1 is
+// exact in int32 and in fp32.
+__device__ __forceinline__ float dp4a_unit_reg2(const uint4 w, const uint4 (&v)[4], float usc, float usm,
+                                                float s, float b, float acc) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    uint32_t a0l = 0u, a0h = 0u;
+    int32_t a1l = 0, a1h = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t lo = ww[i] & 0x0F0F0F0Fu, hi = (ww[i] >> 4) & 0x0F0F0F0Fu;
+        a0l = dp4a_uu(lo, v[i].x, a0l);
+        a0h = dp4a_uu(hi, v[i].y, a0h);
+        a1l = dp4a_us(lo, v[i].z, a1l);
+        a1h = dp4a_us(hi, v[i].w, a1h);
+    }
+    const float d = (float)((int32_t)(a0l + a0h) + ((a1l + a1h) << 8));
     return fmaf(s, d * usc, fmaf(b, usm, acc));
 }
 
@@ -1056,7 +1086,7 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
 #pragma unroll
                 for (int i = 0; i < 8; i++) v[i] = 0.f;
             }
-            plane_word(v, planes + u * DP_PW, wd, uscale + u, usum + u, valid);
+            plane_word2(v, planes + u * DP_PW2, wd, uscale + u, usum + u, valid);
         }
     }
     __syncthreads();
@@ -1064,15 +1094,15 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
     // this lane's units and their planes, in registers for all its rows
     const uint32_t gi = lane / LPR, l = lane % LPR;
     const uint32_t upg = P.gs / 32u;
-    uint4 pv[UPL][6];
+    uint4 pv[UPL][4];
     float usc[UPL], usm[UPL];
     uint32_t grp[UPL];
 #pragma unroll
     for (int i = 0; i < UPL; i++) {
         const uint32_t u = tmin<uint32_t>(l + (uint32_t)i * LPR, nu - 1u);
-        const uint4 *pl = (const uint4 *)(planes + u * DP_PW);
+        const uint4 *pl = (const uint4 *)(planes + u * DP_PW2);
 #pragma unroll
-        for (int t = 0; t < 6; t++) pv[i][t] = pl[t];
+        for (int t = 0; t < 4; t++) pv[i][t] = pl[t];
         usc[i] = uscale[u];
         usm[i] = usum[u];
         grp[i] = tmin<uint32_t>(u / upg, G - 1u);
@@ -1111,8 +1141,8 @@ gemv_aff4_rows(const GemvParams P, uint32_t rows_per_cta) {
                     const uint32_t u = l + (uint32_t)i * LPR;
                     if (u < nu) {
                         const uint4 w = *(const uint4 *)(wrow + 16u * u);
-                        acc[h] = dp4a_unit_reg(w, pv[i], usc[i], usm[i], bf16_bits_to_f32(srow[grp[i]]),
-                                               bf16_bits_to_f32(brow[grp[i]]), acc[h]);
+                        acc[h] = dp4a_unit_reg2(w, pv[i], usc[i], usm[i], bf16_bits_to_f32(srow[grp[i]]),
+                                                bf16_bits_to_f32(brow[grp[i]]), acc[h]);
                     }
                 }
             }

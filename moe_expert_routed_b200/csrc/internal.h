@@ -18,6 +18,7 @@ constexpr uint32_t ROUTE_MAX_E = 1024;      // experts (the out-of-range bucket 
 struct WsLayout {
     size_t err;          // u32 error word at offset 0
     size_t tile_count;   // u32
+    size_t work_counter; // u32: the grouped GEMM's dynamic work counter (zeroed by the routing prologue)
     size_t counts;       // (E+1) u32
     size_t offsets;      // (E+2) u32
     size_t sorted_pairs; // R u32
@@ -35,12 +36,13 @@ constexpr uint32_t MIN_TILE_ROWS = 64;
 bool ws_layout(uint64_t R, uint32_t E, WsLayout *L);
 
 // Routing prologue: histogram -> scan -> stable scatter (+ zero rows of
-// out-of-range pairs when `out` is non-null).
+// out-of-range pairs when `out` is non-null; zeroes *work_counter when non-null).
 cudaError_t launch_route(const uint32_t *ids, uint32_t R, uint32_t E, uint32_t tile_rows,
                          uint32_t *counts, uint32_t *offsets, uint32_t *sorted_pairs,
                          uint32_t *tiles, uint32_t *tile_count, uint32_t max_tiles,
                          uint32_t *chunk_hist, uint32_t *chunk_base, uint32_t chunks,
-                         uint32_t *err, void *out, uint32_t n, int out_dtype, cudaStream_t st);
+                         uint32_t *err, void *out, uint32_t n, int out_dtype, cudaStream_t st,
+                         uint32_t *work_counter = nullptr);
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device:
 // `cache` is a per-kernel array of the largest size already set, per device.
@@ -88,7 +90,7 @@ bool gemm_supported(const QmmArgs &a);
 uint32_t gemm_tile_rows(const QmmArgs &a);
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
-                        uint32_t *err, cudaStream_t st);
+                        uint32_t *err, uint32_t *work_counter, cudaStream_t st);
 
 // moe_qmm_id's scalar validation (MOE_OK or the status moe_qmm_id would return).
 moe_status validate_call(const void *x, const uint32_t *ids, const void *packed, const void *scales,

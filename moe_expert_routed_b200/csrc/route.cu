@@ -93,7 +93,8 @@ __global__ void __launch_bounds__(1024)
 route_scan(const uint32_t *__restrict__ chunk_hist, uint32_t C, uint32_t E, uint32_t R,
            uint32_t tile_rows, uint32_t *__restrict__ counts, uint32_t *__restrict__ offsets,
            uint32_t *__restrict__ chunk_base, uint32_t *__restrict__ tiles,
-           uint32_t *__restrict__ tile_count, uint32_t max_tiles, uint32_t *__restrict__ err) {
+           uint32_t *__restrict__ tile_count, uint32_t max_tiles, uint32_t *__restrict__ err,
+           uint32_t *__restrict__ work_counter) {
     extern __shared__ uint32_t sm[];
     const uint32_t NB = E + 1;
     uint32_t *tot = sm;            // [NB]
@@ -139,6 +140,7 @@ route_scan(const uint32_t *__restrict__ chunk_hist, uint32_t C, uint32_t E, uint
     if (threadIdx.x == 0) {
         offsets[NB] = total_rows;
         *tile_count = min(total_tiles, max_tiles);
+        if (work_counter) *work_counter = 0u;  // the grouped GEMM's dynamic work counter
         if (total_rows != R) atomicOr(err, ERR_INTERNAL);
     }
 }
@@ -206,14 +208,15 @@ cudaError_t launch_route(const uint32_t *ids, uint32_t R, uint32_t E, uint32_t t
                          uint32_t *counts, uint32_t *offsets, uint32_t *sorted_pairs,
                          uint32_t *tiles, uint32_t *tile_count, uint32_t max_tiles,
                          uint32_t *chunk_hist, uint32_t *chunk_base, uint32_t chunks,
-                         uint32_t *err, void *out, uint32_t n, int out_dtype, cudaStream_t st) {
+                         uint32_t *err, void *out, uint32_t n, int out_dtype, cudaStream_t st,
+                         uint32_t *work_counter) {
     const uint32_t NB = E + 1;
     route_hist<<<chunks, ROUTE_THREADS, NB * sizeof(uint32_t), st>>>(ids, R, E, chunk_hist);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     route_scan<<<1, 1024, (NB + 33) * sizeof(uint32_t), st>>>(
         chunk_hist, chunks, E, R, tile_rows, counts, offsets, chunk_base, tiles, tile_count,
-        max_tiles, err);
+        max_tiles, err, work_counter);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t sc_smem = (size_t)NB * ROUTE_WARPS * sizeof(uint32_t);

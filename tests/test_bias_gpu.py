@@ -1,7 +1,7 @@
 """Per-expert output bias (moe_qmm_id_bias) against the oracle plus its bias
 step, element by element, on every kernel path: the one-token decode kernel,
 the TMA-staged and generic decode kernels with routing fused in, the routed
-decode kernel, and the grouped GEMM with 64-, 256- and 320-pair tiles; bias in
+decode kernel, and the grouped GEMM with 64- and 256-pair tiles (one expert over two); bias in
 f32, bf16 and f16; rows of out-of-range ids stay zero."""
 
 import numpy as np
@@ -29,7 +29,7 @@ CASES = [
                         num_experts=12, x_dtype=DT_F16, out_dtype=DT_F16), "grouped", DT_F16),
     ("grouped-256", dict(fmt=FMT_AFFINE, bits=6, group_size=64, m=400, k=512, n=192, n_expert_used=4,
                          num_experts=8, x_dtype=DT_BF16, out_dtype=DT_F32), "grouped", DT_BF16),
-    ("grouped-320", dict(fmt=FMT_NVFP4, bits=4, group_size=16, m=700, k=256, n=160, n_expert_used=2,
+    ("grouped-256x2", dict(fmt=FMT_NVFP4, bits=4, group_size=16, m=700, k=256, n=160, n_expert_used=2,
                          num_experts=4, x_dtype=DT_BF16, out_dtype=DT_BF16), "grouped", DT_F32),
 ]
 

@@ -64,8 +64,8 @@ def _tile_class_sample(P):
     columns for the coldest; for the hottest, all columns of the pairs at each
     64-pair boundary inside the expert, 0, 63, 64, 127, 128, ..., and the
     first, middle and last column of every 128-row block for the others), pairs
-    256..319 of an expert with more than 256 pairs (the second accumulator of
-    320-pair tiles), and the last 128-column block of every pair at a tile
+    256..319 of an expert with more than 256 pairs (the start of its second
+    256-pair tile), and the last 128-column block of every pair at a tile
     boundary. The tile list runs over the experts' pairs in ascending pair index
     (metrale helpers_b.rs, launch_grouped_gemm: expert_offsets / sorted_token_ids)."""
     ids = P.ids.reshape(-1).astype(np.int64)

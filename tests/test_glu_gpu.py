@@ -3,7 +3,7 @@ out = act(gate) * up, gate rows [0, n/2), up rows [n/2, n) of each expert) again
 the oracle and its glu step, element by element, on every kernel that takes a
 gated output: the one-token decode kernel, the generic decode kernel with routing
 fused in or read from the routing prologue, and the grouped GEMM with 64-, 128-,
-256- and 320-pair tiles; SiLU and both GELU forms; with and without an expert
+256-pair tiles (one expert over two); SiLU and both GELU forms; with and without an expert
 bias; ragged n; rows of out-of-range ids stay zero."""
 
 import numpy as np
@@ -41,7 +41,7 @@ CASES = [
                               num_experts=4, x_dtype=DT_F32, out_dtype=DT_F32), "grouped", "gelu_erf", None),
     ("grouped-256", dict(fmt=FMT_AFFINE, bits=6, group_size=64, m=400, k=512, n=192, n_expert_used=4,
                          num_experts=8, x_dtype=DT_BF16, out_dtype=DT_F32), "grouped", "gelu_erf", DT_BF16),
-    ("grouped-320", dict(fmt=FMT_NVFP4, bits=4, group_size=16, m=700, k=256, n=160, n_expert_used=2,
+    ("grouped-256x2", dict(fmt=FMT_NVFP4, bits=4, group_size=16, m=700, k=256, n=160, n_expert_used=2,
                          num_experts=4, x_dtype=DT_BF16, out_dtype=DT_BF16), "grouped", "gelu_tanh", DT_F32),
 ]
 
@@ -71,7 +71,7 @@ def test_decode_gate_up_config(act):
 
 def test_prefill_config_sampled():
     """The prefill shape (NVFP4, m=4096, top-8, k=4096, n=1536) as a fused gate+up
-    projection on the grouped GEMM with 320-pair tiles: sampled outputs."""
+    projection on the grouped GEMM with 256-pair tiles: sampled outputs."""
     P = config_problem("prefill")
     out = run_glu(P, "silu", path="grouped")
     torch.cuda.synchronize()
