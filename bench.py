@@ -50,10 +50,10 @@ GRAPH_STEPS = 1000   # longest graph of timed steps (more steps replay it)
 GRAPH_CALLS = 100    # calls per graph for the per-call figures
 REPEATS = 5          # per-call figures: median of this many graph replays
 # dram__bytes_read.sum + dram__bytes_write.sum of one gate/up launch of the decode
-# kernel, from one ncu capture of it (cold L2); None until captured for the current
-# kernel
-GATE_UP_DRAM_BYTES = None
-GATE_UP_TRAFFIC_NOTE = "not yet captured for the current kernel"
+# kernel, from one ncu capture of it (cold L2): 17,876,992 B read, 0 B written
+GATE_UP_DRAM_BYTES = 17876992
+GATE_UP_TRAFFIC_NOTE = ("ncu capture of the third gate/up launch of `bench.py --probe decode --reps 4` "
+                        "(gemv_aff4_rows<32, 3, 0>, cold L2): dram read 17,876,992 B, write 0 B")
 
 
 def peaks():
@@ -541,7 +541,8 @@ def grouped_entry(name: str, pk: dict) -> dict:
 
     P = config_problem(name)
     d = to_device(P)
-    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    # sized for the gathered x rows: the GEMM loads each tile of x rows with one tensor copy
+    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts, k=P.k, x_dtype=d["x"].dtype)
     out_dt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float16}[P.out_dtype]
     out = torch.empty((P.m, P.n_expert_used, P.n), dtype=out_dt, device="cuda")
 
@@ -603,9 +604,9 @@ def grouped_entry(name: str, pk: dict) -> dict:
                      "peak_source": pk["source"] + " (bf16_tflops burst, hbm_gbs copy)"},
         "repeats_us": rc["repeats_us"], "route_repeats_us": rr["repeats_us"],
         "timing": f"CUDA graph of {GRAPH_CALLS} calls, median of {REPEATS} replays; routing prologue alone "
-                  f"the same way; gemm_us = call - routing",
+                  f"the same way; gemm_us = call - routing (the x gather kernel and the GEMM)",
         "l2": f"weights {P.packed.nbytes / 1e6:.0f} MB + x {P.x.nbytes / 1e6:.0f} MB (> L2 126 MB)",
-        "gpu_launches_per_call": 4,
+        "gpu_launches_per_call": 5,  # routing histogram, scan, scatter; x gather; GEMM
     }
     del d, out, ws, ws_r, rbuf
     torch.cuda.empty_cache()
@@ -807,7 +808,7 @@ def run_grouped(args, dist: Dist):
         "dtype": ent["workload"].split(", ")[-2], "data": "synthetic",
         "config": {"workload": f"{args.config}: {ent['workload']}", "l2": ent["l2"], "timing": ent["timing"]},
         "per_config": {args.config: ent}, "roofline": ent["roofline"],
-        "gpu_launches": 4 * GRAPH_CALLS * REPEATS, "clocks": clocks,
+        "gpu_launches": ent["gpu_launches_per_call"] * GRAPH_CALLS * REPEATS, "clocks": clocks,
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
@@ -850,7 +851,7 @@ def run_crossover(args):
             d_ids = torch.from_numpy(ids.view(np.int32)).cuda()
             d_x = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
             out = torch.empty((calls, m, 8, P.n), dtype=torch.float32, device="cuda")
-            ws = M.new_workspace(m, 8, P.num_experts)
+            ws = M.new_workspace(m, 8, P.num_experts, k=P.k, x_dtype=torch.bfloat16)
             row = {"projection": name.replace("decode_", ""), "m": m, "routings": 8 * m}
             for path in ("decode", "grouped"):
                 def one(c, path=path):
@@ -885,7 +886,7 @@ def run_probe(args):
     for name in names:
         P = config_problem(name)
         d = to_device(P)
-        ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+        ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts, k=P.k, x_dtype=d["x"].dtype)
         out_dt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float16}[P.out_dtype]
         out = torch.empty((P.m, P.n_expert_used, P.n), dtype=out_dt, device="cuda")
         for _ in range(args.reps):

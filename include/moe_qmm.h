@@ -245,6 +245,19 @@ moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed
  * sizes overflow. */
 size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t num_experts);
 
+/* Workspace bytes with room for the grouped path's gathered f32 x rows: the
+ * pairs' x rows in expert order (m * n_expert_used rows of k values, each held as
+ * two bf16 halves, 4 bytes). When a call with f32 x takes the grouped path and its
+ * workspace_bytes reaches this size (and k is a multiple of 8), x is gathered and
+ * split into its bf16 halves once after routing and the GEMM loads each tile of x
+ * rows with one tensor copy per half; with the minimum moe_qmm_id_workspace_bytes
+ * the GEMM copies and splits x rows itself. Results are the same either way. For
+ * bf16 / f16 x it equals moe_qmm_id_workspace_bytes (the GEMM copies 16-bit x rows
+ * straight from x). Returns 0 if the sizes overflow or
+ * x_dtype is not a moe_dtype. */
+size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts,
+                                    moe_dtype x_dtype);
+
 /* Bytes of one packed weight row (mlx-native quantized_matmul_id.rs,
  * expert_weight_bytes per row): AFFINE 4/8 and CODEBOOK ceil(k / (32/bits)) * 4,
  * AFFINE 6 ceil(k / 4) * 3, NVFP4 k / 2. Returns 0 for an invalid (fmt, bits). */
@@ -372,6 +385,16 @@ moe_status moe_qmm_id_poll_error(void *workspace, moe_stream_t stream);
  * it never faults or hangs the GPU. Returns MOE_OK.
  */
 moe_status moe_qmm_test_inject_wait_timeout(uint64_t limit_ns);
+
+/*
+ * moe_qmm_test_x_copies -- test hook (no counterpart on the pages). on = 1: calls
+ * launched afterwards from this process that take the grouped path with f32 x have
+ * the GEMM's loader warps copy x rows and split them into bf16 halves per tile even
+ * when the workspace holds the gathered rows, so that tests can check both ways give
+ * the same bits. on = 0 (the default) restores the tensor copies of gathered rows.
+ * Returns MOE_ERR_INVALID_ARGUMENT for any other value.
+ */
+moe_status moe_qmm_test_x_copies(int on);
 
 /* Static description of a status code. */
 const char *moe_status_str(moe_status s);

@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.moe_qmm_id_path.restype = i32
         L.moe_qmm_id_workspace_bytes.argtypes = [u32, u32, u32]
         L.moe_qmm_id_workspace_bytes.restype = sz
+        L.moe_qmm_id_workspace_bytes_k.argtypes = [u32] * 4 + [i32]
+        L.moe_qmm_id_workspace_bytes_k.restype = sz
+        L.moe_qmm_test_x_copies.argtypes = [i32]
+        L.moe_qmm_test_x_copies.restype = i32
         L.moe_packed_row_bytes.argtypes = [i32, u32, u32]
         L.moe_packed_row_bytes.restype = sz
         L.moe_qmm_id_route.argtypes = [vp, u32, u32, u32, u32, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -99,13 +103,22 @@ def packed_row_bytes(fmt: int, bits: int, k: int) -> int:
     return int(lib().moe_packed_row_bytes(fmt, bits, k))
 
 
-def workspace_bytes(m: int, n_expert_used: int, num_experts: int) -> int:
-    return int(lib().moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
+def workspace_bytes(m: int, n_expert_used: int, num_experts: int, k: int | None = None,
+                    x_dtype: torch.dtype | None = None) -> int:
+    """moe_qmm_id_workspace_bytes; with k and x_dtype, moe_qmm_id_workspace_bytes_k
+    (room for the grouped path's gathered x rows)."""
+    if k is None:
+        return int(lib().moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
+    return int(lib().moe_qmm_id_workspace_bytes_k(m, k, n_expert_used, num_experts,
+                                                  _TORCH_DT[x_dtype or torch.bfloat16]))
 
 
-def new_workspace(m: int, n_expert_used: int, num_experts: int, device="cuda") -> torch.Tensor:
-    """Zero-initialised workspace (the device error word must start at zero)."""
-    nbytes = workspace_bytes(m, n_expert_used, num_experts)
+def new_workspace(m: int, n_expert_used: int, num_experts: int, device="cuda", k: int | None = None,
+                  x_dtype: torch.dtype | None = None) -> torch.Tensor:
+    """Zero-initialised workspace (the device error word must start at zero). With k
+    and x_dtype it has room for the gathered x rows of the grouped path; without, it
+    is the minimum size (the grouped GEMM then gathers x rows itself)."""
+    nbytes = workspace_bytes(m, n_expert_used, num_experts, k, x_dtype)
     if nbytes == 0:
         raise ValueError("sizes overflow the workspace layout")
     return torch.zeros(nbytes, dtype=torch.uint8, device=device)
@@ -228,7 +241,7 @@ def qmm_id(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: tor
     if out is None:
         out = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
     if workspace is None:
-        workspace = new_workspace(m, n_expert_used, num_experts, device)
+        workspace = new_workspace(m, n_expert_used, num_experts, device, k, x.dtype)
     else:
         _check_dev(workspace, "workspace", device)
     if act is not None:
@@ -279,7 +292,7 @@ class Plan:
         out_n = n // 2 if act is not None else n
         out0 = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
         if workspace is None:
-            workspace = new_workspace(m, n_expert_used, num_experts, device)
+            workspace = new_workspace(m, n_expert_used, num_experts, device, k, x_dtype)
         _validate_only(x0, ids0, packed, scales, aux, n=n, group_size=group_size, bits=bits, fmt=fmt,
                        num_experts=num_experts, out=out0, expert_bias=expert_bias, act=act, launch=launch)
         self._keep = (packed, scales, aux, workspace, expert_bias)  # buffers the plan points into
@@ -326,7 +339,7 @@ def qmm_id_ptrs(x: torch.Tensor, ids: torch.Tensor, packed_ptrs: torch.Tensor, s
     m, k = x.shape
     n_expert_used = ids.shape[1]
     if workspace is None:
-        workspace = new_workspace(m, n_expert_used, num_experts, device)
+        workspace = new_workspace(m, n_expert_used, num_experts, device, k, x.dtype)
     st = lib().moe_qmm_id_ptrs(
         x.data_ptr(), ids.data_ptr(), packed_ptrs.data_ptr(), scale_ptrs.data_ptr(),
         bias_ptrs.data_ptr() if bias_ptrs is not None else None,

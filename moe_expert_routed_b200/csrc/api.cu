@@ -15,6 +15,7 @@ namespace moe {
 
 // Wait limit of the failure-detection test hook (0: off).
 static std::atomic<uint64_t> g_fault_wait_ns{0};
+static std::atomic<int> g_x_copies{0};
 
 static inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -40,6 +41,11 @@ bool ws_layout(uint64_t R, uint32_t E, WsLayout *L) {
     return true;
 }
 
+uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype) {
+    if (k % 8u != 0 || x_dtype != DT_F32) return 0;
+    return al256(R * k * 4ull);
+}
+
 static uint64_t row_bytes_of(int fmt, uint32_t bits, uint32_t k) {
     if (fmt == FMT_NVFP4 || fmt == FMT_MXFP4) return k / 2u;
     if (fmt == FMT_AFFINE && bits == 6) return ((uint64_t)k + 3) / 4 * 3;
@@ -63,6 +69,14 @@ size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t n
     WsLayout L;
     if (!ws_layout((uint64_t)m * n_expert_used, num_experts, &L)) return 0;
     return L.total;
+}
+
+size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts,
+                                    moe_dtype x_dtype) {
+    WsLayout L;
+    if ((int)x_dtype < 0 || (int)x_dtype > 2) return 0;
+    if (!ws_layout((uint64_t)m * n_expert_used, num_experts, &L)) return 0;
+    return L.total + (size_t)gathered_x_bytes((uint64_t)m * n_expert_used, k, (int)x_dtype);
 }
 
 const char *moe_status_str(moe_status s) {
@@ -159,6 +173,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     a.out_n = act >= 0 ? n / 2u : n;
     a.launch_flags = launch_flags;
     a.fault_wait_ns = g_fault_wait_ns.load(std::memory_order_relaxed);
+    a.x_copies = g_x_copies.load(std::memory_order_relaxed);
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);
@@ -197,13 +212,17 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         const uint32_t tile_rows = choice == GROUPED ? gemm_tile_rows(a) : MIN_TILE_ROWS;
         const uint32_t max_tiles = (uint32_t)(R / tile_rows + num_experts + 1);
         uint32_t *wc = (uint32_t *)(ws + L.work_counter);
+        // x rows in expert order for the grouped GEMM, when the workspace has room for them
+        const uint64_t gx = choice == GROUPED ? gathered_x_bytes(R, k, (int)x_dtype) : 0;
+        uint16_t *xg = (gx && workspace_bytes >= L.total + gx) ? (uint16_t *)(ws + L.total) : nullptr;
         ce = launch_route(ids, (uint32_t)R, num_experts, tile_rows, counts, offsets, sp, tiles, tc,
                           max_tiles, (uint32_t *)(ws + L.chunk_hist),
                           (uint32_t *)(ws + L.chunk_base), L.chunks, err, out, a.out_n, (int)out_dtype,
                           st, wc);
+        if (ce == cudaSuccess && xg) ce = launch_gather_x(x, (int)x_dtype, sp, (uint32_t)R, k, n_expert_used, xg, st);
         if (ce == cudaSuccess) {
             if (choice == GROUPED)
-                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, st);
+                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, xg, st);
             else
                 ce = launch_gemv_routed(a, counts, offsets, sp, err, st);
         }
@@ -371,6 +390,12 @@ moe_status moe_qmm_id_route(const uint32_t *ids, uint32_t m, uint32_t n_expert_u
 
 moe_status moe_qmm_test_inject_wait_timeout(uint64_t limit_ns) {
     moe::g_fault_wait_ns.store(limit_ns, std::memory_order_relaxed);
+    return MOE_OK;
+}
+
+moe_status moe_qmm_test_x_copies(int on) {
+    if (on != 0 && on != 1) return MOE_ERR_INVALID_ARGUMENT;
+    moe::g_x_copies.store(on, std::memory_order_relaxed);
     return MOE_OK;
 }
 

@@ -72,6 +72,9 @@ constexpr int MMA_WARP = (NDQ + NLD) / 32;
 constexpr int TMA_WARP = MMA_WARP + 1;
 constexpr int EPI_WARP0 = TMA_WARP + 1;
 constexpr int SCHED_WARP = EPI_WARP0 + NEP / 32;
+// how the B operand's x rows reach shared memory
+constexpr uint32_t XM_LOADERS = 0;  // 16-byte copies by the loader warps
+constexpr uint32_t XM_ROWS = 1;     // tensor copies of x rows gathered into expert order beforehand
 constexpr uint32_t RING = 4;                    // work items the scheduler may publish ahead
 // arrivals that release a ring slot: one per dequantiser, loader and epilogue warp,
 // plus the tensor-copy and MMA lanes
@@ -106,6 +109,11 @@ struct GemmParams {
     uint32_t glu_nh;
     int act;
     uint32_t n_mtiles;      // 128-row blocks per expert (work items per tile)
+    // x tiles (XM_*): XM_ROWS reads the x rows gathered in expert order (f32 x: bf16 high
+    // halves in rows [0, xg_R), remainders in rows [xg_R, 2 xg_R)) through the kernel's
+    // second tensor map
+    uint32_t xmode;
+    uint32_t xg_R;
     uint32_t *work_counter; // items claimed beyond each CTA's first (zeroed by the routing prologue)
     // failure-detection test hook: non-zero makes the MMA warp first wait this long on
     // a barrier nothing completes (so the CTA aborts); 0 in normal operation
@@ -466,7 +474,8 @@ struct Item {
 // epilogue), also decided at compile time so that the plain kernels carry none of it.
 template <int KIND, int XT, int BN, bool PTRS, bool GLU>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap) {
+grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap,
+                    const __grid_constant__ CUtensorMap xmap) {
     using C = GemmCfg<KIND, XT, BN>;
     constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
     constexpr uint32_t STAGE = C::STAGE;
@@ -494,7 +503,8 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
 
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
     const uint32_t S = P.stages;
-    const uint32_t n_items = __ldg(P.tile_count) * P.n_mtiles;
+    const uint32_t nm = P.n_mtiles;  // work items per tile
+    const uint32_t n_items = __ldg(P.tile_count) * nm;
 
     const uint32_t base = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - ptx::smem_u32(smem_raw));
@@ -524,10 +534,13 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
     };
 
     const bool tma = !PTRS && KIND != K_CB3 && P.tma != 0;
+    // x tiles: by the loader warps' 16-byte copies, or (f32 x) by tensor copies of rows
+    // gathered beforehand; a compile-time XM_LOADERS for 16-bit x
+    const uint32_t xmode = (XT == DT_F32) ? P.xmode : XM_LOADERS;
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
             ptx::mbar_init(full0 + 8 * s, NDQ);
-            ptx::mbar_init(loaded0 + 8 * s, NLD + (tma ? 1u : 0u));  // + the tensor-copy warp's arrival
+            ptx::mbar_init(loaded0 + 8 * s, NLD + ((tma || xmode != XM_LOADERS) ? 1u : 0u));  // + the tensor-copy warp's
             ptx::mbar_init(empty0 + 8 * s, 1);
         }
         for (uint32_t b = 0; b < 2; b++) {
@@ -564,8 +577,9 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_s;
     const bool gs16 = (P.lg_gs == 4);
-    const uint32_t nm = P.n_mtiles;
     Item<KIND, PTRS> it;
+    // work item w: tile w / nm, 128-row block w % nm
+    auto load_item = [&](uint32_t w) -> bool { return it.load(P, w / nm, w % nm, BN); };
 
     if (warp < LD_WARP0) {
         // -------------------------------------------------------- dequantisers
@@ -574,7 +588,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
         for (uint32_t i = 0;; i++) {
             uint32_t w;
             if (!next_item(i, true, w) || w >= n_items) break;
-            if (!it.load(P, w / nm, w % nm, BN)) continue;
+            if (!load_item(w)) continue;
             const size_t row_in = glu_row(tmin<uint32_t>(it.row0 + r, P.n - 1), GLU ? P.glu_nh : 0u);
             const uint8_t *srow = it.sb + row_in * P.groups * ES;
             const uint8_t *brow = it.bb + row_in * P.groups * 2u;
@@ -589,7 +603,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                 }
                 const uint32_t st = base + s * STAGE;
                 const uint8_t *stp = base_ptr + s * STAGE;
-                if constexpr (BT == 2) {
+                if (BT == 2 && xmode == XM_LOADERS) {
                     // f32 x: elements 0-3 of a chunk landed in the hi tile's slot, 4-7 in the
                     // lo tile's slot; rewrite both as the bf16 hi and lo halves
                     const uint32_t cc = tid & 7u;
@@ -709,15 +723,15 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
         for (uint32_t i = 0; ok; i++) {
             uint32_t w;
             if (!next_item(i, true, w) || w >= n_items) break;
-            if (!it.load(P, w / nm, w % nm, BN)) continue;
+            if (!load_item(w)) continue;
             const uint8_t *xrow[NXL];
 #pragma unroll
             for (int j = 0; j < NXL; j++) {
                 const uint32_t i = xi0 + XR * j;
-                xrow[j] = i < it.nt ? (const uint8_t *)P.x +
-                                          (size_t)(__ldg(P.sorted_pairs + it.off + it.r0 + i) / P.n_expert_used) *
-                                              P.k * XS
-                                    : nullptr;
+                xrow[j] = (xmode == XM_LOADERS && i < it.nt)
+                              ? (const uint8_t *)P.x +
+                                    (size_t)(__ldg(P.sorted_pairs + it.off + it.r0 + i) / P.n_expert_used) * P.k * XS
+                              : nullptr;
             }
             const uint8_t *ebase = it.wb;
             const uint32_t row0 = it.row0;
@@ -735,11 +749,12 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                     break;
                 }
                 const uint32_t st = base + s * STAGE;
-                // x rows of the pairs, straight into the B operand tile (zero past k and nt)
+                // x rows of the pairs, straight into the B operand tile (zero past k and nt),
+                // unless they come by tensor copy
                 const uint32_t kk = kt * KT + xc * 8u;
 #pragma unroll
                 for (int j = 0; j < NXL; j++) {
-                    if (xi0 + XR * j < it.nt_pad) {
+                    if (xmode == XM_LOADERS && xi0 + XR * j < it.nt_pad) {
                         const bool in = xrow[j] != nullptr && kk < P.k;
                         const uint8_t *src = in ? xrow[j] + (size_t)kk * XS : (const uint8_t *)P.x;
                         const uint32_t dst = st + xdst0 + XR * 128u * j;
@@ -802,20 +817,25 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
         }
         ptx::cp_async_wait_all();
     } else if (warp == TMA_WARP) {
-        // ------------------------------------------------------ code tensor copies
+        // ------------------------------------------------------------ tensor copies
         if (lane == 0) {
             // per k-tile two 64-row copies of RB bytes per row (GLU: the 64 gate rows,
-            // then the 64 up rows); rows past the expert's last read a neighbour's rows or
-            // zeros and are never stored. The arrival (with the byte count) is one of the
-            // stage's loaded arrivals. Without TMA staging the lane only reads the ring.
+            // then the 64 up rows; rows past the expert's last read a neighbour's rows or
+            // zeros and are never stored) and, for gathered x rows, the box of BN rows.
+            // The arrival (with the byte count) is one of the stage's loaded arrivals.
+            // Without tensor copies the lane only reads the ring.
             constexpr uint32_t RB = RL::RB;
             if (tma) ptx::prefetch_tensormap(&tmap);
+            if (xmode == XM_ROWS) ptx::prefetch_tensormap(&xmap);
+            // bytes per k-tile: the codes' two 64-row boxes, the x box of BN rows (each row
+            // one 128-byte swizzle line; twice for f32 x)
+            const uint32_t tx = (tma ? 2u * 64u * RB : 0u) + (xmode == XM_ROWS ? (uint32_t)(BT * B_TILE) : 0u);
             uint32_t g = 0, last_s = 0, last_par = 0;
             bool any = false, ok = true;
             for (uint32_t i = 0; ok; i++) {
                 uint32_t w;
                 if (!next_item(i, false, w) || w >= n_items) break;
-                if (!tma || !it.load(P, w / nm, w % nm, BN)) continue;
+                if (!(tma || xmode == XM_ROWS) || !load_item(w)) continue;
                 const int32_t y0 = (int32_t)(it.e * P.n + (GLU ? it.row0 / 2u : it.row0));
                 const int32_t y1 = GLU ? (int32_t)(it.e * P.n + P.glu_nh + it.row0 / 2u) : y0 + 64;
                 for (uint32_t kt = 0; kt < P.ktiles; kt++, g++) {
@@ -826,9 +846,20 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                         break;
                     }
                     const uint32_t bar = loaded0 + 8 * s, raw = base + s * STAGE + RAW_OFF;
-                    ptx::mbar_arrive_expect_tx(bar, 2u * 64u * RB);
-                    ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
-                    ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
+                    ptx::mbar_arrive_expect_tx(bar, tx);
+                    if (tma) {
+                        ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
+                        ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
+                    }
+                    if (xmode == XM_ROWS) {
+                        // gathered rows off + r0 .. + BN - 1: rows past the tile's pairs are other
+                        // pairs' x rows (or zeros past the end) in B rows whose results are not stored
+                        const uint32_t xb = base + s * STAGE + B_OFF;
+                        const int32_t xrow = (int32_t)(it.off + it.r0);
+                        ptx::tma_load_2d(xb, &xmap, (int32_t)(kt * KT), xrow, bar);
+                        if constexpr (BT == 2)
+                            ptx::tma_load_2d(xb + B_TILE, &xmap, (int32_t)(kt * KT), xrow + (int32_t)P.xg_R, bar);
+                    }
                     last_s = s;
                     last_par = (g / S) & 1u;
                     any = true;
@@ -850,7 +881,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                     break;
                 }
                 if (w >= n_items) break;
-                if (!it.load(P, w / nm, w % nm, BN)) continue;
+                if (!load_item(w)) continue;
                 const uint32_t buf = done % NACC, use = done / NACC;
                 // the epilogue has read this accumulator's previous item (a fresh barrier's
                 // preceding phase counts as complete, so the first two items do not wait)
@@ -922,7 +953,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
         for (uint32_t i = 0;; i++) {
             uint32_t w;
             if (!next_item(i, true, w) || w >= n_items) break;
-            if (!it.load(P, w / nm, w % nm, BN)) continue;
+            if (!load_item(w)) continue;
             const uint32_t buf = done % NACC, use = done / NACC;
             if (!ptx::mbar_wait_bounded(accfull0 + 8 * buf, use & 1u, abort_flag, P.err, ERR_TIMEOUT, P.timeout_ns))
                 break;
@@ -1033,8 +1064,8 @@ uint32_t sm_count_gemm() {
 }
 
 template <int KIND, int XT, int BN, bool PTRS, bool GLU>
-cudaError_t launch_tp(const GemmParams &P0, const CUtensorMap &tmap, const GemmPlan &pl, uint32_t n_mtiles,
-                      uint32_t max_tiles, cudaStream_t st) {
+cudaError_t launch_tp(const GemmParams &P0, const CUtensorMap &tmap, const CUtensorMap &xmap, const GemmPlan &pl,
+                      uint32_t n_mtiles, uint32_t max_tiles, cudaStream_t st) {
     GemmParams P = P0;
     P.stages = (uint32_t)pl.stages;
     auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS, GLU>;
@@ -1044,51 +1075,51 @@ cudaError_t launch_tp(const GemmParams &P0, const CUtensorMap &tmap, const GemmP
     // persistent: one CTA per SM, or fewer when there are fewer work items
     const uint64_t items = (uint64_t)n_mtiles * max_tiles;
     const uint32_t ctas = (uint32_t)(items < (uint64_t)sm_count_gemm() ? items : (uint64_t)sm_count_gemm());
-    kern<<<ctas, GEMM_THREADS, pl.smem, st>>>(P, tmap);
+    kern<<<ctas, GEMM_THREADS, pl.smem, st>>>(P, tmap, xmap);
     return cudaGetLastError();
 }
 
 template <int KIND, int XT, int BN>
-cudaError_t launch_t(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, uint32_t n_mtiles,
-                     uint32_t max_tiles, cudaStream_t st) {
-    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true, false>(P, tm, pl, n_mtiles, max_tiles, st);
-    if (P.glu_nh) return launch_tp<KIND, XT, BN, false, true>(P, tm, pl, n_mtiles, max_tiles, st);
-    return launch_tp<KIND, XT, BN, false, false>(P, tm, pl, n_mtiles, max_tiles, st);
+cudaError_t launch_t(const GemmParams &P, const CUtensorMap &tm, const CUtensorMap &xm, const GemmPlan &pl,
+                     uint32_t n_mtiles, uint32_t max_tiles, cudaStream_t st) {
+    if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true, false>(P, tm, xm, pl, n_mtiles, max_tiles, st);
+    if (P.glu_nh) return launch_tp<KIND, XT, BN, false, true>(P, tm, xm, pl, n_mtiles, max_tiles, st);
+    return launch_tp<KIND, XT, BN, false, false>(P, tm, xm, pl, n_mtiles, max_tiles, st);
 }
 
 template <int KIND>
-cudaError_t launch_k(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, int x_dtype, uint32_t nm,
-                     uint32_t mt, cudaStream_t st) {
+cudaError_t launch_k(const GemmParams &P, const CUtensorMap &tm, const CUtensorMap &xm, const GemmPlan &pl,
+                     int x_dtype, uint32_t nm, uint32_t mt, cudaStream_t st) {
     if (x_dtype == DT_F32) {
-        if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, tm, pl, nm, mt, st);
-        return launch_t<KIND, DT_F32, 64>(P, tm, pl, nm, mt, st);
+        if (pl.bn == 128) return launch_t<KIND, DT_F32, 128>(P, tm, xm, pl, nm, mt, st);
+        return launch_t<KIND, DT_F32, 64>(P, tm, xm, pl, nm, mt, st);
     }
     if constexpr (KIND == K_MXFP4) {
         // e2m1 * 2^e can leave the f16 range: only bf16 (and f32, as bf16 halves) x here
         if (x_dtype != DT_BF16) return cudaErrorNotSupported;
-        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, pl, nm, mt, st);
-        return launch_t<KIND, DT_BF16, 64>(P, tm, pl, nm, mt, st);
+        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, xm, pl, nm, mt, st);
+        return launch_t<KIND, DT_BF16, 64>(P, tm, xm, pl, nm, mt, st);
     } else {
     if (x_dtype == DT_BF16) {
-        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, pl, nm, mt, st);
-        return launch_t<KIND, DT_BF16, 64>(P, tm, pl, nm, mt, st);
+        if (pl.bn == 256) return launch_t<KIND, DT_BF16, 256>(P, tm, xm, pl, nm, mt, st);
+        return launch_t<KIND, DT_BF16, 64>(P, tm, xm, pl, nm, mt, st);
     }
-    if (pl.bn == 256) return launch_t<KIND, DT_F16, 256>(P, tm, pl, nm, mt, st);
-    return launch_t<KIND, DT_F16, 64>(P, tm, pl, nm, mt, st);
+    if (pl.bn == 256) return launch_t<KIND, DT_F16, 256>(P, tm, xm, pl, nm, mt, st);
+    return launch_t<KIND, DT_F16, 64>(P, tm, xm, pl, nm, mt, st);
     }
 }
 
-cudaError_t launch_kind(const GemmParams &P, const CUtensorMap &tm, const GemmPlan &pl, int kind, int x_dtype,
-                        uint32_t nm, uint32_t mt, cudaStream_t st) {
+cudaError_t launch_kind(const GemmParams &P, const CUtensorMap &tm, const CUtensorMap &xm, const GemmPlan &pl,
+                        int kind, int x_dtype, uint32_t nm, uint32_t mt, cudaStream_t st) {
     switch (kind) {
-        case K_AFF4: return launch_k<K_AFF4>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_AFF6: return launch_k<K_AFF6>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_AFF8: return launch_k<K_AFF8>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_CB2: return launch_k<K_CB2>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_CB3: return launch_k<K_CB3>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_CB4: return launch_k<K_CB4>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_NVFP4: return launch_k<K_NVFP4>(P, tm, pl, x_dtype, nm, mt, st);
-        case K_MXFP4: return launch_k<K_MXFP4>(P, tm, pl, x_dtype, nm, mt, st);
+        case K_AFF4: return launch_k<K_AFF4>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_AFF6: return launch_k<K_AFF6>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_AFF8: return launch_k<K_AFF8>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_CB2: return launch_k<K_CB2>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_CB3: return launch_k<K_CB3>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_CB4: return launch_k<K_CB4>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_NVFP4: return launch_k<K_NVFP4>(P, tm, xm, pl, x_dtype, nm, mt, st);
+        case K_MXFP4: return launch_k<K_MXFP4>(P, tm, xm, pl, x_dtype, nm, mt, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1118,6 +1149,21 @@ uint32_t ktile_row_bytes(int kind) {
         case K_MXFP4: return RawLayout<K_MXFP4>::RB;
         default: return 0;
     }
+}
+
+// Tensor map of rows of 16-bit x values, a [rows, k] matrix, with boxes of 64
+// values x box_rows rows in the 128-byte swizzle (the B operand's canonical
+// K-major layout). False if it cannot be encoded.
+bool x_tensor_map(const void *x, uint32_t rows, uint32_t k, uint32_t box_rows, CUtensorMap *m) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
+    if (!enc || (uintptr_t)x % 16u != 0 || k % 8u != 0 || box_rows == 0 || box_rows > 256u || rows == 0) return false;
+    const cuuint64_t dims[2] = {k, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)k * 2u};
+    const cuuint32_t box[2] = {64u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void *)x, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Tensor map of the packed codes as a [num_experts * n, row_bytes] byte matrix with
@@ -1166,7 +1212,7 @@ uint32_t gemm_tile_rows(const QmmArgs &a) {
 
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
-                        uint32_t *err, uint32_t *work_counter, cudaStream_t st) {
+                        uint32_t *err, uint32_t *work_counter, const uint16_t *xg, cudaStream_t st) {
     GemmPlan pl;
     if (!gemm_plan(a, &pl)) return cudaErrorNotSupported;
     GemmParams P{};
@@ -1196,7 +1242,16 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     const uint32_t nm = (a.n + BM - 1) / BM;
     P.n_mtiles = nm;
     P.work_counter = work_counter;
-    return launch_kind(P, tmap, pl, a.kind, a.x_dtype, nm, max_tiles, st);
+    CUtensorMap xmap;
+    memset(&xmap, 0, sizeof(xmap));
+    const uint32_t R = a.m * a.n_expert_used;
+    P.xg_R = R;
+    // f32 x: tensor copies of the rows gathered and split after routing, when the
+    // workspace holds them (and no test asks for the loader copies)
+    P.xmode = (a.x_dtype == DT_F32 && !a.x_copies && xg && x_tensor_map(xg, R * 2u, a.k, pl.bn, &xmap))
+                  ? XM_ROWS
+                  : XM_LOADERS;
+    return launch_kind(P, tmap, xmap, pl, a.kind, a.x_dtype, nm, max_tiles, st);
 }
 
 }  // namespace moe

@@ -77,6 +77,7 @@ struct QmmArgs {
     // kernels with bounded waits make one wait per CTA on a barrier nothing
     // completes, giving up after this many ns; 0 in normal operation
     uint64_t fault_wait_ns;
+    int x_copies;  // 1: the grouped GEMM's loader warps copy x rows (test hook)
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).
@@ -85,12 +86,20 @@ cudaError_t launch_gemv_fused(const QmmArgs &a, uint32_t *err, cudaStream_t st);
 cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const uint32_t *offsets,
                                const uint32_t *sorted_pairs, uint32_t *err, cudaStream_t st);
 
-// tcgen05 grouped GEMM over the routing prologue's tiles.
+// f32 x rows in expert order for the grouped GEMM, as bf16 high halves in rows
+// [0, R) and the bf16 roundings of the remainders in rows [R, 2R); k % 8 == 0.
+cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_pairs, uint32_t R, uint32_t k,
+                            uint32_t n_expert_used, uint16_t *xg, cudaStream_t st);
+// Bytes of the gathered x rows (0 when the grouped GEMM does not use them: 16-bit x
+// is gathered by the GEMM's tensor copies straight from x).
+uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype);
+
+// tcgen05 grouped GEMM over the routing prologue's tiles (xg: gathered f32 x rows, or null).
 bool gemm_supported(const QmmArgs &a);
 uint32_t gemm_tile_rows(const QmmArgs &a);
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
-                        uint32_t *err, uint32_t *work_counter, cudaStream_t st);
+                        uint32_t *err, uint32_t *work_counter, const uint16_t *xg, cudaStream_t st);
 
 // moe_qmm_id's scalar validation (MOE_OK or the status moe_qmm_id would return).
 moe_status validate_call(const void *x, const uint32_t *ids, const void *packed, const void *scales,

@@ -10,6 +10,13 @@
 //                 tile list
 //   route_scatter one CTA per chunk: per-warp bucket counts, their prefix over
 //                 the warps, then stable ranks from warp match masks
+// and, for the grouped GEMM with f32 x when the caller's workspace has room for it,
+//   gather_x      the pairs' x rows in expert order (row i = x row of the token of
+//                 sorted pair i) as bf16 high halves (rows 0 .. R-1) and the bf16
+//                 roundings of the remainders (rows R .. 2R-1), so that the GEMM loads
+//                 each tile of x rows with one tensor copy per half and no longer
+//                 splits f32 values per tile (16-bit x needs no such pass: the GEMM
+//                 gathers its rows with 4-row tensor copies)
 #include "common.cuh"
 #include "internal.h"
 
@@ -202,7 +209,48 @@ route_scatter(const uint32_t *__restrict__ ids, uint32_t R, uint32_t E,
     }
 }
 
+// One warp per gathered row, 32-byte loads and 16-byte stores (k % 8 == 0). The split
+// is the one the GEMM applies to f32 x it copies itself: hi = bf16(v), lo = bf16(v - hi),
+// both rounded to nearest even.
+__global__ void __launch_bounds__(256)
+gather_x(const float *__restrict__ x, const uint32_t *__restrict__ sorted_pairs, uint32_t R, uint32_t k,
+         uint32_t n_expert_used, uint16_t *__restrict__ xg) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t k8 = k / 8u;  // 8-element chunks per row
+    for (uint32_t row = blockIdx.x * 8u + (threadIdx.x >> 5); row < R; row += gridDim.x * 8u) {
+        const size_t t = __ldg(sorted_pairs + row) / n_expert_used;
+        const float4 *src = (const float4 *)x + t * k8 * 2u;
+        uint4 *hi = (uint4 *)xg + (size_t)row * k8, *lo = (uint4 *)xg + ((size_t)R + row) * k8;
+        for (uint32_t c = lane; c < k8; c += 32u) {
+            const float4 a = __ldg(src + 2u * c), b = __ldg(src + 2u * c + 1u);
+            const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            uint32_t h[4], l[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+                const float2 hf = __bfloat1622float2(hb);
+                const __nv_bfloat162 lb = __floats2bfloat162_rn(f[2 * i] - hf.x, f[2 * i + 1] - hf.y);
+                h[i] = *reinterpret_cast<const uint32_t *>(&hb);
+                l[i] = *reinterpret_cast<const uint32_t *>(&lb);
+            }
+            hi[c] = make_uint4(h[0], h[1], h[2], h[3]);
+            lo[c] = make_uint4(l[0], l[1], l[2], l[3]);
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_pairs, uint32_t R, uint32_t k,
+                            uint32_t n_expert_used, uint16_t *xg, cudaStream_t st) {
+    const uint32_t rows_per_cta = 8;
+    uint32_t ctas = (R + rows_per_cta - 1) / rows_per_cta;
+    if (ctas > 148u * 16u) ctas = 148u * 16u;
+    if (ctas == 0) return cudaSuccess;
+    if (x_dtype != DT_F32 || k % 8u != 0) return cudaErrorInvalidValue;
+    gather_x<<<ctas, 256, 0, st>>>((const float *)x, sorted_pairs, R, k, n_expert_used, xg);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_route(const uint32_t *ids, uint32_t R, uint32_t E, uint32_t tile_rows,
                          uint32_t *counts, uint32_t *offsets, uint32_t *sorted_pairs,

@@ -55,6 +55,23 @@ def test_workspace_bytes_grows_with_routings():
     assert 0 < a < b and b % 256 == 0
 
 
+def test_workspace_bytes_with_gathered_x():
+    base = M.workspace_bytes(512, 8, 64)
+    bf = M.workspace_bytes(512, 8, 64, k=1024, x_dtype=torch.bfloat16)
+    f32 = M.workspace_bytes(512, 8, 64, k=1024, x_dtype=torch.float32)
+    assert bf == base                                 # 16-bit x: gathered by the GEMM's tensor copies
+    assert f32 == base + 512 * 8 * 1024 * 4          # f32 x: two bf16 halves per element
+    assert M.workspace_bytes(512, 8, 64, k=1028, x_dtype=torch.float32) == base  # k % 8: no room added
+    assert M.lib().moe_qmm_id_workspace_bytes_k(512, 1024, 8, 64, 3) == 0         # not a moe_dtype
+
+
+def test_x_copies_hook_rejects_other_values():
+    L = M.lib()
+    assert L.moe_qmm_test_x_copies(2) == 1
+    assert L.moe_qmm_test_x_copies(-1) == 1
+    assert L.moe_qmm_test_x_copies(0) == 0
+
+
 def _call(**kw):
     args = dict(x=16, ids=16, packed=16, scales=16, aux=16, out=16, m=4, k=256, n=128, gs=32,
                 bits=4, fmt=0, topk=2, E=8, xd=0, od=0, ws=4096, wsb=1 << 20, stream=None, path=0)

@@ -14,7 +14,7 @@ import torch
 import moe_expert_routed_b200 as M
 from tests.gpu_util import check_full, run, to_device
 from workloads import config_problem, make_problem
-from workloads.gen import DT_BF16, DT_F16, DT_F32, FMT_CODEBOOK, FMT_NVFP4
+from workloads.gen import DT_BF16, DT_F16, DT_F32, FMT_AFFINE, FMT_CODEBOOK, FMT_NVFP4
 
 pytestmark = pytest.mark.gpu
 
@@ -36,9 +36,13 @@ def problems():
                                   k=320, n=256, n_expert_used=2, num_experts=4, x_dtype=DT_F16,
                                   out_dtype=DT_F32, seed=62, scale_range=(0.01, 0.05))
     yield "auto", config_problem("decode_gate_up")  # the one-token decode kernel
+    # 256-pair tiles
+    yield "grouped", make_problem("timeout-pair", fmt=FMT_AFFINE, bits=4, group_size=64, m=512, k=512,
+                                  n=384, n_expert_used=2, num_experts=8, x_dtype=DT_BF16,
+                                  out_dtype=DT_F32, seed=63)
 
 
-@pytest.mark.parametrize("case", list(range(3)))
+@pytest.mark.parametrize("case", list(range(4)))
 def test_wait_timeout_is_reported_and_the_next_call_is_exact(case):
     path, P = list(problems())[case]
     dev = to_device(P)
