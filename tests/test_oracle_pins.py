@@ -96,6 +96,18 @@ def test_round_to_f16_matches_numpy():
     np.testing.assert_array_equal(got, ref)
 
 
+def test_scalar_rounding_helpers_match_the_casts():
+    # the scalar entry points are the same RNE casts as the array one
+    rng = np.random.default_rng(13)
+    vals = np.concatenate([rng.standard_normal(500), rng.standard_normal(50) * 1e-39,
+                           np.array([0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1 + 2 ** -11, 65504.0])])
+    bf = np.array([oracle.double_to_bf16(v) for v in vals], dtype=np.uint16)
+    np.testing.assert_array_equal(bf, bf16_bits(vals.astype(np.float32)))
+    with np.errstate(over="ignore"):
+        f16 = vals.astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(np.array([oracle.double_to_f16(v) for v in vals], dtype=np.uint16), f16)
+
+
 # ---------------------------------------------------------------- storage
 
 @pytest.mark.parametrize("fmt,bits,k,expect", [
