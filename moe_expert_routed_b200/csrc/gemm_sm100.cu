@@ -178,21 +178,30 @@ template <> struct Raw<K_CB3> { static constexpr int W = 4; };  // codes SUB .. 
 // Rows are an odd number of 16-byte units apart, so 8 consecutive rows read
 // with 16-byte loads touch all 32 banks once.
 //
-// With TMA staging (contiguous weights, rows a multiple of 16 bytes, not 3-bit)
-// the same area holds instead
+// With TMA staging (contiguous weights, rows a multiple of 16 bytes) the same area
+// holds instead
 //   [0, BM*RB)            the codes, BM rows of RB bytes written by two 64-row
 //                         tensor copies; for RB = 32 / 64 the 16-byte chunks of a
 //                         row are swizzled within 32 / 64 bytes (the copies'
 //                         SWIZZLE_32B / 64B mode), so 8 consecutive rows read with
 //                         16-byte loads touch all 32 banks once
 //   [BM*RB, BM*RB+BM*16)  per row: scale words (8 bytes), then bias words (8 bytes)
+// 3-bit codebook rows (10 codes per word) are a multiple of 8 bytes, so two rows
+// form a "super-row" of a multiple of 16 bytes and the codes come as two tensor
+// copies of 64 super-rows x CB3_WIN bytes: the window of the k-tile's words in the
+// even rows, then in the odd rows, each starting at the 16-byte boundary below
+// the k-tile's first word:
+//   [0, 64*CB3_WIN)              even rows 0, 2, ..., 126
+//   [64*CB3_WIN, 128*CB3_WIN)    odd rows 1, 3, ..., 127
+//   [128*CB3_WIN, +BM*16)        scale and bias words as above
+constexpr uint32_t CB3_WIN = 48;  // up to 12 bytes of offset + 8 words of 10 codes
 template <int KIND> struct RawLayout {
     static constexpr uint32_t RB = KIND == K_CB3 ? 32u : 8u * kind_bits(KIND);
     static constexpr uint32_t SC = RB;  // scale words at SC, bias words at SC + 8
     static constexpr uint32_t STRIDE = ((RB + 16u) / 16u) % 2u ? RB + 16u : RB + 32u;
-    static constexpr uint32_t TILE = BM * STRIDE;
-    static constexpr uint32_t TMA_SC = BM * RB;
-    static_assert(BM * RB + BM * 16u <= TILE, "TMA staging fits the cp.async staging area");
+    static constexpr uint32_t TMA_SC = KIND == K_CB3 ? BM * CB3_WIN : BM * RB;
+    static constexpr uint32_t TILE = KIND == K_CB3 ? BM * CB3_WIN + BM * 16u : BM * STRIDE;
+    static_assert(TMA_SC + BM * 16u <= TILE && BM * STRIDE <= TILE, "both stagings fit the area");
 };
 
 // Byte offset of 16-byte chunk c of staged row sr in the TMA code tile (the
@@ -533,7 +542,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
         return true;
     };
 
-    const bool tma = !PTRS && KIND != K_CB3 && P.tma != 0;
+    const bool tma = !PTRS && P.tma != 0;
     // x tiles: by the loader warps' 16-byte copies, or (f32 x) by tensor copies of rows
     // gathered beforehand; a compile-time XM_LOADERS for 16-bit x
     const uint32_t xmode = (XT == DT_F32) ? P.xmode : XM_LOADERS;
@@ -655,8 +664,14 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                 } else {  // K_CB3: codes from (kt*KT) % 10 + 32h of the window
                     const uint32_t c0 = (kt * KT) % 10u + 32u * h, wi = c0 / 10u;
                     sub = c0 - 10u * wi;
+                    const uint8_t *cr = rr;
+                    if (tma) {
+                        // the row's window in the even- or odd-row copy, from its 16-byte start
+                        const uint32_t odd = r & 1u, byte0 = odd * P.row_bytes + 4u * ((kt * KT) / 10u);
+                        cr = ct + odd * (64u * CB3_WIN) + (r >> 1) * CB3_WIN + (byte0 & 15u);
+                    }
 #pragma unroll
-                    for (int i = 0; i < 4; i++) wv[i] = *(const uint32_t *)(rr + 4u * (wi + i));
+                    for (int i = 0; i < 4; i++) wv[i] = *(const uint32_t *)(cr + 4u * (wi + i));
                 }
                 const uint32_t j0 = kt * KT, gh = (j0 + 32u * h) >> P.lg_gs;
                 if constexpr (KIND == K_NVFP4) {
@@ -829,7 +844,8 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
             if (xmode == XM_ROWS) ptx::prefetch_tensormap(&xmap);
             // bytes per k-tile: the codes' two 64-row boxes, the x box of BN rows (each row
             // one 128-byte swizzle line; twice for f32 x)
-            const uint32_t tx = (tma ? 2u * 64u * RB : 0u) + (xmode == XM_ROWS ? (uint32_t)(BT * B_TILE) : 0u);
+            constexpr uint32_t CODE_TX = KIND == K_CB3 ? 2u * 64u * CB3_WIN : 2u * 64u * RB;
+            const uint32_t tx = (tma ? CODE_TX : 0u) + (xmode == XM_ROWS ? (uint32_t)(BT * B_TILE) : 0u);
             uint32_t g = 0, last_s = 0, last_par = 0;
             bool any = false, ok = true;
             for (uint32_t i = 0; ok; i++) {
@@ -848,8 +864,16 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                     const uint32_t bar = loaded0 + 8 * s, raw = base + s * STAGE + RAW_OFF;
                     ptx::mbar_arrive_expect_tx(bar, tx);
                     if (tma) {
-                        ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
-                        ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
+                        if constexpr (KIND == K_CB3) {
+                            // super-row (e n + row0) / 2 onwards: the even rows' window, then the odd rows'
+                            const uint32_t byte0 = 4u * ((kt * KT) / 10u);
+                            const int32_t ys = (int32_t)((it.e * P.n + it.row0) / 2u);
+                            ptx::tma_load_2d(raw, &tmap, (int32_t)(byte0 & ~15u), ys, bar);
+                            ptx::tma_load_2d(raw + 64u * CB3_WIN, &tmap, (int32_t)((P.row_bytes + byte0) & ~15u), ys, bar);
+                        } else {
+                            ptx::tma_load_2d(raw, &tmap, (int32_t)(kt * RB), y0, bar);
+                            ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
+                        }
                     }
                     if (xmode == XM_ROWS) {
                         // gathered rows off + r0 .. + BN - 1: rows past the tile's pairs are other
@@ -1171,12 +1195,25 @@ bool x_tensor_map(const void *x, uint32_t rows, uint32_t k, uint32_t box_rows, C
 // cannot be staged this way (pointer tables, 3-bit rows, rows not a multiple of
 // 16 bytes, or no driver entry point).
 bool code_tensor_map(const QmmArgs &a, CUtensorMap *m) {
-    const uint32_t rb = ktile_row_bytes(a.kind);
-    if (!rb || a.packed_ptrs || a.row_bytes % 16u != 0 || (uintptr_t)a.packed % 16u != 0) return false;
     const uint64_t rows = (uint64_t)a.num_experts * a.n;
-    if (rows >= (1ull << 31)) return false;
+    if (a.packed_ptrs || (uintptr_t)a.packed % 16u != 0 || rows >= (1ull << 31)) return false;
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
     if (!enc) return false;
+    if (a.kind == K_CB3) {
+        // super-rows of two rows (a multiple of 16 bytes when a row is of 8), never
+        // straddling two experts (n even); not with a gated output, whose A tiles
+        // pair rows from the two halves
+        if (a.row_bytes % 8u != 0 || a.n % 2u != 0 || a.act >= 0) return false;
+        const cuuint64_t dims[2] = {2ull * a.row_bytes, rows / 2};
+        const cuuint64_t strides[1] = {2ull * a.row_bytes};
+        const cuuint32_t box[2] = {CB3_WIN, 64u};
+        const cuuint32_t estr[2] = {1u, 1u};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void *)a.packed, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    const uint32_t rb = ktile_row_bytes(a.kind);
+    if (!rb || a.row_bytes % 16u != 0) return false;
     const cuuint64_t dims[2] = {a.row_bytes, rows};
     const cuuint64_t strides[1] = {a.row_bytes};
     const cuuint32_t box[2] = {rb, 64u};
