@@ -75,6 +75,12 @@ def lib():
         L.oracle_act.restype = ctypes.c_double
         L.oracle_glu_elems.argtypes = [ctypes.c_void_p] * 2 + [u64, i32, ctypes.c_void_p]
         L.oracle_glu_elems.restype = None
+        L.oracle_e2m1_rne.argtypes = [ctypes.c_float]
+        L.oracle_e2m1_rne.restype = ctypes.c_uint8
+        L.oracle_e4m3_rne_satfinite.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_rne_satfinite.restype = ctypes.c_uint8
+        L.oracle_quantize_act_nvfp4.argtypes = [ctypes.c_void_p, i32, u32, u32] + [ctypes.c_void_p] * 4
+        L.oracle_quantize_act_nvfp4.restype = i32
         del u8p, u16p, u32p, dp, vp
         _lib = L
     return _lib
@@ -236,3 +242,41 @@ def route(ids: np.ndarray, num_experts: int, tile_rows: int):
     if nt < 0:
         raise ValueError("tile list overflow")
     return counts, offsets, sp[:R], tiles[:nt]
+
+
+# ------------------------------------------------- W4A4 (NVFP4 activations)
+
+DT_F64 = 3  # oracle-only x dtype: x given exactly as float64
+
+
+def e2m1_rne(v: float) -> int:
+    """Nearest E2M1 code of the f32 value v (ties to even, saturating at 6)."""
+    return int(lib().oracle_e2m1_rne(float(v)))
+
+
+def e4m3_rne_satfinite(v: float) -> int:
+    """Nearest finite E4M3 code of the f32 value v >= 0 (ties to even, saturating at 448)."""
+    return int(lib().oracle_e4m3_rne_satfinite(float(v)))
+
+
+def quantize_act_nvfp4(x: np.ndarray, x_dtype: int, m: int, k: int):
+    """Per-token NVFP4 quantisation of x [m, k] (raw storage): returns codes [m, k/2]
+    uint8 (element 2i in the low nibble), E4M3 block scales [m, k/16] uint8, the
+    per-token f32 scale [m] and the exact dequantised x^ [m, k] float64."""
+    x = np.ascontiguousarray(x)
+    codes = np.zeros((m, k // 2), np.uint8)
+    scales = np.zeros((m, k // 16), np.uint8)
+    g = np.zeros(m, np.float32)
+    xhat = np.zeros((m, k), np.float64)
+    if lib().oracle_quantize_act_nvfp4(_ptr(x), int(x_dtype), m, k, _ptr(codes), _ptr(scales), _ptr(g),
+                                       _ptr(xhat)) != 0:
+        raise ValueError("k must be a positive multiple of 16")
+    return codes, scales, g, xhat
+
+
+def w4a4_problem(P):
+    """The problem the W4A4 operation computes: P with x replaced by its NVFP4
+    quantisation x^ (float64, exact)."""
+    import dataclasses
+    _, _, _, xhat = quantize_act_nvfp4(P.x, P.x_dtype, P.m, P.k)
+    return dataclasses.replace(P, x=xhat, x_dtype=DT_F64)

@@ -58,7 +58,7 @@
 #include <string.h>
 
 enum { O_FMT_AFFINE = 0, O_FMT_CODEBOOK = 1, O_FMT_NVFP4 = 2, O_FMT_MXFP4 = 3 };
-enum { O_DT_F32 = 0, O_DT_BF16 = 1, O_DT_F16 = 2 };
+enum { O_DT_F32 = 0, O_DT_BF16 = 1, O_DT_F16 = 2, O_DT_F64 = 3 /* oracle-only: x given exactly */ };
 
 /* ---------------------------------------------------------------- decoders */
 
@@ -110,6 +110,7 @@ double oracle_e2m1_to_double(uint8_t c) {
 }
 
 static double x_at(const void *x, int dt, uint64_t idx) {
+    if (dt == O_DT_F64) return ((const double *)x)[idx];
     if (dt == O_DT_F32) return (double)((const float *)x)[idx];
     if (dt == O_DT_BF16) return oracle_bf16_to_double(((const uint16_t *)x)[idx]);
     return oracle_f16_to_double(((const uint16_t *)x)[idx]);
@@ -289,7 +290,7 @@ static int make_problem(problem_t *P, const void *x, const uint32_t *ids, const 
     if (fmt == O_FMT_CODEBOOK && bits != 2 && bits != 3 && bits != 4) return -1;
     if (fmt == O_FMT_NVFP4 && (bits != 4 || group_size != 16 || (k & 1))) return -1;
     if (fmt == O_FMT_MXFP4 && (bits != 4 || group_size != 32 || (k & 1))) return -1;
-    if (fmt < 0 || fmt > 3 || x_dtype < 0 || x_dtype > 2) return -1;
+    if (fmt < 0 || fmt > 3 || x_dtype < 0 || x_dtype > 3) return -1;
     P->x = x; P->ids = ids; P->packed = packed; P->scales = scales; P->aux = aux;
     P->m = m; P->k = k; P->n = n; P->group_size = group_size; P->bits = bits;
     P->n_expert_used = n_expert_used; P->num_experts = num_experts;
@@ -412,4 +413,103 @@ double oracle_act(int act, double g) {
 /* out[i] = act(gate[i]) * up[i] for i < count. */
 void oracle_glu_elems(const double *gate, const double *up, uint64_t count, int act, double *out) {
     for (uint64_t i = 0; i < count; i++) out[i] = oracle_act(act, gate[i]) * up[i];
+}
+
+/* ------------------------------------------- W4A4: NVFP4 activation quantisation
+ *
+ * The pages quantise weights to NVFP4 (E2M1 codes, one E4M3 scale per 16 values,
+ * a second-level f32 scale; spark_model helpers_a.rs) and name a grouped NVFP4
+ * GEMM whose activations are NVFP4 too (metrale helpers_b.rs,
+ * build_cutlass_grouped_sfb: per-expert swizzled scale tables for that path), but
+ * they do not say how activations are quantised. The reading here, per token t
+ * (one row of x), with every step in f32 as a GPU kernel would take it:
+ *   a   = max_j |x[t][j]|
+ *   g   = a / 2688   (2688 = 448 * 6: the largest E4M3 scale times the largest
+ *                     E2M1 value), or 0 when a = 0
+ *   per block b of 16 values (k a multiple of 16):
+ *     s_b  = E4M3(max_{j in b} |x[t][j]| / (6 * g)), nearest, ties to even,
+ *            values above 448 taken as 448; 0 when g = 0
+ *     d    = e4m3(s_b) * g
+ *     q_j  = E2M1(x[t][j] / d), nearest, ties to even, magnitudes above 6 taken
+ *            as 6, the sign of the quotient kept; code 0 when d = 0
+ *   x^[t][j] = e2m1(q_j) * e4m3(s_b) * g   (in double: exact)
+ * The matmul then takes x^ in place of x (oracle_qmm_id with O_DT_F64). */
+
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* Nearest E2M1 code of v (ties to the even code, |v| > 6 saturates to 6). The
+ * magnitude codes 0..7 are in increasing order; "even" is the code's low bit. */
+uint8_t oracle_e2m1_rne(float v) {
+    uint8_t sign = signbit(v) ? 8u : 0u;
+    double a = fabs((double)v);
+    if (a >= 6.0) return (uint8_t)(sign | 7u);  /* saturate (also where far-off distances tie) */
+    int best = 0;
+    for (int c = 1; c < 8; c++) {
+        double dc = fabs(E2M1_MAG[c] - a), db = fabs(E2M1_MAG[best] - a);
+        if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+    }
+    return (uint8_t)(sign | (uint8_t)best);
+}
+
+/* Nearest finite E4M3 code of v >= 0 (ties to the even code, values above 448
+ * saturate to 448), by scanning the 127 non-negative finite codes in order. */
+uint8_t oracle_e4m3_rne_satfinite(float v) {
+    double a = (double)v;
+    if (!(a > 0.0)) return 0u;
+    if (a >= 448.0) return 0x7Eu;  /* saturate */
+    int best = 0;
+    for (int c = 1; c <= 0x7E; c++) {
+        double dc = fabs(oracle_e4m3_to_double((uint8_t)c) - a);
+        double db = fabs(oracle_e4m3_to_double((uint8_t)best) - a);
+        if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+    }
+    return (uint8_t)best;
+}
+
+/* Quantise x [m, k] (x_dtype) per the reading above. Any output may be NULL:
+ * codes [m, k/2] (element 2i in the low nibble), scales [m, k/16] E4M3 bytes,
+ * gscale [m] f32, xhat [m, k] double. Returns -1 when k is not a multiple of 16. */
+int oracle_quantize_act_nvfp4(const void *x, int x_dtype, uint32_t m, uint32_t k, uint8_t *codes,
+                              uint8_t *scales, float *gscale, double *xhat) {
+    if (k == 0 || k % 16u != 0 || x_dtype < 0 || x_dtype > 2) return -1;
+    for (uint32_t t = 0; t < m; t++) {
+        float a = 0.0f;
+        for (uint32_t j = 0; j < k; j++) {
+            float v = fabsf((float)x_at(x, x_dtype, (uint64_t)t * k + j));
+            if (v > a) a = v;
+        }
+        volatile float g = a / 2688.0f;  /* f32 division, no contraction */
+        if (gscale) gscale[t] = g;
+        for (uint32_t b = 0; b < k / 16u; b++) {
+            float ab = 0.0f;
+            for (uint32_t i = 0; i < 16; i++) {
+                float v = fabsf((float)x_at(x, x_dtype, (uint64_t)t * k + 16u * b + i));
+                if (v > ab) ab = v;
+            }
+            uint8_t s = 0;
+            if (g > 0.0f) {
+                volatile float six_g = 6.0f * g;
+                volatile float q = ab / six_g;
+                s = oracle_e4m3_rne_satfinite(q);
+            }
+            if (scales) scales[(uint64_t)t * (k / 16u) + b] = s;
+            volatile float sv = (float)oracle_e4m3_to_double(s);
+            volatile float d = sv * g;
+            for (uint32_t i = 0; i < 16; i++) {
+                uint64_t idx = (uint64_t)t * k + 16u * b + i;
+                uint8_t c = 0;
+                if (d > 0.0f) {
+                    volatile float q = (float)x_at(x, x_dtype, idx) / d;
+                    c = oracle_e2m1_rne(q);
+                }
+                if (codes) {
+                    uint8_t *byte = codes + idx / 2;
+                    if (idx % 2 == 0) *byte = (uint8_t)((*byte & 0xF0u) | c);
+                    else *byte = (uint8_t)((*byte & 0x0Fu) | (uint8_t)(c << 4));
+                }
+                if (xhat) xhat[idx] = oracle_e2m1_to_double(c) * (double)sv * (double)g;
+            }
+        }
+    }
+    return 0;
 }

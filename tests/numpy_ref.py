@@ -116,6 +116,8 @@ def dequant_dense(P) -> np.ndarray:
 
 
 def x_f64(P) -> np.ndarray:
+    if P.x_dtype == 3:  # exact float64 x (the oracle's W4A4 problems)
+        return P.x.astype(np.float64)
     if P.x_dtype == DT_F32:
         return P.x.astype(np.float64)
     if P.x_dtype == DT_BF16:
