@@ -258,6 +258,40 @@ size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t n
 size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts,
                                     moe_dtype x_dtype);
 
+/*
+ * W4A4: the operation with NVFP4 activations (spark_model helpers_a.rs quantises
+ * the routed weights to NVFP4; metrale helpers_b.rs, build_cutlass_grouped_sfb,
+ * names the grouped NVFP4 GEMM whose activations are NVFP4 as well). The pages do
+ * not say how activations are quantised; the reading implemented, per token t of x,
+ * every step in f32:
+ *   g_t  = max_j |x[t][j]| / 2688        (2688 = 448 * 6; 0 for an all-zero token)
+ *   s_b  = E4M3(max over the 16 values of block b of |x| / (6 g_t)), round to nearest
+ *          even, saturating at 448
+ *   q_j  = E2M1(x[t][j] / (e4m3(s_b) g_t)), round to nearest even, saturating at 6
+ *   x^   = e2m1(q_j) * e4m3(s_b) * g_t
+ * and the result is moe_qmm_id with x^ in place of x.
+ *
+ * moe_quantize_act_nvfp4 -- the quantisation alone, on `stream`: x [m, k] (x_dtype,
+ *   device), k a multiple of 16 (else MOE_ERR_UNSUPPORTED). Outputs, each optional
+ *   (NULL): codes [m, k/2] bytes, element 2i in the low nibble (8-byte aligned);
+ *   scales [m, k/16] E4M3 bytes; gscale [m] f32; xhat [m, k] f32 (x^ rounded once
+ *   to f32).
+ * moe_qmm_id_w4a4 -- arguments as moe_qmm_id_path (any weight format; the path
+ *   argument may carry launch flags). The workspace holds x^ (f32) followed by the
+ *   operation's own workspace: at least moe_qmm_id_workspace_bytes_w4a4(m, k,
+ *   n_expert_used, num_experts) bytes for the fastest layout, and never less than
+ *   round_up(m*k*4, 256) + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts)
+ *   (else MOE_ERR_WORKSPACE_TOO_SMALL). Errors as moe_qmm_id.
+ */
+size_t moe_qmm_id_workspace_bytes_w4a4(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts);
+moe_status moe_quantize_act_nvfp4(const void *x, uint32_t m, uint32_t k, moe_dtype x_dtype, uint8_t *codes,
+                                  uint8_t *scales, float *gscale, float *xhat, moe_stream_t stream);
+moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                           const void *aux, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
+                           uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts,
+                           moe_dtype x_dtype, moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                           moe_stream_t stream, moe_path path);
+
 /* Bytes of one packed weight row (mlx-native quantized_matmul_id.rs,
  * expert_weight_bytes per row): AFFINE 4/8 and CODEBOOK ceil(k / (32/bits)) * 4,
  * AFFINE 6 ceil(k / 4) * 3, NVFP4 k / 2. Returns 0 for an invalid (fmt, bits). */

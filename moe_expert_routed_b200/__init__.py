@@ -78,6 +78,12 @@ def lib() -> ctypes.CDLL:
         L.moe_qmm_id_workspace_bytes_k.argtypes = [u32] * 4 + [i32]
         L.moe_qmm_id_workspace_bytes_k.restype = sz
         L.moe_qmm_test_x_copies.argtypes = [i32]
+        L.moe_qmm_id_w4a4.argtypes = L.moe_qmm_id.argtypes + [i32]
+        L.moe_qmm_id_w4a4.restype = i32
+        L.moe_quantize_act_nvfp4.argtypes = [vp, u32, u32, i32, vp, vp, vp, vp, vp]
+        L.moe_quantize_act_nvfp4.restype = i32
+        L.moe_qmm_id_workspace_bytes_w4a4.argtypes = [u32] * 4
+        L.moe_qmm_id_workspace_bytes_w4a4.restype = sz
         L.moe_qmm_test_x_copies.restype = i32
         L.moe_packed_row_bytes.argtypes = [i32, u32, u32]
         L.moe_packed_row_bytes.restype = sz
@@ -380,3 +386,56 @@ def route(ids: torch.Tensor, num_experts: int, tile_rows: int,
 def poll_error(workspace: torch.Tensor) -> int:
     """Synchronise the current stream, read and clear the device error word."""
     return int(lib().moe_qmm_id_poll_error(workspace.data_ptr(), _stream_ptr(workspace.device)))
+
+
+def quantize_act_nvfp4(x: torch.Tensor):
+    """moe_quantize_act_nvfp4: per-token NVFP4 quantisation of x [m, k] (f32 / bf16 /
+    f16, k a multiple of 16) on the current stream. Returns (codes [m, k/2] uint8,
+    element 2i in the low nibble; E4M3 scales [m, k/16] uint8; per-token scales [m]
+    f32; x^ [m, k] f32)."""
+    if x.dim() != 2 or not x.is_cuda or not x.is_contiguous() or x.dtype not in _TORCH_DT:
+        raise ValueError("quantize_act_nvfp4: x must be a contiguous 2-D f32/bf16/f16 CUDA tensor")
+    m, k = x.shape
+    dev = x.device
+    codes = torch.empty((m, k // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((m, k // 16), dtype=torch.uint8, device=dev)
+    g = torch.empty(m, dtype=torch.float32, device=dev)
+    xhat = torch.empty((m, k), dtype=torch.float32, device=dev)
+    st = lib().moe_quantize_act_nvfp4(x.data_ptr(), m, k, _TORCH_DT[x.dtype], codes.data_ptr(),
+                                      scales.data_ptr(), g.data_ptr(), xhat.data_ptr(), _stream_ptr(dev))
+    if st != MOE_OK:
+        raise MoeError(st, "moe_quantize_act_nvfp4")
+    return codes, scales, g, xhat
+
+
+def workspace_bytes_w4a4(m: int, k: int, n_expert_used: int, num_experts: int) -> int:
+    return int(lib().moe_qmm_id_workspace_bytes_w4a4(m, k, n_expert_used, num_experts))
+
+
+def qmm_id_w4a4(x: torch.Tensor, ids: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                aux: torch.Tensor, *, n: int, group_size: int, bits: int, fmt: int, num_experts: int,
+                out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float32,
+                workspace: torch.Tensor | None = None, path: str = "auto", launch: str | None = None) -> torch.Tensor:
+    """moe_qmm_id_w4a4: the operation with x quantised per token to NVFP4 first
+    (see moe_quantize_act_nvfp4 in include/moe_qmm.h for the quantisation); the
+    other arguments and checks as qmm_id."""
+    device = x.device
+    m, k, n_expert_used, out_n = _validate_only(x, ids, packed, scales, aux, n=n, group_size=group_size,
+                                                bits=bits, fmt=fmt, num_experts=num_experts, out=out,
+                                                expert_bias=None, act=None, launch=launch)
+    if out is None:
+        out = torch.empty((m, n_expert_used, out_n), dtype=out_dtype, device=device)
+    if workspace is None:
+        nbytes = workspace_bytes_w4a4(m, k, n_expert_used, num_experts)
+        if nbytes == 0:
+            raise ValueError("sizes overflow the workspace layout")
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    else:
+        _check_dev(workspace, "workspace", device)
+    st = lib().moe_qmm_id_w4a4(
+        x.data_ptr(), ids.data_ptr(), packed.data_ptr(), scales.data_ptr(), aux.data_ptr(), out.data_ptr(),
+        m, k, n, group_size, bits, fmt, n_expert_used, num_experts, _TORCH_DT[x.dtype], _TORCH_DT[out.dtype],
+        workspace.data_ptr(), _nbytes(workspace), _stream_ptr(device), _PATHS[path] | _LAUNCH[launch])
+    if st != MOE_OK:
+        raise MoeError(st, "moe_qmm_id_w4a4")
+    return out

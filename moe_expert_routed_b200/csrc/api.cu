@@ -282,6 +282,46 @@ moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed
                stream, path, PtrTables{nullptr, nullptr, nullptr}, (int)act);
 }
 
+size_t moe_qmm_id_workspace_bytes_w4a4(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts) {
+    const size_t rest = moe_qmm_id_workspace_bytes_k(m, k, n_expert_used, num_experts, MOE_F32);
+    if (!rest) return 0;
+    return (size_t)al256((uint64_t)m * k * 4ull) + rest;
+}
+
+moe_status moe_quantize_act_nvfp4(const void *x, uint32_t m, uint32_t k, moe_dtype x_dtype, uint8_t *codes,
+                                  uint8_t *scales, float *gscale, float *xhat, moe_stream_t stream) {
+    if (!x || m == 0 || k == 0 || (int)x_dtype < 0 || (int)x_dtype > 2) return MOE_ERR_INVALID_ARGUMENT;
+    if (((uintptr_t)codes & 7u) || ((uintptr_t)xhat & 3u) || ((uintptr_t)gscale & 3u)) return MOE_ERR_INVALID_ARGUMENT;
+    if (k % 16u != 0) return MOE_ERR_UNSUPPORTED;
+    return moe::launch_quant_act(x, (int)x_dtype, m, k, codes, scales, gscale, xhat, (cudaStream_t)stream) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packed, const void *scales,
+                           const void *aux, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
+                           uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts,
+                           moe_dtype x_dtype, moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                           moe_stream_t stream, moe_path path) {
+    moe_status v = moe::validate_call(x, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt,
+                                      n_expert_used, num_experts, x_dtype, out_dtype);
+    if (v != MOE_OK) return v;
+    if (k % 16u != 0) return MOE_ERR_UNSUPPORTED;
+    if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
+    // x^ (f32) first, then the operation's own workspace
+    const size_t xh = (size_t)al256((uint64_t)m * k * 4ull);
+    if (workspace_bytes < xh + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    float *xhat = (float *)workspace;
+    if (moe::launch_quant_act(x, (int)x_dtype, m, k, nullptr, nullptr, nullptr, xhat, (cudaStream_t)stream) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return moe_qmm_id_path(xhat, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt, n_expert_used,
+                           num_experts, MOE_F32, out_dtype, (uint8_t *)workspace + xh, workspace_bytes - xh, stream,
+                           path);
+}
+
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,
                       const void *aux, void *out, uint32_t m, uint32_t k, uint32_t n,
                       uint32_t group_size, uint32_t bits, moe_fmt fmt, uint32_t n_expert_used,

@@ -90,6 +90,11 @@ cudaError_t launch_gemv_routed(const QmmArgs &a, const uint32_t *counts, const u
 // [0, R) and the bf16 roundings of the remainders in rows [R, 2R); k % 8 == 0.
 cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_pairs, uint32_t R, uint32_t k,
                             uint32_t n_expert_used, uint16_t *xg, cudaStream_t st);
+// W4A4 activations: per-token NVFP4 quantisation of x [m, k] (k % 16 == 0; any output
+// may be null): codes [m, k/2] (8-byte aligned), E4M3 scales [m, k/16], per-token
+// f32 scales [m], and x^ [m, k] f32.
+cudaError_t launch_quant_act(const void *x, int x_dtype, uint32_t m, uint32_t k, uint8_t *codes, uint8_t *scales,
+                             float *gscale, float *xhat, cudaStream_t st);
 // Bytes of the gathered x rows (0 when the grouped GEMM does not use them: 16-bit x
 // is gathered by the GEMM's tensor copies straight from x).
 uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype);
