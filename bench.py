@@ -528,6 +528,62 @@ def grouped_tile_rows(P) -> int:
     return 64
 
 
+def w4a4_entry(pk: dict) -> dict:
+    """The prefill workload with W4A4 (x quantised per token to NVFP4 first,
+    moe_qmm_id_w4a4): per-call time from a CUDA graph of GRAPH_CALLS calls (median of
+    REPEATS replays), and the activation quantisation alone timed the same way."""
+    import moe_expert_routed_b200 as M
+    from workloads import config_problem
+    from workloads.torch_io import to_device
+
+    P = config_problem("prefill")
+    d = to_device(P)
+    ws = torch.zeros(M.workspace_bytes_w4a4(P.m, P.k, P.n_expert_used, P.num_experts), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((P.m, P.n_expert_used, P.n), dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty((P.m, P.k // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((P.m, P.k // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(P.m, dtype=torch.float32, device="cuda")
+    xhat = torch.empty((P.m, P.k), dtype=torch.float32, device="cuda")
+    L = M.lib()
+
+    def call(_i):
+        M.qmm_id_w4a4(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], n=P.n, group_size=P.group_size,
+                      bits=P.bits, fmt=P.fmt, num_experts=P.num_experts, out=out, workspace=ws)
+
+    def quant(_i):
+        st = L.moe_quantize_act_nvfp4(d["x"].data_ptr(), P.m, P.k, 1, codes.data_ptr(), scales.data_ptr(),
+                                      g.data_ptr(), xhat.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        if st != 0:
+            raise RuntimeError(f"moe_quantize_act_nvfp4: status {st}")
+
+    call(0)
+    torch.cuda.synchronize()
+    gc = capture_graph(call, GRAPH_CALLS)
+    rc = per_call(gc, GRAPH_CALLS)
+    del gc
+    gq = capture_graph(quant, GRAPH_CALLS)
+    rq = per_call(gq, GRAPH_CALLS)
+    del gq
+    ids = P.ids.reshape(-1)
+    flops = 2.0 * int((ids < P.num_experts).sum()) * P.n * P.k
+    us = rc["s"] * 1e6
+    tf = flops / us / 1e6
+    ent = {
+        "workload": "prefill with W4A4: x quantised per token to NVFP4 (E2M1 codes, E4M3 scales per 16, f32 "
+                    "per-token scale), then the operation on the dequantised x (f32 operands split into bf16 "
+                    "halves on the tensor cores)",
+        "us_per_call": us, "quantize_us": rq["s"] * 1e6, "TFLOP_per_s": tf,
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tf / pk["bf16_tflops"], "peak_source": pk["source"] + " (bf16_tflops burst)"},
+        "repeats_us": rc["repeats_us"],
+        "timing": f"CUDA graph of {GRAPH_CALLS} calls, median of {REPEATS} replays",
+    }
+    del d, out, ws, codes, scales, g, xhat
+    torch.cuda.empty_cache()
+    return ent
+
+
 def grouped_entry(name: str, pk: dict) -> dict:
     """One grouped-path workload (routing prologue + tcgen05 grouped GEMM), inputs
     resident in HBM: per-call time from a CUDA graph of GRAPH_CALLS calls (median
@@ -776,6 +832,7 @@ def run_ours(args, dist: Dist):
         # the other workloads and the decode m-sweep, on this GPU, outside the timed region
         sampler = clocks_sampler(dev)
         line["per_config"] = {name: grouped_entry(name, pk) for name in ("canvas", "prefill", "skewed")}
+        line["per_config"]["prefill_w4a4"] = w4a4_entry(pk)
         line["sweep"] = decode_sweep(pk)
         line["per_config_clocks"] = clocks_summary(sampler)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:

@@ -273,15 +273,17 @@ size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_us
  *
  * moe_quantize_act_nvfp4 -- the quantisation alone, on `stream`: x [m, k] (x_dtype,
  *   device), k a multiple of 16 (else MOE_ERR_UNSUPPORTED). Outputs, each optional
- *   (NULL): codes [m, k/2] bytes, element 2i in the low nibble (8-byte aligned);
+ *   (NULL): codes [m, k/2] bytes, element 2i in the low nibble (4-byte aligned);
  *   scales [m, k/16] E4M3 bytes; gscale [m] f32; xhat [m, k] f32 (x^ rounded once
- *   to f32).
+ *   to f32; 16-byte aligned).
  * moe_qmm_id_w4a4 -- arguments as moe_qmm_id_path (any weight format; the path
- *   argument may carry launch flags). The workspace holds x^ (f32) followed by the
- *   operation's own workspace: at least moe_qmm_id_workspace_bytes_w4a4(m, k,
- *   n_expert_used, num_experts) bytes for the fastest layout, and never less than
- *   round_up(m*k*4, 256) + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts)
- *   (else MOE_ERR_WORKSPACE_TOO_SMALL). Errors as moe_qmm_id.
+ *   argument may carry launch flags). The CUDA-core paths take x^ as f32 x; the
+ *   grouped GEMM takes e2m1(q) * e4m3(s_b) as bf16 (exact) and multiplies each
+ *   output by its token's g_t before the single rounding. The workspace holds x^
+ *   (f32 [m, k]), the bf16 values [m, k] and g [m] (each section rounded up to 256
+ *   bytes), then the operation's own workspace: at least
+ *   moe_qmm_id_workspace_bytes_w4a4(m, k, n_expert_used, num_experts) bytes (else
+ *   MOE_ERR_WORKSPACE_TOO_SMALL). Errors as moe_qmm_id.
  */
 size_t moe_qmm_id_workspace_bytes_w4a4(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts);
 moe_status moe_quantize_act_nvfp4(const void *x, uint32_t m, uint32_t k, moe_dtype x_dtype, uint8_t *codes,

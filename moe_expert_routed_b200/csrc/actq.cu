@@ -14,7 +14,7 @@
 //   x^  = e2m1(q_j) * e4m3(s_b) * g
 // The conversions are the hardware's round-to-nearest-even, satfinite ones.
 //
-// One CTA per token: a block-wide maximum, then one thread per 16-value block.
+// One CTA per token: a block-wide maximum, then two lanes per 16-value block.
 #include "common.cuh"
 #include "internal.h"
 
@@ -48,17 +48,49 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
     return r;
 }
 
+// Eight consecutive values of x from element i (i a multiple of 8): vector loads
+// when the row is 16-byte aligned, else one at a time.
+__device__ __forceinline__ void load8(const void *x, int dt, size_t i, bool vec, float (&v)[8]) {
+    if (vec && dt == DT_F32) {
+        const float4 a = __ldg((const float4 *)x + i / 4), b = __ldg((const float4 *)x + i / 4 + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else if (vec) {
+        const uint4 q = __ldg((const uint4 *)x + i / 8);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            v[2 * j] = dt == DT_BF16 ? bf16_bits_to_f32(w[j] & 0xFFFFu) : f16_bits_to_f32(w[j] & 0xFFFFu);
+            v[2 * j + 1] = dt == DT_BF16 ? bf16_bits_to_f32(w[j] >> 16) : f16_bits_to_f32(w[j] >> 16);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; j++) v[j] = load_x(x, dt, i + j);
+    }
+}
+
+// One CTA per token. Pass 1: the row's maximum. Pass 2: lanes 2p and 2p+1 of a warp
+// take the two halves of one 16-value block (8 values each), so loads and stores
+// are contiguous across the warp; every thread runs the same number of passes so
+// that the pairs' shuffles always have both lanes.
 __global__ void __launch_bounds__(AQ_THREADS)
 quant_act_nvfp4(const void *__restrict__ x, int x_dtype, uint32_t k, uint8_t *__restrict__ codes,
-                uint8_t *__restrict__ scales, float *__restrict__ gscale, float *__restrict__ xhat) {
+                uint8_t *__restrict__ scales, float *__restrict__ gscale, float *__restrict__ xhat,
+                uint16_t *__restrict__ x16) {
     __shared__ float red[AQ_THREADS / 32];
-    const uint32_t t = blockIdx.x, tid = threadIdx.x;
+    const uint32_t t = blockIdx.x, tid = threadIdx.x, lane = tid & 31u;
     const size_t row = (size_t)t * k;
+    const uint32_t k8 = k / 8u;  // 8-value chunks (even: k is a multiple of 16)
+    const bool vec = ((uintptr_t)x & 15u) == 0;
     float a = 0.f;
-    for (uint32_t j = tid; j < k; j += AQ_THREADS) a = fmaxf(a, fabsf(load_x(x, x_dtype, row + j)));
+    for (uint32_t c = tid; c < k8; c += AQ_THREADS) {
+        float v[8];
+        load8(x, x_dtype, row + 8u * c, vec, v);
+#pragma unroll
+        for (int j = 0; j < 8; j++) a = fmaxf(a, fabsf(v[j]));
+    }
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, d));
-    if ((tid & 31u) == 0) red[tid >> 5] = a;
+    if (lane == 0) red[tid >> 5] = a;
     __syncthreads();
     a = red[0];
 #pragma unroll
@@ -66,38 +98,57 @@ quant_act_nvfp4(const void *__restrict__ x, int x_dtype, uint32_t k, uint8_t *__
     const float g = __fdiv_rn(a, 2688.0f);
     if (tid == 0 && gscale) gscale[t] = g;
     const float six_g = __fmul_rn(6.0f, g);
-    for (uint32_t b = tid; b < k / 16u; b += AQ_THREADS) {
-        float v[16], ab = 0.f;
+    for (uint32_t c0 = 0; c0 < k8; c0 += AQ_THREADS) {
+        const uint32_t c = c0 + tid;
+        const bool valid = c < k8;
+        float v[8], ab = 0.f;
+        if (valid) {
+            load8(x, x_dtype, row + 8u * c, vec, v);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            v[i] = load_x(x, x_dtype, row + 16u * b + i);
-            ab = fmaxf(ab, fabsf(v[i]));
+            for (int j = 0; j < 8; j++) v[j] = 0.f;
         }
+#pragma unroll
+        for (int j = 0; j < 8; j++) ab = fmaxf(ab, fabsf(v[j]));
+        ab = fmaxf(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 1));  // the block's other half
+        if (!valid) continue;
         const uint32_t s = g > 0.f ? e4m3_rn_sat(__fdiv_rn(ab, six_g)) : 0u;
-        if (scales) scales[(size_t)t * (k / 16u) + b] = (uint8_t)s;
+        if (scales && (c & 1u) == 0) scales[row / 16u + c / 2u] = (uint8_t)s;
         const float sv = e4m3_value(s);
         const float d = __fmul_rn(sv, g);
-        uint32_t packed[2] = {0u, 0u};
+        uint32_t cw = 0;
+        float vs[8];
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            const uint32_t c2 = d > 0.f ? e2m1x2_rn_sat(__fdiv_rn(v[i], d), __fdiv_rn(v[i + 1], d)) : 0u;
-            packed[i / 8] |= c2 << (8 * ((i % 8) / 2));
-            if (xhat) {
-                xhat[row + 16u * b + i] = __fmul_rn(__fmul_rn(e2m1_to_f32(c2 & 15u), sv), g);
-                xhat[row + 16u * b + i + 1] = __fmul_rn(__fmul_rn(e2m1_to_f32(c2 >> 4), sv), g);
-            }
+        for (int j = 0; j < 8; j += 2) {
+            const uint32_t c2 = d > 0.f ? e2m1x2_rn_sat(__fdiv_rn(v[j], d), __fdiv_rn(v[j + 1], d)) : 0u;
+            cw |= c2 << (4 * j);
+            vs[j] = e2m1_to_f32(c2 & 15u) * sv;  // exact: at most 6 significant bits
+            vs[j + 1] = e2m1_to_f32(c2 >> 4) * sv;
         }
-        if (codes) *(uint2 *)(codes + (row + 16u * b) / 2) = make_uint2(packed[0], packed[1]);
+        if (codes) *(uint32_t *)(codes + (row + 8u * c) / 2) = cw;
+        if (xhat) {
+            float4 *o = (float4 *)(xhat + row + 8u * c);
+            o[0] = make_float4(__fmul_rn(vs[0], g), __fmul_rn(vs[1], g), __fmul_rn(vs[2], g), __fmul_rn(vs[3], g));
+            o[1] = make_float4(__fmul_rn(vs[4], g), __fmul_rn(vs[5], g), __fmul_rn(vs[6], g), __fmul_rn(vs[7], g));
+        }
+        if (x16) {
+            uint32_t h[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                h[j] = (__float_as_uint(vs[2 * j]) >> 16) | (__float_as_uint(vs[2 * j + 1]) & 0xFFFF0000u);
+            *(uint4 *)(x16 + row + 8u * c) = make_uint4(h[0], h[1], h[2], h[3]);
+        }
     }
 }
 
 }  // namespace
 
 cudaError_t launch_quant_act(const void *x, int x_dtype, uint32_t m, uint32_t k, uint8_t *codes, uint8_t *scales,
-                             float *gscale, float *xhat, cudaStream_t st) {
+                             float *gscale, float *xhat, uint16_t *x16, cudaStream_t st) {
     if (m == 0) return cudaSuccess;
-    if (k == 0 || k % 16u != 0 || ((uintptr_t)codes & 7u)) return cudaErrorInvalidValue;
-    quant_act_nvfp4<<<m, AQ_THREADS, 0, st>>>(x, x_dtype, k, codes, scales, gscale, xhat);
+    if (k == 0 || k % 16u != 0 || ((uintptr_t)codes & 3u) || ((uintptr_t)xhat & 15u) || ((uintptr_t)x16 & 15u))
+        return cudaErrorInvalidValue;
+    quant_act_nvfp4<<<m, AQ_THREADS, 0, st>>>(x, x_dtype, k, codes, scales, gscale, xhat, x16);
     return cudaGetLastError();
 }
 

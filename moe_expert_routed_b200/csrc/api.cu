@@ -41,6 +41,11 @@ bool ws_layout(uint64_t R, uint32_t E, WsLayout *L) {
     return true;
 }
 
+// W4A4 workspace ahead of the operation's own: x^ f32 [m, k], bf16 [m, k], f32 [m].
+size_t w4a4_front_bytes(uint32_t m, uint32_t k) {
+    return al256((uint64_t)m * k * 4ull) + al256((uint64_t)m * k * 2ull) + al256((uint64_t)m * 4ull);
+}
+
 uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype) {
     if (k % 8u != 0 || x_dtype != DT_F32) return 0;
     return al256(R * k * 4ull);
@@ -140,7 +145,8 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
                const void *bias, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
                uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace, size_t workspace_bytes,
-               moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}, int act = -1) {
+               moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}, int act = -1,
+               const uint16_t *w4a4_x16 = nullptr, const float *w4a4_scale = nullptr) {
     moe_status v = validate(x, ids, pt.packed ? (const void *)pt.packed : packed,
                             pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
                             fmt, n_expert_used, num_experts, x_dtype, out_dtype);
@@ -174,6 +180,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     a.launch_flags = launch_flags;
     a.fault_wait_ns = g_fault_wait_ns.load(std::memory_order_relaxed);
     a.x_copies = g_x_copies.load(std::memory_order_relaxed);
+    a.tok_scale = nullptr;
 
     uint8_t *ws = (uint8_t *)workspace;
     uint32_t *err = (uint32_t *)(ws + L.err);
@@ -198,6 +205,17 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         else if (routable && gemm_supported(a)) choice = GROUPED;
         else if (routable) choice = ROUTED_GEMV;
         else return MOE_ERR_UNSUPPORTED;
+    }
+
+    // W4A4 on the grouped GEMM: bf16 e2m1(q) * e4m3(s) (exact) as the B operand and the
+    // per-token factor in the epilogue, instead of the f32 x^ the CUDA-core paths take
+    if (choice == GROUPED && w4a4_x16 && w4a4_scale) {
+        a.x = w4a4_x16;
+        a.x_dtype = DT_BF16;
+        x = w4a4_x16;
+        x_dtype = MOE_BF16;
+        a.tok_scale = w4a4_scale;
+        if (!gemm_supported(a)) return MOE_ERR_UNSUPPORTED;
     }
 
     cudaError_t ce;
@@ -283,17 +301,19 @@ moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed
 }
 
 size_t moe_qmm_id_workspace_bytes_w4a4(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts) {
-    const size_t rest = moe_qmm_id_workspace_bytes_k(m, k, n_expert_used, num_experts, MOE_F32);
+    const size_t rest = moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts);
     if (!rest) return 0;
-    return (size_t)al256((uint64_t)m * k * 4ull) + rest;
+    return moe::w4a4_front_bytes(m, k) + rest;
 }
 
 moe_status moe_quantize_act_nvfp4(const void *x, uint32_t m, uint32_t k, moe_dtype x_dtype, uint8_t *codes,
                                   uint8_t *scales, float *gscale, float *xhat, moe_stream_t stream) {
     if (!x || m == 0 || k == 0 || (int)x_dtype < 0 || (int)x_dtype > 2) return MOE_ERR_INVALID_ARGUMENT;
-    if (((uintptr_t)codes & 7u) || ((uintptr_t)xhat & 3u) || ((uintptr_t)gscale & 3u)) return MOE_ERR_INVALID_ARGUMENT;
+    if (((uintptr_t)codes & 3u) || ((uintptr_t)xhat & 15u) || ((uintptr_t)gscale & 3u))
+        return MOE_ERR_INVALID_ARGUMENT;
     if (k % 16u != 0) return MOE_ERR_UNSUPPORTED;
-    return moe::launch_quant_act(x, (int)x_dtype, m, k, codes, scales, gscale, xhat, (cudaStream_t)stream) ==
+    return moe::launch_quant_act(x, (int)x_dtype, m, k, codes, scales, gscale, xhat, nullptr,
+                                 (cudaStream_t)stream) ==
                    cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
@@ -309,17 +329,21 @@ moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packe
     if (v != MOE_OK) return v;
     if (k % 16u != 0) return MOE_ERR_UNSUPPORTED;
     if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
-    // x^ (f32) first, then the operation's own workspace
-    const size_t xh = (size_t)al256((uint64_t)m * k * 4ull);
-    if (workspace_bytes < xh + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
+    // x^ (f32), the bf16 values without the per-token factor, the per-token factors,
+    // then the operation's own workspace
+    const size_t front = moe::w4a4_front_bytes(m, k);
+    if (workspace_bytes < front + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
         return MOE_ERR_WORKSPACE_TOO_SMALL;
-    float *xhat = (float *)workspace;
-    if (moe::launch_quant_act(x, (int)x_dtype, m, k, nullptr, nullptr, nullptr, xhat, (cudaStream_t)stream) !=
+    uint8_t *w = (uint8_t *)workspace;
+    float *xhat = (float *)w;
+    uint16_t *x16 = (uint16_t *)(w + moe::al256((uint64_t)m * k * 4ull));
+    float *g = (float *)(w + moe::al256((uint64_t)m * k * 4ull) + moe::al256((uint64_t)m * k * 2ull));
+    if (moe::launch_quant_act(x, (int)x_dtype, m, k, nullptr, nullptr, g, xhat, x16, (cudaStream_t)stream) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
-    return moe_qmm_id_path(xhat, ids, packed, scales, aux, out, m, k, n, group_size, bits, fmt, n_expert_used,
-                           num_experts, MOE_F32, out_dtype, (uint8_t *)workspace + xh, workspace_bytes - xh, stream,
-                           path);
+    return moe::run(xhat, ids, packed, scales, aux, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
+                    num_experts, MOE_F32, out_dtype, MOE_F32, w + front, workspace_bytes - front, stream, path,
+                    {nullptr, nullptr, nullptr}, -1, x16, g);
 }
 
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,

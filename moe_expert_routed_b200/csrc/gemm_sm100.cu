@@ -114,6 +114,8 @@ struct GemmParams {
     // second tensor map
     uint32_t xmode;
     uint32_t xg_R;
+    // W4A4: per-token factor of every output (null: none)
+    const float *tok_scale;
     uint32_t *work_counter; // items claimed beyond each CTA's first (zeroed by the routing prologue)
     // failure-detection test hook: non-zero makes the MMA warp first wait this long on
     // a barrier nothing completes (so the CTA aborts); 0 in normal operation
@@ -995,6 +997,12 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
 #pragma unroll
                 for (int i = 0; i < 16; i++) pr[i] = c0 + i < it.nt ? __ldg(pairs + c0 + i) : 0u;
                 ptx::tmem_wait_ld();
+                if (P.tok_scale) {
+                    // W4A4: the token's factor, applied to the fp32 sum before the bias
+#pragma unroll
+                    for (int i = 0; i < 16; i++)
+                        v[i] = __float_as_uint(__uint_as_float(v[i]) * __ldg(P.tok_scale + pr[i] / P.n_expert_used));
+                }
                 if constexpr (GLU) {
                     // even lanes hold gate rows, the next lane the matching up row
 #pragma unroll
@@ -1283,6 +1291,7 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     memset(&xmap, 0, sizeof(xmap));
     const uint32_t R = a.m * a.n_expert_used;
     P.xg_R = R;
+    P.tok_scale = a.tok_scale;
     // f32 x: tensor copies of the rows gathered and split after routing, when the
     // workspace holds them (and no test asks for the loader copies)
     P.xmode = (a.x_dtype == DT_F32 && !a.x_copies && xg && x_tensor_map(xg, R * 2u, a.k, pl.bn, &xmap))

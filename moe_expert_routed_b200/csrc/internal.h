@@ -78,6 +78,9 @@ struct QmmArgs {
     // completes, giving up after this many ns; 0 in normal operation
     uint64_t fault_wait_ns;
     int x_copies;  // 1: the grouped GEMM's loader warps copy x rows (test hook)
+    // W4A4 on the grouped GEMM: the GEMM takes x as these bf16 values and multiplies
+    // each output by tok_scale[token] (null: x as given, no factor)
+    const float *tok_scale;
 };
 
 // CUDA-core GEMV with routing fused in (R <= 64).
@@ -93,8 +96,9 @@ cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_p
 // W4A4 activations: per-token NVFP4 quantisation of x [m, k] (k % 16 == 0; any output
 // may be null): codes [m, k/2] (8-byte aligned), E4M3 scales [m, k/16], per-token
 // f32 scales [m], and x^ [m, k] f32.
+// x16 (optional) [m, k]: e2m1(q) * e4m3(s) as bf16 (exact), x^ without the per-token factor.
 cudaError_t launch_quant_act(const void *x, int x_dtype, uint32_t m, uint32_t k, uint8_t *codes, uint8_t *scales,
-                             float *gscale, float *xhat, cudaStream_t st);
+                             float *gscale, float *xhat, uint16_t *x16, cudaStream_t st);
 // Bytes of the gathered x rows (0 when the grouped GEMM does not use them: 16-bit x
 // is gathered by the GEMM's tensor copies straight from x).
 uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype);

@@ -40,12 +40,18 @@ def _x(rng, m, k, xd):
 
 
 @pytest.mark.parametrize("xd", [DT_F32, DT_BF16, DT_F16])
-@pytest.mark.parametrize("m,k", [(1, 2816), (7, 512), (64, 4096)])
-def test_quantize_matches_oracle(xd, m, k):
+@pytest.mark.parametrize("m,k,offset", [(1, 2816, 0), (7, 512, 0), (64, 4096, 0), (5, 256, 1)])
+def test_quantize_matches_oracle(xd, m, k, offset):
     rng = np.random.default_rng(1000 + m + k + xd)
     xb = _x(rng, m, k, xd)
     dt = {DT_F32: torch.float32, DT_BF16: torch.bfloat16, DT_F16: torch.float16}[xd]
     xt = torch.from_numpy(xb.view(np.float32) if xd == DT_F32 else xb.view(np.int16)).view(dt).cuda()
+    if offset:
+        # x one element off a 16-byte boundary: the kernel's element-wise loads
+        big = torch.zeros(m * k + offset, dtype=dt, device="cuda")
+        big[offset:] = xt.reshape(-1)
+        xt = big[offset:].view(m, k)
+        assert xt.data_ptr() % 16 != 0
     codes, scales, g, xhat = M.quantize_act_nvfp4(xt)
     torch.cuda.synchronize()
     o_codes, o_scales, o_g, o_xhat = oracle.quantize_act_nvfp4(xb, xd, m, k)
