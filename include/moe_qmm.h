@@ -245,16 +245,24 @@ moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed
  * sizes overflow. */
 size_t moe_qmm_id_workspace_bytes(uint32_t m, uint32_t n_expert_used, uint32_t num_experts);
 
-/* Workspace bytes with room for the grouped path's gathered f32 x rows: the
- * pairs' x rows in expert order (m * n_expert_used rows of k values, each held as
- * two bf16 halves, 4 bytes). When a call with f32 x takes the grouped path and its
- * workspace_bytes reaches this size (and k is a multiple of 8), x is gathered and
- * split into its bf16 halves once after routing and the GEMM loads each tile of x
- * rows with one tensor copy per half; with the minimum moe_qmm_id_workspace_bytes
- * the GEMM copies and splits x rows itself. Results are the same either way. For
- * bf16 / f16 x it equals moe_qmm_id_workspace_bytes (the GEMM copies 16-bit x rows
- * straight from x). Returns 0 if the sizes overflow or
- * x_dtype is not a moe_dtype. */
+/* Workspace bytes with room for the grouped path's x operand, which makes that
+ * path faster (results are the same up to the order of fp32 sums, and bit for bit
+ * for f32 x):
+ *   f32 x   -- the pairs' x rows gathered in expert order and split into bf16 halves
+ *              once after routing (m * n_expert_used rows of k values, 4 bytes each),
+ *              loaded by one tensor copy per tile and half;
+ *   bf16 / f16 x -- when the automatic path would take the grouped GEMM with
+ *              256-pair tiles (experts hold 96 or more pairs on average), a tile-major
+ *              f16 image of the B operand ([m*n_expert_used/256 + num_experts + 1]
+ *              tiles x ceil(k/64) x 256 rows x 128 bytes) and one f32 per token (no
+ *              room is added for smaller calls): bf16 x is scaled by a
+ *              power of two per token (exact in f16 above 2^-28 of the token's largest
+ *              value) and the factor is undone in the epilogue. Each k-tile of a tile
+ *              is then one bulk copy. Not for MXFP4 weights, pointer tables or gated
+ *              outputs, which keep the row copies.
+ * With the minimum moe_qmm_id_workspace_bytes the GEMM's loader warps copy x rows
+ * themselves. k must be a multiple of 8 (else no room is added). Returns 0 if the
+ * sizes overflow or x_dtype is not a moe_dtype. */
 size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts,
                                     moe_dtype x_dtype);
 

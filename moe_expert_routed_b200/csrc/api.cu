@@ -80,8 +80,14 @@ size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_us
                                     moe_dtype x_dtype) {
     WsLayout L;
     if ((int)x_dtype < 0 || (int)x_dtype > 2) return 0;
-    if (!ws_layout((uint64_t)m * n_expert_used, num_experts, &L)) return 0;
-    return L.total + (size_t)gathered_x_bytes((uint64_t)m * n_expert_used, k, (int)x_dtype);
+    const uint64_t R = (uint64_t)m * n_expert_used;
+    if (!ws_layout(R, num_experts, &L)) return 0;
+    if (x_dtype == MOE_F32) return L.total + (size_t)gathered_x_bytes(R, k, (int)x_dtype);
+    // 16-bit x: room for the f16 image when the automatic path takes the grouped GEMM
+    if (R <= MOE_DECODE_MAX_ROUTINGS || R <= (uint64_t)MOE_DECODE_MAX_PAIRS_PER_EXPERT * num_experts || k % 8u != 0)
+        return L.total;
+    if (R < 96ull * num_experts) return L.total;  // 64-pair tiles keep the row copies
+    return L.total + (size_t)x_image_bytes(R, num_experts, k, 256u) + al256(4ull * m);
 }
 
 const char *moe_status_str(moe_status s) {
@@ -233,14 +239,35 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         // x rows in expert order for the grouped GEMM, when the workspace has room for them
         const uint64_t gx = choice == GROUPED ? gathered_x_bytes(R, k, (int)x_dtype) : 0;
         uint16_t *xg = (gx && workspace_bytes >= L.total + gx) ? (uint16_t *)(ws + L.total) : nullptr;
+        // 16-bit x with 256-pair tiles: the tile-major f16 image of the B operand (and
+        // bf16's per-token powers of two), when the workspace has room; not for MXFP4
+        // (e2m1 * 2^e can leave f16's range), pointer tables, gated outputs or W4A4's
+        // operand. With 64-pair tiles (a few pairs per expert) writing the image costs
+        // more than the GEMM saves.
+        uint8_t *ximg = nullptr;
+        float *tscale = nullptr;
+        if (choice == GROUPED && tile_rows == 256u && x_dtype != MOE_F32 && a.kind != K_MXFP4 && !a.packed_ptrs &&
+            a.act < 0 && !a.tok_scale && !a.x_copies && ((uintptr_t)x & 15u) == 0) {
+            const uint64_t ib = x_image_bytes(R, num_experts, k, tile_rows);
+            if (workspace_bytes >= L.total + ib + al256(4ull * m)) {
+                ximg = ws + L.total;
+                tscale = (float *)(ws + L.total + ib);
+            }
+        }
         ce = launch_route(ids, (uint32_t)R, num_experts, tile_rows, counts, offsets, sp, tiles, tc,
                           max_tiles, (uint32_t *)(ws + L.chunk_hist),
                           (uint32_t *)(ws + L.chunk_base), L.chunks, err, out, a.out_n, (int)out_dtype,
                           st, wc);
         if (ce == cudaSuccess && xg) ce = launch_gather_x(x, (int)x_dtype, sp, (uint32_t)R, k, n_expert_used, xg, st);
+        if (ce == cudaSuccess && ximg) {
+            ce = launch_x_image(x, (int)x_dtype, m, k, sp, tiles, tc, offsets, n_expert_used, tile_rows, max_tiles,
+                                ximg, tscale, st);
+            a.x_dtype = DT_F16;
+            a.tok_scale = x_dtype == MOE_BF16 ? tscale : nullptr;
+        }
         if (ce == cudaSuccess) {
             if (choice == GROUPED)
-                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, xg, st);
+                ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, xg, ximg, st);
             else
                 ce = launch_gemv_routed(a, counts, offsets, sp, err, st);
         }

@@ -75,6 +75,7 @@ constexpr int SCHED_WARP = EPI_WARP0 + NEP / 32;
 // how the B operand's x rows reach shared memory
 constexpr uint32_t XM_LOADERS = 0;  // 16-byte copies by the loader warps
 constexpr uint32_t XM_ROWS = 1;     // tensor copies of x rows gathered into expert order beforehand
+constexpr uint32_t XM_IMAGE = 2;    // one bulk copy per k-tile of the tile-major, pre-swizzled f16 image
 constexpr uint32_t RING = 4;                    // work items the scheduler may publish ahead
 // arrivals that release a ring slot: one per dequantiser, loader and epilogue warp,
 // plus the tensor-copy and MMA lanes
@@ -114,8 +115,10 @@ struct GemmParams {
     // second tensor map
     uint32_t xmode;
     uint32_t xg_R;
-    // W4A4: per-token factor of every output (null: none)
+    // W4A4, or the f16 image of bf16 x: per-token factor of every output (null: none)
     const float *tok_scale;
+    // XM_IMAGE: the B operand image, tile t's k-tile kt at (t * ktiles + kt) * BN * 128
+    const uint8_t *ximage;
     uint32_t *work_counter; // items claimed beyond each CTA's first (zeroed by the routing prologue)
     // failure-detection test hook: non-zero makes the MMA warp first wait this long on
     // a barrier nothing completes (so the CTA aborts); 0 in normal operation
@@ -483,11 +486,13 @@ struct Item {
 // compile time so that the contiguous case keeps its copy-width and scale-staging
 // branches on kernel parameters). GLU: gated output (glu_row order, act(gate) * up
 // epilogue), also decided at compile time so that the plain kernels carry none of it.
-template <int KIND, int XT, int BN, bool PTRS, bool GLU>
+// XIMG (f16 x only): the B tiles come by one bulk copy per k-tile from the image.
+template <int KIND, int XT, int BN, bool PTRS, bool GLU, bool XIMG = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap,
                     const __grid_constant__ CUtensorMap xmap) {
     using C = GemmCfg<KIND, XT, BN>;
+    static_assert(!XIMG || (XT == DT_F16 && !PTRS && !GLU), "the image is f16, for the plain kernel");
     constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
     constexpr uint32_t STAGE = C::STAGE;
     constexpr uint32_t B_OFF = AT * A_TILE, RAW_OFF = AT * A_TILE + BT * B_TILE;
@@ -547,7 +552,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
     const bool tma = !PTRS && P.tma != 0;
     // x tiles: by the loader warps' 16-byte copies, or (f32 x) by tensor copies of rows
     // gathered beforehand; a compile-time XM_LOADERS for 16-bit x
-    const uint32_t xmode = (XT == DT_F32) ? P.xmode : XM_LOADERS;
+    const uint32_t xmode = XIMG ? XM_IMAGE : (XT == DT_F32) ? P.xmode : XM_LOADERS;
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
             ptx::mbar_init(full0 + 8 * s, NDQ);
@@ -847,13 +852,17 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
             // bytes per k-tile: the codes' two 64-row boxes, the x box of BN rows (each row
             // one 128-byte swizzle line; twice for f32 x)
             constexpr uint32_t CODE_TX = KIND == K_CB3 ? 2u * 64u * CB3_WIN : 2u * 64u * RB;
-            const uint32_t tx = (tma ? CODE_TX : 0u) + (xmode == XM_ROWS ? (uint32_t)(BT * B_TILE) : 0u);
+            const uint32_t tx0 = (tma ? CODE_TX : 0u) + (xmode == XM_ROWS ? (uint32_t)(BT * B_TILE) : 0u);
+            const size_t img_tile = (size_t)P.ktiles * BN * 128u;
             uint32_t g = 0, last_s = 0, last_par = 0;
             bool any = false, ok = true;
             for (uint32_t i = 0; ok; i++) {
                 uint32_t w;
                 if (!next_item(i, false, w) || w >= n_items) break;
-                if (!(tma || xmode == XM_ROWS) || !load_item(w)) continue;
+                if (!(tma || xmode != XM_LOADERS) || !load_item(w)) continue;
+                // with the image: nt_pad lines of 128 bytes per k-tile
+                const uint32_t tx = tx0 + (XIMG ? it.nt_pad * 128u : 0u);
+                const uint8_t *img = XIMG ? P.ximage + (size_t)(w / nm) * img_tile : nullptr;
                 const int32_t y0 = (int32_t)(it.e * P.n + (GLU ? it.row0 / 2u : it.row0));
                 const int32_t y1 = GLU ? (int32_t)(it.e * P.n + P.glu_nh + it.row0 / 2u) : y0 + 64;
                 for (uint32_t kt = 0; kt < P.ktiles; kt++, g++) {
@@ -877,6 +886,8 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                             ptx::tma_load_2d(raw + 64u * RB, &tmap, (int32_t)(kt * RB), y1, bar);
                         }
                     }
+                    if constexpr (XIMG)
+                        ptx::bulk_g2s(base + s * STAGE + B_OFF, img + (size_t)kt * BN * 128u, it.nt_pad * 128u, bar);
                     if (xmode == XM_ROWS) {
                         // gathered rows off + r0 .. + BN - 1: rows past the tile's pairs are other
                         // pairs' x rows (or zeros past the end) in B rows whose results are not stored
@@ -1095,12 +1106,12 @@ uint32_t sm_count_gemm() {
     return (uint32_t)count[dev];
 }
 
-template <int KIND, int XT, int BN, bool PTRS, bool GLU>
+template <int KIND, int XT, int BN, bool PTRS, bool GLU, bool XIMG = false>
 cudaError_t launch_tp(const GemmParams &P0, const CUtensorMap &tmap, const CUtensorMap &xmap, const GemmPlan &pl,
                       uint32_t n_mtiles, uint32_t max_tiles, cudaStream_t st) {
     GemmParams P = P0;
     P.stages = (uint32_t)pl.stages;
-    auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS, GLU>;
+    auto kern = grouped_gemm_kernel<KIND, XT, BN, PTRS, GLU, XIMG>;
     static int smem_set[64];
     cudaError_t e = ensure_dyn_smem(kern, pl.smem, smem_set);
     if (e != cudaSuccess) return e;
@@ -1116,6 +1127,9 @@ cudaError_t launch_t(const GemmParams &P, const CUtensorMap &tm, const CUtensorM
                      uint32_t n_mtiles, uint32_t max_tiles, cudaStream_t st) {
     if (P.packed_ptrs) return launch_tp<KIND, XT, BN, true, false>(P, tm, xm, pl, n_mtiles, max_tiles, st);
     if (P.glu_nh) return launch_tp<KIND, XT, BN, false, true>(P, tm, xm, pl, n_mtiles, max_tiles, st);
+    if constexpr (XT == DT_F16) {
+        if (P.xmode == XM_IMAGE) return launch_tp<KIND, XT, BN, false, false, true>(P, tm, xm, pl, n_mtiles, max_tiles, st);
+    }
     return launch_tp<KIND, XT, BN, false, false>(P, tm, xm, pl, n_mtiles, max_tiles, st);
 }
 
@@ -1257,7 +1271,8 @@ uint32_t gemm_tile_rows(const QmmArgs &a) {
 
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
-                        uint32_t *err, uint32_t *work_counter, const uint16_t *xg, cudaStream_t st) {
+                        uint32_t *err, uint32_t *work_counter, const uint16_t *xg, const uint8_t *ximg,
+                        cudaStream_t st) {
     GemmPlan pl;
     if (!gemm_plan(a, &pl)) return cudaErrorNotSupported;
     GemmParams P{};
@@ -1297,6 +1312,12 @@ cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_
     P.xmode = (a.x_dtype == DT_F32 && !a.x_copies && xg && x_tensor_map(xg, R * 2u, a.k, pl.bn, &xmap))
                   ? XM_ROWS
                   : XM_LOADERS;
+    // 16-bit x as the f16 image (the caller sets a.x_dtype to f16 with it)
+    P.ximage = nullptr;
+    if (ximg && a.x_dtype == DT_F16 && !a.packed_ptrs && a.act < 0) {
+        P.xmode = XM_IMAGE;
+        P.ximage = ximg;
+    }
     return launch_kind(P, tmap, xmap, pl, a.kind, a.x_dtype, nm, max_tiles, st);
 }
 

@@ -99,6 +99,14 @@ cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_p
 // x16 (optional) [m, k]: e2m1(q) * e4m3(s) as bf16 (exact), x^ without the per-token factor.
 cudaError_t launch_quant_act(const void *x, int x_dtype, uint32_t m, uint32_t k, uint8_t *codes, uint8_t *scales,
                              float *gscale, float *xhat, uint16_t *x16, cudaStream_t st);
+// The grouped GEMM's B operand image for 16-bit x (tile-major, 128-byte-swizzled f16
+// lines, [max_tiles][ceil(k/64)][tile_rows][128 B]) and, for bf16 x, the per-token
+// powers of two tok_scale [m] the epilogue applies (img 16-byte aligned).
+cudaError_t launch_x_image(const void *x, int x_dtype, uint32_t m, uint32_t k, const uint32_t *sorted_pairs,
+                           const uint32_t *tiles, const uint32_t *tile_count, const uint32_t *offsets,
+                           uint32_t n_expert_used, uint32_t tile_rows, uint32_t max_tiles, uint8_t *img,
+                           float *tok_scale, cudaStream_t st);
+uint64_t x_image_bytes(uint64_t R, uint32_t E, uint32_t k, uint32_t tile_rows);
 // Bytes of the gathered x rows (0 when the grouped GEMM does not use them: 16-bit x
 // is gathered by the GEMM's tensor copies straight from x).
 uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype);
@@ -108,7 +116,8 @@ bool gemm_supported(const QmmArgs &a);
 uint32_t gemm_tile_rows(const QmmArgs &a);
 cudaError_t launch_gemm(const QmmArgs &a, const uint32_t *offsets, const uint32_t *sorted_pairs,
                         const uint32_t *tiles, const uint32_t *tile_count, uint32_t max_tiles,
-                        uint32_t *err, uint32_t *work_counter, const uint16_t *xg, cudaStream_t st);
+                        uint32_t *err, uint32_t *work_counter, const uint16_t *xg, const uint8_t *ximg,
+                        cudaStream_t st);
 
 // moe_qmm_id's scalar validation (MOE_OK or the status moe_qmm_id would return).
 moe_status validate_call(const void *x, const uint32_t *ids, const void *packed, const void *scales,

@@ -239,6 +239,75 @@ gather_x(const float *__restrict__ x, const uint32_t *__restrict__ sorted_pairs,
     }
 }
 
+// Per-token power of two for the f16 image of bf16 x: with a = max_j |x[t][j]| in
+// [2^(E-1), 2^E), x * 2^(15-E) has its largest magnitude in [2^14, 2^15), inside f16's
+// range, and a bf16 value (8 significant bits) times a power of two is exact in f16
+// unless it falls below f16's normal range (2^-14, i.e. below 2^-28 of the token's
+// largest). tok_scale[t] = 2^(E-15) undoes it in the GEMM's epilogue (1 for a zero row).
+__global__ void __launch_bounds__(256)
+x_token_scale(const uint16_t *__restrict__ x, uint32_t k, float *__restrict__ tok_scale) {
+    __shared__ float red[8];
+    const uint32_t t = blockIdx.x;
+    float a = 0.f;
+    for (uint32_t j = threadIdx.x; j < k; j += 256u) a = fmaxf(a, fabsf(bf16_bits_to_f32(__ldg(x + (size_t)t * k + j))));
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, d));
+    if ((threadIdx.x & 31u) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; w++) a = fmaxf(a, red[w]);
+        const int e = a > 0.f ? ((int)((__float_as_uint(a) >> 23) & 0xFFu) - 126) : 15;  // a < 2^e
+        const int s = e - 15 < -126 ? -126 : (e - 15 > 127 ? 127 : e - 15);
+        tok_scale[t] = __uint_as_float((uint32_t)(s + 127) << 23);
+    }
+}
+
+// The B operand image of the grouped GEMM: for tile t of the routing prologue's tile
+// list and k-tile kt, rows 0 .. nt_pad-1 of the tile (its pairs' x rows; zeros past
+// its pairs and past k) as f16, each row a 128-byte line with 16-byte chunk c at
+// position c ^ (row & 7): block (t, kt) of bn lines starts at (t * ktiles + kt) * bn
+// * 128 and is exactly the shared-memory tile (128-byte swizzle, K-major) the GEMM
+// copies with one bulk copy. bf16 x is scaled per token by 1 / tok_scale; f16 x is
+// copied. One warp per row, each lane a 16-byte chunk of 4 consecutive k-tiles.
+__global__ void __launch_bounds__(256)
+x_image(const uint16_t *__restrict__ x, int x_dtype, uint32_t k, uint32_t ktiles, const uint32_t *__restrict__ sp,
+        const uint32_t *__restrict__ tiles, const uint32_t *__restrict__ tile_count,
+        const uint32_t *__restrict__ offsets, uint32_t n_expert_used, uint32_t bn,
+        const float *__restrict__ tok_scale, uint8_t *__restrict__ img) {
+    const uint32_t t = blockIdx.x;
+    if (t >= __ldg(tile_count)) return;
+    const uint32_t e = __ldg(tiles + 2 * t), r0 = __ldg(tiles + 2 * t + 1);
+    const uint32_t off = __ldg(offsets + e), cnt = __ldg(offsets + e + 1) - off;
+    const uint32_t nt = cnt - r0 < bn ? cnt - r0 : bn, nt_pad = (nt + 15u) & ~15u;
+    const uint32_t lane = threadIdx.x & 31u;
+    for (uint32_t i = blockIdx.y * 8u + (threadIdx.x >> 5); i < nt_pad; i += gridDim.y * 8u) {
+        const bool live = i < nt;
+        const size_t tok = live ? __ldg(sp + off + r0 + i) / n_expert_used : 0;
+        const uint16_t *xr = x + tok * k;
+        float mul = 1.f;
+        if (live && tok_scale) mul = 1.f / __ldg(tok_scale + tok);  // an exact power of two
+        for (uint32_t q = lane; q < ktiles * 8u; q += 32u) {
+            const uint32_t kt = q >> 3, c = q & 7u, j = kt * 64u + c * 8u;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (live && j < k) {
+                v = __ldg((const uint4 *)(xr + j));
+                if (x_dtype == DT_BF16) {
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int h = 0; h < 4; h++) {
+                        const __half2 f = __floats2half2_rn(bf16_bits_to_f32(w[h] & 0xFFFFu) * mul,
+                                                            bf16_bits_to_f32(w[h] >> 16) * mul);
+                        w[h] = *reinterpret_cast<const uint32_t *>(&f);
+                    }
+                    v = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            uint8_t *line = img + (((size_t)t * ktiles + kt) * bn + i) * 128u;
+            *(uint4 *)(line + ((c ^ (i & 7u)) << 4)) = v;
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_pairs, uint32_t R, uint32_t k,
@@ -249,6 +318,31 @@ cudaError_t launch_gather_x(const void *x, int x_dtype, const uint32_t *sorted_p
     if (ctas == 0) return cudaSuccess;
     if (x_dtype != DT_F32 || k % 8u != 0) return cudaErrorInvalidValue;
     gather_x<<<ctas, 256, 0, st>>>((const float *)x, sorted_pairs, R, k, n_expert_used, xg);
+    return cudaGetLastError();
+}
+
+uint64_t x_image_bytes(uint64_t R, uint32_t E, uint32_t k, uint32_t tile_rows) {
+    const uint64_t max_tiles = R / tile_rows + E + 1ull;
+    return max_tiles * ((k + 63ull) / 64ull) * tile_rows * 128ull;
+}
+
+cudaError_t launch_x_image(const void *x, int x_dtype, uint32_t m, uint32_t k, const uint32_t *sorted_pairs,
+                           const uint32_t *tiles, const uint32_t *tile_count, const uint32_t *offsets,
+                           uint32_t n_expert_used, uint32_t tile_rows, uint32_t max_tiles, uint8_t *img,
+                           float *tok_scale, cudaStream_t st) {
+    if (x_dtype == DT_F32 || k % 8u != 0 || (tile_rows & 15u) || ((uintptr_t)x & 15u) || ((uintptr_t)img & 15u))
+        return cudaErrorInvalidValue;
+    const uint16_t *x16 = (const uint16_t *)x;
+    if (x_dtype == DT_BF16) {
+        if (!tok_scale) return cudaErrorInvalidValue;
+        x_token_scale<<<m, 256, 0, st>>>(x16, k, tok_scale);
+    } else {
+        tok_scale = nullptr;
+    }
+    const uint32_t ktiles = (k + 63u) / 64u;
+    const dim3 grid(max_tiles, (tile_rows + 31u) / 32u);
+    x_image<<<grid, 256, 0, st>>>(x16, x_dtype, k, ktiles, sorted_pairs, tiles, tile_count, offsets, n_expert_used,
+                                  tile_rows, tok_scale, img);
     return cudaGetLastError();
 }
 

@@ -56,12 +56,19 @@ def test_workspace_bytes_grows_with_routings():
 
 
 def test_workspace_bytes_with_gathered_x():
+    al = lambda v: (v + 255) // 256 * 256
     base = M.workspace_bytes(512, 8, 64)
-    bf = M.workspace_bytes(512, 8, 64, k=1024, x_dtype=torch.bfloat16)
     f32 = M.workspace_bytes(512, 8, 64, k=1024, x_dtype=torch.float32)
-    assert bf == base                                 # 16-bit x: gathered by the GEMM's tensor copies
     assert f32 == base + 512 * 8 * 1024 * 4          # f32 x: two bf16 halves per element
     assert M.workspace_bytes(512, 8, 64, k=1028, x_dtype=torch.float32) == base  # k % 8: no room added
+    # 16-bit x with 64-pair tiles (fewer than 96 pairs per expert): no room added
+    assert M.workspace_bytes(512, 8, 64, k=1024, x_dtype=torch.bfloat16) == base
+    # 256-pair tiles: the f16 image, [R/256 + E + 1 tiles][k/64][256 rows][128 B], and one f32 per token
+    big = M.workspace_bytes(2048, 8, 64, k=512, x_dtype=torch.float16)
+    assert big == M.workspace_bytes(2048, 8, 64) + (16384 // 256 + 64 + 1) * 8 * 256 * 128 + al(2048 * 4)
+    # decode-sized calls: no image
+    assert M.workspace_bytes(8, 8, 64, k=1024, x_dtype=torch.bfloat16) == M.workspace_bytes(8, 8, 64)
+    assert M.workspace_bytes(16, 8, 64, k=1024, x_dtype=torch.bfloat16) == M.workspace_bytes(16, 8, 64)
     assert M.lib().moe_qmm_id_workspace_bytes_k(512, 1024, 8, 64, 3) == 0         # not a moe_dtype
 
 

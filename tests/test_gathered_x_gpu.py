@@ -1,14 +1,15 @@
-"""The grouped GEMM's two ways of bringing x rows into the B operand tiles give
-the same bits: for f32 x, tensor copies of the rows gathered into expert order
-and split into bf16 halves once after routing (a workspace sized by
-moe_qmm_id_workspace_bytes_k), and 16-byte copies by the loader warps, which
-split f32 x per tile (the minimum workspace, or forced through
-moe_qmm_test_x_copies). 16-bit x always takes the loader copies; its cases
-check that the k-aware workspace and the hook change nothing. The default path is
-also checked element by element against the oracle. Cases span every weight
-format, bf16 / f16 / f32 x, 64- and 256-pair tiles, partial tiles, a ragged last
-k-tile, a ragged last row block, out-of-range ids, a gated output and an expert
-bias."""
+"""The grouped GEMM's ways of bringing x rows into the B operand tiles. For f32 x,
+tensor copies of the rows gathered into expert order and split into bf16 halves
+once after routing (a workspace sized by moe_qmm_id_workspace_bytes_k) and the
+loader warps' 16-byte copies, which split f32 x per tile (the minimum workspace,
+or forced through moe_qmm_test_x_copies), give the same bits. For 16-bit x the
+k-aware workspace holds the tile-major f16 image of the B operand (bf16 x scaled
+per token by a power of two), read with one bulk copy per k-tile, and the
+minimum workspace or the hook keeps the loader copies; the two compute in f16
+and bf16 respectively, so each is checked against the oracle. Every output is
+checked element by element against the oracle. Cases span every weight format,
+bf16 / f16 / f32 x, 64- and 256-pair tiles, partial tiles, a ragged last k-tile,
+a ragged last row block, out-of-range ids, a gated output and an expert bias."""
 
 import pytest
 import torch
@@ -41,7 +42,14 @@ def _ways(P, runner, **kw):
     return outs, ws_k
 
 
-def _same_bits(outs):
+def _same_bits(outs, P=None, check=None):
+    """f32 x: every way gives the default's bits. 16-bit x: each way within the
+    oracle's tolerance (check(P, out) -> (violations, ratio, info))."""
+    if P is not None and P.x_dtype != DT_F32:
+        for i, o in enumerate(outs):
+            nviol, ratio, info = check(P, o)
+            assert nviol == 0, f"x-tile way {i}: {nviol} outside tolerance ({ratio:.3g}, {info})"
+        return
     ref = outs[0].view(torch.uint8)
     for i, o in enumerate(outs[1:], 1):
         assert torch.equal(ref, o.view(torch.uint8)), f"x-tile way {i} differs from the default"
@@ -69,7 +77,7 @@ def test_x_tile_ways_bit_identical_and_match_oracle(fmt, bits, gs, xd, od, m, to
                      out_dtype=od, m=m, k=k, n=n, n_expert_used=topk, num_experts=E)
     outs, ws = _ways(P, run)
     assert M.poll_error(ws) == 0
-    _same_bits(outs)
+    _same_bits(outs, P, check_full)
     nviol, ratio, info = check_full(P, outs[0])
     assert nviol == 0, f"{nviol} outside tolerance ({ratio:.3g}, {info})"
 
@@ -83,7 +91,7 @@ def test_x_tiles_out_of_range_ids():
     P = P.with_ids(ids)
     outs, ws = _ways(P, run)
     assert M.poll_error(ws) == 5
-    _same_bits(outs)
+    _same_bits(outs, P, check_full)
     nviol, ratio, info = check_full(P, outs[0])
     assert nviol == 0, f"{nviol} outside tolerance ({ratio:.3g}, {info})"
 
@@ -93,11 +101,11 @@ def test_x_tiles_gated_and_bias(xd):
     P = make_problem("x-tiles-glu", seed=8950, fmt=FMT_AFFINE, bits=4, group_size=64, x_dtype=xd,
                      out_dtype=DT_F32, m=600, k=768, n=256, n_expert_used=2, num_experts=4)
     outs, _ = _ways(P, run_glu, act="silu")
-    _same_bits(outs)
+    _same_bits(outs, P, lambda P, o: check_full_glu(P, "silu", o))
     nviol, ratio, info = check_full_glu(P, "silu", outs[0])
     assert nviol == 0, f"{nviol} outside tolerance ({ratio:.3g}, {info})"
     bias = expert_bias(8951, P.num_experts, P.n, DT_F32)
     outs, _ = _ways(P, lambda P, **kw: run_bias(P, bias, DT_F32, **kw))
-    _same_bits(outs)
+    _same_bits(outs, P, lambda P, o: check_full_bias(P, o, bias, DT_F32))
     nviol, ratio, info = check_full_bias(P, outs[0], bias, DT_F32)
     assert nviol == 0, f"{nviol} outside tolerance ({ratio:.3g}, {info})"
