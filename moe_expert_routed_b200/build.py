@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe_qmm.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
-SOURCES = ["api.cu", "route.cu", "gemv.cu", "gemm_sm100.cu", "noalloc.cu", "actq.cu"]
+SOURCES = ["api.cu", "route.cu", "gemv.cu", "gemm_sm100.cu", "noalloc.cu", "actq.cu", "gemm_w4a4.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "internal.h", "gemv_common.cuh"]
 
 NVCC_FLAGS = [

@@ -41,9 +41,11 @@ bool ws_layout(uint64_t R, uint32_t E, WsLayout *L) {
     return true;
 }
 
-// W4A4 workspace ahead of the operation's own: x^ f32 [m, k], bf16 [m, k], f32 [m].
+// W4A4 workspace ahead of the operation's own: x^ f32 [m, k], bf16 [m, k], f32 [m],
+// codes [m, k/2], E4M3 factors [m, k/16].
 size_t w4a4_front_bytes(uint32_t m, uint32_t k) {
-    return al256((uint64_t)m * k * 4ull) + al256((uint64_t)m * k * 2ull) + al256((uint64_t)m * 4ull);
+    return al256((uint64_t)m * k * 4ull) + al256((uint64_t)m * k * 2ull) + al256((uint64_t)m * 4ull) +
+           al256((uint64_t)m * k / 2ull) + al256((uint64_t)m * k / 16ull);
 }
 
 uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype) {
@@ -152,7 +154,8 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
                uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace, size_t workspace_bytes,
                moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}, int act = -1,
-               const uint16_t *w4a4_x16 = nullptr, const float *w4a4_scale = nullptr) {
+               const uint16_t *w4a4_x16 = nullptr, const float *w4a4_scale = nullptr,
+               const uint8_t *w4a4_codes = nullptr, const uint8_t *w4a4_xscales = nullptr) {
     moe_status v = validate(x, ids, pt.packed ? (const void *)pt.packed : packed,
                             pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
                             fmt, n_expert_used, num_experts, x_dtype, out_dtype);
@@ -213,9 +216,12 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         else return MOE_ERR_UNSUPPORTED;
     }
 
-    // W4A4 on the grouped GEMM: bf16 e2m1(q) * e4m3(s) (exact) as the B operand and the
+    // W4A4 on the grouped GEMM: the block-scaled MMA on the activations' NVFP4 codes
+    // where it applies; else bf16 e2m1(q) * e4m3(s) (exact) as the B operand and the
     // per-token factor in the epilogue, instead of the f32 x^ the CUDA-core paths take
-    if (choice == GROUPED && w4a4_x16 && w4a4_scale) {
+    const bool w4mma = choice == GROUPED && w4a4_codes && w4a4_xscales && w4a4_scale && !a.x_copies &&
+                       w4a4_mma_supported(a);
+    if (choice == GROUPED && !w4mma && w4a4_x16 && w4a4_scale) {
         a.x = w4a4_x16;
         a.x_dtype = DT_BF16;
         x = w4a4_x16;
@@ -233,11 +239,11 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         uint32_t *sp = (uint32_t *)(ws + L.sorted_pairs);
         uint32_t *tiles = (uint32_t *)(ws + L.tiles);
         uint32_t *tc = (uint32_t *)(ws + L.tile_count);
-        const uint32_t tile_rows = choice == GROUPED ? gemm_tile_rows(a) : MIN_TILE_ROWS;
+        const uint32_t tile_rows = w4mma ? 128u : choice == GROUPED ? gemm_tile_rows(a) : MIN_TILE_ROWS;
         const uint32_t max_tiles = (uint32_t)(R / tile_rows + num_experts + 1);
         uint32_t *wc = (uint32_t *)(ws + L.work_counter);
         // x rows in expert order for the grouped GEMM, when the workspace has room for them
-        const uint64_t gx = choice == GROUPED ? gathered_x_bytes(R, k, (int)x_dtype) : 0;
+        const uint64_t gx = (choice == GROUPED && !w4mma) ? gathered_x_bytes(R, k, (int)x_dtype) : 0;
         uint16_t *xg = (gx && workspace_bytes >= L.total + gx) ? (uint16_t *)(ws + L.total) : nullptr;
         // 16-bit x with 256-pair tiles: the tile-major f16 image of the B operand (and
         // bf16's per-token powers of two), when the workspace has room; not for MXFP4
@@ -246,8 +252,8 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         // more than the GEMM saves.
         uint8_t *ximg = nullptr;
         float *tscale = nullptr;
-        if (choice == GROUPED && tile_rows == 256u && x_dtype != MOE_F32 && a.kind != K_MXFP4 && !a.packed_ptrs &&
-            a.act < 0 && !a.tok_scale && !a.x_copies && ((uintptr_t)x & 15u) == 0) {
+        if (choice == GROUPED && !w4mma && tile_rows == 256u && x_dtype != MOE_F32 && a.kind != K_MXFP4 &&
+            !a.packed_ptrs && a.act < 0 && !a.tok_scale && !a.x_copies && ((uintptr_t)x & 15u) == 0) {
             const uint64_t ib = x_image_bytes(R, num_experts, k, tile_rows);
             if (workspace_bytes >= L.total + ib + al256(4ull * m)) {
                 ximg = ws + L.total;
@@ -266,7 +272,10 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
             a.tok_scale = x_dtype == MOE_BF16 ? tscale : nullptr;
         }
         if (ce == cudaSuccess) {
-            if (choice == GROUPED)
+            if (w4mma)
+                ce = launch_gemm_w4a4(a, w4a4_codes, w4a4_xscales, w4a4_scale, offsets, sp, tiles, tc, max_tiles,
+                                      err, wc, st);
+            else if (choice == GROUPED)
                 ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, xg, ximg, st);
             else
                 ce = launch_gemv_routed(a, counts, offsets, sp, err, st);
@@ -362,15 +371,21 @@ moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packe
     if (workspace_bytes < front + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
         return MOE_ERR_WORKSPACE_TOO_SMALL;
     uint8_t *w = (uint8_t *)workspace;
-    float *xhat = (float *)w;
-    uint16_t *x16 = (uint16_t *)(w + moe::al256((uint64_t)m * k * 4ull));
-    float *g = (float *)(w + moe::al256((uint64_t)m * k * 4ull) + moe::al256((uint64_t)m * k * 2ull));
-    if (moe::launch_quant_act(x, (int)x_dtype, m, k, nullptr, nullptr, g, xhat, x16, (cudaStream_t)stream) !=
-        cudaSuccess)
+    size_t o = 0;
+    float *xhat = (float *)(w + o);
+    o += moe::al256((uint64_t)m * k * 4ull);
+    uint16_t *x16 = (uint16_t *)(w + o);
+    o += moe::al256((uint64_t)m * k * 2ull);
+    float *g = (float *)(w + o);
+    o += moe::al256((uint64_t)m * 4ull);
+    uint8_t *codes = w + o;
+    o += moe::al256((uint64_t)m * k / 2ull);
+    uint8_t *xs = w + o;
+    if (moe::launch_quant_act(x, (int)x_dtype, m, k, codes, xs, g, xhat, x16, (cudaStream_t)stream) != cudaSuccess)
         return MOE_ERR_CUDA;
     return moe::run(xhat, ids, packed, scales, aux, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
                     num_experts, MOE_F32, out_dtype, MOE_F32, w + front, workspace_bytes - front, stream, path,
-                    {nullptr, nullptr, nullptr}, -1, x16, g);
+                    {nullptr, nullptr, nullptr}, -1, x16, g, codes, xs);
 }
 
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,

@@ -1005,14 +1005,20 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
             for (uint32_t c0 = 0; c0 < it.nt; c0 += 16) {
                 uint32_t v[16], pr[16];
                 ptx::tmem_ld16(d + ((q * 32u) << 16) + c0, v);
+                // lane j < 16 fetches column c0 + j's pair (and its token's factor); the
+                // warp shares them by shuffles
+                const uint32_t cj = c0 + (lane & 15u);
+                const uint32_t myp = cj < it.nt ? __ldg(pairs + cj) : 0u;
+                const float myf = P.tok_scale ? __ldg(P.tok_scale + myp / P.n_expert_used) : 1.f;
 #pragma unroll
-                for (int i = 0; i < 16; i++) pr[i] = c0 + i < it.nt ? __ldg(pairs + c0 + i) : 0u;
+                for (int i = 0; i < 16; i++) pr[i] = __shfl_sync(0xFFFFFFFFu, myp, i);
                 ptx::tmem_wait_ld();
                 if (P.tok_scale) {
-                    // W4A4: the token's factor, applied to the fp32 sum before the bias
+                    // the token's factor (W4A4, or the power of two of the f16 image of bf16
+                    // x), applied to the fp32 sum before the bias
 #pragma unroll
                     for (int i = 0; i < 16; i++)
-                        v[i] = __float_as_uint(__uint_as_float(v[i]) * __ldg(P.tok_scale + pr[i] / P.n_expert_used));
+                        v[i] = __float_as_uint(__uint_as_float(v[i]) * __shfl_sync(0xFFFFFFFFu, myf, i));
                 }
                 if constexpr (GLU) {
                     // even lanes hold gate rows, the next lane the matching up row
@@ -1025,11 +1031,18 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                             store_out(P.out, P.out_dtype, (size_t)pr[i] * nh + (grow_e >> 1), glu_act(P.act, y) * up);
                     }
                 } else if (grow_e < P.n) {
+                    const uint32_t nc = tmin<uint32_t>(16u, it.nt - c0);
+                    if (P.out_dtype == DT_BF16) {
 #pragma unroll
-                    for (int i = 0; i < 16; i++) {
-                        const uint32_t col = c0 + i;
-                        if (col < it.nt)
-                            store_out(P.out, P.out_dtype, (size_t)pr[i] * P.n + grow_e, __uint_as_float(v[i]) * s2 + bv);
+                        for (int i = 0; i < 16; i++)
+                            if ((uint32_t)i < nc)
+                                ((__nv_bfloat16 *)P.out)[(size_t)pr[i] * P.n + grow_e] =
+                                    __float2bfloat16_rn(__uint_as_float(v[i]) * s2 + bv);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; i++)
+                            if ((uint32_t)i < nc)
+                                store_out(P.out, P.out_dtype, (size_t)pr[i] * P.n + grow_e, __uint_as_float(v[i]) * s2 + bv);
                     }
                 }
             }

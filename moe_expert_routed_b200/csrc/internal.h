@@ -111,6 +111,14 @@ uint64_t x_image_bytes(uint64_t R, uint32_t E, uint32_t k, uint32_t tile_rows);
 // is gathered by the GEMM's tensor copies straight from x).
 uint64_t gathered_x_bytes(uint64_t R, uint32_t k, int x_dtype);
 
+// W4A4 on the block-scaled MMA (NVFP4 weights, k % 256 == 0, contiguous, no bias or
+// gated output): the activations' codes [m, k/2], E4M3 factors [m, k/16] and
+// per-token scales [m] from launch_quant_act; tiles of up to 128 pairs.
+bool w4a4_mma_supported(const QmmArgs &a);
+cudaError_t launch_gemm_w4a4(const QmmArgs &a, const uint8_t *xcodes, const uint8_t *xscales, const float *gscale,
+                             const uint32_t *offsets, const uint32_t *sorted_pairs, const uint32_t *tiles,
+                             const uint32_t *tile_count, uint32_t max_tiles, uint32_t *err, uint32_t *work_counter,
+                             cudaStream_t st);
 // tcgen05 grouped GEMM over the routing prologue's tiles (xg: gathered f32 x rows, or null).
 bool gemm_supported(const QmmArgs &a);
 uint32_t gemm_tile_rows(const QmmArgs &a);

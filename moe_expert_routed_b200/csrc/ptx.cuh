@@ -254,5 +254,37 @@ __host__ __device__ __forceinline__ uint32_t idesc_f16(uint32_t ab_type, uint32_
     return (1u << 4) | (ab_type << 7) | (ab_type << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// 32 lanes x 16 consecutive 32-bit columns from registers (the store counterpart of
+// tmem_ld16): thread i of the warp writes lane (warp's quarter * 32 + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[128 x N] (+)= A[128 x 64] * B[N x 64]^T with A and B packed E2M1 (two per byte,
+// K-major in the 128-byte swizzle), every 16 values along K scaled by an E4M3 factor
+// held in tensor memory: sfa / sfb address the A and B factors of this K-block.
+__device__ __forceinline__ void mma_nvf4_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with E4M3 block factors (one per 16
+// values): A and B E2M1 (format 1), fp32 D, K-major, M = 128, N = n.
+__host__ __device__ __forceinline__ uint32_t idesc_nvf4(uint32_t n) {
+    return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 }  // namespace ptx
 }  // namespace moe

@@ -286,6 +286,7 @@ x_image(const uint16_t *__restrict__ x, int x_dtype, uint32_t k, uint32_t ktiles
         const uint16_t *xr = x + tok * k;
         float mul = 1.f;
         if (live && tok_scale) mul = 1.f / __ldg(tok_scale + tok);  // an exact power of two
+#pragma unroll 4
         for (uint32_t q = lane; q < ktiles * 8u; q += 32u) {
             const uint32_t kt = q >> 3, c = q & 7u, j = kt * 64u + c * 8u;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);

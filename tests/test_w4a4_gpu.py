@@ -9,6 +9,9 @@
   tolerance) on the one-token decode kernel, the several-token decode path, the
   routed path and the grouped GEMM (16- and 256-pair tiles), with NVFP4 and affine
   weights, and the workspace check.
+- The block-scaled MMA (NVFP4 weights, k a multiple of 256): against the oracle,
+  and against the bf16-operand GEMM (forced through moe_qmm_test_x_copies), with
+  partial tiles, a ragged last row block, bf16 output and out-of-range ids.
 """
 
 import numpy as np
@@ -96,3 +99,37 @@ def test_w4a4_workspace_check():
         M.qmm_id_w4a4(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], n=P.n, group_size=16, bits=4,
                       fmt=FMT_NVFP4, num_experts=4, workspace=small)
     assert exc.value.status == 3
+
+
+@pytest.mark.parametrize("m,topk,E,k,n,od", [
+    (600, 2, 8, 1024, 200, DT_BF16),   # 150 pairs per expert: a full and a partial 128-pair tile
+    (90, 4, 6, 512, 128, DT_F32),      # 60 pairs per expert
+    (2000, 8, 16, 2048, 384, DT_BF16), # 1000 pairs per expert, several k-tiles of 256
+])
+def test_w4a4_block_scaled_mma(m, topk, E, k, n, od):
+    P = make_problem("w4a4-mma", seed=6300 + m + k, fmt=FMT_NVFP4, bits=4, group_size=16, m=m, k=k, n=n,
+                     n_expert_used=topk, num_experts=E, x_dtype=DT_BF16, out_dtype=od)
+    ids = P.ids.copy()
+    ids[1, 0] = P.num_experts          # an out-of-range id: zero row and the error word
+    P = P.with_ids(ids)
+    d = to_device(P)
+    odt = {DT_F32: torch.float32, DT_BF16: torch.bfloat16}[od]
+    ws = torch.zeros(M.workspace_bytes_w4a4(P.m, P.k, P.n_expert_used, P.num_experts), dtype=torch.uint8,
+                     device="cuda")
+    kw = dict(n=P.n, group_size=16, bits=4, fmt=FMT_NVFP4, num_experts=P.num_experts, out_dtype=odt, path="grouped")
+    out = M.qmm_id_w4a4(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], workspace=ws, **kw)
+    torch.cuda.synchronize()
+    assert M.poll_error(ws[M.workspace_bytes_w4a4(P.m, P.k, P.n_expert_used, P.num_experts)
+                           - M.workspace_bytes(P.m, P.n_expert_used, P.num_experts):]) == 5
+    Q = oracle.w4a4_problem(P)
+    nviol, ratio, info = check_full(Q, out)
+    assert nviol == 0, f"block-scaled: {nviol} outside tolerance ({ratio:.3g}, {info})"
+    L = M.lib()
+    assert L.moe_qmm_test_x_copies(1) == 0
+    try:
+        ref = M.qmm_id_w4a4(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], **kw)
+    finally:
+        assert L.moe_qmm_test_x_copies(0) == 0
+    torch.cuda.synchronize()
+    nviol, ratio, info = check_full(Q, ref)
+    assert nviol == 0, f"bf16 operand: {nviol} outside tolerance ({ratio:.3g}, {info})"
