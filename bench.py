@@ -529,9 +529,10 @@ def grouped_tile_rows(P) -> int:
 
 
 def w4a4_entry(pk: dict) -> dict:
-    """The prefill workload with W4A4 (x quantised per token to NVFP4 first,
-    moe_qmm_id_w4a4): per-call time from a CUDA graph of GRAPH_CALLS calls (median of
-    REPEATS replays), and the activation quantisation alone timed the same way."""
+    """The prefill workload with W4A4 (x quantised per token to NVFP4 first, then the
+    block-scaled MMA; moe_qmm_id_w4a4): per-call time from a CUDA graph of GRAPH_CALLS
+    calls (median of REPEATS replays), and the activation quantisation alone timed
+    the same way."""
     import moe_expert_routed_b200 as M
     from workloads import config_problem
     from workloads.torch_io import to_device
@@ -569,13 +570,17 @@ def w4a4_entry(pk: dict) -> dict:
     flops = 2.0 * int((ids < P.num_experts).sum()) * P.n * P.k
     us = rc["s"] * 1e6
     tf = flops / us / 1e6
+    # the block-scaled fp4 MMA's peak: the measured bf16 peak times the nominal dense
+    # ratio of the two (9 / 2.25 PFLOP/s per GPU)
+    fp4_peak = 4.0 * pk["bf16_tflops"]
     ent = {
         "workload": "prefill with W4A4: x quantised per token to NVFP4 (E2M1 codes, E4M3 scales per 16, f32 "
-                    "per-token scale), then the operation on the dequantised x (f32 operands split into bf16 "
-                    "halves on the tensor cores)",
+                    "per-token scale), then the block-scaled tensor-core MMA (kind::mxf4nvf4) on the codes of "
+                    "both operands",
         "us_per_call": us, "quantize_us": rq["s"] * 1e6, "TFLOP_per_s": tf,
-        "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": tf / pk["bf16_tflops"], "peak_source": pk["source"] + " (bf16_tflops burst)"},
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": tf / fp4_peak, "bf16_frac": tf / pk["bf16_tflops"],
+                     "peak_source": pk["source"] + " bf16_tflops x 4 (nominal dense fp4 / bf16 ratio)"},
         "repeats_us": rc["repeats_us"],
         "timing": f"CUDA graph of {GRAPH_CALLS} calls, median of {REPEATS} replays",
     }
@@ -933,12 +938,27 @@ def run_crossover(args):
 def run_probe(args):
     """A few untimed calls of one workload (for profiler captures): decode runs the
     gate/up projection `reps` times, then the down projection `reps` times; the
-    grouped configs run one full call `reps` times."""
+    grouped configs run one full call `reps` times; prefill_w4a4 runs the prefill
+    workload through moe_qmm_id_w4a4 `reps` times."""
     import moe_expert_routed_b200 as M
     from workloads import config_problem
     from workloads.torch_io import to_device
 
     M.lib()
+    if args.probe == "prefill_w4a4":
+        P = config_problem("prefill")
+        d = to_device(P)
+        ws = torch.zeros(M.workspace_bytes_w4a4(P.m, P.k, P.n_expert_used, P.num_experts), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.empty((P.m, P.n_expert_used, P.n), dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.reps):
+            M.qmm_id_w4a4(d["x"], d["ids"], d["packed"], d["scales"], d["aux"], n=P.n, group_size=P.group_size,
+                          bits=P.bits, fmt=P.fmt, num_experts=P.num_experts, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        if M.poll_error(ws) != 0:
+            raise SystemExit("prefill_w4a4: device error word set")
+        print(json.dumps({"probe": args.probe, "reps": args.reps, "status": "ok"}))
+        return
     names = ["decode_gate_up", "decode_down"] if args.probe == "decode" else [args.probe]
     for name in names:
         P = config_problem(name)
@@ -966,7 +986,7 @@ def main():
                     help="decode step without programmatic dependent launch between its calls")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--config", default="decode", choices=["decode", "canvas", "prefill", "skewed"])
-    ap.add_argument("--probe", choices=["decode", "canvas", "prefill", "skewed"],
+    ap.add_argument("--probe", choices=["decode", "canvas", "prefill", "skewed", "prefill_w4a4"],
                     help="run a few untimed calls (for profiler captures) and exit")
     ap.add_argument("--reps", type=int, default=4)
     ap.add_argument("--no-extras", action="store_true",
