@@ -560,6 +560,8 @@ def w4a4_entry(pk: dict) -> dict:
 
     call(0)
     torch.cuda.synchronize()
+    if M.poll_error(ws) != 0:
+        raise RuntimeError("prefill with W4A4: device error word set")
     gc = capture_graph(call, GRAPH_CALLS)
     rc = per_call(gc, GRAPH_CALLS)
     del gc

@@ -285,13 +285,20 @@ size_t moe_qmm_id_workspace_bytes_k(uint32_t m, uint32_t k, uint32_t n_expert_us
  *   scales [m, k/16] E4M3 bytes; gscale [m] f32; xhat [m, k] f32 (x^ rounded once
  *   to f32; 16-byte aligned).
  * moe_qmm_id_w4a4 -- arguments as moe_qmm_id_path (any weight format; the path
- *   argument may carry launch flags). The CUDA-core paths take x^ as f32 x; the
- *   grouped GEMM takes e2m1(q) * e4m3(s_b) as bf16 (exact) and multiplies each
- *   output by its token's g_t before the single rounding. The workspace holds x^
- *   (f32 [m, k]), the bf16 values [m, k] and g [m] (each section rounded up to 256
- *   bytes), then the operation's own workspace: at least
- *   moe_qmm_id_workspace_bytes_w4a4(m, k, n_expert_used, num_experts) bytes (else
- *   MOE_ERR_WORKSPACE_TOO_SMALL). Errors as moe_qmm_id.
+ *   argument may carry launch flags). The CUDA-core paths take x^ as f32 x. The
+ *   grouped GEMM, for NVFP4 weights with k a multiple of 256, no bias, gated output
+ *   or pointer table and 16-byte aligned packed rows, runs the block-scaled
+ *   tensor-core MMA on the E2M1 codes of both operands with their E4M3 block scales;
+ *   otherwise it takes e2m1(q) * e4m3(s_b) as bf16 (exact). Either way each output
+ *   is multiplied by scale2 and its token's g_t before the single rounding.
+ *   workspace: at least moe_qmm_id_workspace_bytes_w4a4(m, k, n_expert_used,
+ *   num_experts) bytes, 16-byte aligned (else MOE_ERR_WORKSPACE_TOO_SMALL). It
+ *   starts with the operation's own workspace, whose first 4 bytes are the device
+ *   error word that moe_qmm_id_poll_error(workspace, ...) reads and clears, as for
+ *   moe_qmm_id; the quantised x (x^ f32 [m, k], the bf16 values [m, k], g [m], the
+ *   codes [m, k/2], the scales [m, k/16], each section rounded up to 256 bytes)
+ *   fills the end, from the last 256-byte boundary that leaves room for it. Errors
+ *   as moe_qmm_id.
  */
 size_t moe_qmm_id_workspace_bytes_w4a4(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts);
 moe_status moe_quantize_act_nvfp4(const void *x, uint32_t m, uint32_t k, moe_dtype x_dtype, uint8_t *codes,

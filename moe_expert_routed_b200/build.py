@@ -64,7 +64,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         objs = list(ex.map(compile_one, SOURCES))
     tmp = LIB + ".tmp"
-    subprocess.check_call([cc, "-shared", "-o", tmp, *objs, "-cudart", "static"])
+    subprocess.check_call([cc, "-shared", *NVCC_FLAGS[:2], "-o", tmp, *objs, "-cudart", "static"])
     os.replace(tmp, LIB)
     if verbose:
         print(f"built {LIB}")

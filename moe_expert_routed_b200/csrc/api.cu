@@ -339,7 +339,7 @@ moe_status moe_qmm_id_glu(const void *x, const uint32_t *ids, const void *packed
 size_t moe_qmm_id_workspace_bytes_w4a4(uint32_t m, uint32_t k, uint32_t n_expert_used, uint32_t num_experts) {
     const size_t rest = moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts);
     if (!rest) return 0;
-    return moe::w4a4_front_bytes(m, k) + rest;
+    return moe::al256(rest) + moe::w4a4_front_bytes(m, k);
 }
 
 moe_status moe_quantize_act_nvfp4(const void *x, uint32_t m, uint32_t k, moe_dtype x_dtype, uint8_t *codes,
@@ -365,12 +365,15 @@ moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packe
     if (v != MOE_OK) return v;
     if (k % 16u != 0) return MOE_ERR_UNSUPPORTED;
     if (!workspace || ((uintptr_t)workspace & 15u)) return MOE_ERR_INVALID_ARGUMENT;
+    // the operation's own workspace first (its error word at the start, as for
+    // moe_qmm_id), then, from the last 256-byte boundary that leaves room for them,
     // x^ (f32), the bf16 values without the per-token factor, the per-token factors,
-    // then the operation's own workspace
+    // the E2M1 codes and the E4M3 block scales
     const size_t front = moe::w4a4_front_bytes(m, k);
-    if (workspace_bytes < front + moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts))
-        return MOE_ERR_WORKSPACE_TOO_SMALL;
-    uint8_t *w = (uint8_t *)workspace;
+    if (workspace_bytes < front) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    const size_t own = (workspace_bytes - front) & ~(size_t)255;
+    if (own < moe_qmm_id_workspace_bytes(m, n_expert_used, num_experts)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *w = (uint8_t *)workspace + own;
     size_t o = 0;
     float *xhat = (float *)(w + o);
     o += moe::al256((uint64_t)m * k * 4ull);
@@ -384,7 +387,7 @@ moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packe
     if (moe::launch_quant_act(x, (int)x_dtype, m, k, codes, xs, g, xhat, x16, (cudaStream_t)stream) != cudaSuccess)
         return MOE_ERR_CUDA;
     return moe::run(xhat, ids, packed, scales, aux, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
-                    num_experts, MOE_F32, out_dtype, MOE_F32, w + front, workspace_bytes - front, stream, path,
+                    num_experts, MOE_F32, out_dtype, MOE_F32, workspace, own, stream, path,
                     {nullptr, nullptr, nullptr}, -1, x16, g, codes, xs);
 }
 

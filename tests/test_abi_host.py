@@ -72,6 +72,23 @@ def test_workspace_bytes_with_gathered_x():
     assert M.lib().moe_qmm_id_workspace_bytes_k(512, 1024, 8, 64, 3) == 0         # not a moe_dtype
 
 
+def test_w4a4_workspace_layout():
+    """The W4A4 call's own workspace (rounded up to 256 bytes) comes first, then x^ f32,
+    the bf16 values, g, the codes and the scales, each rounded up to 256 bytes."""
+    al = lambda v: (v + 255) // 256 * 256
+    for m, k, topk, E in [(3, 256, 2, 5), (4096, 4096, 8, 128), (17, 48, 1, 1)]:
+        front = al(m * k * 4) + al(m * k * 2) + al(m * 4) + al(m * k // 2) + al(m * k // 16)
+        assert M.workspace_bytes_w4a4(m, k, topk, E) == al(M.workspace_bytes(m, topk, E)) + front
+    L = M.lib()
+
+    def call(wsb, k=256):
+        return L.moe_qmm_id_w4a4(16, 16, 16, 16, 16, 16, 4, k, 128, 16, 4, 2, 2, 8, 0, 0, 4096, wsb, None, 0)
+    need = M.workspace_bytes_w4a4(4, 256, 2, 8)
+    assert call(need - 1) == 3        # one byte short: rejected before any CUDA call
+    assert call(64) == 3
+    assert call(need, k=250) == 2     # k not a multiple of the 16-value group: unsupported
+
+
 def test_x_copies_hook_rejects_other_values():
     L = M.lib()
     assert L.moe_qmm_test_x_copies(2) == 1
