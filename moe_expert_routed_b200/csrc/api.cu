@@ -147,15 +147,27 @@ struct PtrTables {
     const uint64_t *packed, *scales, *biases;
 };
 
+// W4A4: the activations to quantise and where each quantised form goes; run()
+// writes only the forms the chosen path reads.
+struct W4A4Front {
+    const void *x;       // [m, k] of x_dtype
+    int x_dtype;
+    float *xhat;         // [m, k] f32 x^ (CUDA-core paths)
+    uint16_t *x16;       // [m, k] bf16 e2m1(q) * e4m3(s) (grouped GEMM on the kind::f16 MMA)
+    float *g;            // [m] per-token factors (grouped GEMM)
+    uint8_t *codes;      // [m, k/2] E2M1 codes (block-scaled MMA)
+    uint8_t *xs;         // [m, k/16] E4M3 block scales (block-scaled MMA)
+};
+
 // moe_qmm_id with an optional per-expert output bias (null: none), optional
 // pointer-table weights and an optional gated output (act >= 0: act(gate) * up).
+// With w4 (W4A4), x is w4->xhat, written here before the path's kernels.
 moe_status run(const void *x, const uint32_t *ids, const void *packed, const void *scales, const void *aux,
                const void *bias, void *out, uint32_t m, uint32_t k, uint32_t n, uint32_t group_size,
                uint32_t bits, moe_fmt fmt, uint32_t n_expert_used, uint32_t num_experts, moe_dtype x_dtype,
                moe_dtype out_dtype, moe_dtype bias_dtype, void *workspace, size_t workspace_bytes,
                moe_stream_t stream, moe_path path, PtrTables pt = {nullptr, nullptr, nullptr}, int act = -1,
-               const uint16_t *w4a4_x16 = nullptr, const float *w4a4_scale = nullptr,
-               const uint8_t *w4a4_codes = nullptr, const uint8_t *w4a4_xscales = nullptr) {
+               const W4A4Front *w4 = nullptr) {
     moe_status v = validate(x, ids, pt.packed ? (const void *)pt.packed : packed,
                             pt.packed ? (const void *)pt.scales : scales, aux, out, m, k, n, group_size, bits,
                             fmt, n_expert_used, num_experts, x_dtype, out_dtype);
@@ -219,16 +231,21 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
     // W4A4 on the grouped GEMM: the block-scaled MMA on the activations' NVFP4 codes
     // where it applies; else bf16 e2m1(q) * e4m3(s) (exact) as the B operand and the
     // per-token factor in the epilogue, instead of the f32 x^ the CUDA-core paths take
-    const bool w4mma = choice == GROUPED && w4a4_codes && w4a4_xscales && w4a4_scale && !a.x_copies &&
-                       w4a4_mma_supported(a);
-    if (choice == GROUPED && !w4mma && w4a4_x16 && w4a4_scale) {
-        a.x = w4a4_x16;
+    const bool w4mma = w4 && choice == GROUPED && !a.x_copies && w4a4_mma_supported(a);
+    const bool w4x16 = w4 && choice == GROUPED && !w4mma;
+    if (w4x16) {
+        a.x = w4->x16;
         a.x_dtype = DT_BF16;
-        x = w4a4_x16;
+        x = w4->x16;
         x_dtype = MOE_BF16;
-        a.tok_scale = w4a4_scale;
+        a.tok_scale = w4->g;
         if (!gemm_supported(a)) return MOE_ERR_UNSUPPORTED;
     }
+    if (w4 && moe::launch_quant_act(w4->x, w4->x_dtype, m, k, w4mma ? w4->codes : nullptr,
+                                    w4mma ? w4->xs : nullptr, (w4mma || w4x16) ? w4->g : nullptr,
+                                    (w4mma || w4x16) ? nullptr : w4->xhat, w4x16 ? w4->x16 : nullptr,
+                                    (cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
 
     cudaError_t ce;
     if (choice == FUSED) {
@@ -273,7 +290,7 @@ moe_status run(const void *x, const uint32_t *ids, const void *packed, const voi
         }
         if (ce == cudaSuccess) {
             if (w4mma)
-                ce = launch_gemm_w4a4(a, w4a4_codes, w4a4_xscales, w4a4_scale, offsets, sp, tiles, tc, max_tiles,
+                ce = launch_gemm_w4a4(a, w4->codes, w4->xs, w4->g, offsets, sp, tiles, tc, max_tiles,
                                       err, wc, st);
             else if (choice == GROUPED)
                 ce = launch_gemm(a, offsets, sp, tiles, tc, max_tiles, err, wc, xg, ximg, st);
@@ -384,11 +401,10 @@ moe_status moe_qmm_id_w4a4(const void *x, const uint32_t *ids, const void *packe
     uint8_t *codes = w + o;
     o += moe::al256((uint64_t)m * k / 2ull);
     uint8_t *xs = w + o;
-    if (moe::launch_quant_act(x, (int)x_dtype, m, k, codes, xs, g, xhat, x16, (cudaStream_t)stream) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    const moe::W4A4Front w4{x, (int)x_dtype, xhat, x16, g, codes, xs};
     return moe::run(xhat, ids, packed, scales, aux, nullptr, out, m, k, n, group_size, bits, fmt, n_expert_used,
                     num_experts, MOE_F32, out_dtype, MOE_F32, workspace, own, stream, path,
-                    {nullptr, nullptr, nullptr}, -1, x16, g, codes, xs);
+                    {nullptr, nullptr, nullptr}, -1, &w4);
 }
 
 moe_status moe_qmm_id(const void *x, const uint32_t *ids, const void *packed, const void *scales,
