@@ -254,10 +254,11 @@ __device__ __forceinline__ void dequant32(const uint32_t (&w)[Raw<KIND>::W], flo
 
 // Store 32 fp32 weights as 4 chunks of 8 16-bit values at chunk positions
 // c0..c0+3 of row r: the 16-bit rounding (hi) and, for two-term formats, the
-// 16-bit rounding of the remainder (lo).
-template <bool F16, bool TWO>
+// 16-bit rounding of the remainder (lo). TM: into the words hw / lw instead (word
+// j holds values 2j and 2j+1), for a store to tensor memory.
+template <bool F16, bool TWO, bool TM = false>
 __device__ __forceinline__ void store_a(const float (&v)[32], uint32_t a_hi, uint32_t a_lo, uint32_t r,
-                                        uint32_t c0) {
+                                        uint32_t c0, uint32_t (&hw)[16], uint32_t (&lw)[16]) {
 #pragma unroll
     for (int cc = 0; cc < 4; cc++) {
         uint32_t hh[4], ll[4];
@@ -270,9 +271,17 @@ __device__ __forceinline__ void store_a(const float (&v)[32], uint32_t a_hi, uin
                 ll[e] = pack2<F16>(x0 - h.x, x1 - h.y);
             }
         }
-        const uint32_t off = swz(r, c0 + cc);
-        sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
-        if constexpr (TWO) sts128(a_lo + off, ll[0], ll[1], ll[2], ll[3]);
+        if constexpr (TM) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                hw[cc * 4 + e] = hh[e];
+                if constexpr (TWO) lw[cc * 4 + e] = ll[e];
+            }
+        } else {
+            const uint32_t off = swz(r, c0 + cc);
+            sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
+            if constexpr (TWO) sts128(a_lo + off, ll[0], ll[1], ll[2], ll[3]);
+        }
     }
 }
 
@@ -325,10 +334,11 @@ __device__ __forceinline__ void nvfp4_store(const uint32_t (&w)[4], __half2 s01,
 // are f16, so cb * s has at most 22 significant bits and hi + lo holds it to
 // within the f16 subnormal spacing (2^-24). Codes of a pair share a word (pairs
 // start at even positions and a 3-bit word holds 10 codes).
-template <int KIND, int SUB>
+template <int KIND, int SUB, bool TM = false>
 __device__ __forceinline__ void cb_pairs_f16(const uint32_t (&w)[Raw<KIND>::W], __half2 s0, __half2 s1,
                                              bool two_groups, const uint32_t *lut2, uint32_t a_hi,
-                                             uint32_t a_lo, uint32_t r, uint32_t c0) {
+                                             uint32_t a_lo, uint32_t r, uint32_t c0, uint32_t (&hw)[16],
+                                             uint32_t (&lw)[16]) {
     constexpr int B = kind_bits(KIND);
 #pragma unroll
     for (int cc = 0; cc < 4; cc++) {
@@ -351,17 +361,25 @@ __device__ __forceinline__ void cb_pairs_f16(const uint32_t (&w)[Raw<KIND>::W], 
             hh[e] = *reinterpret_cast<const uint32_t *>(&hi);
             ll[e] = *reinterpret_cast<const uint32_t *>(&lo);
         }
-        const uint32_t off = swz(r, c0 + cc);
-        sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
-        sts128(a_lo + off, ll[0], ll[1], ll[2], ll[3]);
+        if constexpr (TM) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                hw[cc * 4 + e] = hh[e];
+                lw[cc * 4 + e] = ll[e];
+            }
+        } else {
+            const uint32_t off = swz(r, c0 + cc);
+            sts128(a_hi + off, hh[0], hh[1], hh[2], hh[3]);
+            sts128(a_lo + off, ll[0], ll[1], ll[2], ll[3]);
+        }
     }
 }
 
-template <int KIND, bool F16>
+template <int KIND, bool F16, bool TM = false>
 __device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], uint32_t sub, float s0,
                                              float b0, float s1, float b1, bool two_groups,
                                              const float *cb, uint32_t a_hi, uint32_t a_lo, uint32_t r,
-                                             uint32_t c0) {
+                                             uint32_t c0, uint32_t (&hw)[16], uint32_t (&lw)[16]) {
     static_assert(KIND != K_NVFP4, "NVFP4 tiles go through nvfp4_store");
     constexpr bool TWO = a_terms<KIND>() == 2;
     {
@@ -377,7 +395,7 @@ __device__ __forceinline__ void dequant_tile(const uint32_t (&w)[Raw<KIND>::W], 
         } else {
             dequant32<KIND, 0>(w, s0, b0, s1, b1, two_groups, cb, v);
         }
-        store_a<F16, TWO>(v, a_hi, a_lo, r, c0);
+        store_a<F16, TWO, TM>(v, a_hi, a_lo, r, c0, hw, lw);
     }
 }
 
@@ -426,12 +444,19 @@ __device__ __forceinline__ void global_scale(const uint8_t *srow, const uint8_t 
     }
 }
 
+// ATM: the two-term A operand (affine, codebook) of tiles up to 128 pairs wide lives
+// in tensor memory: the dequantisers store it with tcgen05.st and the MMAs read it
+// from there (A_TM_COLS columns per term and stage after the two accumulators), so
+// the stage in shared memory holds only B and the staged codes. Wider tiles leave no
+// room beside their accumulators and keep A in shared memory.
+constexpr uint32_t A_TM_COLS = KT / 2;  // 16-bit values, two per 32-bit column
 template <int KIND, int XT, int BN>
 struct GemmCfg {
     static constexpr int AT = a_terms<KIND>();
     static constexpr int BT = (XT == DT_F32) ? 2 : 1;
+    static constexpr bool ATM = AT == 2 && BN <= 128;
     static constexpr int B_TILE = BN * KT * 2;
-    static constexpr uint32_t STAGE = AT * A_TILE + BT * B_TILE + RawLayout<KIND>::TILE;
+    static constexpr uint32_t STAGE = (ATM ? 0u : AT * A_TILE) + BT * B_TILE + RawLayout<KIND>::TILE;
 };
 
 // Work item w of the persistent grid: tile w / n_mtiles of the routing prologue's
@@ -495,7 +520,8 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
     static_assert(!XIMG || (XT == DT_F16 && !PTRS && !GLU), "the image is f16, for the plain kernel");
     constexpr int AT = C::AT, BT = C::BT, B_TILE = C::B_TILE;
     constexpr uint32_t STAGE = C::STAGE;
-    constexpr uint32_t B_OFF = AT * A_TILE, RAW_OFF = AT * A_TILE + BT * B_TILE;
+    constexpr bool ATM = C::ATM;
+    constexpr uint32_t B_OFF = ATM ? 0u : AT * A_TILE, RAW_OFF = B_OFF + BT * B_TILE;
     constexpr bool F16 = (XT == DT_F16);
     constexpr uint32_t ES = (KIND == K_NVFP4 || KIND == K_MXFP4) ? 1u : 2u;  // bytes per scale
     constexpr bool AFF = (KIND == K_AFF4 || KIND == K_AFF6 || KIND == K_AFF8);
@@ -504,8 +530,9 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
     // the other
     static_assert(BN == 64 || BN == 128 || BN == 256, "tile widths");
     constexpr uint32_t NACC = 2u;
-    constexpr uint32_t TMEM_COLS = 2u * BN;
+    constexpr uint32_t TMEM_COLS = ATM ? 512u : 2u * BN;
     constexpr uint32_t ACC_STRIDE = BN;
+    constexpr uint32_t ACOL0 = 2u * BN;  // ATM: A of stage s, term t at ACOL0 + (s AT + t) A_TM_COLS
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[3 * MAX_STAGES + 6 + 2 * RING];
@@ -650,6 +677,7 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                 const uint8_t *sw_row = tma ? ct + RL::TMA_SC + 16u * r : rr + RL::SC;
                 uint32_t wv[Raw<KIND>::W];
                 uint32_t sub = 0;
+                uint32_t hw[16], lw[16];  // ATM: this thread's A words (hi and lo terms)
                 if constexpr (KIND == K_AFF4 || KIND == K_CB4 || KIND == K_NVFP4 || KIND == K_MXFP4) {
                     const uint4 q = *(const uint4 *)(tma ? ct + tma_chunk<KIND>(sr, h) : rr + 16u * h);
                     wv[0] = q.x; wv[1] = q.y; wv[2] = q.z; wv[3] = q.w;
@@ -710,20 +738,31 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
                         const __half2 h0 = __float2half2_rn(s0), h1 = __float2half2_rn(s1);  // exact: f16 scales
                         if constexpr (KIND == K_CB3) {
                             switch (sub) {  // first code's position in word 0: 0, 2, 4, 6 or 8
-                                case 0: cb_pairs_f16<KIND, 0>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                                case 2: cb_pairs_f16<KIND, 2>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                                case 4: cb_pairs_f16<KIND, 4>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                                case 6: cb_pairs_f16<KIND, 6>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
-                                default: cb_pairs_f16<KIND, 8>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u); break;
+                                case 0: cb_pairs_f16<KIND, 0, ATM>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u, hw, lw); break;
+                                case 2: cb_pairs_f16<KIND, 2, ATM>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u, hw, lw); break;
+                                case 4: cb_pairs_f16<KIND, 4, ATM>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u, hw, lw); break;
+                                case 6: cb_pairs_f16<KIND, 6, ATM>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u, hw, lw); break;
+                                default: cb_pairs_f16<KIND, 8, ATM>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u, hw, lw); break;
                             }
                         } else {
-                            cb_pairs_f16<KIND, 0>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u);
+                            cb_pairs_f16<KIND, 0, ATM>(wv, h0, h1, gs16, lut2_s, st, st + A_TILE, r, h * 4u, hw, lw);
                         }
                     } else {
-                        dequant_tile<KIND, F16>(wv, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u);
+                        dequant_tile<KIND, F16, ATM>(wv, sub, s0, b0, s1, b1, gs16, cb_s, st, st + A_TILE, r, h * 4u,
+                                                     hw, lw);
                     }
                 }
-                ptx::fence_proxy_async_smem();
+                if constexpr (ATM) {
+                    // this warp's 32 rows (its lane quarter), the thread's half of the k-tile
+                    const uint32_t ta = tmem + ((32u * (warp & 3u)) << 16) + ACOL0 + s * (AT * A_TM_COLS) + h * 16u;
+                    ptx::tmem_st16(ta, hw);
+                    ptx::tmem_st16(ta + A_TM_COLS, lw);
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    if (BT == 2 && xmode == XM_LOADERS) ptx::fence_proxy_async_smem();  // the rewritten B
+                } else {
+                    ptx::fence_proxy_async_smem();
+                }
                 ptx::mbar_arrive(full0 + 8 * s);
             }
             if (!ok) break;
@@ -945,11 +984,19 @@ grouped_gemm_kernel(const GemmParams P, const __grid_constant__ CUtensorMap tmap
 #pragma unroll
                     for (int ks = 0; ks < KT / 16; ks++) {
                         const uint32_t ko = ks * 32u;
-                        ptx::mma_f16_ss(d, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_hi + ko), idesc, accum);
-                        if constexpr (BT == 2)
-                            ptx::mma_f16_ss(d, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_lo + ko), idesc, 1);
-                        if constexpr (AT == 2)
-                            ptx::mma_f16_ss(d, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b_hi + ko), idesc, 1);
+                        if constexpr (ATM) {
+                            // 16 values of K: 8 columns of each A term
+                            const uint32_t ta = tmem + ACOL0 + s * (AT * A_TM_COLS) + ks * 8u;
+                            ptx::mma_f16_ts(d, ta, ptx::sdesc_k128(b_hi + ko), idesc, accum);
+                            if constexpr (BT == 2) ptx::mma_f16_ts(d, ta, ptx::sdesc_k128(b_lo + ko), idesc, 1);
+                            ptx::mma_f16_ts(d, ta + A_TM_COLS, ptx::sdesc_k128(b_hi + ko), idesc, 1);
+                        } else {
+                            ptx::mma_f16_ss(d, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_hi + ko), idesc, accum);
+                            if constexpr (BT == 2)
+                                ptx::mma_f16_ss(d, ptx::sdesc_k128(a_hi + ko), ptx::sdesc_k128(b_lo + ko), idesc, 1);
+                            if constexpr (AT == 2)
+                                ptx::mma_f16_ss(d, ptx::sdesc_k128(a_lo + ko), ptx::sdesc_k128(b_hi + ko), idesc, 1);
+                        }
                         accum = 1;
                     }
                     ptx::mma_commit(empty0 + 8 * s);
@@ -1096,10 +1143,15 @@ bool gemm_plan(const QmmArgs &a, GemmPlan *pl) {
     const bool fp4 = a.kind == K_NVFP4 || a.kind == K_MXFP4;  // single-term A
     const uint32_t bn = big ? (f32x ? 128u : 256u) : 64u;
     const uint32_t at = fp4 ? 1u : 2u, bt = f32x ? 2u : 1u;
-    const size_t stage = (size_t)at * A_TILE + (size_t)bt * bn * KT * 2 + raw_tile(a.kind);
+    const bool atm = at == 2u && bn <= 128u;  // A in tensor memory (GemmCfg::ATM)
+    const size_t stage = (atm ? 0u : (size_t)at * A_TILE) + (size_t)bt * bn * KT * 2 + raw_tile(a.kind);
     if (2 * stage + 1024 > GEMM_SMEM_BUDGET) return false;
     int S = (int)((GEMM_SMEM_BUDGET - 1024) / stage);
     S = S > MAX_STAGES ? MAX_STAGES : S;
+    if (atm) {  // the A terms of every stage beside the two accumulators in 512 columns
+        const int s_tm = (int)((512u - 2u * bn) / (at * A_TM_COLS));
+        S = S > s_tm ? s_tm : S;
+    }
     pl->bn = bn;
     pl->stages = S;
     pl->smem = (size_t)S * stage + 1024;

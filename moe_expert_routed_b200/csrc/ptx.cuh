@@ -208,6 +208,19 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t tmem_d, uint64_t adesc, uint
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16, with A in tensor memory: row m of
+// A in lane m, K along the columns, two 16-bit values per 32-bit column (the lower
+// half holds the even k); a_tmem addresses lane 0 and the first column of the step.
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive (once) on the mbarrier when all tcgen05 operations issued so far by
 // this thread have completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
