@@ -580,6 +580,7 @@ def w4a4_entry(pk: dict) -> dict:
                     "per-token scale), then the block-scaled tensor-core MMA (kind::mxf4nvf4) on the codes of "
                     "both operands",
         "us_per_call": us, "quantize_us": rq["s"] * 1e6, "TFLOP_per_s": tf,
+        "gpu_launches_per_call": 5,  # quantisation; routing histogram, scan, scatter; the block-scaled GEMM
         "roofline": {"bound": "tensor", "achieved": tf, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": tf / fp4_peak, "bf16_frac": tf / pk["bf16_tflops"],
                      "peak_source": pk["source"] + " bf16_tflops x 4 (nominal dense fp4 / bf16 ratio)"},
@@ -667,13 +668,27 @@ def grouped_entry(name: str, pk: dict) -> dict:
                      "peak_source": pk["source"] + " (bf16_tflops burst, hbm_gbs copy)"},
         "repeats_us": rc["repeats_us"], "route_repeats_us": rr["repeats_us"],
         "timing": f"CUDA graph of {GRAPH_CALLS} calls, median of {REPEATS} replays; routing prologue alone "
-                  f"the same way; gemm_us = call - routing (the x gather kernel and the GEMM)",
+                  f"the same way; gemm_us = call - routing (the x pre-pass kernels and the GEMM)",
         "l2": f"weights {P.packed.nbytes / 1e6:.0f} MB + x {P.x.nbytes / 1e6:.0f} MB (> L2 126 MB)",
-        "gpu_launches_per_call": 5,  # routing histogram, scan, scatter; x gather; GEMM
+        "gpu_launches_per_call": grouped_launches(P),
     }
     del d, out, ws, ws_r, rbuf
     torch.cuda.empty_cache()
     return ent
+
+
+def grouped_launches(P) -> int:
+    """Kernels of one grouped call with the k-aware workspace: the routing histogram,
+    scan and scatter; for f32 x the gather of its split rows; for 16-bit x with
+    256-pair tiles the f16 image of B (and, for bf16 x, the per-token factor
+    before it); the GEMM."""
+    R = P.m * P.n_expert_used
+    n = 3 + 1
+    if P.x_dtype == 0:
+        n += 1
+    elif R > 64 and R > 2 * P.num_experts and P.k % 8 == 0 and R >= 96 * P.num_experts:
+        n += 2 if P.x_dtype == 1 else 1
+    return n
 
 
 def decode_sweep(pk: dict) -> list:
