@@ -15,8 +15,11 @@
 // Warp roles (736 threads), each running through the CTA's items and their
 // k-tiles on its own; the stage ring continues from one item to the next:
 //   warps 0-7   dequantisers: per 64-wide k-tile, turn the staged codes of 128
-//               rows x 64 codes into 16-bit values in the 128-byte-swizzled
-//               K-major layout (and split f32 x into two bf16 halves).
+//               rows x 64 codes into 16-bit values: into tensor memory
+//               (tcgen05.st, one lane quarter per warp) for the two-term formats
+//               with tiles of up to 128 pairs, else into shared memory in the
+//               128-byte-swizzled K-major layout (and split f32 x into two bf16
+//               halves when the loaders copied it).
 //   warps 8-15  loaders: cp.async the pairs' x rows straight into the B operand
 //               tile and the packed codes and scale words into a staging area,
 //               up to S k-tiles ahead of the tensor core; each loader's
@@ -24,7 +27,8 @@
 //               engine (cp.async.mbarrier.arrive), so loaders never block on
 //               their own copies.
 //   warp 16     TMEM allocation; one lane issues tcgen05.mma (kind::f16, fp32
-//               accumulation in TMEM) and tcgen05.commit.
+//               accumulation in TMEM; A from tensor or shared memory, B from
+//               shared memory) and tcgen05.commit.
 //   warp 17     with TMA staging, one lane issues the k-tiles' tensor copies of
 //               the packed codes (no multicast), S k-tiles ahead like the loaders.
 //   warps 18-21 epilogue: TMEM -> registers (tcgen05.ld), times scale2 for
