@@ -1,12 +1,16 @@
 """Full-size workloads in the launch configuration the benchmark times (path
-"auto"), checked against the oracle on sampled outputs (the oracle computes them
-one by one) and on properties that hold at any size."""
+"auto", the workspace sized by moe_qmm_id_workspace_bytes_k, so that f32 x takes
+the gathered rows and 16-bit x with 256-pair tiles the f16 image of B), checked
+against the oracle on sampled outputs (the oracle computes them one by one) and on
+properties that hold at any size; the minimum workspace (loader copies of x) and
+W4A4 on the prefill workload (the block-scaled MMA) as well."""
 
 import numpy as np
 import pytest
 import torch
 
 import moe_expert_routed_b200 as M
+import oracle
 from tests.gpu_util import check_sampled, run, to_device
 from workloads import config_problem
 
@@ -22,9 +26,14 @@ def problem(request):
     return P, dev
 
 
+def _bench_workspace(P, dev):
+    """The workspace the benchmark gives a call: room for the grouped path's x pre-pass."""
+    return M.new_workspace(P.m, P.n_expert_used, P.num_experts, k=P.k, x_dtype=dev["x"].dtype)
+
+
 def test_sampled_parity(problem):
     P, dev = problem
-    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    ws = _bench_workspace(P, dev)
     out = run(P, "auto", dev=dev, workspace=ws)
     assert M.poll_error(ws) == 0
     rng = np.random.default_rng(17)
@@ -109,9 +118,46 @@ def _tile_class_sample(P):
 def test_every_tile_class(name):
     P = config_problem(name)
     dev = to_device(P)
-    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    ws = _bench_workspace(P, dev)
     out = run(P, "auto", dev=dev, workspace=ws)
     assert M.poll_error(ws) == 0
     pairs, cols = _tile_class_sample(P)
     nviol, ratio, info = check_sampled(P, out, pairs, cols)
     assert nviol == 0, f"{P.name}: {nviol} of {pairs.size} violations, worst err/bound {ratio:.3g} {info}"
+
+
+@pytest.mark.parametrize("name", ["prefill", "skewed"])
+def test_sampled_parity_minimum_workspace(name):
+    """The minimum workspace: the loader warps copy x rows themselves (f32 x split per
+    tile by the dequantisers)."""
+    P = config_problem(name)
+    dev = to_device(P)
+    ws = M.new_workspace(P.m, P.n_expert_used, P.num_experts)
+    out = run(P, "auto", dev=dev, workspace=ws)
+    assert M.poll_error(ws) == 0
+    rng = np.random.default_rng(23)
+    pairs = np.concatenate([rng.integers(0, P.R, 1500), np.full(64, P.R - 1)])
+    cols = np.concatenate([rng.integers(0, P.n, 1500), np.arange(P.n - 64, P.n)])
+    nviol, ratio, info = check_sampled(P, out, pairs, cols)
+    assert nviol == 0, f"{P.name}: {nviol} violations, worst err/bound {ratio:.3g} {info}"
+
+
+def test_w4a4_prefill_sampled():
+    """W4A4 on the prefill workload as the benchmark runs it (NVFP4 weights: the
+    block-scaled MMA on the codes of both operands), against the oracle's operation
+    on its own quantisation of x, on sampled outputs, whole rows and the last rows."""
+    P = config_problem("prefill")
+    dev = to_device(P)
+    ws = torch.zeros(M.workspace_bytes_w4a4(P.m, P.k, P.n_expert_used, P.num_experts), dtype=torch.uint8,
+                     device="cuda")
+    out = M.qmm_id_w4a4(dev["x"], dev["ids"], dev["packed"], dev["scales"], dev["aux"], n=P.n,
+                        group_size=P.group_size, bits=P.bits, fmt=P.fmt, num_experts=P.num_experts,
+                        out_dtype=torch.bfloat16, workspace=ws)
+    assert M.poll_error(ws) == 0
+    Q = oracle.w4a4_problem(P)
+    rng = np.random.default_rng(29)
+    pairs = np.concatenate([rng.integers(0, P.R, 2000), np.repeat(rng.integers(0, P.R, 2), P.n),
+                            np.full(64, P.R - 1)])
+    cols = np.concatenate([rng.integers(0, P.n, 2000), np.tile(np.arange(P.n), 2), np.arange(P.n - 64, P.n)])
+    nviol, ratio, info = check_sampled(Q, out, pairs, cols)
+    assert nviol == 0, f"W4A4 prefill: {nviol} violations, worst err/bound {ratio:.3g} {info}"
