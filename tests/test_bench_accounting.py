@@ -46,3 +46,16 @@ def test_out_of_range_ids_touch_no_expert():
     ids = np.array([0, 1, P.num_experts, 0xFFFFFFFF], dtype=np.uint32)
     two = bench.alg_bytes(P, ids[:2])
     assert bench.alg_bytes(P, ids) == two
+
+
+def test_grouped_launch_counts():
+    """Kernels per grouped call, as the bench reports them (gpu_launches): routing
+    histogram, scan and scatter, then the GEMM; f32 x adds the gather of its split
+    rows (skewed); bf16 x with 256-pair tiles adds the per-token factor and the f16
+    image of B (prefill); canvas (64-pair tiles, f16 x) adds nothing."""
+    expect = {"canvas": 4, "prefill": 6, "skewed": 5}
+    for name, n in expect.items():
+        c = CONFIGS[name]
+        P = types.SimpleNamespace(m=c["m"], n_expert_used=c["n_expert_used"], num_experts=c["num_experts"],
+                                  k=c["k"], x_dtype=c["x_dtype"])
+        assert bench.grouped_launches(P) == n, name
